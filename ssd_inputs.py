@@ -1,0 +1,236 @@
+"""Seeded synthetic inputs for the bidirectional SSD scan.
+
+This module is shared by the tests, the bench and the smoke check.  It draws
+random numbers and rounds them to the storage dtypes; it holds none of the
+scan's arithmetic.
+
+Generator
+---------
+Every tensor has its own counter-based stream: element ``i`` of tensor
+``tensor_id`` under ``seed`` is a pure function of ``(seed, tensor_id, i)``,
+so any element (or any sampled subset) can be regenerated on its own.
+
+* 64-bit mixing: the SplitMix64 finaliser (Steele, Lea & Flood, "Fast
+  splittable pseudorandom number generators", OOPSLA 2014): add the golden
+  gamma 0x9E3779B97F4A7C15, then ``z ^= z >> 30; z *= 0xBF58476D1CE4E5B9;
+  z ^= z >> 27; z *= 0x94D049BB133111EB; z ^= z >> 31``.
+* uniforms: the top 53 bits of a mixed word, offset by half an ulp, give a
+  double in the open interval (0, 1).
+* normals: Box-Muller, ``sqrt(-2 ln u1) * cos(2 pi u2)``, in float64.
+
+Distributions (the layer-shape workloads of the bidirectional SSD mixer):
+x ~ N(0,1); dt = softplus(N(0,1) - 4) (dt arrives positive, so the scan does
+no softplus of its own); A_h = -exp(U(0, ln 16)) in [-16, -1];
+B, C ~ N(0,1)/sqrt(d_state); D ~ U(0,1); residual ~ N(0,1); gate s ~ U(0, 0.5).
+
+Rounding: values are drawn in float64, rounded to float32 (round to nearest
+even), and, for bf16 tensors, rounded again float32 -> bf16 (nearest even).
+A and D are always float32.
+
+Tensor ids: forward {x:0, dt:1, A:2, B:3, C:4, D:5}; reverse adds 16;
+residual 32; gate 33; step k of a multi-step workload adds 64*k.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_GOLDEN = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+
+TENSOR_IDS = {"x": 0, "dt": 1, "A": 2, "B": 3, "C": 4, "D": 5}
+REV_OFFSET = 16
+RESIDUAL_ID = 32
+GATE_ID = 33
+STEP_STRIDE = 64
+
+_CHUNK = 1 << 22  # elements generated per slice, bounds temporary memory
+
+
+def _mix64(z: np.ndarray) -> np.ndarray:
+    z = z ^ (z >> np.uint64(30))
+    z = z * _M1
+    z = z ^ (z >> np.uint64(27))
+    z = z * _M2
+    return z ^ (z >> np.uint64(31))
+
+
+def _stream_key(seed: int, tensor_id: int) -> np.uint64:
+    with np.errstate(over="ignore"):
+        k = np.array([(seed << 32) | tensor_id], dtype=np.uint64)
+        return _mix64(k + _GOLDEN)[0]
+
+
+def _uniform_pair(key: np.uint64, idx: np.ndarray):
+    """Two independent uniforms in (0,1) for each flat index in ``idx``."""
+    with np.errstate(over="ignore"):
+        base = idx.astype(np.uint64) * np.uint64(2)
+        w1 = _mix64(key + (base + np.uint64(1)) * _GOLDEN)
+        w2 = _mix64(key + (base + np.uint64(2)) * _GOLDEN)
+    scale = 2.0 ** -53
+    u1 = ((w1 >> np.uint64(11)).astype(np.float64) + 0.5) * scale
+    u2 = ((w2 >> np.uint64(11)).astype(np.float64) + 0.5) * scale
+    return u1, u2
+
+
+def uniform(seed: int, tensor_id: int, n: int, idx: np.ndarray | None = None) -> np.ndarray:
+    key = _stream_key(seed, tensor_id)
+    if idx is not None:
+        return _uniform_pair(key, np.asarray(idx))[0]
+    out = np.empty(n, dtype=np.float64)
+    for s in range(0, n, _CHUNK):
+        e = min(n, s + _CHUNK)
+        out[s:e] = _uniform_pair(key, np.arange(s, e, dtype=np.uint64))[0]
+    return out
+
+
+def normal(seed: int, tensor_id: int, n: int, idx: np.ndarray | None = None) -> np.ndarray:
+    key = _stream_key(seed, tensor_id)
+
+    def _bm(ix):
+        u1, u2 = _uniform_pair(key, ix)
+        return np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * math.pi * u2)
+
+    if idx is not None:
+        return _bm(np.asarray(idx))
+    out = np.empty(n, dtype=np.float64)
+    for s in range(0, n, _CHUNK):
+        e = min(n, s + _CHUNK)
+        out[s:e] = _bm(np.arange(s, e, dtype=np.uint64))
+    return out
+
+
+# ---------------------------------------------------------------- rounding
+
+def f64_to_f32(a: np.ndarray) -> np.ndarray:
+    return np.asarray(a, dtype=np.float64).astype(np.float32)  # IEEE RNE
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bit patterns (uint16), round to nearest even (finite inputs)."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    lsb = (u >> np.uint32(16)) & np.uint32(1)
+    r = (u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)
+    return r.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+# ---------------------------------------------------------------- tensors
+
+@dataclass
+class Stored:
+    """One stored tensor: its storage dtype, the stored bits and the exact value as float64."""
+    dtype: str                 # "bf16" or "f32"
+    shape: tuple
+    data: np.ndarray           # uint16 bit patterns (bf16) or float32 values
+
+    def f64(self) -> np.ndarray:
+        if self.dtype == "bf16":
+            return bf16_bits_to_f32(self.data).astype(np.float64).reshape(self.shape)
+        return self.data.astype(np.float64).reshape(self.shape)
+
+    def torch(self, device="cpu"):
+        import torch
+        if self.dtype == "bf16":
+            t = torch.from_numpy(self.data.view(np.int16).reshape(self.shape)).view(torch.bfloat16)
+        else:
+            t = torch.from_numpy(self.data.reshape(self.shape))
+        return t.to(device) if device != "cpu" else t
+
+
+def _store(vals64: np.ndarray, dtype: str, shape) -> Stored:
+    f32 = f64_to_f32(vals64)
+    if dtype == "bf16":
+        return Stored("bf16", tuple(shape), f32_to_bf16_bits(f32))
+    return Stored("f32", tuple(shape), f32)
+
+
+@dataclass
+class Shape:
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int
+    dstate: int
+    ngroups: int = 1
+    io: str = "bf16"           # dtype of x, dt, B, C, y, residual
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.seqlen
+
+
+@dataclass
+class Params:
+    """One direction's parameter set (x, dt, A, B, C, D)."""
+    x: Stored
+    dt: Stored
+    A: Stored
+    B: Stored
+    C: Stored
+    D: Stored
+    extra: dict = field(default_factory=dict)
+
+
+def make_params(shape: Shape, seed: int = 0, offset: int = 0, with_D: bool = True) -> Params:
+    """Generate one direction's parameters; ``offset`` is added to every tensor id."""
+    b, L, H, P, N, G = (shape.batch, shape.seqlen, shape.nheads, shape.headdim,
+                        shape.dstate, shape.ngroups)
+    tid = {k: v + offset for k, v in TENSOR_IDS.items()}
+    x = normal(seed, tid["x"], b * L * H * P)
+    z = normal(seed, tid["dt"], b * L * H)
+    dt = np.log1p(np.exp(z - 4.0))
+    A = -np.exp(uniform(seed, tid["A"], H) * math.log(16.0))
+    Bv = normal(seed, tid["B"], b * L * G * N) / math.sqrt(N)
+    Cv = normal(seed, tid["C"], b * L * G * N) / math.sqrt(N)
+    D = uniform(seed, tid["D"], H) if with_D else np.zeros(H)
+    io = shape.io
+    return Params(
+        x=_store(x, io, (b, L, H, P)),
+        dt=_store(dt, io, (b, L, H)),
+        A=_store(A, "f32", (H,)),
+        B=_store(Bv, io, (b, L, G, N)),
+        C=_store(Cv, io, (b, L, G, N)),
+        D=_store(D, "f32", (H,)),
+        extra={"with_D": with_D},
+    )
+
+
+def make_bidir(shape: Shape, seed: int = 0, step: int = 0, with_D: bool = True):
+    """Forward and reverse parameter sets (independent draws, as two separate layers)."""
+    base = STEP_STRIDE * step
+    return (make_params(shape, seed, base, with_D),
+            make_params(shape, seed, base + REV_OFFSET, with_D))
+
+
+def make_residual(shape: Shape, seed: int = 0, step: int = 0) -> Stored:
+    b, L, H, P = shape.batch, shape.seqlen, shape.nheads, shape.headdim
+    r = normal(seed, RESIDUAL_ID + STEP_STRIDE * step, b * L * H * P)
+    return _store(r, shape.io, (b, L, H * P))
+
+
+def make_gate(seed: int = 0, step: int = 0) -> float:
+    """Gate scalar s ~ U(0, 0.5), stored as float32."""
+    u = uniform(seed, GATE_ID + STEP_STRIDE * step, 1)[0]
+    return float(np.float32(0.5 * u))
+
+
+# ------------------------------------------------------------- workloads
+
+# The five workloads: a tiny fp32 case the oracle checks exhaustively, two
+# bidirectional layer shapes of the DiffuMamba mixer (~240M and ~1.3B
+# models), a batch-1 long-sequence scaling case, and the R2L sidecar block.
+WORKLOADS = {
+    "tiny_f32": dict(shape=Shape(1, 64, 2, 16, 16, 1, "f32"), chunk=16, kind="bidir"),
+    "diffumamba_240m_L2048": dict(shape=Shape(8, 2048, 32, 64, 128, 1, "bf16"), chunk=256, kind="bidir"),
+    "diffumamba_1p3b_L8192": dict(shape=Shape(4, 8192, 64, 64, 128, 1, "bf16"), chunk=256, kind="bidir"),
+    "long_L32768": dict(shape=Shape(1, 32768, 64, 64, 128, 1, "bf16"), chunk=256, kind="bidir"),
+    "long_L131072": dict(shape=Shape(1, 131072, 64, 64, 128, 1, "bf16"), chunk=256, kind="bidir"),
+    "r2l_block_L32": dict(shape=Shape(8, 32, 32, 64, 64, 1, "bf16"), chunk=32, kind="r2l", steps=256),
+}

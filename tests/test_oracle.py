@@ -1,0 +1,212 @@
+"""Pins for the float64 oracle (CPU only).
+
+Every check here ties the oracle to something other than itself: a value
+worked by hand, the explicit semiseparable-matrix sum computed by brute
+force, a closed form (cumulative sum, geometric series, impulse response),
+or an identity of the recurrence (reverse = flip . forward . flip,
+linearity in x, chunk-size invariance of the chunked form).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import ssd_inputs as si
+from pins import matrix_form as _matrix_form, rand_params as _rand_params
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _scan(p, direction, **kw):
+    return oracle.ssd_scan_f64(p["x"], p["dt"], p["A"], p["B"], p["C"], p.get("D"), direction, **kw)
+
+
+# ----------------------------------------------------------------- golden
+
+def test_golden_handworked():
+    g = json.load(open(os.path.join(GOLDEN, "ssd_handworked_L3.json")))
+    p = dict(x=np.array(g["x"])[None, :, None, :], dt=np.array(g["dt"])[None, :, None],
+             A=np.array(g["A"]), B=np.array(g["B"])[None, :, None, :],
+             C=np.array(g["C"])[None, :, None, :], D=np.array(g["D"]))
+    tol = g["tolerance"]
+    yf = _scan(p, 1)[0, :, 0, :]
+    yr = _scan(p, -1)[0, :, 0, :]
+    np.testing.assert_allclose(yf, g["y_forward"], rtol=0, atol=tol)
+    np.testing.assert_allclose(yr, g["y_reverse"], rtol=0, atol=tol)
+    yb = oracle.bidir_f64(p, p)[0, :, 0, :]
+    np.testing.assert_allclose(yb, g["y_bidirectional"], rtol=0, atol=tol)
+    res = np.array(g["residual"])[None]
+    out = oracle.r2l_block_f64(p, g["gate_s"], res)[0]
+    np.testing.assert_allclose(out, g["r2l_out"], rtol=0, atol=tol)
+
+
+# ------------------------------------------------------------ matrix form
+
+@pytest.mark.parametrize("direction", [1, -1])
+def test_matrix_form_tiny_workload(direction):
+    """The tiny fp32 workload (b1 L64 H2 P16 N16), exact stored inputs, both directions."""
+    shape = si.WORKLOADS["tiny_f32"]["shape"]
+    pf, pr = si.make_bidir(shape, seed=0)
+    p = oracle.params_f64(pf if direction > 0 else pr)
+    y = _scan(p, direction)
+    ref = _matrix_form(p, direction)
+    assert oracle.rel_err(y, ref) <= 1e-12
+
+
+@pytest.mark.parametrize("direction", [1, -1])
+def test_matrix_form_groups_ragged(direction):
+    """Two groups over four heads (head h uses group h // 2), odd length, no D."""
+    rng = np.random.default_rng(7)
+    p = _rand_params(rng, 2, 13, 4, 3, 5, 2)
+    p["D"] = None
+    assert oracle.rel_err(_scan(p, direction), _matrix_form(p, direction)) <= 1e-12
+
+
+# ----------------------------------------------------------- closed forms
+
+def test_A_zero_is_cumulative_sum():
+    """A = 0: the state is the running sum of dt x (outer) B, so y_t = C_t . cumsum + D x_t."""
+    rng = np.random.default_rng(1)
+    p = _rand_params(rng, 2, 40, 3, 4, 6, 1, A_zero=True)
+    outer = p["dt"][..., None, None] * p["x"][..., :, None] * p["B"][:, :, 0][:, :, None, None, :]
+    Sc = np.cumsum(outer, axis=1)                                    # [b, L, H, P, N]
+    ref = np.einsum("blhpn,bln->blhp", Sc, p["C"][:, :, 0]) + p["D"][None, None, :, None] * p["x"]
+    assert oracle.rel_err(_scan(p, 1), ref) <= 1e-12
+    Sr = np.cumsum(outer[:, ::-1], axis=1)[:, ::-1]
+    ref_r = np.einsum("blhpn,bln->blhp", Sr, p["C"][:, :, 0]) + p["D"][None, None, :, None] * p["x"]
+    assert oracle.rel_err(_scan(p, -1), ref_r) <= 1e-12
+
+
+def test_scalar_state_is_plain_cumsum():
+    """N = 1, B = C = 1, A = 0, D = 0: the scan is the textbook cumulative sum of dt * x."""
+    rng = np.random.default_rng(2)
+    L = 50
+    x = rng.standard_normal((1, L, 1, 1)); dt = rng.uniform(0.1, 1.0, (1, L, 1))
+    ones = np.ones((1, L, 1, 1))
+    p = dict(x=x, dt=dt, A=np.zeros(1), B=ones, C=ones, D=None)
+    np.testing.assert_allclose(_scan(p, 1)[0, :, 0, 0], np.cumsum(dt[0, :, 0] * x[0, :, 0, 0]),
+                               rtol=1e-13, atol=1e-13)
+
+
+def test_geometric_series():
+    """Constant dt and x, B = C = e1, D = 0: y_t = dt x (1 - a^(t+1)) / (1 - a), a = exp(dt A)."""
+    L, dtv, xv, Av = 60, 0.3, 1.7, -2.5
+    e1 = np.zeros((1, L, 1, 4)); e1[..., 0] = 1.0
+    p = dict(x=np.full((1, L, 1, 1), xv), dt=np.full((1, L, 1), dtv), A=np.array([Av]),
+             B=e1, C=e1, D=None)
+    a = math.exp(dtv * Av)
+    ref = np.array([dtv * xv * (1 - a ** (t + 1)) / (1 - a) for t in range(L)])
+    np.testing.assert_allclose(_scan(p, 1)[0, :, 0, 0], ref, rtol=1e-13)
+    np.testing.assert_allclose(_scan(p, -1)[0, :, 0, 0], ref[::-1], rtol=1e-13)
+
+
+def test_impulse_response():
+    """x nonzero only at s0: y_t = dt_s0 (C_t . B_s0) exp(A sum_{s0<r<=t} dt_r) x_s0 for t >= s0, else 0."""
+    rng = np.random.default_rng(3)
+    p = _rand_params(rng, 1, 30, 1, 2, 8, 1)
+    s0 = 11
+    x = np.zeros_like(p["x"]); x[0, s0, 0] = [1.25, -0.5]; p["x"] = x
+    y = _scan(p, 1)[0, :, 0]
+    dt, A, B, C, D = p["dt"][0, :, 0], p["A"][0], p["B"][0, :, 0], p["C"][0, :, 0], p["D"][0]
+    for t in range(30):
+        if t < s0:
+            ref = np.zeros(2)
+        else:
+            ref = dt[s0] * float(C[t] @ B[s0]) * math.exp(A * dt[s0 + 1:t + 1].sum()) * x[0, s0, 0]
+            if t == s0:
+                ref = ref + D * x[0, s0, 0]
+        np.testing.assert_allclose(y[t], ref, rtol=1e-12, atol=1e-15)
+
+
+def test_single_token():
+    rng = np.random.default_rng(4)
+    p = _rand_params(rng, 3, 1, 2, 4, 8, 1)
+    ref = (p["dt"][..., None] * np.einsum("bgn,bgn->bg", p["C"][:, 0], p["B"][:, 0])[:, None, :, None]
+           * p["x"] + p["D"][None, None, :, None] * p["x"])
+    for d in (1, -1):
+        assert oracle.rel_err(_scan(p, d), ref) <= 1e-14
+
+
+def test_dt_zero_gives_skip_term_exactly():
+    rng = np.random.default_rng(5)
+    p = _rand_params(rng, 2, 9, 2, 4, 4, 1)
+    p["dt"] = np.zeros_like(p["dt"])
+    for d in (1, -1):
+        assert np.array_equal(_scan(p, d), p["D"][None, None, :, None] * p["x"])
+
+
+# ------------------------------------------------------------- identities
+
+def test_reverse_is_flip_forward_flip():
+    rng = np.random.default_rng(6)
+    p = _rand_params(rng, 2, 33, 4, 8, 16, 2)
+    flip = {k: (np.ascontiguousarray(v[:, ::-1]) if k in ("x", "dt", "B", "C") else v) for k, v in p.items()}
+    yr = _scan(p, -1)
+    yff = _scan(flip, 1)[:, ::-1]
+    assert np.max(np.abs(yr - yff)) <= 1e-15 * max(1.0, np.max(np.abs(yr)))
+
+
+def test_linear_in_x():
+    rng = np.random.default_rng(8)
+    p = _rand_params(rng, 1, 24, 2, 4, 8, 1)
+    x2 = rng.standard_normal(p["x"].shape)
+    al, be = 0.75, -1.5
+    q = dict(p, x=al * p["x"] + be * x2)
+    y = _scan(q, 1)
+    ref = al * _scan(p, 1) + be * _scan(dict(p, x=x2), 1)
+    assert oracle.rel_err(y, ref) <= 1e-12
+
+
+def test_thread_count_does_not_change_result():
+    rng = np.random.default_rng(9)
+    p = _rand_params(rng, 3, 20, 5, 4, 8, 1)
+    assert np.array_equal(_scan(p, 1, nthreads=1), _scan(p, 1, nthreads=7))
+
+
+def test_empty_inputs():
+    p = _rand_params(np.random.default_rng(0), 0, 8, 2, 4, 4, 1)
+    assert _scan(p, 1).shape == (0, 8, 2, 4)
+    p = _rand_params(np.random.default_rng(0), 2, 0, 2, 4, 4, 1)
+    assert _scan(p, -1).shape == (2, 0, 2, 4)
+
+
+# ------------------------------------------------------------ chunked form
+
+@pytest.mark.parametrize("chunk", [1, 4, 16, 32, 64])
+@pytest.mark.parametrize("direction", [1, -1])
+def test_chunked_form_matches_recurrence(chunk, direction):
+    rng = np.random.default_rng(10)
+    p = _rand_params(rng, 2, 64, 4, 8, 16, 2)
+    y = oracle.ssd_chunked_f64(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], direction, chunk)
+    assert oracle.rel_err(y, _scan(p, direction)) <= 1e-12
+
+
+def test_chunked_form_tiny_workload_chunk16():
+    shape = si.WORKLOADS["tiny_f32"]["shape"]
+    pf, _ = si.make_bidir(shape, seed=0)
+    p = oracle.params_f64(pf)
+    y = oracle.ssd_chunked_f64(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], 1, 16)
+    assert oracle.rel_err(y, _matrix_form(p, 1)) <= 1e-12
+
+
+# ------------------------------------------------------------------- gate
+
+def test_gate_zero_returns_residual_bitwise():
+    rng = np.random.default_rng(11)
+    p = _rand_params(rng, 2, 8, 2, 4, 4, 1)
+    res = rng.standard_normal((2, 8, 8))
+    res[0, 0, 0] = -0.0
+    out = oracle.r2l_block_f64(p, 0.0, res)
+    assert np.array_equal(out.view(np.uint64), res.view(np.uint64))
+
+
+def test_gate_nonzero():
+    rng = np.random.default_rng(12)
+    p = _rand_params(rng, 2, 8, 2, 4, 4, 1)
+    res = rng.standard_normal((2, 8, 8))
+    out = oracle.r2l_block_f64(p, 0.3, res)
+    ref = res + 0.3 * _matrix_form(p, -1).reshape(res.shape)
+    assert oracle.rel_err(out, ref) <= 1e-12
