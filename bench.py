@@ -1,0 +1,396 @@
+"""Benchmark: bidirectional SSD scan throughput (tokens/s) at the DiffuMamba ~1.3B layer shape.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step is one full bidirectional scan call (forward + reverse + sum) over a
+batch of synthetic seeded inputs already resident in HBM.  The default
+workload is batch 4 x L 8192, 64 heads x headdim 64, d_state 128, chunk 256,
+bf16 io with float32 state.  Under torchrun every rank runs its own batch of
+the same size (independent sequences, no data-path collective: weak scaling);
+the timed region is bracketed by a barrier and device synchronisation and the
+reported time is the maximum over ranks.
+
+The JSON line carries, besides the contract keys:
+  roofline      algorithmic bytes of the dominant kernel per launch / its
+                CUDA-event duration, against the measured HBM copy bandwidth
+  cpu_baseline  the float64 oracle timed on this host's cores on a bounded
+                sample of the same workload (rank 0, N = 1 only)
+  e2e           the same metric through the public API with pinned host
+                buffers, host->device inputs and device->host output copies
+                inside the timed region
+  clocks        SM clocks and throttle reasons sampled during the timed region
+``--impl reference`` times the oracle alone (the CPU reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import ssd_inputs as si  # noqa: E402
+
+METRIC = "bidirectional SSD scan tokens/s at 1.3B shape L=8192; % of HBM/tensor roofline"
+DEFAULT_WORKLOAD = "diffumamba_1p3b_L8192"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ------------------------------------------------------------------ accounting
+
+def algorithmic_bytes_per_token(shape: si.Shape, directions: int = 2) -> int:
+    """Bytes that must cross HBM once per token: each direction's x, dt, B, C read once, y written once."""
+    e = 2 if shape.io == "bf16" else 4
+    H, P, N, G = shape.nheads, shape.headdim, shape.dstate, shape.ngroups
+    per_dir = e * (H * P + H + 2 * G * N)
+    return directions * per_dir + e * H * P
+
+
+def shard_plan(rank: int, world: int, workload: str) -> dict:
+    """Weak scaling: every rank owns one full batch of independent sequences, drawn with its own seed."""
+    w = si.WORKLOADS[workload]
+    return {"rank": rank, "world": world, "seed": rank, "shape": w["shape"], "chunk": w["chunk"],
+            "tokens": w["shape"].tokens}
+
+
+def max_over_ranks(value: float, dist) -> float:
+    """Maximum of a per-rank float over the process group (the slowest rank sets the time)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    import torch
+    backend = dist.get_backend()
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Polls NVML for SM clock and clock-event (throttle) reasons in a background thread."""
+    REASONS = {0x2: "applications_clocks", 0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clocks"}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self._stop, self._th, self._h = period_s, threading.Event(), None, None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._th = threading.Thread(target=self._run, daemon=True)
+            self._th.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._th is not None:
+            self._th.join()
+
+    def summary(self) -> dict:
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ peaks and profiles
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def _kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bidirectional_mamba_ssd_bidir_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current kernel source."""
+    prof = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(prof):
+        return None
+    src_hash = _kernel_source_hash()
+    for f in sorted(os.listdir(prof)):
+        if not f.endswith(".md"):
+            continue
+        text = open(os.path.join(prof, f)).read()
+        m = re.search(r"traffic-record: kernel=(\S+) workload=(\S+) source=(\S+) bytes_per_launch=(\d+)", text)
+        if m and m.group(1) == kernel and m.group(2) == workload and m.group(3) == src_hash:
+            return int(m.group(4))
+    return None
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(shape: si.Shape, seed: int, heads: int, seqlen: int | None = None):
+    """Inputs for a bounded sample of the workload: batch 0, the first ``heads`` heads, the first ``seqlen`` tokens."""
+    import numpy as np
+    L = seqlen or shape.seqlen
+    sub = si.Shape(1, shape.seqlen, shape.nheads, shape.headdim, shape.dstate, shape.ngroups, shape.io)
+    pf, pr = si.make_bidir(sub, seed=seed)
+    import oracle
+    out = []
+    for p in (pf, pr):
+        q = oracle.params_f64(p)
+        q = {"x": np.ascontiguousarray(q["x"][:, :L, :heads]), "dt": np.ascontiguousarray(q["dt"][:, :L, :heads]),
+             "A": q["A"][:heads], "B": np.ascontiguousarray(q["B"][:, :L]), "C": np.ascontiguousarray(q["C"][:, :L]),
+             "D": q["D"][:heads]}
+        out.append(q)
+    return out
+
+
+def time_oracle(shape: si.Shape, seed: int, heads: int, seqlen: int | None = None, repeats: int = 1):
+    import oracle
+    qf, qr = oracle_sample(shape, seed, heads, seqlen)
+    L = qf["x"].shape[1]
+    threads = oracle.default_threads()
+    oracle.bidir_f64(qf, qr, nthreads=threads)                        # warm the library
+    times = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        oracle.bidir_f64(qf, qr, nthreads=threads)
+        times.append(time.perf_counter() - t0)
+    # tokens/s of the whole workload: the sample covers heads/H of each of L tokens
+    tok_per_s = [L * heads / shape.nheads / t for t in times]
+    return tok_per_s, threads, L
+
+
+def cpu_baseline(shape: si.Shape, target_s: float = 15.0) -> dict:
+    """Times the oracle on a bounded sample: batch 0, all tokens, as many heads as ~target_s of CPU work allows."""
+    import oracle
+    cores = oracle.default_threads()
+    qf, qr = oracle_sample(shape, 0, 1)
+    t0 = time.perf_counter()
+    oracle.bidir_f64(qf, qr, nthreads=1)
+    one_head = max(time.perf_counter() - t0, 1e-4)            # CPU seconds for one head, both directions
+    heads = int(min(shape.nheads, max(1, round(target_s / one_head))))
+    if heads >= cores:
+        heads -= heads % cores                                 # whole rounds of threads
+    tps, threads, L = time_oracle(shape, 0, heads)
+    return {"value": tps[0], "unit": "tokens/s", "cores": min(threads, heads), "kind": "oracle",
+            "sample": f"float64 recurrence, both directions, batch 0, {heads} of {shape.nheads} heads, "
+                      f"all {L} tokens (about {heads * one_head:.0f} s of CPU work); "
+                      f"tokens/s scaled by heads/{shape.nheads}"}
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args) -> None:
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    import bidirectional_mamba_ssd_bidir_b200 as ssd
+
+    plan = shard_plan(rank, world, args.workload)
+    shape, chunk = plan["shape"], plan["chunk"]
+    pf, pr = si.make_bidir(shape, seed=plan["seed"])
+    host = {}
+    for tag, p in (("f", pf), ("r", pr)):
+        for k in ("x", "dt", "A", "B", "C", "D"):
+            host[tag + k] = getattr(p, k).torch().pin_memory()
+    devt = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+    fwd = {k: devt["f" + k] for k in ("x", "dt", "A", "B", "C", "D")}
+    rev = {k: devt["r" + k] for k in ("x", "dt", "A", "B", "C", "D")}
+    y = torch.empty_like(fwd["x"])
+    dims = (shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate, shape.ngroups)
+    ws = torch.empty(max(256, ssd.workspace_bytes(dims, fwd["x"].dtype, chunk)), dtype=torch.uint8, device=dev)
+    path = ssd.path_for(dims, fwd["x"].dtype, chunk)
+    launches_per_step = ssd.kernel_launches(dims, fwd["x"].dtype, chunk, "bidir")
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize()
+
+    def step():
+        ssd.bidir_ssd(fwd, rev, chunk=chunk, out=y, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- device-timed region: inputs resident in HBM, larger than L2
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    per_launch_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    ssd.workspace_status(ws)
+    total_ms = max_over_ranks(total_ms, dist)
+    ms_per_step = total_ms / args.steps
+    tokens_all = plan["tokens"] * world
+    value = tokens_all / (ms_per_step / 1e3)
+
+    # ---- end to end through the public API with host buffers
+    out_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    e2e_steps = max(1, min(args.steps, 20))
+
+    def e2e_step():
+        for k, v in host.items():
+            devt[k].copy_(v, non_blocking=True)
+        step()
+        out_host.copy_(y, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(s2.elapsed_time(e2), dist) / e2e_steps
+    e2e_value = tokens_all / (e2e_ms / 1e3)
+
+    if rank == 0:
+        peaks = measured_peaks()
+        bpt = algorithmic_bytes_per_token(shape)
+        alg_bytes = bpt * plan["tokens"]
+        achieved = alg_bytes / (per_launch_ms / 1e3) / 1e9
+        kernel = "ssd_bidir_tc" if path == 1 else "simt_call(6 kernels)"
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if shape.io == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": args.workload, "global_batch": shape.batch * world, "seq_len": shape.seqlen,
+                       "nheads": shape.nheads, "headdim": shape.headdim, "dstate": shape.dstate,
+                       "ngroups": shape.ngroups, "chunk": chunk, "parallelism": f"dp{world} (independent sequences)",
+                       "path": "tcgen05" if path == 1 else "simt",
+                       "l2": f"inputs+output {alg_bytes / 1e6:.0f} MB per step > L2 {L2_BYTES / 1e6:.0f} MB, no flush"},
+            "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": profiled_traffic(kernel, args.workload),
+                         "algorithmic_bytes_per_launch": alg_bytes, "bytes_per_token": bpt,
+                         "launch_ms": per_launch_ms, "peak_source": peaks["source"] + " hbm_gbs"},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms, "steps": e2e_steps},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(shape, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    w = si.WORKLOADS[args.workload]
+    shape = w["shape"]
+    import oracle
+    cores = oracle.default_threads()
+    # size each step so that warmup + steps stay within ~args.ref_budget seconds
+    per_step_budget = max(0.05, args.ref_budget / max(1, args.steps + args.warmup))
+    probe, _, _ = time_oracle(shape, 0, min(cores, shape.nheads), seqlen=min(shape.seqlen, 1024))
+    # probe throughput in "whole-workload tokens per second" -> seconds per token per head
+    sec_per_tok_head = 1.0 / (probe[0] * shape.nheads)
+    heads = min(shape.nheads, max(1, cores))
+    L = int(min(shape.seqlen, max(64, per_step_budget / (sec_per_tok_head * heads))))
+    qf, qr = oracle_sample(shape, 0, heads, L)
+    for _ in range(args.warmup):
+        oracle.bidir_f64(qf, qr, nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.bidir_f64(qf, qr, nthreads=cores)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = L * heads / shape.nheads / dt
+    sample = (f"float64 recurrence, both directions, batch 0, {heads} of {shape.nheads} heads, first {L} of "
+              f"{shape.seqlen} tokens per step; tokens/s scaled by heads/{shape.nheads}")
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.workload, "global_batch": shape.batch, "seq_len": shape.seqlen,
+                       "nheads": shape.nheads, "headdim": shape.headdim, "dstate": shape.dstate,
+                       "chunk": w["chunk"], "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[k for k, v in si.WORKLOADS.items()
+                                                                      if v["kind"] == "bidir"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU work of the oracle baseline sample")
+    ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds for the reference arm's steps")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

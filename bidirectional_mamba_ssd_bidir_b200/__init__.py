@@ -1,0 +1,197 @@
+"""Bidirectional Mamba-2 SSD scan for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libbidirssd.so`` (declared in
+``include/bidir_ssd.h``).  This module only marshals arguments: it checks
+dtypes, shapes and devices, takes device memory for the output and the
+workspace from PyTorch, and passes raw pointers and the current CUDA stream
+to the library.  Every step of the scan runs in the library's CUDA kernels;
+there is no CPU or PyTorch fallback, and importing this package fails if the
+library has not been built.
+
+Entry points (same names as the C ABI):
+  ssd_scan(x, dt, A, B, C, D=None, direction=1, chunk=256)   one direction
+  bidir_ssd(fwd, rev, chunk=256)                              y_fwd + flip(scan(flip(.)))
+  r2l_block_scan(p, s, residual, chunk=32)                    residual + s * y_rev
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["ssd_scan", "bidir_ssd", "r2l_block_scan", "workspace_bytes", "path_for",
+           "kernel_launches", "workspace_status", "SSDError", "library_path", "lib"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libbidirssd.so")
+
+if not os.path.exists(library_path):
+    raise ImportError(
+        f"{library_path} is missing: build the CUDA library first "
+        "(python -c 'import __graft_entry__ as g; g.build()' from the repository root)")
+
+lib = ctypes.CDLL(library_path)
+
+SSD_BF16, SSD_F32 = 0, 1
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "CUDA error", 4: "device wait timed out"}
+
+
+class _Shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("seqlen", ctypes.c_int), ("nheads", ctypes.c_int),
+                ("headdim", ctypes.c_int), ("dstate", ctypes.c_int), ("ngroups", ctypes.c_int),
+                ("io", ctypes.c_int)]
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("dt", ctypes.c_void_p), ("A", ctypes.c_void_p),
+                ("B", ctypes.c_void_p), ("C", ctypes.c_void_p), ("D", ctypes.c_void_p)]
+
+
+_SP, _PP, _VP, _SZ = ctypes.POINTER(_Shape), ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_size_t
+lib.ssd_workspace_bytes.argtypes = [_SP, ctypes.c_int]
+lib.ssd_workspace_bytes.restype = _SZ
+lib.ssd_path_for.argtypes = [_SP, ctypes.c_int]
+lib.ssd_path_for.restype = ctypes.c_int
+lib.ssd_kernel_launches.argtypes = [_SP, ctypes.c_int, ctypes.c_int]
+lib.ssd_kernel_launches.restype = ctypes.c_int
+lib.ssd_scan.argtypes = [_SP, _PP, ctypes.c_int, ctypes.c_int, _VP, _VP, _SZ, _VP]
+lib.ssd_scan.restype = ctypes.c_int
+lib.bidir_ssd.argtypes = [_SP, _PP, _PP, ctypes.c_int, _VP, _VP, _SZ, _VP]
+lib.bidir_ssd.restype = ctypes.c_int
+lib.r2l_block_scan.argtypes = [_SP, _PP, ctypes.c_float, _VP, ctypes.c_int, _VP, _VP, _SZ, _VP]
+lib.r2l_block_scan.restype = ctypes.c_int
+lib.ssd_workspace_status.argtypes = [_VP, _SZ, _VP]
+lib.ssd_workspace_status.restype = ctypes.c_int
+lib.ssd_status_string.argtypes = [ctypes.c_int]
+lib.ssd_status_string.restype = ctypes.c_char_p
+lib.ssd_last_error.argtypes = []
+lib.ssd_last_error.restype = ctypes.c_char_p
+
+
+class SSDError(RuntimeError):
+    def __init__(self, status: int):
+        self.status = status
+        msg = lib.ssd_last_error().decode() or ""
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+
+
+def _check(status: int):
+    if status != 0:
+        raise SSDError(status)
+
+
+def _io(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SSD_BF16
+    if t.dtype == torch.float32:
+        return SSD_F32
+    raise TypeError(f"unsupported io dtype {t.dtype} (bfloat16 or float32)")
+
+
+def _shape_of(x, B) -> _Shape:
+    if x.dim() != 4 or B.dim() != 4:
+        raise ValueError("x must be [batch, seqlen, nheads, headdim] and B/C [batch, seqlen, ngroups, dstate]")
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    return _Shape(b, L, H, P, N, G, _io(x))
+
+
+def _params(x, dt, A, B, C, D) -> _Params:
+    b, L, H, P = x.shape
+    io = x.dtype
+    for name, t, shp in (("dt", dt, (b, L, H)), ("B", B, None), ("C", C, tuple(B.shape))):
+        if shp is not None and tuple(t.shape) != shp:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shp}")
+    if B.shape[:2] != x.shape[:2]:
+        raise ValueError("B must be [batch, seqlen, ngroups, dstate]")
+    for name, t in (("x", x), ("dt", dt), ("B", B), ("C", C)):
+        if t.dtype != io:
+            raise TypeError(f"{name} is {t.dtype}; x, dt, B, C must share one dtype")
+    for name, t in (("A", A), ("D", D)):
+        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != (H,)):
+            raise TypeError(f"{name} must be float32 of shape ({H},)")
+    dev = x.device
+    for name, t in (("x", x), ("dt", dt), ("A", A), ("B", B), ("C", C), ("D", D)):
+        if t is None:
+            continue
+        if t.device != dev or dev.type != "cuda":
+            raise ValueError(f"{name} must be a CUDA tensor on {dev}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    return _Params(x.data_ptr(), dt.data_ptr(), A.data_ptr(), B.data_ptr(), C.data_ptr(),
+                   D.data_ptr() if D is not None else None)
+
+
+def _stream(dev) -> int:
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
+def workspace_bytes(shape: tuple, io: torch.dtype, chunk: int) -> int:
+    """Workspace size for (batch, seqlen, nheads, headdim, dstate, ngroups) at this chunk."""
+    s = _Shape(*shape, SSD_BF16 if io == torch.bfloat16 else SSD_F32)
+    return int(lib.ssd_workspace_bytes(ctypes.byref(s), int(chunk)))
+
+
+def path_for(shape: tuple, io: torch.dtype, chunk: int) -> int:
+    """1 = tensor-core path, 0 = SIMT path, -1 = refused."""
+    s = _Shape(*shape, SSD_BF16 if io == torch.bfloat16 else SSD_F32)
+    return int(lib.ssd_path_for(ctypes.byref(s), int(chunk)))
+
+
+def kernel_launches(shape: tuple, io: torch.dtype, chunk: int, op: str) -> int:
+    """Kernels one call launches: op in {"scan", "bidir", "r2l"}."""
+    s = _Shape(*shape, SSD_BF16 if io == torch.bfloat16 else SSD_F32)
+    return int(lib.ssd_kernel_launches(ctypes.byref(s), int(chunk), {"scan": 0, "bidir": 1, "r2l": 2}[op]))
+
+
+def _workspace(shape: _Shape, chunk: int, dev, workspace):
+    need = int(lib.ssd_workspace_bytes(ctypes.byref(shape), int(chunk)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def ssd_scan(x, dt, A, B, C, D=None, direction: int = 1, chunk: int = 256, out=None, workspace=None):
+    """One direction of the scan; returns y shaped like x."""
+    shape = _shape_of(x, B)
+    prm = _params(x, dt, A, B, C, D)
+    y = torch.empty_like(x) if out is None else out
+    ws, nbytes = _workspace(shape, chunk, x.device, workspace)
+    _check(lib.ssd_scan(ctypes.byref(shape), ctypes.byref(prm), int(direction), int(chunk),
+                        y.data_ptr(), ws.data_ptr(), nbytes, _stream(x.device)))
+    return y
+
+
+def bidir_ssd(fwd: dict, rev: dict, chunk: int = 256, out=None, workspace=None):
+    """DiffuMamba mixer: y = scan(fwd, +1) + scan(rev, -1).  Each dict holds x, dt, A, B, C and D (or None)."""
+    shape = _shape_of(fwd["x"], fwd["B"])
+    if tuple(rev["x"].shape) != tuple(fwd["x"].shape) or tuple(rev["B"].shape) != tuple(fwd["B"].shape):
+        raise ValueError("forward and reverse parameters must have the same shapes")
+    pf = _params(fwd["x"], fwd["dt"], fwd["A"], fwd["B"], fwd["C"], fwd.get("D"))
+    pr = _params(rev["x"], rev["dt"], rev["A"], rev["B"], rev["C"], rev.get("D"))
+    y = torch.empty_like(fwd["x"]) if out is None else out
+    ws, nbytes = _workspace(shape, chunk, fwd["x"].device, workspace)
+    _check(lib.bidir_ssd(ctypes.byref(shape), ctypes.byref(pf), ctypes.byref(pr), int(chunk),
+                         y.data_ptr(), ws.data_ptr(), nbytes, _stream(fwd["x"].device)))
+    return y
+
+
+def r2l_block_scan(p: dict, s: float, residual, chunk: int = 32, out=None, workspace=None):
+    """R2LM sidecar block: out = residual + s * scan(p, -1); s == 0 returns the residual bit for bit."""
+    shape = _shape_of(p["x"], p["B"])
+    prm = _params(p["x"], p["dt"], p["A"], p["B"], p["C"], p.get("D"))
+    b, L, H, P = p["x"].shape
+    if tuple(residual.shape) != (b, L, H * P) or residual.dtype != p["x"].dtype or not residual.is_contiguous():
+        raise ValueError(f"residual must be contiguous {p['x'].dtype} of shape {(b, L, H * P)}")
+    o = torch.empty_like(residual) if out is None else out
+    ws, nbytes = _workspace(shape, chunk, p["x"].device, workspace)
+    _check(lib.r2l_block_scan(ctypes.byref(shape), ctypes.byref(prm), ctypes.c_float(s), residual.data_ptr(),
+                              int(chunk), o.data_ptr(), ws.data_ptr(), nbytes, _stream(p["x"].device)))
+    return o
+
+
+def workspace_status(workspace) -> None:
+    """Raise SSDError if a bounded device-side wait gave up in a call that used ``workspace``."""
+    dev = workspace.device
+    _check(lib.ssd_workspace_status(workspace.data_ptr(), workspace.numel(), _stream(dev)))

@@ -1,0 +1,236 @@
+// ssd_api.cu -- the C ABI declared in include/bidir_ssd.h: argument checks,
+// workspace layout, path choice and stream-ordered launches.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/bidir_ssd.h"
+#include "ssd_internal.cuh"
+#include "ssd_tc.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+ssd_status fail(ssd_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return s;
+}
+
+ssd_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(SSD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 256;   // device status word + padding
+
+size_t round_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool is_pow2_in(int v, const int *set, int n) {
+    for (int i = 0; i < n; ++i)
+        if (v == set[i]) return true;
+    return false;
+}
+
+bool aligned16(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ssd_status check_shape(const ssd_shape *s, int chunk) {
+    if (!s) return fail(SSD_ERR_INVALID_ARG, "shape is NULL");
+    if (s->batch < 0 || s->seqlen < 0 || s->nheads <= 0 || s->headdim <= 0 || s->dstate <= 0 || s->ngroups <= 0)
+        return fail(SSD_ERR_INVALID_ARG, "negative or zero size in shape");
+    if (s->io != SSD_BF16 && s->io != SSD_F32) return fail(SSD_ERR_INVALID_ARG, "unknown io dtype %d", (int)s->io);
+    static const int P_ok[] = {16, 32, 64}, N_ok[] = {16, 32, 64, 128}, Q_ok[] = {16, 32, 64, 128, 256};
+    if (!is_pow2_in(s->headdim, P_ok, 3)) return fail(SSD_ERR_UNSUPPORTED, "headdim %d not in {16,32,64}", s->headdim);
+    if (!is_pow2_in(s->dstate, N_ok, 4)) return fail(SSD_ERR_UNSUPPORTED, "dstate %d not in {16,32,64,128}", s->dstate);
+    if (!is_pow2_in(chunk, Q_ok, 5)) return fail(SSD_ERR_UNSUPPORTED, "chunk %d not in {16,32,64,128,256}", chunk);
+    if (s->nheads % s->ngroups != 0)
+        return fail(SSD_ERR_UNSUPPORTED, "nheads %d not a multiple of ngroups %d", s->nheads, s->ngroups);
+    if (s->seqlen % chunk != 0) return fail(SSD_ERR_INVALID_ARG, "seqlen %d not a multiple of chunk %d", s->seqlen, chunk);
+    const double elems = (double)s->batch * s->seqlen * s->nheads * s->headdim;
+    if (elems > 4.0e9) return fail(SSD_ERR_UNSUPPORTED, "tensor too large (%.3g elements)", elems);
+    return SSD_OK;
+}
+
+ssd_status check_params(const ssd_params *p, const char *which) {
+    if (!p) return fail(SSD_ERR_INVALID_ARG, "%s params is NULL", which);
+    if (!aligned16(p->x) || !aligned16(p->B) || !aligned16(p->C))
+        return fail(SSD_ERR_INVALID_ARG, "%s: x, B and C must be non-NULL and 16-byte aligned", which);
+    if (!p->dt || !p->A) return fail(SSD_ERR_INVALID_ARG, "%s: dt and A must be non-NULL", which);
+    if ((reinterpret_cast<uintptr_t>(p->dt) & 3u) || (reinterpret_cast<uintptr_t>(p->A) & 3u) ||
+        (reinterpret_cast<uintptr_t>(p->D) & 3u))
+        return fail(SSD_ERR_INVALID_ARG, "%s: dt, A, D must be 4-byte aligned", which);
+    return SSD_OK;
+}
+
+// SIMT-path workspace: [status | decays (batch*H*nc floats) | states (batch*H*nc*P*N floats)]
+size_t simt_ws_bytes(const ssd_shape *s, int chunk) {
+    const size_t units = (size_t)s->batch * s->nheads * (s->seqlen / chunk);
+    if (s->seqlen / chunk <= 1) return kStatusBytes;
+    return kStatusBytes + round_up(units * sizeof(float)) + round_up(units * s->headdim * s->dstate * sizeof(float));
+}
+
+int choose_path(const ssd_shape *s, int chunk) {
+    return ssd::tc_supported(s->io == SSD_BF16, s->batch, s->seqlen, s->nheads, s->headdim, s->dstate,
+                             s->ngroups, chunk) ? 1 : 0;
+}
+
+size_t path_ws_bytes(const ssd_shape *s, int chunk) {
+    if (choose_path(s, chunk) == 1)
+        return kStatusBytes + round_up(ssd::tc_workspace_bytes(s->batch, s->seqlen, s->nheads, chunk));
+    return simt_ws_bytes(s, chunk);
+}
+
+ssd::ScanArgs make_args(const ssd_shape *s, const ssd_params *p, int dir, int chunk, void *y, void *ws) {
+    ssd::ScanArgs a{};
+    a.batch = s->batch; a.L = s->seqlen; a.H = s->nheads; a.P = s->headdim; a.N = s->dstate;
+    a.G = s->ngroups; a.Q = chunk; a.nc = s->seqlen / chunk; a.dir = dir;
+    a.x = p->x; a.dt = p->dt; a.B = p->B; a.C = p->C; a.A = p->A; a.D = p->D;
+    a.y = y; a.residual = nullptr; a.gate = 0.f; a.mode = ssd::OUT_WRITE;
+    char *w = static_cast<char *>(ws) + kStatusBytes;
+    const size_t units = (size_t)s->batch * s->nheads * a.nc;
+    a.decays = reinterpret_cast<float *>(w);
+    a.states = reinterpret_cast<float *>(w + round_up(units * sizeof(float)));
+    return a;
+}
+
+ssd_status common_checks(const ssd_shape *s, int chunk, void *out, void *ws, size_t ws_bytes) {
+    ssd_status st = check_shape(s, chunk);
+    if (st != SSD_OK) return st;
+    if (!aligned16(out)) return fail(SSD_ERR_INVALID_ARG, "output must be non-NULL and 16-byte aligned");
+    const size_t need = path_ws_bytes(s, chunk);
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
+        return fail(SSD_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+    if (ws_bytes < need) return fail(SSD_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    return SSD_OK;
+}
+
+ssd_status run_simt(const ssd_shape *s, const ssd_params *p, int dir, int chunk, void *y, void *ws,
+                    int mode, const void *residual, float gate, cudaStream_t st) {
+    ssd::ScanArgs a = make_args(s, p, dir, chunk, y, ws);
+    a.mode = mode; a.residual = residual; a.gate = gate;
+    cudaError_t e = ssd::launch_simt_scan(a, s->io == SSD_BF16, st);
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, "SIMT scan launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ssd_workspace_bytes(const ssd_shape *shape, int chunk) {
+    if (check_shape(shape, chunk) != SSD_OK) return 0;
+    return path_ws_bytes(shape, chunk);
+}
+
+int ssd_path_for(const ssd_shape *shape, int chunk) {
+    if (check_shape(shape, chunk) != SSD_OK) return -1;
+    return choose_path(shape, chunk);
+}
+
+int ssd_kernel_launches(const ssd_shape *shape, int chunk, int op) {
+    if (check_shape(shape, chunk) != SSD_OK || op < 0 || op > 2) return -1;
+    if (shape->batch == 0 || shape->seqlen == 0) return 0;
+    const int dirs = op == 1 ? 2 : 1;
+    if (op != 2 && choose_path(shape, chunk) == 1) return ssd::tc_launches(op == 1);
+    return dirs * (shape->seqlen / chunk > 1 ? 3 : 1);
+}
+
+ssd_status ssd_scan(const ssd_shape *shape, const ssd_params *p, int direction, int chunk, void *y,
+                    void *workspace, size_t workspace_bytes, void *stream) {
+    g_err.clear();
+    ssd_status st = common_checks(shape, chunk, y, workspace, workspace_bytes);
+    if (st != SSD_OK) return st;
+    if (direction != 1 && direction != -1) return fail(SSD_ERR_INVALID_ARG, "direction must be +1 or -1");
+    if ((st = check_params(p, "scan")) != SSD_OK) return st;
+    if (shape->batch == 0 || shape->seqlen == 0) return SSD_OK;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (choose_path(shape, chunk) == 1) {
+        ssd::TcArgs t = ssd::make_tc_args(shape->batch, shape->seqlen, shape->nheads, chunk,
+                                          static_cast<char *>(workspace) + kStatusBytes,
+                                          static_cast<int *>(workspace));
+        ssd::tc_set_direction(t, 0, direction, p->x, p->dt, p->A, p->B, p->C, p->D);
+        cudaError_t e = ssd::launch_tc(t, /*bidir=*/false, y, cs);
+        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "tensor-core scan launch");
+    }
+    return run_simt(shape, p, direction, chunk, y, workspace, ssd::OUT_WRITE, nullptr, 0.f, cs);
+}
+
+ssd_status bidir_ssd(const ssd_shape *shape, const ssd_params *fwd, const ssd_params *rev, int chunk, void *y,
+                     void *workspace, size_t workspace_bytes, void *stream) {
+    g_err.clear();
+    ssd_status st = common_checks(shape, chunk, y, workspace, workspace_bytes);
+    if (st != SSD_OK) return st;
+    if ((st = check_params(fwd, "forward")) != SSD_OK) return st;
+    if ((st = check_params(rev, "reverse")) != SSD_OK) return st;
+    if (shape->batch == 0 || shape->seqlen == 0) return SSD_OK;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (choose_path(shape, chunk) == 1) {
+        ssd::TcArgs t = ssd::make_tc_args(shape->batch, shape->seqlen, shape->nheads, chunk,
+                                          static_cast<char *>(workspace) + kStatusBytes,
+                                          static_cast<int *>(workspace));
+        ssd::tc_set_direction(t, 0, 1, fwd->x, fwd->dt, fwd->A, fwd->B, fwd->C, fwd->D);
+        ssd::tc_set_direction(t, 1, -1, rev->x, rev->dt, rev->A, rev->B, rev->C, rev->D);
+        cudaError_t e = ssd::launch_tc(t, /*bidir=*/true, y, cs);
+        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "tensor-core bidirectional launch");
+    }
+    st = run_simt(shape, fwd, 1, chunk, y, workspace, ssd::OUT_WRITE, nullptr, 0.f, cs);
+    if (st != SSD_OK) return st;
+    return run_simt(shape, rev, -1, chunk, y, workspace, ssd::OUT_ACCUM, nullptr, 0.f, cs);
+}
+
+ssd_status r2l_block_scan(const ssd_shape *shape, const ssd_params *p, float s, const void *residual, int chunk,
+                          void *out, void *workspace, size_t workspace_bytes, void *stream) {
+    g_err.clear();
+    ssd_status st = common_checks(shape, chunk, out, workspace, workspace_bytes);
+    if (st != SSD_OK) return st;
+    if ((st = check_params(p, "r2l")) != SSD_OK) return st;
+    if (!aligned16(residual)) return fail(SSD_ERR_INVALID_ARG, "residual must be non-NULL and 16-byte aligned");
+    if (shape->batch == 0 || shape->seqlen == 0) return SSD_OK;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (s == 0.0f) {
+        // Gate at its initial value: the block is returned untouched, bit for bit.
+        if (out == residual) return SSD_OK;
+        const size_t bytes = (size_t)shape->batch * shape->seqlen * shape->nheads * shape->headdim *
+                             (shape->io == SSD_BF16 ? 2 : 4);
+        cudaError_t e = cudaMemcpyAsync(out, residual, bytes, cudaMemcpyDeviceToDevice, cs);
+        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "residual copy");
+    }
+    return run_simt(shape, p, -1, chunk, out, workspace, ssd::OUT_GATE, residual, s, cs);
+}
+
+ssd_status ssd_workspace_status(void *workspace, size_t workspace_bytes, void *stream) {
+    g_err.clear();
+    if (!workspace || workspace_bytes < kStatusBytes) return fail(SSD_ERR_INVALID_ARG, "workspace too small");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    int word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return cuda_fail(e, "status read");
+    if (word != 0) {
+        e = cudaMemsetAsync(workspace, 0, sizeof(int), cs);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+        if (e != cudaSuccess) return cuda_fail(e, "status clear");
+        return fail(SSD_ERR_TIMEOUT, "a bounded device wait gave up (code %d)", word);
+    }
+    return SSD_OK;
+}
+
+const char *ssd_status_string(ssd_status s) {
+    switch (s) {
+        case SSD_OK: return "ok";
+        case SSD_ERR_INVALID_ARG: return "invalid argument";
+        case SSD_ERR_UNSUPPORTED: return "unsupported shape";
+        case SSD_ERR_CUDA: return "CUDA error";
+        case SSD_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+const char *ssd_last_error(void) { return g_err.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+// ssd_internal.cuh -- definitions shared by the launch layer and the kernels.
+//
+// Notation used throughout the kernels: k is a position in SCAN order
+// (0..L-1).  The forward scan reads token t = k; the reverse scan reads token
+// t = L-1-k.  Doing every computation in scan order and mapping only the
+// addresses is the "flip, scan, flip back" of the R2LM right-to-left stream
+// ("Bifocal Diffusion Language Models", section 2, mechanism) without
+// materialising a flipped copy.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssd {
+
+enum OutMode : int {
+    OUT_WRITE = 0,   // y = value
+    OUT_ACCUM = 1,   // y = y + value   (second direction of the bidirectional mixer)
+    OUT_GATE = 2     // out = residual + gate * value   (R2L sidecar, gate != 0)
+};
+
+struct ScanArgs {
+    int batch, L, H, P, N, G, Q, nc;
+    int dir;                 // +1 forward, -1 reverse
+    const void *x, *dt, *B, *C;
+    const float *A, *D;      // D may be null
+    void *y;                 // output (y, or out for OUT_GATE)
+    const void *residual;    // OUT_GATE only
+    float gate;              // OUT_GATE only
+    int mode;
+    float *states;           // [batch][H][nc][P][N] chunk states -> incoming states
+    float *decays;           // [batch][H][nc] chunk decay exp(cs_last)
+};
+
+// token index in memory for scan position k
+__device__ __forceinline__ int tok(int k, int L, int dir) { return dir > 0 ? k : L - 1 - k; }
+
+template <typename T> __device__ __forceinline__ float ldf(const T *p, size_t i);
+template <> __device__ __forceinline__ float ldf<float>(const float *p, size_t i) { return p[i]; }
+template <> __device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16 *p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+template <typename T> __device__ __forceinline__ void stf(T *p, size_t i, float v);
+template <> __device__ __forceinline__ void stf<float>(float *p, size_t i, float v) { p[i] = v; }
+template <> __device__ __forceinline__ void stf<__nv_bfloat16>(__nv_bfloat16 *p, size_t i, float v) {
+    p[i] = __float2bfloat16_rn(v);
+}
+
+// Launchers (defined in the kernel translation units).  All return the
+// cudaError_t of the launch.
+cudaError_t launch_simt_scan(const ScanArgs &a, bool bf16, cudaStream_t st);
+
+}  // namespace ssd

@@ -1,0 +1,264 @@
+// ssd_simt.cu -- chunked SSD scan on the CUDA cores (float32 FFMA).
+//
+// This is the general path: any supported headdim/dstate/chunk, float32 or
+// bf16 storage, both directions.  It evaluates the scan in the chunked
+// (state-passing) form, exactly as the recurrence
+//     S <- exp(dt A) S + dt x (outer) B,   y = C.S + D x
+// unrolls over a chunk of Q tokens (cs_k = A * sum_{j<=k in chunk} dt_j):
+//     intra-chunk  y_diag[k] = sum_{s<=k} (C_k . B_s) exp(cs_k - cs_s) dt_s x_s
+//     chunk state  S_c       = sum_s exp(cs_last - cs_s) dt_s x_s (outer) B_s
+//     passing      Sin_0 = 0, Sin_{c+1} = exp(cs_last) Sin_c + S_c
+//     from state   y_off[k]  = exp(cs_k) C_k . Sin_c
+// in three launches: chunk states (all chunks in parallel), the sequential
+// pass over chunks, and the outputs (all chunks in parallel).  A single-chunk
+// sequence skips the first two.
+#include "ssd_internal.cuh"
+
+namespace ssd {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kRows = 16;    // output rows per CTA in the output kernel
+constexpr int kSTile = 32;   // tokens per staged tile
+
+// Inclusive prefix sum of dt over one chunk (scan order), times A, into cs[];
+// dts[] receives dt.  Every kernel uses this same routine, so the chunk's
+// cumulative decays are bit-identical wherever they are recomputed.
+template <typename T>
+__device__ void chunk_cumsum(const ScanArgs &a, const T *dt, int b, int h, int c, float *cs, float *dts) {
+    __shared__ float warp_tot[kThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int Q = a.Q;
+    float v = 0.f;
+    if (tid < Q) {
+        const int t = tok(c * Q + tid, a.L, a.dir);
+        v = ldf<T>(dt, ((size_t)b * a.L + t) * a.H + h);
+        dts[tid] = v;
+    }
+    float s = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        float u = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += u;
+    }
+    if (lane == 31) warp_tot[warp] = s;
+    __syncthreads();
+    float base = 0.f;
+    for (int w = 0; w < warp; ++w) base += warp_tot[w];
+    if (tid < Q) cs[tid] = a.A[h] * (base + s);
+    __syncthreads();
+}
+
+template <typename T, int P, int N>
+__global__ void __launch_bounds__(kThreads) k_chunk_state(ScanArgs a) {
+    constexpr int E = P * N / kThreads;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int Q = a.Q, g = h / (a.H / a.G);
+    const T *x = (const T *)a.x, *B = (const T *)a.B;
+    extern __shared__ float sm[];
+    float *cs = sm, *dts = cs + Q, *xs = dts + Q, *bs = xs + kSTile * P;
+    chunk_cumsum<T>(a, (const T *)a.dt, b, h, c, cs, dts);
+    const float cl = cs[Q - 1];
+    float acc[E];
+#pragma unroll
+    for (int j = 0; j < E; ++j) acc[j] = 0.f;
+    const int n = threadIdx.x % N;
+    for (int s0 = 0; s0 < Q; s0 += kSTile) {
+        // rows past the chunk end (chunk shorter than a tile) are zero
+        for (int i = threadIdx.x; i < kSTile * P; i += kThreads) {
+            const int r = i / P, p = i % P, k = s0 + r;
+            float v = 0.f;
+            if (k < Q) {
+                const int t = tok(c * Q + k, a.L, a.dir);
+                v = expf(cl - cs[k]) * dts[k] * ldf<T>(x, (((size_t)b * a.L + t) * a.H + h) * P + p);
+            }
+            xs[i] = v;
+        }
+        for (int i = threadIdx.x; i < kSTile * N; i += kThreads) {
+            const int r = i / N, nn = i % N, k = s0 + r;
+            float v = 0.f;
+            if (k < Q) {
+                const int t = tok(c * Q + k, a.L, a.dir);
+                v = ldf<T>(B, (((size_t)b * a.L + t) * a.G + g) * N + nn);
+            }
+            bs[i] = v;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int r = 0; r < kSTile; ++r) {
+            const float bv = bs[r * N + n];
+#pragma unroll
+            for (int j = 0; j < E; ++j) {
+                const int p = (threadIdx.x + kThreads * j) / N;
+                acc[j] = fmaf(xs[r * P + p], bv, acc[j]);
+            }
+        }
+        __syncthreads();
+    }
+    float *S = a.states + (((size_t)b * a.H + h) * a.nc + c) * P * N;
+#pragma unroll
+    for (int j = 0; j < E; ++j) S[threadIdx.x + kThreads * j] = acc[j];
+    if (threadIdx.x == 0) a.decays[((size_t)b * a.H + h) * a.nc + c] = expf(cl);
+}
+
+template <int P, int N>
+__global__ void __launch_bounds__(kThreads) k_state_pass(ScanArgs a) {
+    constexpr int E = P * N / kThreads;
+    const int h = blockIdx.x, b = blockIdx.y;
+    float run[E];
+#pragma unroll
+    for (int j = 0; j < E; ++j) run[j] = 0.f;
+    const size_t base = ((size_t)b * a.H + h) * a.nc;
+    for (int c = 0; c < a.nc; ++c) {
+        float *S = a.states + (base + c) * P * N;
+        const float dc = a.decays[base + c];
+#pragma unroll
+        for (int j = 0; j < E; ++j) {
+            const int e = threadIdx.x + kThreads * j;
+            const float sc = S[e];
+            S[e] = run[j];                       // state entering chunk c
+            run[j] = fmaf(dc, run[j], sc);
+        }
+    }
+}
+
+template <typename T, int P, int N>
+__global__ void __launch_bounds__(kThreads) k_chunk_output(ScanArgs a, int have_state) {
+    constexpr int NP = N + 1;                       // padded row stride (bank spread)
+    constexpr int EO = kRows * P / kThreads;        // outputs per thread
+    constexpr int EG = kRows * kSTile / kThreads;   // decayed-score entries per thread
+    const int tiles = a.Q / kRows;
+    const int c = blockIdx.x / tiles, k0 = (blockIdx.x % tiles) * kRows;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int Q = a.Q, g = h / (a.H / a.G);
+    const T *x = (const T *)a.x, *B = (const T *)a.B, *Cm = (const T *)a.C;
+    extern __shared__ float sm[];
+    float *cs = sm, *dts = cs + Q, *Cs = dts + Q, *Sin = Cs + kRows * N;
+    float *Bs = Sin + (have_state ? P * NP : 0), *xs = Bs + kSTile * NP, *Ms = xs + kSTile * P;
+    chunk_cumsum<T>(a, (const T *)a.dt, b, h, c, cs, dts);
+    for (int i = threadIdx.x; i < kRows * N; i += kThreads) {
+        const int r = i / N, n = i % N;
+        const int t = tok(c * Q + k0 + r, a.L, a.dir);
+        Cs[i] = ldf<T>(Cm, (((size_t)b * a.L + t) * a.G + g) * N + n);
+    }
+    if (have_state) {
+        const float *S = a.states + (((size_t)b * a.H + h) * a.nc + c) * P * N;
+        for (int i = threadIdx.x; i < P * N; i += kThreads) Sin[(i / N) * NP + (i % N)] = S[i];
+    }
+    __syncthreads();
+
+    float yv[EO];
+#pragma unroll
+    for (int j = 0; j < EO; ++j) {
+        const int o = threadIdx.x + kThreads * j, r = o / P, p = o % P;
+        float acc = 0.f;
+        if (have_state) {
+#pragma unroll 8
+            for (int n = 0; n < N; ++n) acc = fmaf(Cs[r * N + n], Sin[p * NP + n], acc);
+            acc *= expf(cs[k0 + r]);
+        }
+        yv[j] = acc;
+    }
+
+    const int send = k0 + kRows;                    // tokens s < send can reach these rows
+    for (int s0 = 0; s0 < send; s0 += kSTile) {
+        for (int i = threadIdx.x; i < kSTile * N; i += kThreads) {
+            const int r = i / N, n = i % N, s = s0 + r;
+            float v = 0.f;
+            if (s < Q) {
+                const int t = tok(c * Q + s, a.L, a.dir);
+                v = ldf<T>(B, (((size_t)b * a.L + t) * a.G + g) * N + n);
+            }
+            Bs[r * NP + n] = v;
+        }
+        for (int i = threadIdx.x; i < kSTile * P; i += kThreads) {
+            const int r = i / P, p = i % P, s = s0 + r;
+            float v = 0.f;
+            if (s < Q) {
+                const int t = tok(c * Q + s, a.L, a.dir);
+                v = ldf<T>(x, (((size_t)b * a.L + t) * a.H + h) * P + p);
+            }
+            xs[i] = v;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < EG; ++j) {
+            const int e = threadIdx.x + kThreads * j, r = e / kSTile, sp = e % kSTile;
+            const int k = k0 + r, s = s0 + sp;
+            float m = 0.f;
+            if (s <= k) {
+                float d = 0.f;
+#pragma unroll 8
+                for (int n = 0; n < N; ++n) d = fmaf(Cs[r * N + n], Bs[sp * NP + n], d);
+                m = d * expf(cs[k] - cs[s]) * dts[s];
+            }
+            Ms[r * kSTile + sp] = m;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < EO; ++j) {
+            const int o = threadIdx.x + kThreads * j, r = o / P, p = o % P;
+            float acc = yv[j];
+#pragma unroll 8
+            for (int sp = 0; sp < kSTile; ++sp) acc = fmaf(Ms[r * kSTile + sp], xs[sp * P + p], acc);
+            yv[j] = acc;
+        }
+        __syncthreads();
+    }
+
+    const float dh = a.D ? a.D[h] : 0.f;
+#pragma unroll
+    for (int j = 0; j < EO; ++j) {
+        const int o = threadIdx.x + kThreads * j, r = o / P, p = o % P;
+        const int t = tok(c * Q + k0 + r, a.L, a.dir);
+        const size_t idx = (((size_t)b * a.L + t) * a.H + h) * P + p;   // same as [b][t][h*P+p]
+        const float v = fmaf(dh, ldf<T>(x, idx), yv[j]);
+        T *y = (T *)a.y;
+        if (a.mode == OUT_WRITE) {
+            stf<T>(y, idx, v);
+        } else if (a.mode == OUT_ACCUM) {
+            stf<T>(y, idx, ldf<T>(y, idx) + v);
+        } else {
+            stf<T>(y, idx, fmaf(a.gate, v, ldf<T>((const T *)a.residual, idx)));
+        }
+    }
+}
+
+template <typename T, int P, int N>
+cudaError_t launch_typed(const ScanArgs &a, cudaStream_t st) {
+    const bool multi = a.nc > 1;
+    const size_t sm_state = sizeof(float) * (2 * a.Q + kSTile * P + kSTile * N);
+    const size_t sm_out = sizeof(float) * (2 * a.Q + kRows * N + (multi ? P * (N + 1) : 0) +
+                                           kSTile * (N + 1) + kSTile * P + kRows * kSTile);
+    cudaError_t e;
+    if (multi) {
+        e = cudaFuncSetAttribute(k_chunk_state<T, P, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_state);
+        if (e != cudaSuccess) return e;
+        k_chunk_state<T, P, N><<<dim3(a.nc, a.H, a.batch), kThreads, sm_state, st>>>(a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        k_state_pass<P, N><<<dim3(a.H, a.batch), kThreads, 0, st>>>(a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    e = cudaFuncSetAttribute(k_chunk_output<T, P, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out);
+    if (e != cudaSuccess) return e;
+    k_chunk_output<T, P, N><<<dim3(a.nc * (a.Q / kRows), a.H, a.batch), kThreads, sm_out, st>>>(a, multi ? 1 : 0);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_dtype(const ScanArgs &a, cudaStream_t st) {
+#define SSD_CASE(PP, NN) if (a.P == PP && a.N == NN) return launch_typed<T, PP, NN>(a, st);
+    SSD_CASE(16, 16) SSD_CASE(16, 32) SSD_CASE(16, 64) SSD_CASE(16, 128)
+    SSD_CASE(32, 16) SSD_CASE(32, 32) SSD_CASE(32, 64) SSD_CASE(32, 128)
+    SSD_CASE(64, 16) SSD_CASE(64, 32) SSD_CASE(64, 64) SSD_CASE(64, 128)
+#undef SSD_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_simt_scan(const ScanArgs &a, bool bf16, cudaStream_t st) {
+    return bf16 ? launch_dtype<__nv_bfloat16>(a, st) : launch_dtype<float>(a, st);
+}
+
+}  // namespace ssd

@@ -1,0 +1,30 @@
+// ssd_tc.cuh -- launch interface of the tensor-core (tcgen05) path.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace ssd {
+
+struct TcDir {
+    const void *x, *dt, *B, *C;
+    const float *A, *D;
+    int dir;
+};
+
+struct TcArgs {
+    int batch, L, H, chunk;
+    TcDir d[2];
+    void *ws;          // path scratch (after the status word)
+    int *status;       // device status word
+};
+
+bool tc_supported(bool bf16, int batch, int L, int H, int P, int N, int G, int chunk);
+size_t tc_workspace_bytes(int batch, int L, int H, int chunk);
+TcArgs make_tc_args(int batch, int L, int H, int chunk, void *ws, int *status);
+void tc_set_direction(TcArgs &t, int slot, int dir, const void *x, const void *dt, const float *A,
+                      const void *B, const void *C, const float *D);
+int tc_launches(bool bidir);
+cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st);
+
+}  // namespace ssd

@@ -1,0 +1,146 @@
+/*
+ * bidir_ssd.h -- C ABI of the bidirectional selective state-space (SSD) scan
+ * library for NVIDIA B200 (sm_100a).
+ *
+ * The operation.  Per batch b and head h (group g = h / (nheads/ngroups)),
+ * with a state S in R^{headdim x dstate} that starts at zero, the scan visits
+ * the tokens in order and computes
+ *
+ *     S   <- exp(dt[b,t,h] * A[h]) * S + dt[b,t,h] * x[b,t,h,:] (outer) B[b,t,g,:]
+ *     y[b,t,h,p] = sum_n C[b,t,g,n] * S[p,n] + D[h] * x[b,t,h,p]
+ *
+ * This is the Mamba-2 selective scan named by "DiffuMamba: High-Throughput
+ * Diffusion LMs with Mamba Backbone" (technical summary, section 2
+ * Methodology: the attention mixer is replaced by bidirectional Mamba-2
+ * layers) and by "Bifocal Diffusion Language Models" (section 2, mechanism:
+ * the right-to-left stream flips the sequence, applies the selective scan and
+ * flips back).  The pages do not print the recurrence; the standard Mamba-2
+ * form with one scalar decay per head is the one implemented.
+ *
+ * Layouts.  Every tensor is row-major and contiguous:
+ *     x, y      [batch][seqlen][nheads][headdim]      (io dtype)
+ *     dt        [batch][seqlen][nheads]               (io dtype, already positive)
+ *     B, C      [batch][seqlen][ngroups][dstate]      (io dtype)
+ *     A, D      [nheads]                              (float32 always; D may be NULL = no skip term)
+ *     residual, out  [batch][seqlen][nheads*headdim]  (io dtype)
+ * Arithmetic is float32 (the state is float32) for both io dtypes; bf16
+ * outputs are rounded to nearest even once at the end.
+ *
+ * Ownership.  The caller allocates every buffer; all data pointers are DEVICE
+ * pointers on the current CUDA device.  The library allocates nothing on any
+ * call below.  Calls are asynchronous and ordered on `stream` (a
+ * cudaStream_t passed as void*; NULL = the legacy default stream).  `y` must
+ * not overlap any input.  `out` may be the same buffer as `residual`.
+ * Data pointers must be 16-byte aligned.
+ *
+ * Workspace.  Some paths keep scratch data in global memory (chunk states,
+ * direction hand-off flags, the device status word).  Query its size with
+ * ssd_workspace_bytes() for the exact shape and chunk and pass a device
+ * buffer of at least that size; its contents need no initialisation and are
+ * not meaningful after the call.  Calls that share a workspace must not run
+ * concurrently.
+ *
+ * Errors.  Every entry point returns an ssd_status; no exception or abort
+ * crosses the ABI.  Arguments are checked on the host before anything is
+ * launched: SSD_ERR_INVALID_ARG for NULL/misaligned pointers, negative sizes,
+ * seqlen % chunk != 0 or a short workspace; SSD_ERR_UNSUPPORTED for sizes
+ * outside the supported set (headdim in {16,32,64}, dstate in {16,32,64,128},
+ * chunk in {16,32,64,128,256}, nheads % ngroups == 0).  A launch failure
+ * returns SSD_ERR_CUDA.  Device-side waits are bounded: a wait that gives up
+ * records SSD_ERR_TIMEOUT in the workspace status word, which
+ * ssd_workspace_status() reports.  ssd_last_error() gives a text for the most
+ * recent failure on the calling thread.  There is no CPU fallback: a shape
+ * the GPU kernels do not cover is refused.
+ */
+#ifndef BIDIR_SSD_H
+#define BIDIR_SSD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,
+    SSD_ERR_UNSUPPORTED = 2,
+    SSD_ERR_CUDA = 3,
+    SSD_ERR_TIMEOUT = 4
+} ssd_status;
+
+typedef enum { SSD_BF16 = 0, SSD_F32 = 1 } ssd_dtype;
+
+typedef struct {
+    int batch, seqlen, nheads, headdim, dstate, ngroups;
+    ssd_dtype io;             /* dtype of x, dt, B, C, y, residual, out */
+} ssd_shape;
+
+typedef struct {
+    const void *x;            /* [batch][seqlen][nheads][headdim] */
+    const void *dt;           /* [batch][seqlen][nheads], positive */
+    const float *A;           /* [nheads], the per-head decay rate (negative) */
+    const void *B;            /* [batch][seqlen][ngroups][dstate] */
+    const void *C;            /* [batch][seqlen][ngroups][dstate] */
+    const float *D;           /* [nheads] or NULL */
+} ssd_params;
+
+/* Bytes of device workspace that ssd_scan, bidir_ssd and r2l_block_scan need
+ * for this shape and chunk (the largest of the three).  Returns 0 for shapes
+ * the library refuses (the call itself then reports why). */
+size_t ssd_workspace_bytes(const ssd_shape *shape, int chunk);
+
+/* One direction of the scan.  direction = +1 visits t = 0..L-1; direction = -1
+ * visits t = L-1..0, i.e. y = flip(scan(flip(x, dt, B, C))) with the flip done
+ * in the address arithmetic ("Bifocal Diffusion Language Models", section 2,
+ * mechanism).  `chunk` is the length of the blocks of the chunked
+ * (state-passing) evaluation; the result is the same for every chunk up to
+ * float32 rounding.  Writes y. */
+ssd_status ssd_scan(const ssd_shape *shape, const ssd_params *p, int direction, int chunk,
+                    void *y, void *workspace, size_t workspace_bytes, void *stream);
+
+/* The DiffuMamba bidirectional mixer ("DiffuMamba", technical summary,
+ * section 2: a forward and a reverse Mamba layer, independent of each other,
+ * for a symmetric context): y = scan(fwd, +1) + scan(rev, -1), the two
+ * directions with their own parameter sets (pass the same pointers twice to
+ * share them).  Writes y. */
+ssd_status bidir_ssd(const ssd_shape *shape, const ssd_params *fwd, const ssd_params *rev,
+                     int chunk, void *y, void *workspace, size_t workspace_bytes, void *stream);
+
+/* The R2LM right-to-left sidecar over one generation block ("Bifocal
+ * Diffusion Language Models", section 2: the reverse scan's output is a
+ * residual correction scaled by the learnable scalar s, initialised to 0 so
+ * the model starts bit-identical to its causal baseline; at decode time only
+ * the generation block is scanned, with nothing entering from the right):
+ *     out = residual + s * scan(p, -1)   for s != 0
+ *     out = residual (bit for bit)        for s == 0
+ * residual/out are [batch][seqlen][nheads*headdim]. */
+ssd_status r2l_block_scan(const ssd_shape *shape, const ssd_params *p, float s,
+                          const void *residual, int chunk, void *out,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/* Waits for `stream`, then reads and clears the device status word in
+ * `workspace` (SSD_OK, or SSD_ERR_TIMEOUT if a bounded device-side wait gave
+ * up during an earlier call that used this workspace). */
+ssd_status ssd_workspace_status(void *workspace, size_t workspace_bytes, void *stream);
+
+/* Static text for a status code. */
+const char *ssd_status_string(ssd_status s);
+
+/* Text describing the most recent failure on the calling thread ("" if none). */
+const char *ssd_last_error(void);
+
+/* Number of kernels one call launches for this shape and chunk; op: 0 =
+ * ssd_scan, 1 = bidir_ssd, 2 = r2l_block_scan with s != 0.  -1 if refused. */
+int ssd_kernel_launches(const ssd_shape *shape, int chunk, int op);
+
+/* Which kernel family a call with this shape and chunk runs:
+ * 1 = tensor-core (tcgen05) path, 0 = SIMT path, -1 = refused. */
+int ssd_path_for(const ssd_shape *shape, int chunk);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BIDIR_SSD_H */

@@ -32,7 +32,11 @@ residual 32; gate 33; step k of a multi-step workload adds 64*k.
 """
 from __future__ import annotations
 
+import ctypes
 import math
+import os
+import subprocess
+import threading
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -46,9 +50,6 @@ REV_OFFSET = 16
 RESIDUAL_ID = 32
 GATE_ID = 33
 STEP_STRIDE = 64
-
-_CHUNK = 1 << 22  # elements generated per slice, bounds temporary memory
-
 
 def _mix64(z: np.ndarray) -> np.ndarray:
     z = z ^ (z >> np.uint64(30))
@@ -65,7 +66,7 @@ def _stream_key(seed: int, tensor_id: int) -> np.uint64:
 
 
 def _uniform_pair(key: np.uint64, idx: np.ndarray):
-    """Two independent uniforms in (0,1) for each flat index in ``idx``."""
+    """Two independent uniforms in (0,1) for each flat index in ``idx`` (numpy restatement of gen.c)."""
     with np.errstate(over="ignore"):
         base = idx.astype(np.uint64) * np.uint64(2)
         w1 = _mix64(key + (base + np.uint64(1)) * _GOLDEN)
@@ -76,31 +77,54 @@ def _uniform_pair(key: np.uint64, idx: np.ndarray):
     return u1, u2
 
 
-def uniform(seed: int, tensor_id: int, n: int, idx: np.ndarray | None = None) -> np.ndarray:
-    key = _stream_key(seed, tensor_id)
+_GEN_SRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "gen.c")
+_GEN_LIB = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssdgen.so")
+_gen = None
+_gen_lock = threading.Lock()
+
+
+def _genlib():
+    """The compiled bulk generator (gcc, built on first use)."""
+    global _gen
+    with _gen_lock:
+        if _gen is None:
+            if (not os.path.exists(_GEN_LIB)) or os.path.getmtime(_GEN_LIB) < os.path.getmtime(_GEN_SRC):
+                tmp = _GEN_LIB + f".tmp{os.getpid()}"
+                subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-pthread",
+                                       "-o", tmp, _GEN_SRC, "-lm"])
+                os.replace(tmp, _GEN_LIB)
+            lib = ctypes.CDLL(_GEN_LIB)
+            lib.gen_stream.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int, ctypes.c_int64,
+                                       ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int]
+            lib.gen_stream.restype = ctypes.c_int
+            _gen = lib
+    return _gen
+
+
+def _threads() -> int:
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+
+
+def _stream(seed: int, tensor_id: int, normal_dist: bool, n: int, idx, start: int = 0) -> np.ndarray:
     if idx is not None:
-        return _uniform_pair(key, np.asarray(idx))[0]
+        idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int64))
+        n = idx.size
     out = np.empty(n, dtype=np.float64)
-    for s in range(0, n, _CHUNK):
-        e = min(n, s + _CHUNK)
-        out[s:e] = _uniform_pair(key, np.arange(s, e, dtype=np.uint64))[0]
+    rc = _genlib().gen_stream(seed, tensor_id, 1 if normal_dist else 0, start,
+                              idx.ctypes.data if idx is not None else None, n, out.ctypes.data, _threads())
+    if rc != 0:
+        raise MemoryError("input generator failed")
     return out
 
 
-def normal(seed: int, tensor_id: int, n: int, idx: np.ndarray | None = None) -> np.ndarray:
-    key = _stream_key(seed, tensor_id)
+def uniform(seed: int, tensor_id: int, n: int, idx=None) -> np.ndarray:
+    """Uniform(0,1) stream: n elements, or the elements at flat indices ``idx``."""
+    return _stream(seed, tensor_id, False, n, idx)
 
-    def _bm(ix):
-        u1, u2 = _uniform_pair(key, ix)
-        return np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * math.pi * u2)
 
-    if idx is not None:
-        return _bm(np.asarray(idx))
-    out = np.empty(n, dtype=np.float64)
-    for s in range(0, n, _CHUNK):
-        e = min(n, s + _CHUNK)
-        out[s:e] = _bm(np.arange(s, e, dtype=np.uint64))
-    return out
+def normal(seed: int, tensor_id: int, n: int, idx=None) -> np.ndarray:
+    """Standard normal stream (Box-Muller): n elements, or the elements at flat indices ``idx``."""
+    return _stream(seed, tensor_id, True, n, idx)
 
 
 # ---------------------------------------------------------------- rounding
@@ -151,6 +175,23 @@ def _store(vals64: np.ndarray, dtype: str, shape) -> Stored:
     return Stored("f32", tuple(shape), f32)
 
 
+_SLICE = 1 << 25
+
+
+def _gen_tensor(seed: int, tensor_id: int, shape, dtype: str, normal_dist: bool, transform=None) -> Stored:
+    """Draws a whole tensor slice by slice (bounded float64 temporaries) and rounds it to ``dtype``."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint16 if dtype == "bf16" else np.float32)
+    for s0 in range(0, n, _SLICE):
+        m = min(_SLICE, n - s0)
+        v = _stream(seed, tensor_id, normal_dist, m, None, start=s0)
+        if transform is not None:
+            v = transform(v)
+        f32 = f64_to_f32(v)
+        out[s0:s0 + m] = f32_to_bf16_bits(f32) if dtype == "bf16" else f32
+    return Stored(dtype, tuple(shape), out)
+
+
 @dataclass
 class Shape:
     batch: int
@@ -183,20 +224,15 @@ def make_params(shape: Shape, seed: int = 0, offset: int = 0, with_D: bool = Tru
     b, L, H, P, N, G = (shape.batch, shape.seqlen, shape.nheads, shape.headdim,
                         shape.dstate, shape.ngroups)
     tid = {k: v + offset for k, v in TENSOR_IDS.items()}
-    x = normal(seed, tid["x"], b * L * H * P)
-    z = normal(seed, tid["dt"], b * L * H)
-    dt = np.log1p(np.exp(z - 4.0))
-    A = -np.exp(uniform(seed, tid["A"], H) * math.log(16.0))
-    Bv = normal(seed, tid["B"], b * L * G * N) / math.sqrt(N)
-    Cv = normal(seed, tid["C"], b * L * G * N) / math.sqrt(N)
-    D = uniform(seed, tid["D"], H) if with_D else np.zeros(H)
     io = shape.io
+    A = -np.exp(uniform(seed, tid["A"], H) * math.log(16.0))
+    D = uniform(seed, tid["D"], H) if with_D else np.zeros(H)
     return Params(
-        x=_store(x, io, (b, L, H, P)),
-        dt=_store(dt, io, (b, L, H)),
+        x=_gen_tensor(seed, tid["x"], (b, L, H, P), io, True),
+        dt=_gen_tensor(seed, tid["dt"], (b, L, H), io, True, lambda z: np.log1p(np.exp(z - 4.0))),
         A=_store(A, "f32", (H,)),
-        B=_store(Bv, io, (b, L, G, N)),
-        C=_store(Cv, io, (b, L, G, N)),
+        B=_gen_tensor(seed, tid["B"], (b, L, G, N), io, True, lambda z: z / math.sqrt(N)),
+        C=_gen_tensor(seed, tid["C"], (b, L, G, N), io, True, lambda z: z / math.sqrt(N)),
         D=_store(D, "f32", (H,)),
         extra={"with_D": with_D},
     )
@@ -211,8 +247,7 @@ def make_bidir(shape: Shape, seed: int = 0, step: int = 0, with_D: bool = True):
 
 def make_residual(shape: Shape, seed: int = 0, step: int = 0) -> Stored:
     b, L, H, P = shape.batch, shape.seqlen, shape.nheads, shape.headdim
-    r = normal(seed, RESIDUAL_ID + STEP_STRIDE * step, b * L * H * P)
-    return _store(r, shape.io, (b, L, H * P))
+    return _gen_tensor(seed, RESIDUAL_ID + STEP_STRIDE * step, (b, L, H * P), shape.io, True)
 
 
 def make_gate(seed: int = 0, step: int = 0) -> float:

@@ -56,3 +56,15 @@ def test_directions_and_steps_are_independent():
     assert not np.array_equal(pf.x.data, pr.x.data)
     pf1, _ = si.make_bidir(shape, seed=0, step=1)
     assert not np.array_equal(pf.x.data, pf1.x.data)
+
+
+def test_bulk_generator_matches_numpy_restatement():
+    """gen.c and the numpy restatement of the same stream definition agree."""
+    key = si._stream_key(5, 9)
+    idx = np.arange(0, 4096, dtype=np.uint64) * np.uint64(977)
+    u1, u2 = si._uniform_pair(key, idx)
+    ref_n = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * math.pi * u2)
+    got_n = si.normal(5, 9, 0, idx=idx.astype(np.int64))
+    got_u = si.uniform(5, 9, 0, idx=idx.astype(np.int64))
+    assert np.array_equal(got_u, u1)
+    assert np.max(np.abs(got_n - ref_n)) <= 1e-15

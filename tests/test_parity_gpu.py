@@ -1,0 +1,199 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on the same seeded inputs.
+
+Metric: max|y - y_ref| / max|y_ref| over the output.  Bars: 2e-2 for bf16 io
+(float32 state), 1e-4 for float32 io.  Every bf16/f32 case is checked twice:
+on the full output and on the "SSD-only" output (D = None on both sides),
+because the skip term D*x dominates |y| and would hide an error in the scan.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ssd_inputs as si
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"bf16": 2e-2, "f32": 1e-4}
+
+
+@pytest.fixture(scope="module")
+def ssd():
+    import bidirectional_mamba_ssd_bidir_b200 as m
+    return m
+
+
+def _dev(p, with_D=True):
+    dev = torch.device("cuda")
+    d = {k: getattr(p, k).torch(dev) for k in ("x", "dt", "A", "B", "C")}
+    d["D"] = p.D.torch(dev) if with_D else None
+    return d
+
+
+def _f64(y):
+    return y.detach().double().cpu().numpy()
+
+
+def _bidir_case(ssd, shape, chunk, with_D, seed=0):
+    pf, pr = si.make_bidir(shape, seed=seed, with_D=with_D)
+    y = ssd.bidir_ssd(_dev(pf, with_D), _dev(pr, with_D), chunk=chunk)
+    torch.cuda.synchronize()
+    ref = oracle.bidir_f64(oracle.params_f64(pf), oracle.params_f64(pr))
+    return oracle.rel_err(_f64(y), ref)
+
+
+SHAPES = [
+    # (batch, L, H, P, N, G, io), chunk
+    (si.Shape(1, 64, 2, 16, 16, 1, "f32"), 16),            # the tiny float32 workload
+    (si.Shape(2, 512, 8, 64, 128, 1, "bf16"), 256),        # layer shape, several chunks
+    (si.Shape(1, 768, 6, 64, 128, 1, "bf16"), 256),        # odd chunk count, 6 heads
+    (si.Shape(3, 384, 4, 64, 128, 1, "bf16"), 128),        # 3 chunks of 128
+    (si.Shape(2, 256, 4, 32, 64, 1, "bf16"), 64),
+    (si.Shape(1, 256, 4, 16, 16, 1, "bf16"), 16),
+    (si.Shape(2, 192, 4, 64, 64, 2, "bf16"), 64),          # two groups
+    (si.Shape(1, 96, 3, 16, 32, 1, "f32"), 32),
+    (si.Shape(2, 256, 2, 64, 128, 1, "f32"), 128),
+]
+
+
+@pytest.mark.parametrize("shape,chunk", SHAPES, ids=lambda v: str(v) if isinstance(v, int) else
+                         f"b{v.batch}L{v.seqlen}H{v.nheads}P{v.headdim}N{v.dstate}G{v.ngroups}{v.io}")
+@pytest.mark.parametrize("with_D", [True, False], ids=["full", "ssd_only"])
+def test_bidir_parity(ssd, shape, chunk, with_D):
+    err = _bidir_case(ssd, shape, chunk, with_D)
+    assert err <= TOL[shape.io], f"rel err {err:.3e}"
+
+
+@pytest.mark.parametrize("direction", [1, -1])
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_single_direction_parity(ssd, direction, io):
+    shape = si.Shape(2, 512, 4, 64, 128, 1, io)
+    p = si.make_params(shape, seed=3, with_D=False)
+    y = ssd.ssd_scan(**_dev(p, False), direction=direction, chunk=128)
+    torch.cuda.synchronize()
+    q = oracle.params_f64(p)
+    ref = oracle.ssd_scan_f64(q["x"], q["dt"], q["A"], q["B"], q["C"], None, direction)
+    assert oracle.rel_err(_f64(y), ref) <= TOL[io]
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64, 128, 256])
+def test_chunk_size_invariance(ssd, chunk):
+    shape = si.Shape(1, 512, 4, 64, 128, 1, "bf16")
+    err = _bidir_case(ssd, shape, chunk, with_D=False, seed=5)
+    assert err <= TOL["bf16"]
+
+
+def _flip(p):
+    q = {}
+    for k, v in p.items():
+        q[k] = v.flip(1).contiguous() if (v is not None and k in ("x", "dt", "B", "C")) else v
+    return q
+
+
+@pytest.mark.parametrize("io,chunk", [("f32", 16), ("bf16", 64), ("bf16", 256)])
+def test_reverse_is_flip_forward_flip(ssd, io, chunk):
+    shape = si.Shape(2, 512, 4, 64, 128, 1, io)
+    p = _dev(si.make_params(shape, seed=6))
+    yr = ssd.ssd_scan(**p, direction=-1, chunk=chunk)
+    yf = ssd.ssd_scan(**_flip(p), direction=1, chunk=chunk).flip(1)
+    torch.cuda.synchronize()
+    if ssd.path_for((2, 512, 4, 64, 128, 1), p["x"].dtype, chunk) == 0:
+        assert torch.equal(yr, yf)      # same arithmetic in scan order: bit for bit
+    else:
+        assert oracle.rel_err(_f64(yr), _f64(yf)) <= 1e-2
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_bidir_is_sum_of_directions(ssd, io):
+    shape = si.Shape(2, 512, 4, 64, 128, 1, io)
+    pf, pr = si.make_bidir(shape, seed=8)
+    df, dr = _dev(pf), _dev(pr)
+    yb = ssd.bidir_ssd(df, dr, chunk=128).double()
+    yf = ssd.ssd_scan(**df, direction=1, chunk=128).double()
+    yr = ssd.ssd_scan(**dr, direction=-1, chunk=128).double()
+    torch.cuda.synchronize()
+    s = yf + yr
+    if io == "f32":
+        assert torch.max(torch.abs(yb - s)).item() <= 1e-5 * torch.max(torch.abs(s)).item()
+    else:
+        # two roundings to bf16 (8-bit significand) on each side
+        bound = 2.0 ** -7 * torch.maximum(torch.maximum(yf.abs(), yr.abs()), s.abs())
+        assert bool(torch.all(torch.abs(yb - s) <= bound))
+
+
+def test_dt_zero_gives_skip_term_bitwise(ssd):
+    shape = si.Shape(1, 128, 4, 64, 128, 1, "f32")
+    p = _dev(si.make_params(shape, seed=9))
+    p["dt"] = torch.zeros_like(p["dt"])
+    for d in (1, -1):
+        y = ssd.ssd_scan(**p, direction=d, chunk=64)
+        torch.cuda.synchronize()
+        assert torch.equal(y, p["D"][None, None, :, None] * p["x"])
+
+
+def test_deterministic(ssd):
+    shape = si.Shape(2, 512, 8, 64, 128, 1, "bf16")
+    pf, pr = si.make_bidir(shape, seed=10)
+    df, dr = _dev(pf), _dev(pr)
+    y1 = ssd.bidir_ssd(df, dr, chunk=256)
+    y2 = ssd.bidir_ssd(df, dr, chunk=256)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_empty_batch(ssd):
+    shape = si.Shape(0, 256, 4, 64, 128, 1, "bf16")
+    x = torch.empty(0, 256, 4, 64, dtype=torch.bfloat16, device="cuda")
+    B = torch.empty(0, 256, 1, 128, dtype=torch.bfloat16, device="cuda")
+    dt = torch.empty(0, 256, 4, dtype=torch.bfloat16, device="cuda")
+    A = -torch.ones(4, device="cuda")
+    y = ssd.ssd_scan(x, dt, A, B, B, None, 1, 256)
+    assert y.shape == x.shape
+
+
+def test_refuses_unsupported_shape(ssd):
+    x = torch.zeros(1, 64, 2, 48, dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros(1, 64, 1, 16, dtype=torch.bfloat16, device="cuda")
+    dt = torch.zeros(1, 64, 2, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ssd.SSDError):
+        ssd.ssd_scan(x, dt, -torch.ones(2, device="cuda"), B, B, None, 1, 16)
+
+
+# ------------------------------------------------------------------ R2L sidecar
+
+def _r2l_step(ssd, shape, chunk, step, s=None):
+    p = si.make_params(shape, seed=0, offset=si.STEP_STRIDE * step + si.REV_OFFSET)
+    res = si.make_residual(shape, seed=0, step=step)
+    gate = si.make_gate(0, step) if s is None else s
+    out = ssd.r2l_block_scan(_dev(p), gate, res.torch("cuda"), chunk=chunk)
+    torch.cuda.synchronize()
+    return p, res, gate, out
+
+
+def test_r2l_gate_zero_is_bit_identical(ssd):
+    shape = si.WORKLOADS["r2l_block_L32"]["shape"]
+    p, res, _, out = _r2l_step(ssd, shape, 32, 0, s=0.0)
+    assert torch.equal(out.cpu().view(torch.int16), res.torch().view(torch.int16))
+    # in place: out is the residual buffer itself
+    r = res.torch("cuda")
+    ref = r.clone()
+    o = ssd.r2l_block_scan(_dev(p), 0.0, r, chunk=32, out=r)
+    torch.cuda.synchronize()
+    assert torch.equal(o.view(torch.int16), ref.view(torch.int16))
+
+
+@pytest.mark.parametrize("chunk", [32, 16])
+def test_r2l_block_parity(ssd, chunk):
+    """Full output against the oracle, then the scan alone: zero residual and no D, so out = s * y_rev."""
+    shape = si.WORKLOADS["r2l_block_L32"]["shape"]
+    for step in range(4):
+        p, res, gate, out = _r2l_step(ssd, shape, chunk, step)
+        ref = oracle.r2l_block_f64(oracle.params_f64(p), gate, res.f64())
+        assert oracle.rel_err(_f64(out), ref) <= TOL["bf16"]
+        q = si.make_params(shape, seed=0, offset=si.STEP_STRIDE * step + si.REV_OFFSET, with_D=False)
+        zero = torch.zeros(shape.batch, shape.seqlen, shape.nheads * shape.headdim,
+                           dtype=torch.bfloat16, device="cuda")
+        o2 = ssd.r2l_block_scan(_dev(q, False), gate, zero, chunk=chunk)
+        torch.cuda.synchronize()
+        ref2 = oracle.r2l_block_f64(oracle.params_f64(q), gate, np.zeros(zero.shape))
+        assert oracle.rel_err(_f64(o2), ref2) <= TOL["bf16"]
