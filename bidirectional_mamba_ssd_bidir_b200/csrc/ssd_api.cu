@@ -99,9 +99,14 @@ ssd::ScanArgs make_args(const ssd_shape *s, const ssd_params *p, int dir, int ch
     return a;
 }
 
-ssd_status common_checks(const ssd_shape *s, int chunk, void *out, void *ws, size_t ws_bytes) {
+// Validates the shape and, for a non-empty problem, the output and workspace.
+// *empty is set when there is nothing to compute (batch or seqlen zero): the
+// call then succeeds without looking at any pointer.
+ssd_status common_checks(const ssd_shape *s, int chunk, void *out, void *ws, size_t ws_bytes, bool *empty) {
     ssd_status st = check_shape(s, chunk);
     if (st != SSD_OK) return st;
+    *empty = s->batch == 0 || s->seqlen == 0;
+    if (*empty) return SSD_OK;
     if (!aligned16(out)) return fail(SSD_ERR_INVALID_ARG, "output must be non-NULL and 16-byte aligned");
     const size_t need = path_ws_bytes(s, chunk);
     if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
@@ -143,11 +148,12 @@ int ssd_kernel_launches(const ssd_shape *shape, int chunk, int op) {
 ssd_status ssd_scan(const ssd_shape *shape, const ssd_params *p, int direction, int chunk, void *y,
                     void *workspace, size_t workspace_bytes, void *stream) {
     g_err.clear();
-    ssd_status st = common_checks(shape, chunk, y, workspace, workspace_bytes);
+    bool empty = false;
+    ssd_status st = common_checks(shape, chunk, y, workspace, workspace_bytes, &empty);
     if (st != SSD_OK) return st;
     if (direction != 1 && direction != -1) return fail(SSD_ERR_INVALID_ARG, "direction must be +1 or -1");
+    if (empty) return SSD_OK;
     if ((st = check_params(p, "scan")) != SSD_OK) return st;
-    if (shape->batch == 0 || shape->seqlen == 0) return SSD_OK;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (choose_path(shape, chunk) == 1) {
         ssd::TcArgs t = ssd::make_tc_args(shape->batch, shape->seqlen, shape->nheads, chunk,
@@ -163,11 +169,11 @@ ssd_status ssd_scan(const ssd_shape *shape, const ssd_params *p, int direction, 
 ssd_status bidir_ssd(const ssd_shape *shape, const ssd_params *fwd, const ssd_params *rev, int chunk, void *y,
                      void *workspace, size_t workspace_bytes, void *stream) {
     g_err.clear();
-    ssd_status st = common_checks(shape, chunk, y, workspace, workspace_bytes);
-    if (st != SSD_OK) return st;
+    bool empty = false;
+    ssd_status st = common_checks(shape, chunk, y, workspace, workspace_bytes, &empty);
+    if (st != SSD_OK || empty) return st;
     if ((st = check_params(fwd, "forward")) != SSD_OK) return st;
     if ((st = check_params(rev, "reverse")) != SSD_OK) return st;
-    if (shape->batch == 0 || shape->seqlen == 0) return SSD_OK;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (choose_path(shape, chunk) == 1) {
         ssd::TcArgs t = ssd::make_tc_args(shape->batch, shape->seqlen, shape->nheads, chunk,
@@ -186,11 +192,11 @@ ssd_status bidir_ssd(const ssd_shape *shape, const ssd_params *fwd, const ssd_pa
 ssd_status r2l_block_scan(const ssd_shape *shape, const ssd_params *p, float s, const void *residual, int chunk,
                           void *out, void *workspace, size_t workspace_bytes, void *stream) {
     g_err.clear();
-    ssd_status st = common_checks(shape, chunk, out, workspace, workspace_bytes);
-    if (st != SSD_OK) return st;
+    bool empty = false;
+    ssd_status st = common_checks(shape, chunk, out, workspace, workspace_bytes, &empty);
+    if (st != SSD_OK || empty) return st;
     if ((st = check_params(p, "r2l")) != SSD_OK) return st;
     if (!aligned16(residual)) return fail(SSD_ERR_INVALID_ARG, "residual must be non-NULL and 16-byte aligned");
-    if (shape->batch == 0 || shape->seqlen == 0) return SSD_OK;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (s == 0.0f) {
         // Gate at its initial value: the block is returned untouched, bit for bit.

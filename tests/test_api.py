@@ -88,6 +88,7 @@ def test_validation_statuses():
     need = _ws(s, 16)
     assert _call_scan(s, _fake_params(), chunk=24, y=good, ws=good, wsb=need) == 2         # unsupported chunk
     assert _call_scan(_shape(L=60), _fake_params(), y=good, ws=good, wsb=need) == 1       # ragged length
+    assert b"multiple of chunk" in ssd.lib.ssd_last_error()
     assert _call_scan(s, None, y=good, ws=good, wsb=need) == 1                            # NULL params
     assert _call_scan(s, _fake_params(), y=None, ws=good, wsb=need) == 1                  # NULL output
     assert _call_scan(s, _fake_params(), y=good + 4, ws=good, wsb=need) == 1              # misaligned output
@@ -96,13 +97,13 @@ def test_validation_statuses():
     assert _call_scan(s, _fake_params(), direction=0, y=good, ws=good, wsb=need) == 1     # bad direction
     assert _call_scan(s, _fake_params(good + 8), y=good, ws=good, wsb=need) == 1          # misaligned x
     assert _call_scan(_shape(P=48), _fake_params(), y=good, ws=good, wsb=need) == 2
-    assert b"multiple" in ssd.lib.ssd_last_error() or True
     assert ssd.lib.ssd_status_string(4) == b"device wait timed out"
 
 
 def test_empty_problem_is_a_no_op():
     s = _shape(b=0)
     assert _call_scan(s, _fake_params(), y=1 << 20, ws=1 << 20, wsb=_ws(s, 16)) == 0
+    assert _call_scan(s, None, y=None, ws=None, wsb=0) == 0   # nothing to compute: pointers unused
 
 
 def test_python_binding_refuses_cpu_tensors():
