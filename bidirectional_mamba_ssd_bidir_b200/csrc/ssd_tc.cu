@@ -68,6 +68,23 @@ enum Bar {
 constexpr long long kWaitCycles = 4000000000LL;        // ~2 s at B200 clocks
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Optional phase timeline for profiling builds (-DSSD_TRACE): %globaltimer
+// stamps of CTA 0, first kTraceBlocks blocks, per role and phase.
+#ifdef SSD_TRACE
+constexpr int kTraceBlocks = 8, kTracePts = 16;
+__device__ unsigned long long g_trace[3][kTraceBlocks][kTracePts];
+__device__ __forceinline__ void trace_pt(int role, int j, int k) {
+    if (blockIdx.x == 0 && j < kTraceBlocks) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        g_trace[role][j][k] = t;
+    }
+}
+#define SSD_TRACE_PT(role, j, k) trace_pt(role, j, k)
+#else
+#define SSD_TRACE_PT(role, j, k) ((void)0)
+#endif
+
 struct TcParams {
     int batch, L, H, nblk, dir, accumulate;
     const __nv_bfloat16 *dt;
@@ -262,11 +279,13 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
                 const int row = b * L + cm * kBlk;
                 const int st = j & 1;
                 if (j >= 2 && !mbar_wait(bar(B_XEMPTY0 + st), ((j >> 1) - 1) & 1, MASK, abort_flag, prm.status, 11)) break;
+                SSD_TRACE_PT(0, j, 0);
                 mbar_expect_tx(bar(B_XFULL0 + st), 2 * kTileBytes);
                 for (int h = 0; h < 2; ++h)
                     tma_load_2d(sbase + kOffX + (st * 2 + h) * kTileBytes, &map_x, (h0 + h) * kP, row,
                                 bar(B_XFULL0 + st));
                 if (j >= 1 && !mbar_wait(bar(B_BCEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 12)) break;
+                SSD_TRACE_PT(0, j, 1);
                 mbar_expect_tx(bar(B_BCFULL), 4 * kTileBytes);
                 for (int q = 0; q < 2; ++q) {
                     tma_load_2d(sbase + kOffB + q * kTileBytes, &map_b, q * 64, row, bar(B_BCFULL));
@@ -295,6 +314,7 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
                 // G = C B^T  (M = rows, N = source rows, K = n)
                 if (!mbar_wait(bar(B_BCFULL), j & 1, MASK, abort_flag, prm.status, 21)) break;
                 if (j >= 1 && !mbar_wait(bar(B_GEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 22)) break;
+                SSD_TRACE_PT(1, j, 0);
                 tc_fence_after();
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = (ks >> 2) * kTileBytes + (ks & 3) * 32;
@@ -304,6 +324,7 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
                 // S^T = B^T (w x)  (M = n, N = (head, p), K = rows); both operands MN-major
                 if (!mbar_wait(bar(B_WXREADY), j & 1, MASK, abort_flag, prm.status, 23)) break;
                 if (j >= 1 && !mbar_wait(bar(B_SEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 24)) break;
+                SSD_TRACE_PT(1, j, 1);
                 tc_fence_after();
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = ks * 2048;
@@ -315,6 +336,7 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
                 if (j >= 1) {
                     if (!mbar_wait(bar(B_SPREADY), (j - 1) & 1, MASK, abort_flag, prm.status, 25)) break;
                     if (!mbar_wait(bar(B_YEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 26)) break;
+                    SSD_TRACE_PT(1, j, 2);
                     tc_fence_after();
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t offc = (ks >> 2) * kTileBytes + (ks & 3) * 32;
@@ -328,6 +350,7 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
                 if (!mbar_wait(bar(B_MREADY), j & 1, MASK, abort_flag, prm.status, 27)) break;
                 if (j >= 1 && !mbar_wait(bar(B_RSREADY), (j - 1) & 1, MASK, abort_flag, prm.status, 28)) break;
                 if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 29)) break;
+                SSD_TRACE_PT(1, j, 3);
                 tc_fence_after();
                 for (int h = 0; h < 2; ++h)
                     for (int ks = 0; ks < 8; ++ks)
@@ -378,6 +401,7 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
             if (__any_sync(0xffffffffu, *abort_flag)) break;
             const int st = j & 1;
             const int t = tok_of(j);
+            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 0);
             const float dtr = dt_next;
             if (j + 1 < nblk) dt_next = __bfloat162float(prm.dt[((size_t)b * L + tok_of(j + 1)) * prm.H + h]);
 
@@ -407,6 +431,7 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
 
             // w (.) x -> wX tile (same swizzled layout as the X tile)
             if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 41)) break;
+            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 1);
             const uint8_t *xt = sm + kOffX + (st * 2 + wg) * kTileBytes;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -420,10 +445,12 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
             }
             fence_async_smem();
             if (!wg_sync(53)) break;           // cs2/dts of all rows visible to this WG
+            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 2);
             if (lane == 0) mbar_arrive(bar(B_WXREADY));
 
             // M_h = G (.) decay (.) dt over the causal triangle, bf16 into TMEM
             if (!mbar_wait(bar(B_GFULL), j & 1, MASK, abort_flag, prm.status, 42)) break;
+            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 3);
             tc_fence_after();
             for (int kb = 0; kb < 4; ++kb) {
                 const bool need = dir > 0 ? kb <= wq : kb >= wq;
@@ -449,9 +476,11 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_GEMPTY));
+            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 10);
 
             // state: S' <- exp(cs_last) S' + S, thread r holds state row n = r
             if (!mbar_wait(bar(B_SFULL), j & 1, MASK, abort_flag, prm.status, 43)) break;
+            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 4);
             tc_fence_after();
             {
                 float sv[32];
@@ -469,6 +498,7 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
             if (j + 1 < nblk) {
                 // the previous state tile must have been consumed by this block's Y = C S'^T
                 if (j >= 1 && !mbar_wait(bar(B_YOFFFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 44)) break;
+                if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 5);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     uint4 o;
@@ -486,6 +516,7 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
             // Y (from the incoming state) scaled by exp(cs_r), before the intra-block term is added
             if (j >= 1) {
                 if (!mbar_wait(bar(B_YOFFFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 45)) break;
+                if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 6);
                 tc_fence_after();
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -505,7 +536,9 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
             if (lane == 0) mbar_arrive(bar(B_MREADY));
 
             // epilogue: y = Y + D x, bf16, 128 contiguous bytes per thread
+            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 7);
             if (!mbar_wait(bar(B_YFULL), j & 1, MASK, abort_flag, prm.status, 46)) break;
+            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 8);
             tc_fence_after();
             float yv[64];
             tmem_ld32(tl + kColY + 64 * wg, yv);
@@ -543,6 +576,7 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_XEMPTY0 + st));
+            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 9);
         }
     }
 
@@ -608,6 +642,14 @@ void tc_set_direction(TcArgs &t, int slot, int dir, const void *x, const void *d
 }
 
 int tc_launches(bool bidir) { return bidir ? 2 : 1; }
+
+#ifdef SSD_TRACE
+extern "C" int ssd_debug_trace(unsigned long long *out, int n) {
+    const int total = 3 * kTraceBlocks * kTracePts;
+    if (n < total) return -1;
+    return cudaMemcpyFromSymbol(out, g_trace, sizeof(unsigned long long) * total) == cudaSuccess ? total : -2;
+}
+#endif
 
 cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
     static std::once_flag once;

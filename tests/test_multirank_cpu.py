@@ -1,0 +1,72 @@
+"""Multi-rank host logic of the bench on CPU (gloo, world size 2).
+
+The scan shards into independent (batch, head, direction) chains, so the
+multi-GPU bench gives every rank its own batch of sequences (weak scaling)
+and exchanges nothing but the timing: a barrier and a MAX all-reduce.  These
+tests run that logic with two gloo ranks on the host.
+"""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import sys
+    sys.path.insert(0, ROOT)
+    from datetime import timedelta
+
+    import torch.distributed as dist
+
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    plan = bench.shard_plan(rank, world, bench.DEFAULT_WORKLOAD)
+    t = bench.max_over_ranks(1.5 + rank, dist)          # rank 1 is the slow one
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, plan["seed"], plan["tokens"], tuple(vars(plan["shape"]).values()), t))
+
+
+def test_two_ranks_shard_and_max():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    res.sort()
+    (r0, s0, n0, sh0, t0), (r1, s1, n1, sh1, t1) = res
+    assert s0 != s1                      # independent sequences per rank
+    assert sh0 == sh1 and n0 == n1       # same per-rank work: weak scaling
+    assert t0 == t1 == 2.5               # everyone reports the slowest rank
+
+
+def test_single_process_max_is_identity():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.25, None) == 3.25
+
+
+def test_algorithmic_bytes_per_token():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import ssd_inputs as si
+    shape = si.WORKLOADS[bench.DEFAULT_WORKLOAD]["shape"]
+    # per direction: x 64*64*2 + dt 64*2 + B,C 2*128*2; y 64*64*2 written once
+    assert bench.algorithmic_bytes_per_token(shape) == 2 * (8192 + 128 + 512) + 8192 == 25856
