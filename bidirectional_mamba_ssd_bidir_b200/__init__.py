@@ -65,6 +65,8 @@ lib.ssd_workspace_status.argtypes = [_VP, _SZ, _VP]
 lib.ssd_workspace_status.restype = ctypes.c_int
 lib.ssd_status_string.argtypes = [ctypes.c_int]
 lib.ssd_status_string.restype = ctypes.c_char_p
+lib.ssd_debug_fault.argtypes = [ctypes.c_int, ctypes.c_double]
+lib.ssd_debug_fault.restype = ctypes.c_int
 lib.ssd_last_error.argtypes = []
 lib.ssd_last_error.restype = ctypes.c_char_p
 

@@ -3,6 +3,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <string>
 
 #include "../../include/bidir_ssd.h"
@@ -12,6 +13,19 @@
 namespace {
 
 thread_local std::string g_err;
+
+// Process-wide test hooks (ssd_debug_fault): bound of device-side waits and an
+// injected fault.  Defaults: 2 s, no fault.
+std::atomic<int> g_fault{0};
+std::atomic<long long> g_wait_ns{2000000000LL};
+
+long long wait_cycles_now() {
+    int dev = 0, khz = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev) != cudaSuccess ||
+        khz <= 0)
+        khz = 2000000;
+    return (long long)((double)g_wait_ns.load() * 1e-9 * (double)khz * 1e3);
+}
 
 ssd_status fail(ssd_status s, const char *fmt, ...) {
     char buf[512];
@@ -159,6 +173,8 @@ ssd_status ssd_scan(const ssd_shape *shape, const ssd_params *p, int direction, 
         ssd::TcArgs t = ssd::make_tc_args(shape->batch, shape->seqlen, shape->nheads, chunk,
                                           static_cast<char *>(workspace) + kStatusBytes,
                                           static_cast<int *>(workspace));
+        t.wait_cycles = wait_cycles_now();
+        t.fault = g_fault.load();
         ssd::tc_set_direction(t, 0, direction, p->x, p->dt, p->A, p->B, p->C, p->D);
         cudaError_t e = ssd::launch_tc(t, /*bidir=*/false, y, cs);
         return e == cudaSuccess ? SSD_OK : cuda_fail(e, "tensor-core scan launch");
@@ -179,6 +195,8 @@ ssd_status bidir_ssd(const ssd_shape *shape, const ssd_params *fwd, const ssd_pa
         ssd::TcArgs t = ssd::make_tc_args(shape->batch, shape->seqlen, shape->nheads, chunk,
                                           static_cast<char *>(workspace) + kStatusBytes,
                                           static_cast<int *>(workspace));
+        t.wait_cycles = wait_cycles_now();
+        t.fault = g_fault.load();
         ssd::tc_set_direction(t, 0, 1, fwd->x, fwd->dt, fwd->A, fwd->B, fwd->C, fwd->D);
         ssd::tc_set_direction(t, 1, -1, rev->x, rev->dt, rev->A, rev->B, rev->C, rev->D);
         cudaError_t e = ssd::launch_tc(t, /*bidir=*/true, y, cs);
@@ -238,5 +256,15 @@ const char *ssd_status_string(ssd_status s) {
 }
 
 const char *ssd_last_error(void) { return g_err.c_str(); }
+
+ssd_status ssd_debug_fault(int mode, double wait_limit_seconds) {
+    g_err.clear();
+    if (mode < 0 || mode > 1) return fail(SSD_ERR_INVALID_ARG, "unknown fault mode %d", mode);
+    if (!(wait_limit_seconds >= 1e-4 && wait_limit_seconds <= 60.0))
+        return fail(SSD_ERR_INVALID_ARG, "wait limit must be within [1e-4, 60] seconds");
+    g_fault.store(mode);
+    g_wait_ns.store((long long)(wait_limit_seconds * 1e9));
+    return SSD_OK;
+}
 
 }  // extern "C"

@@ -12,26 +12,45 @@
 //   Y    = C S'^T_prev                 tcgen05, N = 2 heads x 64       TMEM [384,512)
 //   Y   *= exp(cs_r) per row           CUDA cores (TMEM ld/st)
 //   Y   += M_h X_h                     tcgen05, A from TMEM, N = 64
-//   y    = Y + D x                     CUDA cores -> bf16 global stores
+//   y    = Y + D x                     CUDA cores -> smem -> coalesced rows
 //   S'   = exp(cs_last) S' + S         CUDA cores, float32 registers -> bf16 smem
 //
 // This is the chunked evaluation of the recurrence S <- exp(dt A) S +
-// dt x (outer) B, y = C.S + D x that the Mamba-2 layers of the DiffuMamba mixer
-// ("DiffuMamba", technical summary, section 2) and the R2LM right-to-left
-// stream ("Bifocal Diffusion Language Models", section 2, mechanism) run.
-// The reverse direction walks the blocks from the end and uses suffix sums
-// and the upper triangle: the flip lives in the address arithmetic only.
+// dt x (outer) B, y = C.S + D x that the Mamba-2 layers of the DiffuMamba
+// mixer ("DiffuMamba", technical summary, section 2) and the R2LM
+// right-to-left stream ("Bifocal Diffusion Language Models", section 2,
+// mechanism) run.  The reverse direction walks the blocks from the end and
+// uses suffix sums and the upper triangle: the flip lives in the address
+// arithmetic only.
 //
-// Warp roles (384 threads): warp 0 issues TMA loads, warp 1 owns TMEM and
-// issues the MMAs (one thread), warps 4-7 do the CUDA-core work of head h0
-// and warps 8-11 that of head h0+1 (thread r <-> TMEM lane r).  Every
-// mbarrier wait is bounded; a wait that runs out records SSD_ERR_TIMEOUT in
-// the status word and the CTA winds down without touching more data.
+// Decay mask.  Inside a block the 128 rows split into four 32-row quarters
+// (= the four TMEM lane quarters).  For a source s in an earlier quarter than
+// the output row r, exp(cs_r - cs_s) = exp(cs_r - cs_ref) * exp(cs_ref - cs_s)
+// with ref the quarter boundary between them; both factors are <= 1, so the
+// product never overflows, and the mask becomes (row factor) x (column table)
+// with no exponential per element.  Only the 32 x 32 diagonal sub-blocks take
+// a direct exponential.
+//
+// Bidirectional mixer in one launch.  The CTAs of the forward and reverse
+// scans of one head pair are neighbours in the grid.  For every output block
+// the first of the two to finish writes its part of y, the second adds its
+// own part to it: an epoch-tagged ticket per (batch, head, block) decides the
+// order and an epoch-tagged ready word publishes the first part.  The first
+// never waits, so the hand-off cannot deadlock whatever the residency.
+//
+// Warp roles (320 threads): warps 0-3 do the CUDA-core work of head h0 and
+// warps 4-7 that of head h0+1 (thread r <-> TMEM lane r), warp 8 issues the
+// TMA loads, warp 9 owns TMEM and issues the MMAs (one thread).  Every wait is
+// bounded; a wait that runs out records SSD_ERR_TIMEOUT in the status word and
+// the CTA winds down without touching more data.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <chrono>
+#include <cstring>
 #include <mutex>
 
 #include "ssd_tc.cuh"
@@ -41,56 +60,75 @@ namespace {
 
 constexpr int kBlk = 128;            // tokens per block (MMA M)
 constexpr int kP = 64, kN = 128;
-constexpr int kThreads = 384;
+constexpr int kThreads = 320;        // warps 0-7: two head warpgroups; 8: TMA; 9: MMA + TMEM
+constexpr int kWarpTma = 8, kWarpMma = 9;
 constexpr uint32_t kTileBytes = kBlk * 64 * 2;        // one [128][64] bf16 swizzled tile = 16 KB
+constexpr uint32_t kDtBytes = kBlk * 8 * 2;           // dt box: 128 tokens x 8 heads, bf16
+constexpr uint32_t kStageBytes = 2 * kTileBytes + kDtBytes;   // x of 2 heads + dt = 34 KB
 
 // TMEM column map
 constexpr uint32_t kColG = 0, kColM = 128, kColS = 256, kColY = 384;
 
 // shared memory map (offsets from a 1024-aligned base)
-constexpr uint32_t kOffX = 0;                          // 2 stages x 2 heads x 16 KB
-constexpr uint32_t kOffB = kOffX + 2 * 2 * kTileBytes; // 2 sub-tiles (n 0..63, 64..127)
+constexpr uint32_t kOffX = 0;                          // 2 stages: [x h0 | x h1 | dt]
+constexpr uint32_t kOffB = kOffX + 2 * kStageBytes;    // 2 sub-tiles (n 0..63, 64..127)
 constexpr uint32_t kOffC = kOffB + 2 * kTileBytes;
 constexpr uint32_t kOffWX = kOffC + 2 * kTileBytes;    // 2 heads
 constexpr uint32_t kOffSP = kOffWX + 2 * kTileBytes;   // 2 heads, rows = state index n
 constexpr uint32_t kOffCS = kOffSP + 2 * kTileBytes;   // float cs2[2][128], dt[2][128]
-constexpr uint32_t kOffRed = kOffCS + 4 * kBlk * 4;    // per-WG cross-warp scan scratch
-constexpr uint32_t kOffBar = kOffRed + 2 * 8 * 4;
+constexpr uint32_t kOffW = kOffCS + 4 * kBlk * 4;      // float W[2][4][128]: off-diagonal column factors
+constexpr uint32_t kOffRed = kOffW + 2 * 4 * kBlk * 4; // per-WG cross-warp scan scratch + epilogue word
+constexpr uint32_t kOffBar = kOffRed + 2 * 16 * 4;
 constexpr uint32_t kNumBars = 20;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+static_assert(kStageBytes % 1024 == 0, "x tiles must stay 1024-byte aligned");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 enum Bar {
     B_XFULL0 = 0, B_XFULL1, B_XEMPTY0, B_XEMPTY1, B_BCFULL, B_BCEMPTY, B_GFULL, B_GEMPTY,
     B_WXREADY, B_SFULL, B_SEMPTY, B_SPREADY, B_YOFFFULL, B_MREADY, B_RSREADY, B_YFULL, B_YEMPTY, B_DONE, B_WG0, B_WG1
 };
 
-constexpr long long kWaitCycles = 4000000000LL;        // ~2 s at B200 clocks
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Optional phase timeline for profiling builds (-DSSD_TRACE): %globaltimer
-// stamps of CTA 0, first kTraceBlocks blocks, per role and phase.
+// stamps of CTA 0, first kTraceBlocks blocks, per warp and phase.
 #ifdef SSD_TRACE
-constexpr int kTraceBlocks = 8, kTracePts = 16;
-__device__ unsigned long long g_trace[3][kTraceBlocks][kTracePts];
-__device__ __forceinline__ void trace_pt(int role, int j, int k) {
-    if (blockIdx.x == 0 && j < kTraceBlocks) {
+constexpr int kTraceWarps = 10, kTraceBlocks = 8, kTracePts = 24;
+__device__ unsigned long long g_trace[kTraceWarps][kTraceBlocks][kTracePts];
+__device__ __forceinline__ void trace_pt(int w, int j, int k) {
+    if (blockIdx.x == 0 && j < kTraceBlocks && (threadIdx.x & 31) == 0) {
         unsigned long long t;
         asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-        g_trace[role][j][k] = t;
+        g_trace[w][j][k] = t;
     }
 }
-#define SSD_TRACE_PT(role, j, k) trace_pt(role, j, k)
+#define SSD_TRACE_PT(w, j, k) trace_pt(w, j, k)
 #else
-#define SSD_TRACE_PT(role, j, k) ((void)0)
+#define SSD_TRACE_PT(w, j, k) ((void)0)
 #endif
 
-struct TcParams {
-    int batch, L, H, nblk, dir, accumulate;
-    const __nv_bfloat16 *dt;
+struct TcDirParams {
     const float *A, *D;
+};
+
+struct TcParams {
+    int batch, L, H, nblk;
+    int bidir;                          // 1: slot = blockIdx & 1, forward/reverse hand-off through flags
+    int dir_single;                     // direction of slot 0 when bidir == 0
+    TcDirParams d[2];
     __nv_bfloat16 *y;
     int *status;
+    unsigned long long *ticket;         // [batch][H][nblk], epoch-tagged
+    unsigned long long *ready;          // [batch][H][nblk], epoch-tagged
+    unsigned long long epoch;
+    long long wait_cycles;              // bound of every device-side wait
+    int fault;                          // test hook: 1 = the first direction never publishes its part
+};
+
+struct TcMaps {
+    CUtensorMap x[2], dt[2], b[2], c[2];
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -110,43 +148,50 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 }
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     uint32_t ok;
+    // the suspend-time hint lets a waiting warp sleep until the phase completes (or 1 us passes)
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(1000u)
         : "memory");
     return ok != 0;
 }
 
-// Bounded wait on phase `parity` by the lanes in `mask` (all of them call it).
-// Returns false (after raising the CTA abort flag and the global status word)
-// if the phase does not complete in time, or if another thread of the CTA has
-// already aborted; the result is the same for every lane in `mask`.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t mask, volatile int *abort_flag,
-                                       int *status, int code) {
-    bool ok = mbar_try(bar, parity);
-    if (!ok) {
-        const long long t0 = clock64();
-        while (true) {
-            if (mbar_try(bar, parity)) { ok = true; break; }
-            if (*abort_flag) break;
-            if (clock64() - t0 > kWaitCycles) {
-                *abort_flag = 1;
-                atomicExch(status, code);
-                break;
-            }
+// Slow path of mbar_wait: polls until the phase completes, the CTA aborts or
+// the time limit passes (then raises the abort flag and the status word).
+__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *status,
+                                            int code) {
+    const long long t0 = clock64();
+    const long long limit = *reinterpret_cast<volatile long long *>(abort_flag + 1);
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > limit) {
+            *abort_flag = 1;
+            atomicExch(status, code);
+            return false;
         }
     }
+}
+
+// Bounded wait on phase `parity` by the lanes in `mask` (all of them call it).
+// Returns false if the phase did not complete in time or the CTA aborted; the
+// result is the same for every lane in `mask`.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t mask, volatile int *abort_flag,
+                                          int *status, int code) {
+    bool ok = mbar_try(bar, parity);
+    if (__all_sync(mask, ok)) return true;
+    if (!ok) ok = mbar_wait_slow(bar, parity, abort_flag, status, code);
     return __all_sync(mask, ok);
 }
 
 // Bounded wait that ignores the abort flag: used on the way out to let
 // copies already in flight land before the CTA releases its shared memory.
-__device__ __noinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, long long limit) {
     const long long t0 = clock64();
-    while (!mbar_try(bar, parity) && clock64() - t0 < kWaitCycles) {
+    while (!mbar_try(bar, parity) && clock64() - t0 < limit) {
     }
 }
 
@@ -230,11 +275,20 @@ __device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u &
 __device__ __forceinline__ uint32_t swz(int r, int q) { return (uint32_t)(r * 128 + ((q ^ (r & 7)) << 4)); }
 
 
+// ------------------------------------------------------------------ global-memory hand-off helpers
+
+__device__ __forceinline__ void st_release(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
 // ------------------------------------------------------------------ the kernel
 
-__global__ void __launch_bounds__(kThreads, 1)
-k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
-         const __grid_constant__ CUtensorMap map_c, TcParams prm) {
+__global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ TcMaps maps, TcParams prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -243,21 +297,32 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);
     float *cs2_s = reinterpret_cast<float *>(sm + kOffCS);          // [2][128] cs * log2(e)
     float *dt_s = cs2_s + 2 * kBlk;                                  // [2][128] dt
-    float *red = reinterpret_cast<float *>(sm + kOffRed);            // [2 WG][8]
+    float *wtab_s = reinterpret_cast<float *>(sm + kOffW);           // [2][4][128]
+    float *red = reinterpret_cast<float *>(sm + kOffRed);            // [2 WG][16]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int npairs = prm.H / 2;
-    const int b = blockIdx.x / npairs, hp = blockIdx.x % npairs;
+    const int unit = prm.bidir ? (blockIdx.x >> 1) : blockIdx.x;
+    const int slot = prm.bidir ? (blockIdx.x & 1) : 0;
+    const int dir = prm.bidir ? (slot == 0 ? 1 : -1) : prm.dir_single;
+    const int b = unit / npairs, hp = unit % npairs;
     const int h0 = 2 * hp;
-    const int nblk = prm.nblk, dir = prm.dir, L = prm.L;
+    const int nblk = prm.nblk, L = prm.L;
+    const CUtensorMap *map_x = &maps.x[slot], *map_dt = &maps.dt[slot], *map_b = &maps.b[slot],
+                      *map_c = &maps.c[slot];
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
-        const uint32_t counts[kNumBars] = {1, 1, 8, 8, 1, 1, 1, 8, 8, 1, 8, 8, 1, 8, 8, 1, 8, 1, 4, 4};
-        for (int i = 0; i < (int)kNumBars; ++i) mbar_init(bar(i), counts[i]);
+        *reinterpret_cast<volatile long long *>(abort_flag + 1) = prm.wait_cycles;
+        // arrival counts: 8 = one per CUDA-core warp, 4 = one per warp of a warpgroup, 1 = one thread / commit
+        constexpr uint32_t k8 = (1u << B_XEMPTY0) | (1u << B_XEMPTY1) | (1u << B_GEMPTY) | (1u << B_WXREADY) |
+                                (1u << B_SEMPTY) | (1u << B_SPREADY) | (1u << B_MREADY) | (1u << B_RSREADY) |
+                                (1u << B_YEMPTY);
+        constexpr uint32_t k4 = (1u << B_WG0) | (1u << B_WG1);
+        for (int i = 0; i < (int)kNumBars; ++i) mbar_init(bar(i), (k8 >> i) & 1 ? 8 : (k4 >> i) & 1 ? 4 : 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(tmem_slot)));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
@@ -266,42 +331,44 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp == kWarpTma) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
             const uint32_t MASK = 1u;
             int issued = 0;   // blocks whose loads were issued
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_x)) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_b)) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_c)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map_x)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map_dt)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map_b)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map_c)) : "memory");
             for (int j = 0; j < nblk; ++j) {
                 const int cm = dir > 0 ? j : nblk - 1 - j;
                 const int row = b * L + cm * kBlk;
                 const int st = j & 1;
                 if (j >= 2 && !mbar_wait(bar(B_XEMPTY0 + st), ((j >> 1) - 1) & 1, MASK, abort_flag, prm.status, 11)) break;
-                SSD_TRACE_PT(0, j, 0);
-                mbar_expect_tx(bar(B_XFULL0 + st), 2 * kTileBytes);
+                SSD_TRACE_PT(8, j, 0);
+                const uint32_t stage = sbase + kOffX + st * kStageBytes;
+                mbar_expect_tx(bar(B_XFULL0 + st), kStageBytes);
                 for (int h = 0; h < 2; ++h)
-                    tma_load_2d(sbase + kOffX + (st * 2 + h) * kTileBytes, &map_x, (h0 + h) * kP, row,
-                                bar(B_XFULL0 + st));
+                    tma_load_2d(stage + h * kTileBytes, map_x, (h0 + h) * kP, row, bar(B_XFULL0 + st));
+                tma_load_2d(stage + 2 * kTileBytes, map_dt, h0 & ~7, row, bar(B_XFULL0 + st));
                 if (j >= 1 && !mbar_wait(bar(B_BCEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 12)) break;
-                SSD_TRACE_PT(0, j, 1);
+                SSD_TRACE_PT(8, j, 1);
                 mbar_expect_tx(bar(B_BCFULL), 4 * kTileBytes);
                 for (int q = 0; q < 2; ++q) {
-                    tma_load_2d(sbase + kOffB + q * kTileBytes, &map_b, q * 64, row, bar(B_BCFULL));
-                    tma_load_2d(sbase + kOffC + q * kTileBytes, &map_c, q * 64, row, bar(B_BCFULL));
+                    tma_load_2d(sbase + kOffB + q * kTileBytes, map_b, q * 64, row, bar(B_BCFULL));
+                    tma_load_2d(sbase + kOffC + q * kTileBytes, map_c, q * 64, row, bar(B_BCFULL));
                 }
                 issued = j + 1;
             }
             if (*abort_flag && issued > 0) {
                 // let copies still in flight land before the CTA exits
                 const int j = issued - 1;
-                mbar_drain(bar(B_XFULL0 + (j & 1)), (j >> 1) & 1);
-                if (j >= 1) mbar_drain(bar(B_XFULL0 + ((j - 1) & 1)), ((j - 1) >> 1) & 1);
-                mbar_drain(bar(B_BCFULL), j & 1);
+                mbar_drain(bar(B_XFULL0 + (j & 1)), (j >> 1) & 1, prm.wait_cycles);
+                if (j >= 1) mbar_drain(bar(B_XFULL0 + ((j - 1) & 1)), ((j - 1) >> 1) & 1, prm.wait_cycles);
+                mbar_drain(bar(B_BCFULL), j & 1, prm.wait_cycles);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == kWarpMma) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t MASK = 1u;
@@ -310,11 +377,11 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
             const uint32_t aB = sbase + kOffB, aC = sbase + kOffC, aWX = sbase + kOffWX, aSP = sbase + kOffSP;
             for (int j = 0; j < nblk; ++j) {
                 const int st = j & 1;
-                const uint32_t aX = sbase + kOffX + st * 2 * kTileBytes;
+                const uint32_t aX = sbase + kOffX + st * kStageBytes;
                 // G = C B^T  (M = rows, N = source rows, K = n)
                 if (!mbar_wait(bar(B_BCFULL), j & 1, MASK, abort_flag, prm.status, 21)) break;
                 if (j >= 1 && !mbar_wait(bar(B_GEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 22)) break;
-                SSD_TRACE_PT(1, j, 0);
+                SSD_TRACE_PT(9, j, 0);
                 tc_fence_after();
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = (ks >> 2) * kTileBytes + (ks & 3) * 32;
@@ -324,7 +391,7 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
                 // S^T = B^T (w x)  (M = n, N = (head, p), K = rows); both operands MN-major
                 if (!mbar_wait(bar(B_WXREADY), j & 1, MASK, abort_flag, prm.status, 23)) break;
                 if (j >= 1 && !mbar_wait(bar(B_SEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 24)) break;
-                SSD_TRACE_PT(1, j, 1);
+                SSD_TRACE_PT(9, j, 1);
                 tc_fence_after();
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = ks * 2048;
@@ -336,7 +403,7 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
                 if (j >= 1) {
                     if (!mbar_wait(bar(B_SPREADY), (j - 1) & 1, MASK, abort_flag, prm.status, 25)) break;
                     if (!mbar_wait(bar(B_YEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 26)) break;
-                    SSD_TRACE_PT(1, j, 2);
+                    SSD_TRACE_PT(9, j, 2);
                     tc_fence_after();
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t offc = (ks >> 2) * kTileBytes + (ks & 3) * 32;
@@ -350,7 +417,7 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
                 if (!mbar_wait(bar(B_MREADY), j & 1, MASK, abort_flag, prm.status, 27)) break;
                 if (j >= 1 && !mbar_wait(bar(B_RSREADY), (j - 1) & 1, MASK, abort_flag, prm.status, 28)) break;
                 if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 29)) break;
-                SSD_TRACE_PT(1, j, 3);
+                SSD_TRACE_PT(9, j, 3);
                 tc_fence_after();
                 for (int h = 0; h < 2; ++h)
                     for (int ks = 0; ks < 8; ++ks)
@@ -360,18 +427,24 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
             }
             // drain: every MMA issued above has completed before TMEM is released
             mma_commit(bar(B_DONE));
-            mbar_drain(bar(B_DONE), 0);
+            mbar_drain(bar(B_DONE), 0, prm.wait_cycles);
         }
-    } else if (warp >= 4) {
+    } else {
         // ---------------------------------------------------------- per-head CUDA-core work
-        const int wg = (warp - 4) >> 2;            // 0: head h0, 1: head h0+1
-        const int wq = warp & 3;                   // TMEM lane quarter
+        const uint32_t MASK = 0xffffffffu;
+        const int wg = warp >> 2;                  // 0: head h0, 1: head h0+1
+        const int wq = warp & 3;                   // TMEM lane quarter = 32-row quarter of the block
         const int r = wq * 32 + lane;              // row in block == TMEM lane
         const int h = h0 + wg;
+        const int tid_wg = threadIdx.x - 128 * wg;
+        const bool leader = (wq == 0 && lane == 0);
         const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
-        const float A2 = prm.A[h] * kLog2e;        // log2 units: exp(a) = exp2(a * log2 e)
-        const float Dh = prm.D ? prm.D[h] : 0.f;
-        const uint32_t MASK = 0xffffffffu;
+        const float A2 = prm.d[slot].A[h] * kLog2e;   // log2 units: exp(a) = exp2(a * log2 e)
+        const float Dh = prm.d[slot].D ? prm.d[slot].D[h] : 0.f;
+        float *cs2 = cs2_s + wg * kBlk, *dts = dt_s + wg * kBlk, *wtab = wtab_s + wg * 4 * kBlk;
+        float *redw = red + wg * 16;
+        uint8_t *wx_tile = sm + kOffWX + wg * kTileBytes;
+        uint8_t *sp_tile = sm + kOffSP + wg * kTileBytes;
         uint32_t wg_phase = 0;   // completions of this WG's sync barrier so far
         // bounded replacement for a named barrier over the 4 warps of this WG
         auto wg_sync = [&](int code) -> bool {
@@ -391,19 +464,23 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
         float state[kP];
 #pragma unroll
         for (int i = 0; i < kP; ++i) state[i] = 0.f;
-        float *cs2 = cs2_s + wg * kBlk, *dts = dt_s + wg * kBlk;
-        uint8_t *wx_tile = sm + kOffWX + wg * kTileBytes;
-        uint8_t *sp_tile = sm + kOffSP + wg * kTileBytes;
-        auto tok_of = [&](int j) { return (dir > 0 ? j : nblk - 1 - j) * kBlk + r; };
-        float dt_next = __bfloat162float(prm.dt[((size_t)b * L + tok_of(0)) * prm.H + h]);
+        const size_t flag_base = ((size_t)b * prm.H + h) * nblk;
+        unsigned long long ticket = 0;
 
         for (int j = 0; j < nblk; ++j) {
             if (__any_sync(0xffffffffu, *abort_flag)) break;
+            SSD_TRACE_PT(warp, j, 0);
             const int st = j & 1;
-            const int t = tok_of(j);
-            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 0);
-            const float dtr = dt_next;
-            if (j + 1 < nblk) dt_next = __bfloat162float(prm.dt[((size_t)b * L + tok_of(j + 1)) * prm.H + h]);
+            const int cm = dir > 0 ? j : nblk - 1 - j;
+            if (prm.bidir && leader) ticket = atomicExch(prm.ticket + flag_base + cm, prm.epoch);
+
+            // x, dt of this block
+            if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 41)) break;
+            SSD_TRACE_PT(warp, j, 1);
+            uint8_t *xt = sm + kOffX + st * kStageBytes + wg * kTileBytes;
+            const __nv_bfloat16 *dtt =
+                reinterpret_cast<const __nv_bfloat16 *>(sm + kOffX + st * kStageBytes + 2 * kTileBytes);
+            const float dtr = __bfloat162float(dtt[r * 8 + (h & 7)]);
 
             // cumulative A*dt in scan order (prefix over rows forward, suffix over rows reverse)
             float s = dtr;
@@ -412,27 +489,48 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
                 const float u = dir > 0 ? __shfl_up_sync(0xffffffffu, s, o) : __shfl_down_sync(0xffffffffu, s, o);
                 if (dir > 0 ? lane >= o : lane + o < 32) s += u;
             }
-            if (!wg_sync(51)) break;           // previous block's readers of red/cs are done
-            if (lane == (dir > 0 ? 31 : 0)) red[wg * 8 + wq] = s;
+            if (!wg_sync(51)) break;           // previous block's readers of red/cs/W are done
+            SSD_TRACE_PT(warp, j, 3);
+            if (lane == (dir > 0 ? 31 : 0)) redw[wq] = s;
             if (!wg_sync(52)) break;
-            float base = 0.f, total = 0.f;
+            SSD_TRACE_PT(warp, j, 4);
+            float tot[4], base = 0.f, total = 0.f;
+#pragma unroll
             for (int w = 0; w < 4; ++w) {
-                const float v = red[wg * 8 + w];
-                total += v;
-                if (dir > 0 ? w < wq : w > wq) base += v;
+                tot[w] = redw[w];
+                total += tot[w];
+                if (dir > 0 ? w < wq : w > wq) base += tot[w];
+            }
+            // cs (log2 units) at the quarter boundaries: the reference rows of the factorised mask
+            float ref2[4];
+            {
+                float acc = 0.f;
+                if (dir > 0) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) { ref2[q] = A2 * acc; acc += tot[q]; }   // row 32q-1
+                } else {
+#pragma unroll
+                    for (int q = 3; q >= 0; --q) { ref2[q] = A2 * acc; acc += tot[q]; }  // row 32(q+1)
+                }
             }
             const float c2 = A2 * (base + s);                 // cs_r * log2 e
             const float cl2 = A2 * total;                     // cs at the block's last scan position
             cs2[r] = c2;
             dts[r] = dtr;
+            // column factors of the off-diagonal quarters: W[q][s] = exp(cs_ref(q) - cs_s) dt_s
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const bool off = dir > 0 ? wq < q : wq > q;    // this row is a source for quarter q
+                if (off) wtab[q * kBlk + r] = exp2f(ref2[q] - c2) * dtr;
+            }
+            const float ref_own = wq == 0 ? ref2[0] : wq == 1 ? ref2[1] : wq == 2 ? ref2[2] : ref2[3];
+            const float e1 = exp2f(c2 - ref_own);            // row factor towards the quarter boundary
             const float wr = exp2f(cl2 - c2) * dtr;           // weight of row r in the block's state
             const float er = exp2f(c2);                       // decay from the block start to row r
             const float ablk = exp2f(cl2);                    // decay across the whole block
+            SSD_TRACE_PT(warp, j, 5);
 
             // w (.) x -> wX tile (same swizzled layout as the X tile)
-            if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 41)) break;
-            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 1);
-            const uint8_t *xt = sm + kOffX + (st * 2 + wg) * kTileBytes;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const uint4 v = *reinterpret_cast<const uint4 *>(xt + swz(r, q));
@@ -443,44 +541,63 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
                 o.w = pack_bf16(bf16lo(v.w) * wr, bf16hi(v.w) * wr);
                 *reinterpret_cast<uint4 *>(wx_tile + swz(r, q)) = o;
             }
+            SSD_TRACE_PT(warp, j, 6);
             fence_async_smem();
-            if (!wg_sync(53)) break;           // cs2/dts of all rows visible to this WG
-            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 2);
+            SSD_TRACE_PT(warp, j, 7);
+            if (!wg_sync(53)) break;           // cs2/dts/W of all rows visible to this WG
+            SSD_TRACE_PT(warp, j, 8);
             if (lane == 0) mbar_arrive(bar(B_WXREADY));
 
             // M_h = G (.) decay (.) dt over the causal triangle, bf16 into TMEM
             if (!mbar_wait(bar(B_GFULL), j & 1, MASK, abort_flag, prm.status, 42)) break;
-            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 3);
+            SSD_TRACE_PT(warp, j, 9);
             tc_fence_after();
-            for (int kb = 0; kb < 4; ++kb) {
-                const bool need = dir > 0 ? kb <= wq : kb >= wq;
-                if (!need) continue;           // entirely outside the triangle: stays zero from set-up
-                float g[32];
-                tmem_ld32(tl + kColG + kb * 32, g);
-                tmem_wait_ld();
-                uint32_t m[16];
+            {
+                const float *wrow = wtab + wq * kBlk;
+#pragma unroll 1
+                for (int kb = 0; kb < 4; ++kb) {
+                    const bool offd = dir > 0 ? kb < wq : kb > wq;
+                    if (!offd && kb != wq) continue;   // outside the triangle: stays zero from set-up
+                    float g[32];
+                    tmem_ld32(tl + kColG + kb * 32, g);
+                    tmem_wait_ld();
+                    uint32_t m[16];
+                    if (offd) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float mv[2];
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 wv = *reinterpret_cast<const float4 *>(wrow + kb * 32 + 4 * i);
+                            m[2 * i] = pack_bf16(g[4 * i] * wv.x * e1, g[4 * i + 1] * wv.y * e1);
+                            m[2 * i + 1] = pack_bf16(g[4 * i + 2] * wv.z * e1, g[4 * i + 3] * wv.w * e1);
+                        }
+                    } else {
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int sidx = kb * 32 + 2 * i + e;
-                        const bool in = dir > 0 ? sidx <= r : sidx >= r;
-                        mv[e] = in ? g[2 * i + e] * exp2f(c2 - cs2[sidx]) * dts[sidx] : 0.f;
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 cv = *reinterpret_cast<const float4 *>(cs2 + kb * 32 + 4 * i);
+                            const float4 dv = *reinterpret_cast<const float4 *>(dts + kb * 32 + 4 * i);
+                            const float cc[4] = {cv.x, cv.y, cv.z, cv.w}, dd[4] = {dv.x, dv.y, dv.z, dv.w};
+                            float mv[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int sl = 4 * i + e;   // source lane within the quarter
+                                const bool in = dir > 0 ? sl <= lane : sl >= lane;
+                                mv[e] = in ? g[sl] * exp2f(c2 - cc[e]) * dd[e] : 0.f;
+                            }
+                            m[2 * i] = pack_bf16(mv[0], mv[1]);
+                            m[2 * i + 1] = pack_bf16(mv[2], mv[3]);
+                        }
                     }
-                    m[i] = pack_bf16(mv[0], mv[1]);
+                    tmem_st16(tl + kColM + 64 * wg + kb * 16, m);
                 }
-                tmem_st16(tl + kColM + 64 * wg + kb * 16, m);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_GEMPTY));
-            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 10);
+            SSD_TRACE_PT(warp, j, 10);
 
             // state: S' <- exp(cs_last) S' + S, thread r holds state row n = r
             if (!mbar_wait(bar(B_SFULL), j & 1, MASK, abort_flag, prm.status, 43)) break;
-            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 4);
+            SSD_TRACE_PT(warp, j, 11);
             tc_fence_after();
             {
                 float sv[32];
@@ -495,10 +612,11 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_SEMPTY));
+            SSD_TRACE_PT(warp, j, 12);
             if (j + 1 < nblk) {
                 // the previous state tile must have been consumed by this block's Y = C S'^T
                 if (j >= 1 && !mbar_wait(bar(B_YOFFFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 44)) break;
-                if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 5);
+                SSD_TRACE_PT(warp, j, 13);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     uint4 o;
@@ -511,12 +629,12 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_SPREADY));
+                SSD_TRACE_PT(warp, j, 14);
             }
 
             // Y (from the incoming state) scaled by exp(cs_r), before the intra-block term is added
             if (j >= 1) {
                 if (!mbar_wait(bar(B_YOFFFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 45)) break;
-                if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 6);
                 tc_fence_after();
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -531,58 +649,118 @@ k_ssd_tc(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUte
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_RSREADY));
+                SSD_TRACE_PT(warp, j, 15);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_MREADY));
 
-            // epilogue: y = Y + D x, bf16, 128 contiguous bytes per thread
-            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 7);
+            // epilogue: y = Y + D x (+ the other direction's part), staged through the x tile
+            // (free once the intra-block MMA is done) so that y is written in whole 128-byte rows
             if (!mbar_wait(bar(B_YFULL), j & 1, MASK, abort_flag, prm.status, 46)) break;
-            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 8);
+            SSD_TRACE_PT(warp, j, 16);
+            __nv_bfloat16 *ytile = prm.y + (((size_t)b * L + (size_t)cm * kBlk) * prm.H + h) * kP;
+            const size_t ystride = (size_t)prm.H * kP;      // elements between consecutive tokens
+            // who writes first: the ticket taken at the block start (bidirectional mixer only)
+            bool second = false;
+            if (prm.bidir) {
+                if (leader) {
+                    int sec = ticket == prm.epoch;
+                    if (sec) {
+                        // the other direction's part of this block: wait until it is published
+                        const unsigned long long *rp = prm.ready + flag_base + cm;
+                        const long long t0 = clock64();
+                        while (ld_acquire(rp) != prm.epoch) {
+                            if (*abort_flag) { sec = 2; break; }
+                            if (clock64() - t0 > prm.wait_cycles) {
+                                *abort_flag = 1;
+                                atomicExch(prm.status, 47);
+                                sec = 2;
+                                break;
+                            }
+                            __nanosleep(256);
+                        }
+                    }
+                    redw[8] = __int_as_float(sec);
+                }
+                if (!wg_sync(54)) break;
+                SSD_TRACE_PT(warp, j, 17);
+                const int sec = __float_as_int(redw[8]);
+                if (sec == 2) break;
+                second = sec == 1;
+            }
+            if (second) {
+                // the published part, as whole rows, into the w(.)x tile (read by this block's S MMA, done)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int c = tid_wg + 128 * i, rr = c >> 3, q = c & 7;
+                    const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(ytile + rr * ystride + 8 * q));
+                    *reinterpret_cast<uint4 *>(wx_tile + swz(rr, q)) = v;
+                }
+                if (!wg_sync(55)) break;
+            }
             tc_fence_after();
-            float yv[64];
-            tmem_ld32(tl + kColY + 64 * wg, yv);
-            tmem_ld32(tl + kColY + 64 * wg + 32, yv + 32);
-            tmem_wait_ld();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float yv[32];
+                tmem_ld32(tl + kColY + 64 * wg + 32 * half, yv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const int q = 4 * half + qq;
+                    const uint4 xv = *reinterpret_cast<const uint4 *>(xt + swz(r, q));
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                    float o[8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        o[2 * i] = fmaf(Dh, bf16lo(xw[i]), yv[8 * qq + 2 * i]);
+                        o[2 * i + 1] = fmaf(Dh, bf16hi(xw[i]), yv[8 * qq + 2 * i + 1]);
+                    }
+                    if (second) {
+                        const uint4 pv = *reinterpret_cast<const uint4 *>(wx_tile + swz(r, q));
+                        const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            o[2 * i] += bf16lo(pw[i]);
+                            o[2 * i + 1] += bf16hi(pw[i]);
+                        }
+                    }
+                    uint4 ov;
+                    ov.x = pack_bf16(o[0], o[1]);
+                    ov.y = pack_bf16(o[2], o[3]);
+                    ov.z = pack_bf16(o[4], o[5]);
+                    ov.w = pack_bf16(o[6], o[7]);
+                    *reinterpret_cast<uint4 *>(xt + swz(r, q)) = ov;
+                }
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_YEMPTY));
-            __nv_bfloat16 *yrow = prm.y + (((size_t)b * L + t) * prm.H + h) * kP;
+            SSD_TRACE_PT(warp, j, 18);
+            if (!wg_sync(56)) break;
+            SSD_TRACE_PT(warp, j, 19);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const uint4 xv = *reinterpret_cast<const uint4 *>(xt + swz(r, q));
-                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                float o[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    o[2 * i] = fmaf(Dh, bf16lo(xw[i]), yv[8 * q + 2 * i]);
-                    o[2 * i + 1] = fmaf(Dh, bf16hi(xw[i]), yv[8 * q + 2 * i + 1]);
-                }
-                if (prm.accumulate) {
-                    const uint4 pv = *reinterpret_cast<const uint4 *>(yrow + 8 * q);
-                    const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        o[2 * i] += bf16lo(pw[i]);
-                        o[2 * i + 1] += bf16hi(pw[i]);
-                    }
-                }
-                uint4 ov;
-                ov.x = pack_bf16(o[0], o[1]);
-                ov.y = pack_bf16(o[2], o[3]);
-                ov.z = pack_bf16(o[4], o[5]);
-                ov.w = pack_bf16(o[6], o[7]);
-                *reinterpret_cast<uint4 *>(yrow + 8 * q) = ov;
+            for (int i = 0; i < 8; ++i) {
+                const int c = tid_wg + 128 * i, rr = c >> 3, q = c & 7;
+                const uint4 v = *reinterpret_cast<const uint4 *>(xt + swz(rr, q));
+                *reinterpret_cast<uint4 *>(ytile + rr * ystride + 8 * q) = v;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_XEMPTY0 + st));
-            if (warp == 4 && lane == 0) SSD_TRACE_PT(2, j, 9);
+            SSD_TRACE_PT(warp, j, 20);
+            if (prm.bidir && !second) {
+                // publish this direction's part of the block
+                __threadfence();
+                SSD_TRACE_PT(warp, j, 21);
+                if (!wg_sync(57)) break;
+                if (leader && prm.fault != 1) st_release(prm.ready + flag_base + cm, prm.epoch);
+                SSD_TRACE_PT(warp, j, 22);
+            }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
     }
@@ -607,28 +785,39 @@ EncodeTiled get_encode() {
     return fn;
 }
 
-// [rows][cols] bf16 matrix, row-major; box [128 rows][64 cols], 128-byte swizzle
-bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols) {
+// [rows][cols] bf16 matrix, row-major; box [128 rows][box_cols columns]
+bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols, bool swizzle) {
     EncodeTiled enc = get_encode();
     if (!enc) return false;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)kBlk};
+    const cuuint32_t box[2] = {box_cols, (cuuint32_t)kBlk};
     const cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+unsigned long long next_epoch() {
+    // distinct per call in this process; the random start keeps a fresh workspace's
+    // leftover contents from matching (flags are compared for equality)
+    static std::atomic<unsigned long long> counter{
+        0x9E3779B97F4A7C15ull ^ (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() ^
+        ((unsigned long long)(uintptr_t)&counter << 17)};
+    return counter.fetch_add(0x100000001ull) | 1ull;
 }
 
 }  // namespace
 
 bool tc_supported(bool bf16, int batch, int L, int H, int P, int N, int G, int chunk) {
-    (void)batch;
-    return bf16 && P == kP && N == kN && G == 1 && H % 2 == 0 && chunk % kBlk == 0 && L % kBlk == 0 &&
-           (long long)batch * L <= (1ll << 31) - 1 && get_encode() != nullptr;
+    return bf16 && P == kP && N == kN && G == 1 && H % 2 == 0 && H % 8 == 0 && chunk % kBlk == 0 &&
+           L % kBlk == 0 && (long long)batch * L <= (1ll << 31) - 1 && get_encode() != nullptr;
 }
 
-size_t tc_workspace_bytes(int, int, int, int) { return 0; }
+size_t tc_workspace_bytes(int batch, int L, int H, int) {
+    // epoch-tagged ticket and ready words per (batch, head, block)
+    return 2 * sizeof(unsigned long long) * (size_t)batch * H * (L / kBlk);
+}
 
 TcArgs make_tc_args(int batch, int L, int H, int chunk, void *ws, int *status) {
     TcArgs t{};
@@ -641,11 +830,11 @@ void tc_set_direction(TcArgs &t, int slot, int dir, const void *x, const void *d
     t.d[slot] = TcDir{x, dt, B, C, A, D, dir};
 }
 
-int tc_launches(bool bidir) { return bidir ? 2 : 1; }
+int tc_launches(bool) { return 1; }
 
 #ifdef SSD_TRACE
 extern "C" int ssd_debug_trace(unsigned long long *out, int n) {
-    const int total = 3 * kTraceBlocks * kTracePts;
+    const int total = kTraceWarps * kTraceBlocks * kTracePts;
     if (n < total) return -1;
     return cudaMemcpyFromSymbol(out, g_trace, sizeof(unsigned long long) * total) == cudaSuccess ? total : -2;
 }
@@ -659,24 +848,33 @@ cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
     });
     if (attr_err != cudaSuccess) return attr_err;
     const int ndir = bidir ? 2 : 1;
+    const uint64_t rows = (uint64_t)t.batch * t.L;
+    TcMaps maps;
+    memset(&maps, 0, sizeof maps);
+    TcParams p{};
     for (int s = 0; s < ndir; ++s) {
         const TcDir &d = t.d[s];
-        CUtensorMap mx, mb, mc;
-        const uint64_t rows = (uint64_t)t.batch * t.L;
-        if (!make_map(&mx, d.x, rows, (uint64_t)t.H * kP) || !make_map(&mb, d.B, rows, kN) ||
-            !make_map(&mc, d.C, rows, kN))
+        if (!make_map(&maps.x[s], d.x, rows, (uint64_t)t.H * kP, 64, true) ||
+            !make_map(&maps.dt[s], d.dt, rows, (uint64_t)t.H, 8, false) ||
+            !make_map(&maps.b[s], d.B, rows, kN, 64, true) || !make_map(&maps.c[s], d.C, rows, kN, 64, true))
             return cudaErrorInvalidValue;
-        TcParams p{};
-        p.batch = t.batch; p.L = t.L; p.H = t.H; p.nblk = t.L / kBlk; p.dir = d.dir; p.accumulate = s;
-        p.dt = static_cast<const __nv_bfloat16 *>(d.dt);
-        p.A = d.A; p.D = d.D;
-        p.y = static_cast<__nv_bfloat16 *>(y);
-        p.status = t.status;
-        k_ssd_tc<<<t.batch * (t.H / 2), kThreads, kSmemBytes, st>>>(mx, mb, mc, p);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
+        p.d[s].A = d.A;
+        p.d[s].D = d.D;
     }
-    return cudaSuccess;
+    p.batch = t.batch; p.L = t.L; p.H = t.H; p.nblk = t.L / kBlk;
+    p.bidir = bidir ? 1 : 0;
+    p.dir_single = t.d[0].dir;
+    p.y = static_cast<__nv_bfloat16 *>(y);
+    p.status = t.status;
+    const size_t nflags = (size_t)t.batch * t.H * p.nblk;
+    p.ticket = static_cast<unsigned long long *>(t.ws);
+    p.ready = p.ticket + nflags;
+    p.epoch = next_epoch();
+    p.wait_cycles = t.wait_cycles;
+    p.fault = t.fault;
+    const int grid = t.batch * (t.H / 2) * ndir;
+    k_ssd_tc<<<grid, kThreads, kSmemBytes, st>>>(maps, p);
+    return cudaGetLastError();
 }
 
 }  // namespace ssd

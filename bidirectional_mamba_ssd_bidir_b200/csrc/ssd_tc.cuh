@@ -17,6 +17,8 @@ struct TcArgs {
     TcDir d[2];
     void *ws;          // path scratch (after the status word)
     int *status;       // device status word
+    long long wait_cycles;   // bound of every device-side wait, in SM clock cycles
+    int fault;               // test hook (0 = none)
 };
 
 bool tc_supported(bool bf16, int batch, int L, int H, int P, int N, int G, int chunk);

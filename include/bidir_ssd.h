@@ -135,6 +135,17 @@ const char *ssd_last_error(void);
  * ssd_scan, 1 = bidir_ssd, 2 = r2l_block_scan with s != 0.  -1 if refused. */
 int ssd_kernel_launches(const ssd_shape *shape, int chunk, int op);
 
+/* Test hook for failure detection (process-wide; not for production use).
+ * Sets the bound of every device-side wait (default 2 s) and an injected
+ * fault: mode 0 = none; mode 1 = in the tensor-core bidirectional mixer the
+ * direction that finishes a block first never publishes its part, so the
+ * other direction's bounded wait runs out and the call records
+ * SSD_ERR_TIMEOUT in the workspace status word (read it with
+ * ssd_workspace_status).  No GPU fault, trap or hang is involved: the waiting
+ * CTA gives up, drains its copies and exits.  Returns SSD_ERR_INVALID_ARG for
+ * an unknown mode or a limit outside [1e-4, 60] s. */
+ssd_status ssd_debug_fault(int mode, double wait_limit_seconds);
+
 /* Which kernel family a call with this shape and chunk runs:
  * 1 = tensor-core (tcgen05) path, 0 = SIMT path, -1 = refused. */
 int ssd_path_for(const ssd_shape *shape, int chunk);
