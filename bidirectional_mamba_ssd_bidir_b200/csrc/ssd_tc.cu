@@ -7,13 +7,15 @@
 // TMEM lane r = token t0 + r), with cs the cumulative A*dt in scan order:
 //
 //   G    = C B^T                      tcgen05, shared by both heads   TMEM [0,128)
-//   M_h  = G (.) decay_h (.) dt        CUDA cores -> bf16 A operand    TMEM [128,256)
-//   S^T  = B^T (w (.) X)               tcgen05, N = 2 heads x 64       TMEM [256,384)
-//   Y    = C S'^T_prev                 tcgen05, N = 2 heads x 64       TMEM [384,512)
+//   M_h  = G (.) decay_h (.) dt        CUDA cores, bf16, written over the G columns it
+//                                      came from (A operand of the next MMA)
+//   S^T  = B^T (w (.) X)               tcgen05, N = 2 heads x 64       TMEM [128,256)
+//   Y    = C S'^T_prev                 tcgen05, N = 2 heads x 64       TMEM [256,384)
 //   Y   *= exp(cs_r) per row           CUDA cores (TMEM ld/st)
 //   Y   += M_h X_h                     tcgen05, A from TMEM, N = 64
 //   y    = Y + D x                     CUDA cores -> smem -> coalesced rows
-//   S'   = exp(cs_last) S' + S         CUDA cores, float32 registers -> bf16 smem
+//   S'   = exp(cs_last) S' + S         CUDA cores; float32 state in TMEM [384,512),
+//                                      bf16 copy in smem for the next block
 //
 // This is the chunked evaluation of the recurrence S <- exp(dt A) S +
 // dt x (outer) B, y = C.S + D x that the Mamba-2 layers of the DiffuMamba
@@ -67,7 +69,7 @@ constexpr uint32_t kDtBytes = kBlk * 8 * 2;           // dt box: 128 tokens x 8 
 constexpr uint32_t kStageBytes = 2 * kTileBytes + kDtBytes;   // x of 2 heads + dt = 34 KB
 
 // TMEM column map
-constexpr uint32_t kColG = 0, kColM = 128, kColS = 256, kColY = 384;
+constexpr uint32_t kColG = 0, kColS = 128, kColY = 256, kColST = 384;
 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr uint32_t kOffX = 0;                          // 2 stages: [x h0 | x h1 | dt]
@@ -77,7 +79,8 @@ constexpr uint32_t kOffWX = kOffC + 2 * kTileBytes;    // 2 heads
 constexpr uint32_t kOffSP = kOffWX + 2 * kTileBytes;   // 2 heads, rows = state index n
 constexpr uint32_t kOffCS = kOffSP + 2 * kTileBytes;   // float cs2[2][128], dt[2][128]
 constexpr uint32_t kOffW = kOffCS + 4 * kBlk * 4;      // float W[2][4][128]: off-diagonal column factors
-constexpr uint32_t kOffRed = kOffW + 2 * 4 * kBlk * 4; // per-WG cross-warp scan scratch + epilogue word
+constexpr uint32_t kOffE1 = kOffW + 2 * 4 * kBlk * 4;  // float e1[2][128]: off-diagonal row factors
+constexpr uint32_t kOffRed = kOffE1 + 2 * kBlk * 4;    // per-WG cross-warp scan scratch + epilogue word
 constexpr uint32_t kOffBar = kOffRed + 2 * 16 * 4;
 constexpr uint32_t kNumBars = 20;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
@@ -148,6 +151,15 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 }
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     uint32_t ok;
+#ifdef SSD_EXP_TESTWAIT
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+#else
     // the suspend-time hint lets a waiting warp sleep until the phase completes (or 1 us passes)
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -156,6 +168,7 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
         : "=r"(ok)
         : "r"(bar), "r"(parity), "r"(1000u)
         : "memory");
+#endif
     return ok != 0;
 }
 
@@ -234,22 +247,57 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+// TMEM loads complete asynchronously: the wait is part of the same asm statement,
+// so no instruction that uses the loaded registers can be scheduled before it.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
     uint32_t r[32];
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
+        : "r"(taddr)
+        : "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+// two 16-column loads, one wait
+__device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, float *va, float *vb) {
+    uint32_t a[16], b[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
+          "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]),
+          "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]),
+          "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15])
+        : "r"(ta), "r"(tb)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) { va[i] = __uint_as_float(a[i]); vb[i] = __uint_as_float(b[i]); }
+}
+// TMEM stores: the wait is part of the asm, so the source registers are not reused while
+// the store may still read them and later TMEM reads of these columns see the new values.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
         "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
@@ -380,7 +428,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 const uint32_t aX = sbase + kOffX + st * kStageBytes;
                 // G = C B^T  (M = rows, N = source rows, K = n)
                 if (!mbar_wait(bar(B_BCFULL), j & 1, MASK, abort_flag, prm.status, 21)) break;
-                if (j >= 1 && !mbar_wait(bar(B_GEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 22)) break;
+                // the previous block's M (read by its intra-block MMA) occupies the G columns
+                if (j >= 1 && !mbar_wait(bar(B_YFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 22)) break;
                 SSD_TRACE_PT(9, j, 0);
                 tc_fence_after();
                 for (int ks = 0; ks < 8; ++ks) {
@@ -421,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 tc_fence_after();
                 for (int h = 0; h < 2; ++h)
                     for (int ks = 0; ks < 8; ++ks)
-                        mma_ts(tmem + kColY + 64 * h, tmem + kColM + 64 * h + 8 * ks,
+                        mma_ts(tmem + kColY + 64 * h, tmem + kColG + 16 * ks + 8 * h,
                                sdesc(aX + h * kTileBytes + ks * 2048, kTileBytes, 1024), id_yd, (j >= 1) || (ks > 0));
                 mma_commit(bar(B_YFULL));
             }
@@ -446,24 +495,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
         uint8_t *wx_tile = sm + kOffWX + wg * kTileBytes;
         uint8_t *sp_tile = sm + kOffSP + wg * kTileBytes;
         uint32_t wg_phase = 0;   // completions of this WG's sync barrier so far
-        // bounded replacement for a named barrier over the 4 warps of this WG
-        auto wg_sync = [&](int code) -> bool {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_WG0 + wg));
-            const bool ok = mbar_wait(bar(B_WG0 + wg), wg_phase & 1, MASK, abort_flag, prm.status, code);
-            ++wg_phase;
-            return ok;
-        };
-        {
-            // M_h outside the causal triangle is never written: start it at zero
-            const uint32_t z[16] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll
-            for (int c = 0; c < 64; c += 16) tmem_st16(tl + kColM + 64 * wg + c, z);
-            tmem_wait_st();
-        }
-        float state[kP];
-#pragma unroll
-        for (int i = 0; i < kP; ++i) state[i] = 0.f;
+        // bounded replacement for a named barrier over the 4 warps of this warpgroup
+#define WG_SYNC(code)                                                                                     \
+    ([&]() __attribute__((always_inline)) {                                                              \
+        __syncwarp();                                                                                     \
+        if (lane == 0) mbar_arrive(bar(B_WG0 + wg));                                                      \
+        const bool ok_ = mbar_wait(bar(B_WG0 + wg), wg_phase & 1, MASK, abort_flag, prm.status, (code));  \
+        ++wg_phase;                                                                                       \
+        return ok_;                                                                                       \
+    }())
+        float *e1_s = reinterpret_cast<float *>(sm + kOffE1);   // [2][128]
         const size_t flag_base = ((size_t)b * prm.H + h) * nblk;
         unsigned long long ticket = 0;
 
@@ -472,7 +513,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             SSD_TRACE_PT(warp, j, 0);
             const int st = j & 1;
             const int cm = dir > 0 ? j : nblk - 1 - j;
-            if (prm.bidir && leader) ticket = atomicExch(prm.ticket + flag_base + cm, prm.epoch);
 
             // x, dt of this block
             if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 41)) break;
@@ -489,10 +529,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 const float u = dir > 0 ? __shfl_up_sync(0xffffffffu, s, o) : __shfl_down_sync(0xffffffffu, s, o);
                 if (dir > 0 ? lane >= o : lane + o < 32) s += u;
             }
-            if (!wg_sync(51)) break;           // previous block's readers of red/cs/W are done
+            if (!WG_SYNC(51)) break;           // previous block's readers of red/cs/W are done
             SSD_TRACE_PT(warp, j, 3);
             if (lane == (dir > 0 ? 31 : 0)) redw[wq] = s;
-            if (!wg_sync(52)) break;
+            if (!WG_SYNC(52)) break;
             SSD_TRACE_PT(warp, j, 4);
             float tot[4], base = 0.f, total = 0.f;
 #pragma unroll
@@ -524,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 if (off) wtab[q * kBlk + r] = exp2f(ref2[q] - c2) * dtr;
             }
             const float ref_own = wq == 0 ? ref2[0] : wq == 1 ? ref2[1] : wq == 2 ? ref2[2] : ref2[3];
-            const float e1 = exp2f(c2 - ref_own);            // row factor towards the quarter boundary
+            e1_s[wg * kBlk + r] = exp2f(c2 - ref_own);      // row factor towards the quarter boundary
             const float wr = exp2f(cl2 - c2) * dtr;           // weight of row r in the block's state
             const float er = exp2f(c2);                       // decay from the block start to row r
             const float ablk = exp2f(cl2);                    // decay across the whole block
@@ -544,93 +584,121 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             SSD_TRACE_PT(warp, j, 6);
             fence_async_smem();
             SSD_TRACE_PT(warp, j, 7);
-            if (!wg_sync(53)) break;           // cs2/dts/W of all rows visible to this WG
+            if (!WG_SYNC(53)) break;           // cs2/dts/W of all rows visible to this WG
             SSD_TRACE_PT(warp, j, 8);
             if (lane == 0) mbar_arrive(bar(B_WXREADY));
 
-            // M_h = G (.) decay (.) dt over the causal triangle, bf16 into TMEM
+            // M_h = G (.) decay (.) dt over the causal triangle, bf16, for both heads.  This
+            // warpgroup takes every other 16-source K-step; the two heads' bf16 results for a
+            // K-step replace the 16 float32 G columns they were computed from.
             if (!mbar_wait(bar(B_GFULL), j & 1, MASK, abort_flag, prm.status, 42)) break;
+            // both heads' decay tables of this block are read below: the other warpgroup must have
+            // finished writing them (all 8 warps arrive on this barrier after their preparation)
+            if (!mbar_wait(bar(B_WXREADY), j & 1, MASK, abort_flag, prm.status, 48)) break;
             SSD_TRACE_PT(warp, j, 9);
             tc_fence_after();
             {
-                const float *wrow = wtab + wq * kBlk;
+                const float c2h[2] = {cs2_s[r], cs2_s[kBlk + r]};
+                const float e1h[2] = {e1_s[r], e1_s[kBlk + r]};
 #pragma unroll 1
-                for (int kb = 0; kb < 4; ++kb) {
-                    const bool offd = dir > 0 ? kb < wq : kb > wq;
-                    if (!offd && kb != wq) continue;   // outside the triangle: stays zero from set-up
-                    float g[32];
-                    tmem_ld32(tl + kColG + kb * 32, g);
-                    tmem_wait_ld();
+                for (int ks = wg; ks < 8; ks += 2) {
+                    const int sq = ks >> 1;                          // source quarter
+                    const bool offd = dir > 0 ? sq < wq : sq > wq;
+                    const bool diag = sq == wq;
                     uint32_t m[16];
-                    if (offd) {
+                    if (offd || diag) {
+                        float g[16];
+                        tmem_ld16(tl + kColG + 16 * ks, g);
+                        tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float4 wv = *reinterpret_cast<const float4 *>(wrow + kb * 32 + 4 * i);
-                            m[2 * i] = pack_bf16(g[4 * i] * wv.x * e1, g[4 * i + 1] * wv.y * e1);
-                            m[2 * i + 1] = pack_bf16(g[4 * i + 2] * wv.z * e1, g[4 * i + 3] * wv.w * e1);
+                        for (int hh = 0; hh < 2; ++hh) {
+                            if (offd) {
+                                const float *wrow = wtab_s + (hh * 4 + wq) * kBlk + 16 * ks;
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    const float4 wv = *reinterpret_cast<const float4 *>(wrow + 4 * i);
+                                    m[8 * hh + 2 * i] = pack_bf16(g[4 * i] * wv.x * e1h[hh], g[4 * i + 1] * wv.y * e1h[hh]);
+                                    m[8 * hh + 2 * i + 1] =
+                                        pack_bf16(g[4 * i + 2] * wv.z * e1h[hh], g[4 * i + 3] * wv.w * e1h[hh]);
+                                }
+                            } else {
+                                const float *csrc = cs2_s + hh * kBlk + 16 * ks, *dsrc = dt_s + hh * kBlk + 16 * ks;
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    const float4 cv = *reinterpret_cast<const float4 *>(csrc + 4 * i);
+                                    const float4 dv = *reinterpret_cast<const float4 *>(dsrc + 4 * i);
+                                    const float cc[4] = {cv.x, cv.y, cv.z, cv.w}, dd[4] = {dv.x, dv.y, dv.z, dv.w};
+                                    float mv[4];
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        const int sidx = 16 * ks + 4 * i + e;
+                                        const bool in = dir > 0 ? sidx <= r : sidx >= r;
+                                        mv[e] = in ? g[4 * i + e] * exp2f(c2h[hh] - cc[e]) * dd[e] : 0.f;
+                                    }
+                                    m[8 * hh + 2 * i] = pack_bf16(mv[0], mv[1]);
+                                    m[8 * hh + 2 * i + 1] = pack_bf16(mv[2], mv[3]);
+                                }
+                            }
                         }
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float4 cv = *reinterpret_cast<const float4 *>(cs2 + kb * 32 + 4 * i);
-                            const float4 dv = *reinterpret_cast<const float4 *>(dts + kb * 32 + 4 * i);
-                            const float cc[4] = {cv.x, cv.y, cv.z, cv.w}, dd[4] = {dv.x, dv.y, dv.z, dv.w};
-                            float mv[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int sl = 4 * i + e;   // source lane within the quarter
-                                const bool in = dir > 0 ? sl <= lane : sl >= lane;
-                                mv[e] = in ? g[sl] * exp2f(c2 - cc[e]) * dd[e] : 0.f;
-                            }
-                            m[2 * i] = pack_bf16(mv[0], mv[1]);
-                            m[2 * i + 1] = pack_bf16(mv[2], mv[3]);
-                        }
+                        for (int i = 0; i < 16; ++i) m[i] = 0u;       // outside the causal triangle
                     }
-                    tmem_st16(tl + kColM + 64 * wg + kb * 16, m);
+                    tmem_st16(tl + kColG + 16 * ks, m);
                 }
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_GEMPTY));
+            if (lane == 0) mbar_arrive(bar(B_MREADY));
             SSD_TRACE_PT(warp, j, 10);
 
-            // state: S' <- exp(cs_last) S' + S, thread r holds state row n = r
+            // state: S' <- exp(cs_last) S' + S; thread r holds state row n = r, the float32 state
+            // lives in TMEM and a bf16 copy goes to smem as the next block's MMA operand
             if (!mbar_wait(bar(B_SFULL), j & 1, MASK, abort_flag, prm.status, 43)) break;
             SSD_TRACE_PT(warp, j, 11);
+            // the previous state tile must have been consumed by this block's Y = C S'^T
+            if (j + 1 < nblk && j >= 1 &&
+                !mbar_wait(bar(B_YOFFFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 44))
+                break;
             tc_fence_after();
-            {
-                float sv[32];
+#pragma unroll 1
+            for (int qd = 0; qd < 4; ++qd) {
+                float sv[16], pv[16];
+                if (j > 0) {
+                    tmem_ld16x2(tl + kColS + 64 * wg + 16 * qd, tl + kColST + 64 * wg + 16 * qd, sv, pv);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tl + kColS + 64 * wg + 32 * half, sv);
-                    tmem_wait_ld();
+                    for (int i = 0; i < 16; ++i) sv[i] = fmaf(ablk, pv[i], sv[i]);
+                } else {
+                    tmem_ld16(tl + kColS + 64 * wg + 16 * qd, sv);
+                }
+                uint32_t w16[16];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) state[32 * half + i] = fmaf(ablk, state[32 * half + i], sv[i]);
+                for (int i = 0; i < 16; ++i) w16[i] = __float_as_uint(sv[i]);
+                tmem_st16(tl + kColST + 64 * wg + 16 * qd, w16);
+                if (j + 1 < nblk) {
+#pragma unroll
+                    for (int qq = 0; qq < 2; ++qq) {
+                        uint4 o;
+                        o.x = pack_bf16(sv[8 * qq + 0], sv[8 * qq + 1]);
+                        o.y = pack_bf16(sv[8 * qq + 2], sv[8 * qq + 3]);
+                        o.z = pack_bf16(sv[8 * qq + 4], sv[8 * qq + 5]);
+                        o.w = pack_bf16(sv[8 * qq + 6], sv[8 * qq + 7]);
+                        *reinterpret_cast<uint4 *>(sp_tile + swz(r, 2 * qd + qq)) = o;
+                    }
                 }
             }
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_SEMPTY));
             SSD_TRACE_PT(warp, j, 12);
             if (j + 1 < nblk) {
-                // the previous state tile must have been consumed by this block's Y = C S'^T
-                if (j >= 1 && !mbar_wait(bar(B_YOFFFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 44)) break;
-                SSD_TRACE_PT(warp, j, 13);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    uint4 o;
-                    o.x = pack_bf16(state[8 * q + 0], state[8 * q + 1]);
-                    o.y = pack_bf16(state[8 * q + 2], state[8 * q + 3]);
-                    o.z = pack_bf16(state[8 * q + 4], state[8 * q + 5]);
-                    o.w = pack_bf16(state[8 * q + 6], state[8 * q + 7]);
-                    *reinterpret_cast<uint4 *>(sp_tile + swz(r, q)) = o;
-                }
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_SPREADY));
-                SSD_TRACE_PT(warp, j, 14);
             }
+            SSD_TRACE_PT(warp, j, 14);
 
             // Y (from the incoming state) scaled by exp(cs_r), before the intra-block term is added
             if (j >= 1) {
@@ -651,59 +719,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 if (lane == 0) mbar_arrive(bar(B_RSREADY));
                 SSD_TRACE_PT(warp, j, 15);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_MREADY));
 
-            // epilogue: y = Y + D x (+ the other direction's part), staged through the x tile
-            // (free once the intra-block MMA is done) so that y is written in whole 128-byte rows
+            // epilogue: o = Y + D x goes through the x tile (free once the intra-block MMA is done)
+            // so that y is written in whole 128-byte rows.  Bidirectional mixer: the ticket is
+            // taken only now, when this block's part is complete, so the first of the two
+            // directions stores and publishes with no further wait, and the second adds the
+            // published part while copying (its wait can only be for that store).
             if (!mbar_wait(bar(B_YFULL), j & 1, MASK, abort_flag, prm.status, 46)) break;
             SSD_TRACE_PT(warp, j, 16);
-            __nv_bfloat16 *ytile = prm.y + (((size_t)b * L + (size_t)cm * kBlk) * prm.H + h) * kP;
-            const size_t ystride = (size_t)prm.H * kP;      // elements between consecutive tokens
-            // who writes first: the ticket taken at the block start (bidirectional mixer only)
-            bool second = false;
-            if (prm.bidir) {
-                if (leader) {
-                    int sec = ticket == prm.epoch;
-                    if (sec) {
-                        // the other direction's part of this block: wait until it is published
-                        const unsigned long long *rp = prm.ready + flag_base + cm;
-                        const long long t0 = clock64();
-                        while (ld_acquire(rp) != prm.epoch) {
-                            if (*abort_flag) { sec = 2; break; }
-                            if (clock64() - t0 > prm.wait_cycles) {
-                                *abort_flag = 1;
-                                atomicExch(prm.status, 47);
-                                sec = 2;
-                                break;
-                            }
-                            __nanosleep(256);
-                        }
-                    }
-                    redw[8] = __int_as_float(sec);
-                }
-                if (!wg_sync(54)) break;
-                SSD_TRACE_PT(warp, j, 17);
-                const int sec = __float_as_int(redw[8]);
-                if (sec == 2) break;
-                second = sec == 1;
-            }
-            if (second) {
-                // the published part, as whole rows, into the w(.)x tile (read by this block's S MMA, done)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int c = tid_wg + 128 * i, rr = c >> 3, q = c & 7;
-                    const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(ytile + rr * ystride + 8 * q));
-                    *reinterpret_cast<uint4 *>(wx_tile + swz(rr, q)) = v;
-                }
-                if (!wg_sync(55)) break;
-            }
+            if (prm.bidir && leader) ticket = atomicExch(prm.ticket + flag_base + cm, prm.epoch);
             tc_fence_after();
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float yv[32];
                 tmem_ld32(tl + kColY + 64 * wg + 32 * half, yv);
-                tmem_wait_ld();
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
                     const int q = 4 * half + qq;
@@ -714,15 +743,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                     for (int i = 0; i < 4; ++i) {
                         o[2 * i] = fmaf(Dh, bf16lo(xw[i]), yv[8 * qq + 2 * i]);
                         o[2 * i + 1] = fmaf(Dh, bf16hi(xw[i]), yv[8 * qq + 2 * i + 1]);
-                    }
-                    if (second) {
-                        const uint4 pv = *reinterpret_cast<const uint4 *>(wx_tile + swz(r, q));
-                        const uint32_t pw[4] = {pv.x, pv.y, pv.z, pv.w};
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            o[2 * i] += bf16lo(pw[i]);
-                            o[2 * i + 1] += bf16hi(pw[i]);
-                        }
                     }
                     uint4 ov;
                     ov.x = pack_bf16(o[0], o[1]);
@@ -735,14 +755,66 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_YEMPTY));
+            SSD_TRACE_PT(warp, j, 17);
+            bool second = false;
+            if (prm.bidir) {
+                if (leader) {
+                    int sec = ticket == prm.epoch;
+                    if (sec) {
+                        // the other direction took its ticket first: its part is being stored now
+                        const unsigned long long *rp = prm.ready + flag_base + cm;
+                        const long long t0 = clock64();
+                        while (ld_acquire(rp) != prm.epoch) {
+                            if (*abort_flag) { sec = 2; break; }
+                            if (clock64() - t0 > prm.wait_cycles) {
+                                *abort_flag = 1;
+                                atomicExch(prm.status, 47);
+                                sec = 2;
+                                break;
+                            }
+                            __nanosleep(64);
+                        }
+                    }
+                    redw[8] = __int_as_float(sec);
+                }
+            }
+            if (!WG_SYNC(56)) break;                   // tile rows complete (and the ticket known)
+            if (prm.bidir) {
+                const int sec = __float_as_int(redw[8]);
+                if (sec == 2) break;
+                second = sec == 1;
+            }
             SSD_TRACE_PT(warp, j, 18);
-            if (!wg_sync(56)) break;
-            SSD_TRACE_PT(warp, j, 19);
+            __nv_bfloat16 *ytile = prm.y + (((size_t)b * L + (size_t)cm * kBlk) * prm.H + h) * kP;
+            const size_t ystride = (size_t)prm.H * kP;      // elements between consecutive tokens
+            {
+                // thread t copies chunk (t & 7) of rows (t >> 3) + 16 i: rows 16 apart keep the
+                // swizzle phase, so one shared offset and one global pointer serve all 8 copies
+                const int rr0 = tid_wg >> 3, q = tid_wg & 7;
+                __nv_bfloat16 *gp = ytile + (size_t)rr0 * ystride + 8 * q;
+                const uint8_t *sp = xt + swz(rr0, q);
+                if (second) {
+#pragma unroll 4
+                    for (int i = 0; i < 8; ++i) {
+                        const uint4 a = *reinterpret_cast<const uint4 *>(sp);
+                        const uint4 pv = __ldcg(reinterpret_cast<const uint4 *>(gp));
+                        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, pw[4] = {pv.x, pv.y, pv.z, pv.w};
+                        uint32_t ow[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int c = tid_wg + 128 * i, rr = c >> 3, q = c & 7;
-                const uint4 v = *reinterpret_cast<const uint4 *>(xt + swz(rr, q));
-                *reinterpret_cast<uint4 *>(ytile + rr * ystride + 8 * q) = v;
+                        for (int k = 0; k < 4; ++k)
+                            ow[k] = pack_bf16(bf16lo(aw[k]) + bf16lo(pw[k]), bf16hi(aw[k]) + bf16hi(pw[k]));
+                        *reinterpret_cast<uint4 *>(gp) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                        gp += 16 * ystride;
+                        sp += 16 * 128;
+                    }
+                } else {
+#pragma unroll 4
+                    for (int i = 0; i < 8; ++i) {
+                        *reinterpret_cast<uint4 *>(gp) = *reinterpret_cast<const uint4 *>(sp);
+                        gp += 16 * ystride;
+                        sp += 16 * 128;
+                    }
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_XEMPTY0 + st));
@@ -750,11 +822,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             if (prm.bidir && !second) {
                 // publish this direction's part of the block
                 __threadfence();
-                SSD_TRACE_PT(warp, j, 21);
-                if (!wg_sync(57)) break;
+                if (!WG_SYNC(57)) break;
                 if (leader && prm.fault != 1) st_release(prm.ready + flag_base + cm, prm.epoch);
-                SSD_TRACE_PT(warp, j, 22);
             }
+            SSD_TRACE_PT(warp, j, 21);
         }
     }
 

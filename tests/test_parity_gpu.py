@@ -45,9 +45,12 @@ def _bidir_case(ssd, shape, chunk, with_D, seed=0):
 SHAPES = [
     # (batch, L, H, P, N, G, io), chunk
     (si.Shape(1, 64, 2, 16, 16, 1, "f32"), 16),            # the tiny float32 workload
-    (si.Shape(2, 512, 8, 64, 128, 1, "bf16"), 256),        # layer shape, several chunks
-    (si.Shape(1, 768, 6, 64, 128, 1, "bf16"), 256),        # odd chunk count, 6 heads
-    (si.Shape(3, 384, 4, 64, 128, 1, "bf16"), 128),        # 3 chunks of 128
+    (si.Shape(2, 512, 8, 64, 128, 1, "bf16"), 256),        # layer shape, tensor-core path, 4 blocks
+    (si.Shape(1, 128, 8, 64, 128, 1, "bf16"), 128),        # tensor-core path, a single block
+    (si.Shape(3, 384, 16, 64, 128, 1, "bf16"), 128),       # tensor-core path, odd block count, 8 head pairs
+    (si.Shape(1, 1280, 24, 64, 128, 1, "bf16"), 256),      # tensor-core path, 10 blocks, 12 head pairs
+    (si.Shape(1, 768, 6, 64, 128, 1, "bf16"), 256),        # SIMT path (6 heads), odd chunk count
+    (si.Shape(3, 384, 4, 64, 128, 1, "bf16"), 128),        # SIMT path, 3 chunks of 128
     (si.Shape(2, 256, 4, 32, 64, 1, "bf16"), 64),
     (si.Shape(1, 256, 4, 16, 16, 1, "bf16"), 16),
     (si.Shape(2, 192, 4, 64, 64, 2, "bf16"), 64),          # two groups
@@ -67,7 +70,7 @@ def test_bidir_parity(ssd, shape, chunk, with_D):
 @pytest.mark.parametrize("direction", [1, -1])
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 def test_single_direction_parity(ssd, direction, io):
-    shape = si.Shape(2, 512, 4, 64, 128, 1, io)
+    shape = si.Shape(2, 512, 8, 64, 128, 1, io)
     p = si.make_params(shape, seed=3, with_D=False)
     y = ssd.ssd_scan(**_dev(p, False), direction=direction, chunk=128)
     torch.cuda.synchronize()
@@ -78,7 +81,7 @@ def test_single_direction_parity(ssd, direction, io):
 
 @pytest.mark.parametrize("chunk", [16, 32, 64, 128, 256])
 def test_chunk_size_invariance(ssd, chunk):
-    shape = si.Shape(1, 512, 4, 64, 128, 1, "bf16")
+    shape = si.Shape(1, 512, 8, 64, 128, 1, "bf16")
     err = _bidir_case(ssd, shape, chunk, with_D=False, seed=5)
     assert err <= TOL["bf16"]
 
@@ -92,12 +95,12 @@ def _flip(p):
 
 @pytest.mark.parametrize("io,chunk", [("f32", 16), ("bf16", 64), ("bf16", 256)])
 def test_reverse_is_flip_forward_flip(ssd, io, chunk):
-    shape = si.Shape(2, 512, 4, 64, 128, 1, io)
+    shape = si.Shape(2, 512, 8, 64, 128, 1, io)
     p = _dev(si.make_params(shape, seed=6))
     yr = ssd.ssd_scan(**p, direction=-1, chunk=chunk)
     yf = ssd.ssd_scan(**_flip(p), direction=1, chunk=chunk).flip(1)
     torch.cuda.synchronize()
-    if ssd.path_for((2, 512, 4, 64, 128, 1), p["x"].dtype, chunk) == 0:
+    if ssd.path_for((2, 512, 8, 64, 128, 1), p["x"].dtype, chunk) == 0:
         assert torch.equal(yr, yf)      # same arithmetic in scan order: bit for bit
     else:
         assert oracle.rel_err(_f64(yr), _f64(yf)) <= 1e-2
@@ -105,7 +108,7 @@ def test_reverse_is_flip_forward_flip(ssd, io, chunk):
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 def test_bidir_is_sum_of_directions(ssd, io):
-    shape = si.Shape(2, 512, 4, 64, 128, 1, io)
+    shape = si.Shape(2, 512, 8, 64, 128, 1, io)
     pf, pr = si.make_bidir(shape, seed=8)
     df, dr = _dev(pf), _dev(pr)
     yb = ssd.bidir_ssd(df, dr, chunk=128).double()
@@ -122,13 +125,38 @@ def test_bidir_is_sum_of_directions(ssd, io):
 
 
 def test_dt_zero_gives_skip_term_bitwise(ssd):
-    shape = si.Shape(1, 128, 4, 64, 128, 1, "f32")
+    shape = si.Shape(1, 128, 8, 64, 128, 1, "f32")
     p = _dev(si.make_params(shape, seed=9))
     p["dt"] = torch.zeros_like(p["dt"])
     for d in (1, -1):
         y = ssd.ssd_scan(**p, direction=d, chunk=64)
         torch.cuda.synchronize()
         assert torch.equal(y, p["D"][None, None, :, None] * p["x"])
+
+
+def test_dt_zero_tensor_core_path(ssd):
+    """dt = 0 on the tensor-core path: the state never moves, y = bf16(D x)."""
+    shape = si.Shape(1, 256, 8, 64, 128, 1, "bf16")
+    p = _dev(si.make_params(shape, seed=9))
+    p["dt"] = torch.zeros_like(p["dt"])
+    for d in (1, -1):
+        y = ssd.ssd_scan(**p, direction=d, chunk=128)
+        torch.cuda.synchronize()
+        ref = (p["D"][None, None, :, None] * p["x"].float()).to(torch.bfloat16)
+        assert torch.equal(y, ref)
+
+
+def test_paths_agree(ssd):
+    """The tensor-core path (chunk 128) and the SIMT path (chunk 64) on the same inputs."""
+    shape = si.Shape(2, 512, 8, 64, 128, 1, "bf16")
+    dims = (2, 512, 8, 64, 128, 1)
+    assert ssd.path_for(dims, torch.bfloat16, 64) == 0
+    pf, pr = si.make_bidir(shape, seed=12, with_D=False)
+    df, dr = _dev(pf, False), _dev(pr, False)
+    a = ssd.bidir_ssd(df, dr, chunk=128).double()
+    b = ssd.bidir_ssd(df, dr, chunk=64).double()
+    torch.cuda.synchronize()
+    assert oracle.rel_err(a.cpu().numpy(), b.cpu().numpy()) <= 2e-2
 
 
 def test_deterministic(ssd):
