@@ -36,13 +36,17 @@
 // Bidirectional mixer in one launch.  The CTAs of the forward and reverse
 // scans of one head pair are neighbours in the grid.  For every output block
 // the first of the two to finish writes its part of y, the second adds its
-// own part to it: an epoch-tagged ticket per (batch, head, block) decides the
-// order and an epoch-tagged ready word publishes the first part.  The first
-// never waits, so the hand-off cannot deadlock whatever the residency.
+// own part to it: an epoch-tagged ticket per (batch, head, block), taken by a
+// store warp once the block's part is complete, decides the order, and an
+// epoch-tagged ready word publishes the first part.  The first never waits,
+// and a second only waits for a first that has already passed every earlier
+// block of its own walk, so the hand-off cannot deadlock whatever the residency.
 //
-// Warp roles (320 threads): warps 0-3 do the CUDA-core work of head h0 and
+// Warp roles (384 threads): warps 0-3 do the CUDA-core work of head h0 and
 // warps 4-7 that of head h0+1 (thread r <-> TMEM lane r), warp 8 issues the
-// TMA loads, warp 9 owns TMEM and issues the MMAs (one thread).  Every wait is
+// TMA loads, warp 9 owns TMEM and issues the MMAs (one thread), warps 10 and
+// 11 write y for heads h0 and h0+1 (TMA stores, and the forward/reverse
+// hand-off), so the CUDA-core warpgroups never wait on global memory.  Every wait is
 // bounded; a wait that runs out records SSD_ERR_TIMEOUT in the status word and
 // the CTA winds down without touching more data.
 #include <cuda.h>
@@ -62,8 +66,8 @@ namespace {
 
 constexpr int kBlk = 128;            // tokens per block (MMA M)
 constexpr int kP = 64, kN = 128;
-constexpr int kThreads = 320;        // warps 0-7: two head warpgroups; 8: TMA; 9: MMA + TMEM
-constexpr int kWarpTma = 8, kWarpMma = 9;
+constexpr int kThreads = 384;        // warps 0-7: two head warpgroups; 8: TMA; 9: MMA + TMEM; 10-11: y stores
+constexpr int kWarpTma = 8, kWarpMma = 9, kWarpStore = 10;
 constexpr uint32_t kTileBytes = kBlk * 64 * 2;        // one [128][64] bf16 swizzled tile = 16 KB
 constexpr uint32_t kDtBytes = kBlk * 8 * 2;           // dt box: 128 tokens x 8 heads, bf16
 constexpr uint32_t kStageBytes = 2 * kTileBytes + kDtBytes;   // x of 2 heads + dt = 34 KB
@@ -80,9 +84,8 @@ constexpr uint32_t kOffSP = kOffWX + 2 * kTileBytes;   // 2 heads, rows = state 
 constexpr uint32_t kOffCS = kOffSP + 2 * kTileBytes;   // float cs2[2][128], dt[2][128]
 constexpr uint32_t kOffW = kOffCS + 4 * kBlk * 4;      // float W[2][4][128]: off-diagonal column factors
 constexpr uint32_t kOffE1 = kOffW + 2 * 4 * kBlk * 4;  // float e1[2][128]: off-diagonal row factors
-constexpr uint32_t kOffRed = kOffE1 + 2 * kBlk * 4;    // per-WG cross-warp scan scratch + epilogue word
-constexpr uint32_t kOffBar = kOffRed + 2 * 16 * 4;
-constexpr uint32_t kNumBars = 20;
+constexpr uint32_t kOffBar = kOffE1 + 2 * kBlk * 4;
+constexpr uint32_t kNumBars = 22;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
 static_assert(kStageBytes % 1024 == 0, "x tiles must stay 1024-byte aligned");
@@ -90,7 +93,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 enum Bar {
     B_XFULL0 = 0, B_XFULL1, B_XEMPTY0, B_XEMPTY1, B_BCFULL, B_BCEMPTY, B_GFULL, B_GEMPTY,
-    B_WXREADY, B_SFULL, B_SEMPTY, B_SPREADY, B_YOFFFULL, B_MREADY, B_RSREADY, B_YFULL, B_YEMPTY, B_DONE, B_WG0, B_WG1
+    B_WXREADY, B_SFULL, B_SEMPTY, B_SPREADY, B_YOFFFULL, B_MREADY, B_RSREADY, B_YFULL, B_YEMPTY, B_DONE, B_WG0, B_WG1, B_TILE0, B_TILE1
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -108,7 +111,20 @@ __device__ __forceinline__ void trace_pt(int w, int j, int k) {
     }
 }
 #define SSD_TRACE_PT(w, j, k) trace_pt(w, j, k)
+__device__ unsigned long long g_cta_time[4096][3];     // start, end, SM id
+#define SSD_TRACE_CTA(k)                                                              \
+    do {                                                                              \
+        if (threadIdx.x == 0 && blockIdx.x < 4096) {                                  \
+            unsigned long long t_;                                                    \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                    \
+            g_cta_time[blockIdx.x][k] = t_;                                           \
+            unsigned smid_;                                                           \
+            asm volatile("mov.u32 %0, %%smid;" : "=r"(smid_));                        \
+            g_cta_time[blockIdx.x][2] = smid_;                                        \
+        }                                                                             \
+    } while (0)
 #else
+#define SSD_TRACE_CTA(k) ((void)0)
 #define SSD_TRACE_PT(w, j, k) ((void)0)
 #endif
 
@@ -131,7 +147,7 @@ struct TcParams {
 };
 
 struct TcMaps {
-    CUtensorMap x[2], dt[2], b[2], c[2];
+    CUtensorMap x[2], dt[2], b[2], c[2], y;
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -334,6 +350,16 @@ __device__ __forceinline__ unsigned long long ld_acquire(const unsigned long lon
     return v;
 }
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ------------------------------------------------------------------ the kernel
 
 __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ TcMaps maps, TcParams prm) {
@@ -346,7 +372,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
     float *cs2_s = reinterpret_cast<float *>(sm + kOffCS);          // [2][128] cs * log2(e)
     float *dt_s = cs2_s + 2 * kBlk;                                  // [2][128] dt
     float *wtab_s = reinterpret_cast<float *>(sm + kOffW);           // [2][4][128]
-    float *red = reinterpret_cast<float *>(sm + kOffRed);            // [2 WG][16]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int npairs = prm.H / 2;
@@ -363,11 +388,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
         *abort_flag = 0;
         *reinterpret_cast<volatile long long *>(abort_flag + 1) = prm.wait_cycles;
         // arrival counts: 8 = one per CUDA-core warp, 4 = one per warp of a warpgroup, 1 = one thread / commit
-        constexpr uint32_t k8 = (1u << B_XEMPTY0) | (1u << B_XEMPTY1) | (1u << B_GEMPTY) | (1u << B_WXREADY) |
-                                (1u << B_SEMPTY) | (1u << B_SPREADY) | (1u << B_MREADY) | (1u << B_RSREADY) |
-                                (1u << B_YEMPTY);
-        constexpr uint32_t k4 = (1u << B_WG0) | (1u << B_WG1);
-        for (int i = 0; i < (int)kNumBars; ++i) mbar_init(bar(i), (k8 >> i) & 1 ? 8 : (k4 >> i) & 1 ? 4 : 1);
+        // arrival counts: 8 = one per CUDA-core warp, 4 = one per warp of a warpgroup,
+        // 2 = one per store warp, 1 = one thread / one MMA commit
+        constexpr uint32_t k8 = (1u << B_GEMPTY) | (1u << B_WXREADY) | (1u << B_SEMPTY) | (1u << B_SPREADY) |
+                                (1u << B_MREADY) | (1u << B_RSREADY) | (1u << B_YEMPTY);
+        constexpr uint32_t k4 = (1u << B_WG0) | (1u << B_WG1) | (1u << B_TILE0) | (1u << B_TILE1);
+        constexpr uint32_t k2 = (1u << B_XEMPTY0) | (1u << B_XEMPTY1);
+        for (int i = 0; i < (int)kNumBars; ++i)
+            mbar_init(bar(i), (k8 >> i) & 1 ? 8 : (k4 >> i) & 1 ? 4 : (k2 >> i) & 1 ? 2 : 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kWarpMma) {
@@ -378,6 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    SSD_TRACE_CTA(0);
 
     if (warp == kWarpTma) {
         // ---------------------------------------------------------- TMA producer
@@ -478,6 +507,78 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             mma_commit(bar(B_DONE));
             mbar_drain(bar(B_DONE), 0, prm.wait_cycles);
         }
+    } else if (warp >= kWarpStore) {
+        // ---------------------------------------------------------- y stores, one warp per head
+        const uint32_t MASK = 0xffffffffu;
+        const int hs = warp - kWarpStore;
+        const int h = h0 + hs;
+        const size_t flag_base = ((size_t)b * prm.H + h) * nblk;
+        const size_t ystride = (size_t)prm.H * kP;      // elements between consecutive tokens
+        for (int j = 0; j < nblk; ++j) {
+            const int st = j & 1;
+            const int cm = dir > 0 ? j : nblk - 1 - j;
+            if (!mbar_wait(bar(B_TILE0 + hs), j & 1, MASK, abort_flag, prm.status, 61)) break;
+            const uint32_t tile = sbase + kOffX + st * kStageBytes + hs * kTileBytes;
+            int sec = 0;
+            if (prm.bidir) {
+                if (lane == 0) {
+                    // this direction's part of the block is complete: first or second?
+                    sec = atomicExch(prm.ticket + flag_base + cm, prm.epoch) == prm.epoch;
+                    if (sec) {
+                        // the other direction's store warp took the block first and is storing it
+                        const unsigned long long *rp = prm.ready + flag_base + cm;
+                        const long long t0 = clock64();
+                        while (ld_acquire(rp) != prm.epoch) {
+                            if (*abort_flag) { sec = 2; break; }
+                            if (clock64() - t0 > prm.wait_cycles) {
+                                *abort_flag = 1;
+                                atomicExch(prm.status, 47);
+                                sec = 2;
+                                break;
+                            }
+                            __nanosleep(64);
+                        }
+                    }
+                }
+                sec = __shfl_sync(MASK, sec, 0);
+                if (sec == 2) break;
+            }
+            if (sec == 0) {
+                if (lane == 0) {
+                    tma_store_2d(&maps.y, tile, h * kP, b * L + cm * kBlk);
+                    bulk_commit();
+                    bulk_wait_read0();                    // the tile may be overwritten from here on
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(bar(B_XEMPTY0 + st));
+                    if (prm.bidir) {
+                        bulk_wait0();                     // this part of y is in global memory
+                        asm volatile("fence.proxy.async.global;" ::: "memory");
+                        if (prm.fault != 1) st_release(prm.ready + flag_base + cm, prm.epoch);
+                    }
+                }
+            } else {
+                // y = published part + this part, four whole 128-byte rows per instruction
+                __nv_bfloat16 *ytile = prm.y + (((size_t)b * L + (size_t)cm * kBlk) * prm.H + h) * kP;
+                const uint8_t *tp = sm + kOffX + st * kStageBytes + hs * kTileBytes;
+#pragma unroll 8
+                for (int i = 0; i < 32; ++i) {
+                    const int c = lane + 32 * i, rr = c >> 3, q = c & 7;
+                    const uint4 a = *reinterpret_cast<const uint4 *>(tp + swz(rr, q));
+                    const uint4 pv = __ldcg(reinterpret_cast<const uint4 *>(ytile + rr * ystride + 8 * q));
+                    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, pw[4] = {pv.x, pv.y, pv.z, pv.w};
+                    uint32_t ow[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        ow[k] = pack_bf16(bf16lo(aw[k]) + bf16lo(pw[k]), bf16hi(aw[k]) + bf16hi(pw[k]));
+                    *reinterpret_cast<uint4 *>(ytile + rr * ystride + 8 * q) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_XEMPTY0 + st));
+            }
+        }
+        if (lane == 0) bulk_wait0();                      // every store has landed before the CTA exits
     } else {
         // ---------------------------------------------------------- per-head CUDA-core work
         const uint32_t MASK = 0xffffffffu;
@@ -485,34 +586,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
         const int wq = warp & 3;                   // TMEM lane quarter = 32-row quarter of the block
         const int r = wq * 32 + lane;              // row in block == TMEM lane
         const int h = h0 + wg;
-        const int tid_wg = threadIdx.x - 128 * wg;
-        const bool leader = (wq == 0 && lane == 0);
         const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
         const float A2 = prm.d[slot].A[h] * kLog2e;   // log2 units: exp(a) = exp2(a * log2 e)
         const float Dh = prm.d[slot].D ? prm.d[slot].D[h] : 0.f;
         float *cs2 = cs2_s + wg * kBlk, *dts = dt_s + wg * kBlk, *wtab = wtab_s + wg * 4 * kBlk;
-        float *redw = red + wg * 16;
         uint8_t *wx_tile = sm + kOffWX + wg * kTileBytes;
         uint8_t *sp_tile = sm + kOffSP + wg * kTileBytes;
-        uint32_t wg_phase = 0;   // completions of this WG's sync barrier so far
-        // bounded replacement for a named barrier over the 4 warps of this warpgroup
-#define WG_SYNC(code)                                                                                     \
-    ([&]() __attribute__((always_inline)) {                                                              \
-        __syncwarp();                                                                                     \
-        if (lane == 0) mbar_arrive(bar(B_WG0 + wg));                                                      \
-        const bool ok_ = mbar_wait(bar(B_WG0 + wg), wg_phase & 1, MASK, abort_flag, prm.status, (code));  \
-        ++wg_phase;                                                                                       \
-        return ok_;                                                                                       \
-    }())
         float *e1_s = reinterpret_cast<float *>(sm + kOffE1);   // [2][128]
-        const size_t flag_base = ((size_t)b * prm.H + h) * nblk;
-        unsigned long long ticket = 0;
 
         for (int j = 0; j < nblk; ++j) {
             if (__any_sync(0xffffffffu, *abort_flag)) break;
             SSD_TRACE_PT(warp, j, 0);
             const int st = j & 1;
-            const int cm = dir > 0 ? j : nblk - 1 - j;
 
             // x, dt of this block
             if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 41)) break;
@@ -522,24 +607,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 reinterpret_cast<const __nv_bfloat16 *>(sm + kOffX + st * kStageBytes + 2 * kTileBytes);
             const float dtr = __bfloat162float(dtt[r * 8 + (h & 7)]);
 
-            // cumulative A*dt in scan order (prefix over rows forward, suffix over rows reverse)
+            // cumulative A*dt in scan order (prefix over rows forward, suffix over rows reverse):
+            // warp shuffles inside the quarter, and every warp reduces all four quarter totals
+            // itself from the dt tile, so no exchange between warps is needed
             float s = dtr;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float u = dir > 0 ? __shfl_up_sync(0xffffffffu, s, o) : __shfl_down_sync(0xffffffffu, s, o);
                 if (dir > 0 ? lane >= o : lane + o < 32) s += u;
             }
-            if (!WG_SYNC(51)) break;           // previous block's readers of red/cs/W are done
-            SSD_TRACE_PT(warp, j, 3);
-            if (lane == (dir > 0 ? 31 : 0)) redw[wq] = s;
-            if (!WG_SYNC(52)) break;
-            SSD_TRACE_PT(warp, j, 4);
             float tot[4], base = 0.f, total = 0.f;
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
-                tot[w] = redw[w];
-                total += tot[w];
-                if (dir > 0 ? w < wq : w > wq) base += tot[w];
+                float v = __bfloat162float(dtt[(32 * w + lane) * 8 + (h & 7)]);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                tot[w] = v;
+                total += v;
+                if (dir > 0 ? w < wq : w > wq) base += v;
             }
             // cs (log2 units) at the quarter boundaries: the reference rows of the factorised mask
             float ref2[4];
@@ -582,9 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 *reinterpret_cast<uint4 *>(wx_tile + swz(r, q)) = o;
             }
             SSD_TRACE_PT(warp, j, 6);
-            fence_async_smem();
-            SSD_TRACE_PT(warp, j, 7);
-            if (!WG_SYNC(53)) break;           // cs2/dts/W of all rows visible to this WG
+            fence_async_smem();                // w(.)x is read by the tensor core
             SSD_TRACE_PT(warp, j, 8);
             if (lane == 0) mbar_arrive(bar(B_WXREADY));
 
@@ -720,14 +803,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 SSD_TRACE_PT(warp, j, 15);
             }
 
-            // epilogue: o = Y + D x goes through the x tile (free once the intra-block MMA is done)
-            // so that y is written in whole 128-byte rows.  Bidirectional mixer: the ticket is
-            // taken only now, when this block's part is complete, so the first of the two
-            // directions stores and publishes with no further wait, and the second adds the
-            // published part while copying (its wait can only be for that store).
+            // epilogue: o = Y + D x, bf16, written over this row of the x tile (free once the
+            // intra-block MMA is done); a store warp then writes the tile to y in whole rows
             if (!mbar_wait(bar(B_YFULL), j & 1, MASK, abort_flag, prm.status, 46)) break;
             SSD_TRACE_PT(warp, j, 16);
-            if (prm.bidir && leader) ticket = atomicExch(prm.ticket + flag_base + cm, prm.epoch);
             tc_fence_after();
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -752,78 +831,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                     *reinterpret_cast<uint4 *>(xt + swz(r, q)) = ov;
                 }
             }
+            fence_async_smem();                // the tile is read by a TMA store
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_YEMPTY));
-            SSD_TRACE_PT(warp, j, 17);
-            bool second = false;
-            if (prm.bidir) {
-                if (leader) {
-                    int sec = ticket == prm.epoch;
-                    if (sec) {
-                        // the other direction took its ticket first: its part is being stored now
-                        const unsigned long long *rp = prm.ready + flag_base + cm;
-                        const long long t0 = clock64();
-                        while (ld_acquire(rp) != prm.epoch) {
-                            if (*abort_flag) { sec = 2; break; }
-                            if (clock64() - t0 > prm.wait_cycles) {
-                                *abort_flag = 1;
-                                atomicExch(prm.status, 47);
-                                sec = 2;
-                                break;
-                            }
-                            __nanosleep(64);
-                        }
-                    }
-                    redw[8] = __int_as_float(sec);
-                }
-            }
-            if (!WG_SYNC(56)) break;                   // tile rows complete (and the ticket known)
-            if (prm.bidir) {
-                const int sec = __float_as_int(redw[8]);
-                if (sec == 2) break;
-                second = sec == 1;
-            }
-            SSD_TRACE_PT(warp, j, 18);
-            __nv_bfloat16 *ytile = prm.y + (((size_t)b * L + (size_t)cm * kBlk) * prm.H + h) * kP;
-            const size_t ystride = (size_t)prm.H * kP;      // elements between consecutive tokens
-            {
-                // thread t copies chunk (t & 7) of rows (t >> 3) + 16 i: rows 16 apart keep the
-                // swizzle phase, so one shared offset and one global pointer serve all 8 copies
-                const int rr0 = tid_wg >> 3, q = tid_wg & 7;
-                __nv_bfloat16 *gp = ytile + (size_t)rr0 * ystride + 8 * q;
-                const uint8_t *sp = xt + swz(rr0, q);
-                if (second) {
-#pragma unroll 4
-                    for (int i = 0; i < 8; ++i) {
-                        const uint4 a = *reinterpret_cast<const uint4 *>(sp);
-                        const uint4 pv = __ldcg(reinterpret_cast<const uint4 *>(gp));
-                        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, pw[4] = {pv.x, pv.y, pv.z, pv.w};
-                        uint32_t ow[4];
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            ow[k] = pack_bf16(bf16lo(aw[k]) + bf16lo(pw[k]), bf16hi(aw[k]) + bf16hi(pw[k]));
-                        *reinterpret_cast<uint4 *>(gp) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                        gp += 16 * ystride;
-                        sp += 16 * 128;
-                    }
-                } else {
-#pragma unroll 4
-                    for (int i = 0; i < 8; ++i) {
-                        *reinterpret_cast<uint4 *>(gp) = *reinterpret_cast<const uint4 *>(sp);
-                        gp += 16 * ystride;
-                        sp += 16 * 128;
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_XEMPTY0 + st));
-            SSD_TRACE_PT(warp, j, 20);
-            if (prm.bidir && !second) {
-                // publish this direction's part of the block
-                __threadfence();
-                if (!WG_SYNC(57)) break;
-                if (leader && prm.fault != 1) st_release(prm.ready + flag_base + cm, prm.epoch);
+            if (lane == 0) {
+                mbar_arrive(bar(B_YEMPTY));
+                mbar_arrive(bar(B_TILE0 + wg));
             }
             SSD_TRACE_PT(warp, j, 21);
         }
@@ -831,6 +844,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
 
     tc_fence_before();
     __syncthreads();
+    SSD_TRACE_CTA(1);
     if (warp == kWarpMma) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
@@ -904,6 +918,10 @@ void tc_set_direction(TcArgs &t, int slot, int dir, const void *x, const void *d
 int tc_launches(bool) { return 1; }
 
 #ifdef SSD_TRACE
+extern "C" int ssd_debug_cta_times(unsigned long long *out, int n) {
+    if (n < 4096 * 3) return -1;
+    return cudaMemcpyFromSymbol(out, g_cta_time, sizeof(unsigned long long) * 4096 * 3) == cudaSuccess ? 4096 : -2;
+}
 extern "C" int ssd_debug_trace(unsigned long long *out, int n) {
     const int total = kTraceWarps * kTraceBlocks * kTracePts;
     if (n < total) return -1;
@@ -932,6 +950,7 @@ cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
         p.d[s].A = d.A;
         p.d[s].D = d.D;
     }
+    if (!make_map(&maps.y, y, rows, (uint64_t)t.H * kP, 64, true)) return cudaErrorInvalidValue;
     p.batch = t.batch; p.L = t.L; p.H = t.H; p.nblk = t.L / kBlk;
     p.bidir = bidir ? 1 : 0;
     p.dir_single = t.d[0].dir;
