@@ -19,11 +19,17 @@ thread_local std::string g_err;
 std::atomic<int> g_fault{0};
 std::atomic<long long> g_wait_ns{2000000000LL};
 
+// SM clock (kHz) of each device, queried once: converts the wait bound to cycles.
+std::atomic<int> g_clock_khz[64];
+
 long long wait_cycles_now() {
-    int dev = 0, khz = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev) != cudaSuccess ||
-        khz <= 0)
-        khz = 2000000;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    int khz = (dev >= 0 && dev < 64) ? g_clock_khz[dev].load(std::memory_order_relaxed) : 0;
+    if (khz <= 0) {
+        if (cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev) != cudaSuccess || khz <= 0) khz = 2000000;
+        if (dev >= 0 && dev < 64) g_clock_khz[dev].store(khz, std::memory_order_relaxed);
+    }
     return (long long)((double)g_wait_ns.load() * 1e-9 * (double)khz * 1e3);
 }
 

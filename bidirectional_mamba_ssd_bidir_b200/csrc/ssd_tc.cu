@@ -356,6 +356,12 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t sr
                  "r"(src), "r"(c0), "r"(c1)
                  : "memory");
 }
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, uint32_t src, int c0, int c1) {
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -513,7 +519,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
         const int hs = warp - kWarpStore;
         const int h = h0 + hs;
         const size_t flag_base = ((size_t)b * prm.H + h) * nblk;
-        const size_t ystride = (size_t)prm.H * kP;      // elements between consecutive tokens
         for (int j = 0; j < nblk; ++j) {
             const int st = j & 1;
             const int cm = dir > 0 ? j : nblk - 1 - j;
@@ -559,20 +564,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                     }
                 }
             } else {
-                // y = published part + this part, four whole 128-byte rows per instruction
-                __nv_bfloat16 *ytile = prm.y + (((size_t)b * L + (size_t)cm * kBlk) * prm.H + h) * kP;
-                const uint8_t *tp = sm + kOffX + st * kStageBytes + hs * kTileBytes;
-#pragma unroll 8
-                for (int i = 0; i < 32; ++i) {
-                    const int c = lane + 32 * i, rr = c >> 3, q = c & 7;
-                    const uint4 a = *reinterpret_cast<const uint4 *>(tp + swz(rr, q));
-                    const uint4 pv = __ldcg(reinterpret_cast<const uint4 *>(ytile + rr * ystride + 8 * q));
-                    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, pw[4] = {pv.x, pv.y, pv.z, pv.w};
-                    uint32_t ow[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        ow[k] = pack_bf16(bf16lo(aw[k]) + bf16lo(pw[k]), bf16hi(aw[k]) + bf16hi(pw[k]));
-                    *reinterpret_cast<uint4 *>(ytile + rr * ystride + 8 * q) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                // y += this part: a bulk tensor reduction (bf16 add in L2) onto the published part
+                if (lane == 0) {
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                    tma_reduce_add_2d(&maps.y, tile, h * kP, b * L + cm * kBlk);
+                    bulk_commit();
+                    bulk_wait_read0();
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_XEMPTY0 + st));
