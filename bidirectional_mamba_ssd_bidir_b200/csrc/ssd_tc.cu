@@ -42,11 +42,11 @@
 // and a second only waits for a first that has already passed every earlier
 // block of its own walk, so the hand-off cannot deadlock whatever the residency.
 //
-// Warp roles (384 threads): warps 0-3 do the CUDA-core work of head h0 and
-// warps 4-7 that of head h0+1 (thread r <-> TMEM lane r), warp 8 issues the
-// TMA loads, warp 9 owns TMEM and issues the MMAs (one thread), warps 10 and
-// 11 write y for heads h0 and h0+1 (TMA stores, and the forward/reverse
-// hand-off), so the CUDA-core warpgroups never wait on global memory.  Every wait is
+// Warp roles (640 threads): warps 0-15 form four warpgroups doing the CUDA-core
+// work (thread r <-> TMEM lane r; warpgroup g = 2*head + column half), warp 16
+// issues the TMA loads, warp 17 owns TMEM and issues the MMAs (one thread),
+// warps 18 and 19 write y for heads h0 and h0+1 (TMA stores, and the
+// forward/reverse hand-off), so the CUDA-core warps never wait on global memory.  Every wait is
 // bounded; a wait that runs out records SSD_ERR_TIMEOUT in the status word and
 // the CTA winds down without touching more data.
 #include <cuda.h>
@@ -66,8 +66,8 @@ namespace {
 
 constexpr int kBlk = 128;            // tokens per block (MMA M)
 constexpr int kP = 64, kN = 128;
-constexpr int kThreads = 384;        // warps 0-7: two head warpgroups; 8: TMA; 9: MMA + TMEM; 10-11: y stores
-constexpr int kWarpTma = 8, kWarpMma = 9, kWarpStore = 10;
+constexpr int kThreads = 640;        // warps 0-15: four warpgroups; 16: TMA; 17: MMA + TMEM; 18-19: y stores
+constexpr int kWarpTma = 16, kWarpMma = 17, kWarpStore = 18;
 constexpr uint32_t kTileBytes = kBlk * 64 * 2;        // one [128][64] bf16 swizzled tile = 16 KB
 constexpr uint32_t kDtBytes = kBlk * 8 * 2;           // dt box: 128 tokens x 8 heads, bf16
 constexpr uint32_t kStageBytes = 2 * kTileBytes + kDtBytes;   // x of 2 heads + dt = 34 KB
@@ -101,7 +101,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Optional phase timeline for profiling builds (-DSSD_TRACE): %globaltimer
 // stamps of CTA 0, first kTraceBlocks blocks, per warp and phase.
 #ifdef SSD_TRACE
-constexpr int kTraceWarps = 10, kTraceBlocks = 8, kTracePts = 24;
+constexpr int kTraceWarps = 20, kTraceBlocks = 8, kTracePts = 24;
 __device__ unsigned long long g_trace[kTraceWarps][kTraceBlocks][kTracePts];
 __device__ __forceinline__ void trace_pt(int w, int j, int k) {
     if (blockIdx.x == 0 && j < kTraceBlocks && (threadIdx.x & 31) == 0) {
@@ -394,14 +394,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
         *abort_flag = 0;
         *reinterpret_cast<volatile long long *>(abort_flag + 1) = prm.wait_cycles;
         // arrival counts: 8 = one per CUDA-core warp, 4 = one per warp of a warpgroup, 1 = one thread / commit
-        // arrival counts: 8 = one per CUDA-core warp, 4 = one per warp of a warpgroup,
-        // 2 = one per store warp, 1 = one thread / one MMA commit
-        constexpr uint32_t k8 = (1u << B_GEMPTY) | (1u << B_WXREADY) | (1u << B_SEMPTY) | (1u << B_SPREADY) |
-                                (1u << B_MREADY) | (1u << B_RSREADY) | (1u << B_YEMPTY);
-        constexpr uint32_t k4 = (1u << B_WG0) | (1u << B_WG1) | (1u << B_TILE0) | (1u << B_TILE1);
+        // arrival counts: 16 = one per CUDA-core warp, 8 = one per warp of a head's two
+        // warpgroups, 2 = one per store warp, 1 = one thread / one MMA commit
+        constexpr uint32_t k16 = (1u << B_GEMPTY) | (1u << B_WXREADY) | (1u << B_SEMPTY) | (1u << B_SPREADY) |
+                                 (1u << B_MREADY) | (1u << B_RSREADY) | (1u << B_YEMPTY);
+        constexpr uint32_t k8 = (1u << B_TILE0) | (1u << B_TILE1);
         constexpr uint32_t k2 = (1u << B_XEMPTY0) | (1u << B_XEMPTY1);
         for (int i = 0; i < (int)kNumBars; ++i)
-            mbar_init(bar(i), (k8 >> i) & 1 ? 8 : (k4 >> i) & 1 ? 4 : (k2 >> i) & 1 ? 2 : 1);
+            mbar_init(bar(i), (k16 >> i) & 1 ? 16 : (k8 >> i) & 1 ? 8 : (k2 >> i) & 1 ? 2 : 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kWarpMma) {
@@ -428,14 +428,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 const int row = b * L + cm * kBlk;
                 const int st = j & 1;
                 if (j >= 2 && !mbar_wait(bar(B_XEMPTY0 + st), ((j >> 1) - 1) & 1, MASK, abort_flag, prm.status, 11)) break;
-                SSD_TRACE_PT(8, j, 0);
+                SSD_TRACE_PT(kWarpTma, j, 0);
                 const uint32_t stage = sbase + kOffX + st * kStageBytes;
                 mbar_expect_tx(bar(B_XFULL0 + st), kStageBytes);
                 for (int h = 0; h < 2; ++h)
                     tma_load_2d(stage + h * kTileBytes, map_x, (h0 + h) * kP, row, bar(B_XFULL0 + st));
                 tma_load_2d(stage + 2 * kTileBytes, map_dt, h0 & ~7, row, bar(B_XFULL0 + st));
                 if (j >= 1 && !mbar_wait(bar(B_BCEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 12)) break;
-                SSD_TRACE_PT(8, j, 1);
+                SSD_TRACE_PT(kWarpTma, j, 1);
                 mbar_expect_tx(bar(B_BCFULL), 4 * kTileBytes);
                 for (int q = 0; q < 2; ++q) {
                     tma_load_2d(sbase + kOffB + q * kTileBytes, map_b, q * 64, row, bar(B_BCFULL));
@@ -465,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 if (!mbar_wait(bar(B_BCFULL), j & 1, MASK, abort_flag, prm.status, 21)) break;
                 // the previous block's M (read by its intra-block MMA) occupies the G columns
                 if (j >= 1 && !mbar_wait(bar(B_YFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 22)) break;
-                SSD_TRACE_PT(9, j, 0);
+                SSD_TRACE_PT(kWarpMma, j, 0);
                 tc_fence_after();
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = (ks >> 2) * kTileBytes + (ks & 3) * 32;
@@ -475,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 // S^T = B^T (w x)  (M = n, N = (head, p), K = rows); both operands MN-major
                 if (!mbar_wait(bar(B_WXREADY), j & 1, MASK, abort_flag, prm.status, 23)) break;
                 if (j >= 1 && !mbar_wait(bar(B_SEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 24)) break;
-                SSD_TRACE_PT(9, j, 1);
+                SSD_TRACE_PT(kWarpMma, j, 1);
                 tc_fence_after();
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = ks * 2048;
@@ -487,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 if (j >= 1) {
                     if (!mbar_wait(bar(B_SPREADY), (j - 1) & 1, MASK, abort_flag, prm.status, 25)) break;
                     if (!mbar_wait(bar(B_YEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 26)) break;
-                    SSD_TRACE_PT(9, j, 2);
+                    SSD_TRACE_PT(kWarpMma, j, 2);
                     tc_fence_after();
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t offc = (ks >> 2) * kTileBytes + (ks & 3) * 32;
@@ -501,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 if (!mbar_wait(bar(B_MREADY), j & 1, MASK, abort_flag, prm.status, 27)) break;
                 if (j >= 1 && !mbar_wait(bar(B_RSREADY), (j - 1) & 1, MASK, abort_flag, prm.status, 28)) break;
                 if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 29)) break;
-                SSD_TRACE_PT(9, j, 3);
+                SSD_TRACE_PT(kWarpMma, j, 3);
                 tc_fence_after();
                 for (int h = 0; h < 2; ++h)
                     for (int ks = 0; ks < 8; ++ks)
@@ -577,19 +577,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
         }
         if (lane == 0) bulk_wait0();                      // every store has landed before the CTA exits
     } else {
-        // ---------------------------------------------------------- per-head CUDA-core work
+        // ---------------------------------------------------------- CUDA-core work
+        // Four warpgroups: g = 2 * head + half.  Each handles one head's rows and one half
+        // (32 of 64) of its headdim columns in the per-head passes, and a quarter of the
+        // 16-source K-steps (both heads) in the decay-mask pass.
         const uint32_t MASK = 0xffffffffu;
-        const int wg = warp >> 2;                  // 0: head h0, 1: head h0+1
+        const int g = warp >> 2;                   // warpgroup 0..3
+        const int hs = g >> 1, c = g & 1;          // head within the pair, column half
         const int wq = warp & 3;                   // TMEM lane quarter = 32-row quarter of the block
         const int r = wq * 32 + lane;              // row in block == TMEM lane
-        const int h = h0 + wg;
+        const int h = h0 + hs;
         const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
         const float A2 = prm.d[slot].A[h] * kLog2e;   // log2 units: exp(a) = exp2(a * log2 e)
         const float Dh = prm.d[slot].D ? prm.d[slot].D[h] : 0.f;
-        float *cs2 = cs2_s + wg * kBlk, *dts = dt_s + wg * kBlk, *wtab = wtab_s + wg * 4 * kBlk;
-        uint8_t *wx_tile = sm + kOffWX + wg * kTileBytes;
-        uint8_t *sp_tile = sm + kOffSP + wg * kTileBytes;
+        float *cs2 = cs2_s + hs * kBlk, *dts = dt_s + hs * kBlk, *wtab = wtab_s + hs * 4 * kBlk;
+        uint8_t *wx_tile = sm + kOffWX + hs * kTileBytes;
+        uint8_t *sp_tile = sm + kOffSP + hs * kTileBytes;
         float *e1_s = reinterpret_cast<float *>(sm + kOffE1);   // [2][128]
+        const uint32_t colS = kColS + 64 * hs + 32 * c, colST = kColST + 64 * hs + 32 * c,
+                       colY = kColY + 64 * hs + 32 * c;
 
         for (int j = 0; j < nblk; ++j) {
             if (__any_sync(0xffffffffu, *abort_flag)) break;
@@ -599,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             // x, dt of this block
             if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 41)) break;
             SSD_TRACE_PT(warp, j, 1);
-            uint8_t *xt = sm + kOffX + st * kStageBytes + wg * kTileBytes;
+            uint8_t *xt = sm + kOffX + st * kStageBytes + hs * kTileBytes;
             const __nv_bfloat16 *dtt =
                 reinterpret_cast<const __nv_bfloat16 *>(sm + kOffX + st * kStageBytes + 2 * kTileBytes);
             const float dtr = __bfloat162float(dtt[r * 8 + (h & 7)]);
@@ -637,24 +643,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             }
             const float c2 = A2 * (base + s);                 // cs_r * log2 e
             const float cl2 = A2 * total;                     // cs at the block's last scan position
-            cs2[r] = c2;
-            dts[r] = dtr;
-            // column factors of the off-diagonal quarters: W[q][s] = exp(cs_ref(q) - cs_s) dt_s
+            if (c == 0) {
+                // decay tables of this head (written once; both halves compute the same values)
+                cs2[r] = c2;
+                dts[r] = dtr;
+                // column factors of the off-diagonal quarters: W[q][s] = exp(cs_ref(q) - cs_s) dt_s
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const bool off = dir > 0 ? wq < q : wq > q;    // this row is a source for quarter q
-                if (off) wtab[q * kBlk + r] = exp2f(ref2[q] - c2) * dtr;
+                for (int q = 0; q < 4; ++q) {
+                    const bool off = dir > 0 ? wq < q : wq > q;    // this row is a source for quarter q
+                    if (off) wtab[q * kBlk + r] = exp2f(ref2[q] - c2) * dtr;
+                }
+                const float ref_own = wq == 0 ? ref2[0] : wq == 1 ? ref2[1] : wq == 2 ? ref2[2] : ref2[3];
+                e1_s[hs * kBlk + r] = exp2f(c2 - ref_own);      // row factor towards the quarter boundary
             }
-            const float ref_own = wq == 0 ? ref2[0] : wq == 1 ? ref2[1] : wq == 2 ? ref2[2] : ref2[3];
-            e1_s[wg * kBlk + r] = exp2f(c2 - ref_own);      // row factor towards the quarter boundary
             const float wr = exp2f(cl2 - c2) * dtr;           // weight of row r in the block's state
             const float er = exp2f(c2);                       // decay from the block start to row r
             const float ablk = exp2f(cl2);                    // decay across the whole block
             SSD_TRACE_PT(warp, j, 5);
 
-            // w (.) x -> wX tile (same swizzled layout as the X tile)
+            // w (.) x -> wX tile (same swizzled layout as the X tile), this half's 4 chunks
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int qq = 0; qq < 4; ++qq) {
+                const int q = 4 * c + qq;
                 const uint4 v = *reinterpret_cast<const uint4 *>(xt + swz(r, q));
                 uint4 o;
                 o.x = pack_bf16(bf16lo(v.x) * wr, bf16hi(v.x) * wr);
@@ -663,17 +673,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 o.w = pack_bf16(bf16lo(v.w) * wr, bf16hi(v.w) * wr);
                 *reinterpret_cast<uint4 *>(wx_tile + swz(r, q)) = o;
             }
-            SSD_TRACE_PT(warp, j, 6);
             fence_async_smem();                // w(.)x is read by the tensor core
             SSD_TRACE_PT(warp, j, 8);
             if (lane == 0) mbar_arrive(bar(B_WXREADY));
 
             // M_h = G (.) decay (.) dt over the causal triangle, bf16, for both heads.  This
-            // warpgroup takes every other 16-source K-step; the two heads' bf16 results for a
-            // K-step replace the 16 float32 G columns they were computed from.
+            // warpgroup takes K-steps g and g + 4; the two heads' bf16 results for a K-step
+            // replace the 16 float32 G columns they were computed from.
             if (!mbar_wait(bar(B_GFULL), j & 1, MASK, abort_flag, prm.status, 42)) break;
-            // both heads' decay tables of this block are read below: the other warpgroup must have
-            // finished writing them (all 8 warps arrive on this barrier after their preparation)
+            // both heads' decay tables of this block are read below: every warp arrives on this
+            // barrier after its preparation
             if (!mbar_wait(bar(B_WXREADY), j & 1, MASK, abort_flag, prm.status, 48)) break;
             SSD_TRACE_PT(warp, j, 9);
             tc_fence_after();
@@ -681,15 +690,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 const float c2h[2] = {cs2_s[r], cs2_s[kBlk + r]};
                 const float e1h[2] = {e1_s[r], e1_s[kBlk + r]};
 #pragma unroll 1
-                for (int ks = wg; ks < 8; ks += 2) {
+                for (int ks = g; ks < 8; ks += 4) {
                     const int sq = ks >> 1;                          // source quarter
                     const bool offd = dir > 0 ? sq < wq : sq > wq;
                     const bool diag = sq == wq;
                     uint32_t m[16];
                     if (offd || diag) {
-                        float g[16];
-                        tmem_ld16(tl + kColG + 16 * ks, g);
-                        tmem_wait_ld();
+                        float gv[16];
+                        tmem_ld16(tl + kColG + 16 * ks, gv);
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             if (offd) {
@@ -697,9 +705,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
 #pragma unroll
                                 for (int i = 0; i < 4; ++i) {
                                     const float4 wv = *reinterpret_cast<const float4 *>(wrow + 4 * i);
-                                    m[8 * hh + 2 * i] = pack_bf16(g[4 * i] * wv.x * e1h[hh], g[4 * i + 1] * wv.y * e1h[hh]);
+                                    m[8 * hh + 2 * i] = pack_bf16(gv[4 * i] * wv.x * e1h[hh], gv[4 * i + 1] * wv.y * e1h[hh]);
                                     m[8 * hh + 2 * i + 1] =
-                                        pack_bf16(g[4 * i + 2] * wv.z * e1h[hh], g[4 * i + 3] * wv.w * e1h[hh]);
+                                        pack_bf16(gv[4 * i + 2] * wv.z * e1h[hh], gv[4 * i + 3] * wv.w * e1h[hh]);
                                 }
                             } else {
                                 const float *csrc = cs2_s + hh * kBlk + 16 * ks, *dsrc = dt_s + hh * kBlk + 16 * ks;
@@ -713,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                                     for (int e = 0; e < 4; ++e) {
                                         const int sidx = 16 * ks + 4 * i + e;
                                         const bool in = dir > 0 ? sidx <= r : sidx >= r;
-                                        mv[e] = in ? g[4 * i + e] * exp2f(c2h[hh] - cc[e]) * dd[e] : 0.f;
+                                        mv[e] = in ? gv[4 * i + e] * exp2f(c2h[hh] - cc[e]) * dd[e] : 0.f;
                                     }
                                     m[8 * hh + 2 * i] = pack_bf16(mv[0], mv[1]);
                                     m[8 * hh + 2 * i + 1] = pack_bf16(mv[2], mv[3]);
@@ -727,14 +735,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                     tmem_st16(tl + kColG + 16 * ks, m);
                 }
             }
-            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_MREADY));
             SSD_TRACE_PT(warp, j, 10);
 
-            // state: S' <- exp(cs_last) S' + S; thread r holds state row n = r, the float32 state
-            // lives in TMEM and a bf16 copy goes to smem as the next block's MMA operand
+            // state: S' <- exp(cs_last) S' + S; thread r holds state row n = r (this half's 32
+            // columns), the float32 state lives in TMEM and a bf16 copy goes to smem as the next
+            // block's MMA operand
             if (!mbar_wait(bar(B_SFULL), j & 1, MASK, abort_flag, prm.status, 43)) break;
             SSD_TRACE_PT(warp, j, 11);
             // the previous state tile must have been consumed by this block's Y = C S'^T
@@ -743,19 +751,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 break;
             tc_fence_after();
 #pragma unroll 1
-            for (int qd = 0; qd < 4; ++qd) {
+            for (int qd = 0; qd < 2; ++qd) {
                 float sv[16], pv[16];
                 if (j > 0) {
-                    tmem_ld16x2(tl + kColS + 64 * wg + 16 * qd, tl + kColST + 64 * wg + 16 * qd, sv, pv);
+                    tmem_ld16x2(tl + colS + 16 * qd, tl + colST + 16 * qd, sv, pv);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) sv[i] = fmaf(ablk, pv[i], sv[i]);
                 } else {
-                    tmem_ld16(tl + kColS + 64 * wg + 16 * qd, sv);
+                    tmem_ld16(tl + colS + 16 * qd, sv);
                 }
                 uint32_t w16[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) w16[i] = __float_as_uint(sv[i]);
-                tmem_st16(tl + kColST + 64 * wg + 16 * qd, w16);
+                tmem_st16(tl + colST + 16 * qd, w16);
                 if (j + 1 < nblk) {
 #pragma unroll
                     for (int qq = 0; qq < 2; ++qq) {
@@ -764,11 +772,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                         o.y = pack_bf16(sv[8 * qq + 2], sv[8 * qq + 3]);
                         o.z = pack_bf16(sv[8 * qq + 4], sv[8 * qq + 5]);
                         o.w = pack_bf16(sv[8 * qq + 6], sv[8 * qq + 7]);
-                        *reinterpret_cast<uint4 *>(sp_tile + swz(r, 2 * qd + qq)) = o;
+                        *reinterpret_cast<uint4 *>(sp_tile + swz(r, 4 * c + 2 * qd + qq)) = o;
                     }
                 }
             }
-            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_SEMPTY));
@@ -784,16 +791,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             if (j >= 1) {
                 if (!mbar_wait(bar(B_YOFFFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 45)) break;
                 tc_fence_after();
+                float yv[32];
+                tmem_ld32(tl + colY, yv);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float yv[32];
-                    tmem_ld32(tl + kColY + 64 * wg + 32 * half, yv);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) yv[i] *= er;
-                    tmem_st32(tl + kColY + 64 * wg + 32 * half, yv);
-                }
-                tmem_wait_st();
+                for (int i = 0; i < 32; ++i) yv[i] *= er;
+                tmem_st32(tl + colY, yv);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_RSREADY));
@@ -805,13 +807,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             if (!mbar_wait(bar(B_YFULL), j & 1, MASK, abort_flag, prm.status, 46)) break;
             SSD_TRACE_PT(warp, j, 16);
             tc_fence_after();
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            {
                 float yv[32];
-                tmem_ld32(tl + kColY + 64 * wg + 32 * half, yv);
+                tmem_ld32(tl + colY, yv);
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
-                    const int q = 4 * half + qq;
+                    const int q = 4 * c + qq;
                     const uint4 xv = *reinterpret_cast<const uint4 *>(xt + swz(r, q));
                     const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
                     float o[8];
@@ -833,7 +834,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(bar(B_YEMPTY));
-                mbar_arrive(bar(B_TILE0 + wg));
+                mbar_arrive(bar(B_TILE0 + hs));
             }
             SSD_TRACE_PT(warp, j, 21);
         }
