@@ -12,6 +12,8 @@ Entry points (same names as the C ABI):
   ssd_scan(x, dt, A, B, C, D=None, direction=1, chunk=256)   one direction
   bidir_ssd(fwd, rev, chunk=256)                              y_fwd + flip(scan(flip(.)))
   r2l_block_scan(p, s, residual, chunk=32)                    residual + s * y_rev
+  bidir_ssd_noalloc(fwd, rev, out, chunk=256)                 bidir_ssd into a caller-owned `out`,
+                                                              scratch inside the library
 """
 from __future__ import annotations
 
@@ -20,7 +22,7 @@ import os
 
 import torch
 
-__all__ = ["ssd_scan", "bidir_ssd", "r2l_block_scan", "workspace_bytes", "path_for",
+__all__ = ["ssd_scan", "bidir_ssd", "r2l_block_scan", "bidir_ssd_noalloc", "noalloc_status", "workspace_bytes", "path_for",
            "kernel_launches", "workspace_status", "SSDError", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -62,6 +64,8 @@ lib.bidir_ssd.restype = ctypes.c_int
 lib.r2l_block_scan.argtypes = [_SP, _PP, ctypes.c_float, _VP, ctypes.c_int, _VP, _VP, _SZ, _VP]
 lib.r2l_block_scan.restype = ctypes.c_int
 lib.ssd_workspace_status.argtypes = [_VP, _SZ, _VP]
+lib.bidir_ssd_noalloc.argtypes = [_SP, _PP, _PP, ctypes.c_int, _VP, _VP, ctypes.POINTER(ctypes.c_void_p)]
+lib.bidir_ssd_noalloc.restype = ctypes.c_int
 lib.ssd_workspace_status.restype = ctypes.c_int
 lib.ssd_status_string.argtypes = [ctypes.c_int]
 lib.ssd_status_string.restype = ctypes.c_char_p
@@ -197,3 +201,34 @@ def workspace_status(workspace) -> None:
     """Raise SSDError if a bounded device-side wait gave up in a call that used ``workspace``."""
     dev = workspace.device
     _check(lib.ssd_workspace_status(workspace.data_ptr(), workspace.numel(), _stream(dev)))
+
+
+def bidir_ssd_noalloc(fwd: dict, rev: dict, out, chunk: int = 256) -> int:
+    """``bidir_ssd`` for callers that cannot allocate device memory at the call.
+
+    Writes y into ``out`` (preallocated, contiguous, shaped like ``fwd["x"]``).
+    The scratch the kernels need is a fixed array inside the library, so
+    neither this function nor the library allocates anything; shapes whose
+    scratch exceeds that array raise SSDError (unsupported shape).  Calls
+    that overlap on the GPU share the array and race: order them on one
+    stream.  Returns the device address of the scratch's status area, for
+    ``noalloc_status``.
+    """
+    shape = _shape_of(fwd["x"], fwd["B"])
+    if tuple(rev["x"].shape) != tuple(fwd["x"].shape) or tuple(rev["B"].shape) != tuple(fwd["B"].shape):
+        raise ValueError("forward and reverse parameters must have the same shapes")
+    x = fwd["x"]
+    if out.shape != x.shape or out.dtype != x.dtype or out.device != x.device or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {x.dtype} tensor of shape {tuple(x.shape)} on {x.device}")
+    pf = _params(x, fwd["dt"], fwd["A"], fwd["B"], fwd["C"], fwd.get("D"))
+    pr = _params(rev["x"], rev["dt"], rev["A"], rev["B"], rev["C"], rev.get("D"))
+    area = ctypes.c_void_p()
+    _check(lib.bidir_ssd_noalloc(ctypes.byref(shape), ctypes.byref(pf), ctypes.byref(pr), int(chunk),
+                                 out.data_ptr(), _stream(x.device), ctypes.byref(area)))
+    return int(area.value or 0)
+
+
+def noalloc_status(area: int, device=None) -> None:
+    """Raise SSDError if a bounded device-side wait gave up in the last ``bidir_ssd_noalloc`` call."""
+    if area:
+        _check(lib.ssd_workspace_status(area, 256, _stream(device or torch.cuda.current_device())))

@@ -274,3 +274,65 @@ ssd_status ssd_debug_fault(int mode, double wait_limit_seconds) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// bidir_ssd_noalloc: the bidirectional mixer with its scratch in a fixed
+// device array of this library instead of a caller-supplied workspace.
+
+namespace {
+
+// The scratch: status area first, then what the chosen path keeps between the
+// kernels (hand-off flags on the tensor-core path, chunk decays and states on
+// the SIMT path).  Zero at module load; the parts that must start at zero are
+// cleared again at every call.
+__device__ __align__(256) unsigned char g_noalloc_scratch[SSD_NOALLOC_MAX_SCRATCH_BYTES];
+
+// Its device address, per device, looked up by the first call on that device.
+std::atomic<void *> g_noalloc_ptr[64];
+
+ssd_status noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(SSD_ERR_UNSUPPORTED, "device ordinal %d above 63", dev);
+    void *ptr = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+    if (!ptr) {
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the scratch array");
+        if (!ptr) return fail(SSD_ERR_CUDA, "cudaGetSymbolAddress returned NULL");
+        g_noalloc_ptr[dev].store(ptr, std::memory_order_release);
+    }
+    *out = ptr;
+    return SSD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+ssd_status bidir_ssd_noalloc(const ssd_shape *shape, const ssd_params *fwd, const ssd_params *rev, int chunk,
+                             void *y, void *stream, void **status_area) {
+    g_err.clear();
+    if (status_area) *status_area = nullptr;
+    ssd_status st = check_shape(shape, chunk);
+    if (st != SSD_OK) return st;
+    if (shape->batch == 0 || shape->seqlen == 0) return SSD_OK;
+    const size_t need = path_ws_bytes(shape, chunk);
+    if (need > (size_t)SSD_NOALLOC_MAX_SCRATCH_BYTES)
+        return fail(SSD_ERR_UNSUPPORTED,
+                    "this shape needs %zu bytes of scratch, more than the %zu the no-allocation entry point "
+                    "holds; call bidir_ssd with a workspace instead",
+                    need, (size_t)SSD_NOALLOC_MAX_SCRATCH_BYTES);
+    void *ws = nullptr;
+    if ((st = noalloc_scratch(&ws)) != SSD_OK) return st;
+    // the status word, and on the tensor-core path the hand-off flags, start at zero
+    const size_t clear = choose_path(shape, chunk) == 1 ? need : kStatusBytes;
+    cudaError_t e = cudaMemsetAsync(ws, 0, clear, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "scratch clear");
+    st = bidir_ssd(shape, fwd, rev, chunk, y, ws, (size_t)SSD_NOALLOC_MAX_SCRATCH_BYTES, stream);
+    if (st == SSD_OK && status_area) *status_area = ws;
+    return st;
+}
+
+}  // extern "C"
+

@@ -120,6 +120,38 @@ ssd_status r2l_block_scan(const ssd_shape *shape, const ssd_params *p, float s,
                           const void *residual, int chunk, void *out,
                           void *workspace, size_t workspace_bytes, void *stream);
 
+/* Largest scratch, in bytes, that bidir_ssd_noalloc holds (status area plus
+ * what the chosen path needs; ssd_workspace_bytes gives that figure). */
+#define SSD_NOALLOC_MAX_SCRATCH_BYTES (2u << 20)
+
+/* bidir_ssd without a workspace argument.  The pages have no counterpart: it
+ * is a convenience of this library for callers that cannot allocate device
+ * memory at the point of the call -- a host program whose device memory is
+ * all handed out up front (a serving engine's fixed pool), or a latency-bound
+ * loop that cannot afford cudaMalloc/cudaFree, which may synchronise the whole
+ * device.  The scratch is a fixed 2 MiB array inside this library (one per
+ * device); nothing is allocated, by this call or by the library.
+ *
+ * Same operation, arguments, layouts and results as bidir_ssd.  Shapes whose
+ * scratch (ssd_workspace_bytes) exceeds SSD_NOALLOC_MAX_SCRATCH_BYTES are
+ * refused with SSD_ERR_UNSUPPORTED before anything is launched; use
+ * bidir_ssd with a workspace for them.  Each call first clears, on `stream`,
+ * the part of the scratch that must start at zero (the status word and the
+ * forward/reverse hand-off flags).
+ *
+ * The first call on a device (with that device current) looks up the
+ * array's device address once; make that first call before any stream
+ * capture.  All calls on one device share the one array: two calls whose
+ * work overlaps on the GPU (different streams, no ordering between them) race
+ * on it and give wrong results.  Order them on one stream, or with events.
+ *
+ * status_area (may be NULL) receives the device address of the scratch's
+ * 256-byte status area; pass it to ssd_workspace_status(area, 256, stream)
+ * to learn whether a bounded device-side wait gave up.  The next call clears
+ * it. */
+ssd_status bidir_ssd_noalloc(const ssd_shape *shape, const ssd_params *fwd, const ssd_params *rev,
+                             int chunk, void *y, void *stream, void **status_area);
+
 /* Waits for `stream`, then reads and clears the device status word in
  * `workspace` (SSD_OK, or SSD_ERR_TIMEOUT if a bounded device-side wait gave
  * up during an earlier call that used this workspace). */
