@@ -3,19 +3,22 @@
 //
 // One CTA owns (batch b, head pair {h0, h0+1}, direction) and walks the
 // sequence in scan order in blocks of 128 tokens, carrying the float32 state
-// of both heads in registers.  Per block (rows r = 0..127 in memory order,
-// TMEM lane r = token t0 + r), with cs the cumulative A*dt in scan order:
+// of both heads in TMEM.  Per block (rows r = 0..127 in memory order, TMEM
+// lane r = token t0 + r), with cs the cumulative A*dt in scan order:
 //
-//   G    = C B^T                      tcgen05, shared by both heads   TMEM [0,128)
-//   M_h  = G (.) decay_h (.) dt        CUDA cores, bf16, written over the G columns it
-//                                      came from (A operand of the next MMA)
-//   S^T  = B^T (w (.) X)               tcgen05, N = 2 heads x 64       TMEM [128,256)
-//   Y    = C S'^T_prev                 tcgen05, N = 2 heads x 64       TMEM [256,384)
-//   Y   *= exp(cs_r) per row           CUDA cores (TMEM ld/st)
-//   Y   += M_h X_h                     tcgen05, A from TMEM, N = 64
-//   y    = Y + D x                     CUDA cores -> smem -> coalesced rows
-//   S'   = exp(cs_last) S' + S         CUDA cores; float32 state in TMEM [384,512),
-//                                      bf16 copy in smem for the next block
+//   tables: cs, dt, decay factors      CUDA cores, from a dt ring loaded one block ahead;
+//                                      written during the previous block's Y_diag MMA
+//                                      (smem, 2 buffers)
+//   G      = C B^T                     tcgen05, shared by both heads   TMEM [0,128)
+//   M_h    = G (.) decay_h (.) dt      CUDA cores, bf16, written over the G columns it
+//                                      came from (A operand of the intra-block MMA)
+//   Y_off  = C S'^T                    tcgen05, N = 2 heads x 64       TMEM [384,512)
+//                                      (S' = state entering the block, bf16 copy in smem)
+//   S'    <- exp(cs_last) S'           CUDA cores, in place in TMEM [128,256)
+//   S'    += B^T (w (.) X)             tcgen05, N = 2 heads x 64, accumulates into S'
+//   Y_diag = M_h X_h                   tcgen05, A from TMEM, N = 64    TMEM [256,384)
+//   y      = Y_diag + exp(cs_r) Y_off + D x
+//                                      CUDA cores -> smem tile -> TMA store
 //
 // This is the chunked evaluation of the recurrence S <- exp(dt A) S +
 // dt x (outer) B, y = C.S + D x that the Mamba-2 layers of the DiffuMamba
@@ -30,8 +33,11 @@
 // the output row r, exp(cs_r - cs_s) = exp(cs_r - cs_ref) * exp(cs_ref - cs_s)
 // with ref the quarter boundary between them; both factors are <= 1, so the
 // product never overflows, and the mask becomes (row factor) x (column table)
-// with no exponential per element.  Only the 32 x 32 diagonal sub-blocks take
-// a direct exponential.
+// with no exponential per element.  Inside the diagonal quarter the same is done
+// at 16-row granularity: exp(cs_r - cs_s) = R16[r] * D16[s] within one 16-row
+// sub-block (masked to the causal half) and R16[r] * O16[s] from the sub-block
+// before.  D16 grows across its sub-block, so a sub-block whose decay exceeds
+// 2^120 falls back to one exponential per element.
 //
 // Bidirectional mixer in one launch.  The CTAs of the forward and reverse
 // scans of one head pair are neighbours in the grid.  For every output block
@@ -66,34 +72,55 @@ namespace {
 
 constexpr int kBlk = 128;            // tokens per block (MMA M)
 constexpr int kP = 64, kN = 128;
-constexpr int kThreads = 640;        // warps 0-15: four warpgroups; 16: TMA; 17: MMA + TMEM; 18-19: y stores
+constexpr int kThreads = 640;        // warps 0-15: four warpgroups; 16: TMA; 17: MMA + TMEM;
+                                     // 18-19: decay tables and y stores, one warp per head
 constexpr int kWarpTma = 16, kWarpMma = 17, kWarpStore = 18;
 constexpr uint32_t kTileBytes = kBlk * 64 * 2;        // one [128][64] bf16 swizzled tile = 16 KB
 constexpr uint32_t kDtBytes = kBlk * 8 * 2;           // dt box: 128 tokens x 8 heads, bf16
-constexpr uint32_t kStageBytes = 2 * kTileBytes + kDtBytes;   // x of 2 heads + dt = 34 KB
+constexpr uint32_t kStageBytes = 2 * kTileBytes;      // x of 2 heads = 32 KB
 
-// TMEM column map
-constexpr uint32_t kColG = 0, kColS = 128, kColY = 256, kColST = 384;
+// TMEM column map: G (then M over it), running state S', Y_diag, Y_off
+constexpr uint32_t kColG = 0, kColST = 128, kColYD = 256, kColYO = 384;
 
 // shared memory map (offsets from a 1024-aligned base)
-constexpr uint32_t kOffX = 0;                          // 2 stages: [x h0 | x h1 | dt]
+constexpr uint32_t kOffX = 0;                          // 2 stages: [x h0 | x h1]
 constexpr uint32_t kOffB = kOffX + 2 * kStageBytes;    // 2 sub-tiles (n 0..63, 64..127)
 constexpr uint32_t kOffC = kOffB + 2 * kTileBytes;
 constexpr uint32_t kOffWX = kOffC + 2 * kTileBytes;    // 2 heads
 constexpr uint32_t kOffSP = kOffWX + 2 * kTileBytes;   // 2 heads, rows = state index n
-constexpr uint32_t kOffCS = kOffSP + 2 * kTileBytes;   // float cs2[2][128], dt[2][128]
-constexpr uint32_t kOffW = kOffCS + 4 * kBlk * 4;      // float W[2][4][128]: off-diagonal column factors
-constexpr uint32_t kOffE1 = kOffW + 2 * 4 * kBlk * 4;  // float e1[2][128]: off-diagonal row factors
-constexpr uint32_t kOffBar = kOffE1 + 2 * kBlk * 4;
-constexpr uint32_t kNumBars = 22;
+// Decay tables of one block, both heads (float, log2 units where noted), double-buffered by
+// block parity: the CUDA-core warps write block j+1's while the tensor core computes block
+// j's intra-block output.
+constexpr uint32_t kTabCS = 0;                          // cs2[2][128]: cs_r * log2 e, scan order
+constexpr uint32_t kTabDT = kTabCS + 2 * kBlk;          // dt[2][128]
+constexpr uint32_t kTabW = kTabDT + 2 * kBlk;           // W[2][4][128]: off-diagonal column factors
+constexpr uint32_t kTabE1 = kTabW + 8 * kBlk;           // e1[2][128]: off-diagonal row factors
+constexpr uint32_t kTabWR = kTabE1 + 2 * kBlk;          // wr[2][128]: weight of row r in the block state
+constexpr uint32_t kTabER = kTabWR + 2 * kBlk;          // er[2][128]: decay from the block start to row r
+constexpr uint32_t kTabR16 = kTabER + 2 * kBlk;        // R16[2][128]: row factor to the 16-row sub-block start
+constexpr uint32_t kTabD16 = kTabR16 + 2 * kBlk;       // D16[2][128]: column factor, same sub-block
+constexpr uint32_t kTabO16 = kTabD16 + 2 * kBlk;       // O16[2][128]: column factor, next sub-block
+constexpr uint32_t kTabBig = kTabO16 + 2 * kBlk;       // big[2][8]: sub-block needs exact exponentials
+constexpr uint32_t kTabA = kTabBig + 16;               // ablk[2]: decay across the block
+constexpr uint32_t kTabFloats = kTabA + 4;
+constexpr uint32_t kOffTab = kOffSP + 2 * kTileBytes;   // 2 buffers
+constexpr uint32_t kOffDT = (kOffTab + 2 * kTabFloats * 4 + 127) / 128 * 128;   // dt ring, 2 slots
+constexpr uint32_t kOffBar = kOffDT + 2 * kDtBytes;
+constexpr uint32_t kNumBars = 24;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
 static_assert(kStageBytes % 1024 == 0, "x tiles must stay 1024-byte aligned");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
+// Every barrier completes at most once more before each of its waiters has
+// passed its wait for the previous completion (a waiter tells completions
+// apart by phase parity only).  Where a producer could otherwise run two
+// completions ahead, the barrier is per buffer: B_TILE (per head and x stage),
+// B_TABREADY (per table buffer), B_DTFULL and B_DTEMPTY (per dt slot).
 enum Bar {
-    B_XFULL0 = 0, B_XFULL1, B_XEMPTY0, B_XEMPTY1, B_BCFULL, B_BCEMPTY, B_GFULL, B_GEMPTY,
-    B_WXREADY, B_SFULL, B_SEMPTY, B_SPREADY, B_YOFFFULL, B_MREADY, B_RSREADY, B_YFULL, B_YEMPTY, B_DONE, B_WG0, B_WG1, B_TILE0, B_TILE1
+    B_XFULL0 = 0, B_XFULL1, B_XEMPTY0, B_XEMPTY1, B_BCFULL, B_BCEMPTY, B_GFULL, B_WXREADY, B_SPREADY, B_STFULL,
+    B_MREADY, B_YFULL, B_YEMPTY, B_DONE, B_TILE00, B_TILE01, B_TILE10, B_TILE11, B_TABREADY0, B_TABREADY1,
+    B_DTFULL0, B_DTFULL1, B_DTEMPTY0, B_DTEMPTY1
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -105,9 +132,7 @@ constexpr int kTraceWarps = 20, kTraceBlocks = 8, kTracePts = 24;
 __device__ unsigned long long g_trace[kTraceWarps][kTraceBlocks][kTracePts];
 __device__ __forceinline__ void trace_pt(int w, int j, int k) {
     if (blockIdx.x == 0 && j < kTraceBlocks && (threadIdx.x & 31) == 0) {
-        unsigned long long t;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-        g_trace[w][j][k] = t;
+        g_trace[w][j][k] = (unsigned long long)clock64();   // SM cycles: exact within the CTA
     }
 }
 #define SSD_TRACE_PT(w, j, k) trace_pt(w, j, k)
@@ -325,14 +350,25 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v) {
     tmem_st16(taddr, r);
     tmem_st16(taddr + 16, r + 16);
 }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // .x = lo (low 16 bits), .y = hi
     return *reinterpret_cast<uint32_t *>(&v);
 }
 __device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
+// 2^x by the PTX ex2.approx.ftz instruction (relative error about 2^-22; results below
+// 2^-126 flush to zero, far below what a bf16 output resolves)
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// (lo, hi) bf16 pair times a bf16 scalar, one packed multiply rounded to nearest even
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t v, uint32_t w2) {
+    uint32_t o;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(o) : "r"(v), "r"(w2));
+    return o;
+}
 __device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
 // byte offset of 16-byte chunk q of row r in a [rows][64] bf16 tile with 128-byte swizzle
@@ -375,9 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
     auto bar = [&](int i) { return sbase + kOffBar + 8u * i; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);
-    float *cs2_s = reinterpret_cast<float *>(sm + kOffCS);          // [2][128] cs * log2(e)
-    float *dt_s = cs2_s + 2 * kBlk;                                  // [2][128] dt
-    float *wtab_s = reinterpret_cast<float *>(sm + kOffW);           // [2][4][128]
+    float *tab_s = reinterpret_cast<float *>(sm + kOffTab);         // [2 buffers][kTabFloats]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int npairs = prm.H / 2;
@@ -393,12 +427,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         *reinterpret_cast<volatile long long *>(abort_flag + 1) = prm.wait_cycles;
-        // arrival counts: 8 = one per CUDA-core warp, 4 = one per warp of a warpgroup, 1 = one thread / commit
         // arrival counts: 16 = one per CUDA-core warp, 8 = one per warp of a head's two
         // warpgroups, 2 = one per store warp, 1 = one thread / one MMA commit
-        constexpr uint32_t k16 = (1u << B_GEMPTY) | (1u << B_WXREADY) | (1u << B_SEMPTY) | (1u << B_SPREADY) |
-                                 (1u << B_MREADY) | (1u << B_RSREADY) | (1u << B_YEMPTY);
-        constexpr uint32_t k8 = (1u << B_TILE0) | (1u << B_TILE1);
+        constexpr uint32_t k16 = (1u << B_WXREADY) | (1u << B_SPREADY) | (1u << B_MREADY) | (1u << B_YEMPTY) |
+                                 (1u << B_TABREADY0) | (1u << B_TABREADY1) | (1u << B_DTEMPTY0) | (1u << B_DTEMPTY1);
+        constexpr uint32_t k8 = (1u << B_TILE00) | (1u << B_TILE01) | (1u << B_TILE10) | (1u << B_TILE11);
         constexpr uint32_t k2 = (1u << B_XEMPTY0) | (1u << B_XEMPTY1);
         for (int i = 0; i < (int)kNumBars; ++i)
             mbar_init(bar(i), (k16 >> i) & 1 ? 16 : (k8 >> i) & 1 ? 8 : (k2 >> i) & 1 ? 2 : 1);
@@ -423,7 +456,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map_dt)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map_b)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map_c)) : "memory");
-            for (int j = 0; j < nblk; ++j) {
+            // dt of block jj into slot jj & 1 of the dt ring (one block ahead of x)
+            int dt_issued = 0, x_issued = 0;
+            auto load_dt = [&](int jj) -> bool {
+                const int sl = jj & 1;
+                if (jj >= 2 && !mbar_wait(bar(B_DTEMPTY0 + sl), ((jj >> 1) - 1) & 1, MASK, abort_flag, prm.status, 13))
+                    return false;
+                const int cmj = dir > 0 ? jj : nblk - 1 - jj;
+                mbar_expect_tx(bar(B_DTFULL0 + sl), kDtBytes);
+                tma_load_2d(sbase + kOffDT + sl * kDtBytes, map_dt, h0 & ~7, b * L + cmj * kBlk, bar(B_DTFULL0 + sl));
+                dt_issued = jj + 1;
+                return true;
+            };
+            bool ok = load_dt(0);
+            for (int j = 0; j < nblk && ok; ++j) {
                 const int cm = dir > 0 ? j : nblk - 1 - j;
                 const int row = b * L + cm * kBlk;
                 const int st = j & 1;
@@ -433,7 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 mbar_expect_tx(bar(B_XFULL0 + st), kStageBytes);
                 for (int h = 0; h < 2; ++h)
                     tma_load_2d(stage + h * kTileBytes, map_x, (h0 + h) * kP, row, bar(B_XFULL0 + st));
-                tma_load_2d(stage + 2 * kTileBytes, map_dt, h0 & ~7, row, bar(B_XFULL0 + st));
+                x_issued = j + 1;
+                if (j + 1 < nblk && !load_dt(j + 1)) break;
                 if (j >= 1 && !mbar_wait(bar(B_BCEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 12)) break;
                 SSD_TRACE_PT(kWarpTma, j, 1);
                 mbar_expect_tx(bar(B_BCFULL), 4 * kTileBytes);
@@ -443,12 +490,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 }
                 issued = j + 1;
             }
-            if (*abort_flag && issued > 0) {
-                // let copies still in flight land before the CTA exits
-                const int j = issued - 1;
-                mbar_drain(bar(B_XFULL0 + (j & 1)), (j >> 1) & 1, prm.wait_cycles);
-                if (j >= 1) mbar_drain(bar(B_XFULL0 + ((j - 1) & 1)), ((j - 1) >> 1) & 1, prm.wait_cycles);
-                mbar_drain(bar(B_BCFULL), j & 1, prm.wait_cycles);
+            if (*abort_flag) {
+                // let copies still in flight land before the CTA exits: the last two x stages,
+                // the last B/C load and the last two dt slots
+                for (int jj = x_issued - 1; jj >= 0 && jj >= x_issued - 2; --jj)
+                    mbar_drain(bar(B_XFULL0 + (jj & 1)), (jj >> 1) & 1, prm.wait_cycles);
+                if (issued > 0) mbar_drain(bar(B_BCFULL), (issued - 1) & 1, prm.wait_cycles);
+                for (int jj = dt_issued - 1; jj >= 0 && jj >= dt_issued - 2; --jj)
+                    mbar_drain(bar(B_DTFULL0 + (jj & 1)), (jj >> 1) & 1, prm.wait_cycles);
             }
         }
     } else if (warp == kWarpMma) {
@@ -472,48 +521,47 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                     mma_ss(tmem + kColG, sdesc(aC + off, 16, 1024), sdesc(aB + off, 16, 1024), id_g, ks > 0);
                 }
                 mma_commit(bar(B_GFULL));
-                // S^T = B^T (w x)  (M = n, N = (head, p), K = rows); both operands MN-major
-                if (!mbar_wait(bar(B_WXREADY), j & 1, MASK, abort_flag, prm.status, 23)) break;
-                if (j >= 1 && !mbar_wait(bar(B_SEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 24)) break;
-                SSD_TRACE_PT(kWarpMma, j, 1);
-                tc_fence_after();
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t off = ks * 2048;
-                    mma_ss(tmem + kColS, sdesc(aB + off, kTileBytes, 1024), sdesc(aWX + off, kTileBytes, 1024), id_s,
-                           ks > 0);
-                }
-                mma_commit(bar(B_SFULL));
-                // Y = C S'^T of the state entering this block (M = rows, N = (head, p), K = n)
                 if (j >= 1) {
-                    if (!mbar_wait(bar(B_SPREADY), (j - 1) & 1, MASK, abort_flag, prm.status, 25)) break;
-                    if (!mbar_wait(bar(B_YEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 26)) break;
-                    SSD_TRACE_PT(kWarpMma, j, 2);
+                    // Y_off = C S'^T of the state entering this block (M = rows, N = (head, p), K = n);
+                    // SP holds bf16(S') and the float32 state has been scaled by this block's decay
+                    if (!mbar_wait(bar(B_SPREADY), (j - 1) & 1, MASK, abort_flag, prm.status, 23)) break;
+                    // the previous block's epilogue has read both Y accumulators
+                    if (!mbar_wait(bar(B_YEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 24)) break;
+                    SSD_TRACE_PT(kWarpMma, j, 1);
                     tc_fence_after();
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t offc = (ks >> 2) * kTileBytes + (ks & 3) * 32;
-                        mma_ss(tmem + kColY, sdesc(aC + offc, 16, 1024), sdesc(aSP + ks * 2048, kTileBytes, 1024), id_yo,
-                               ks > 0);
+                        mma_ss(tmem + kColYO, sdesc(aC + offc, 16, 1024), sdesc(aSP + ks * 2048, kTileBytes, 1024),
+                               id_yo, ks > 0);
                     }
-                    mma_commit(bar(B_YOFFFULL));
                 }
+                // S'^T (+)= B^T (w x)  (M = n, N = (head, p), K = rows); both operands MN-major
+                if (!mbar_wait(bar(B_WXREADY), j & 1, MASK, abort_flag, prm.status, 25)) break;
+                SSD_TRACE_PT(kWarpMma, j, 2);
+                tc_fence_after();
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t off = ks * 2048;
+                    mma_ss(tmem + kColST, sdesc(aB + off, kTileBytes, 1024), sdesc(aWX + off, kTileBytes, 1024), id_s,
+                           (j > 0) || (ks > 0));
+                }
+                mma_commit(bar(B_STFULL));
                 mma_commit(bar(B_BCEMPTY));
-                // Y += M_h X_h  (A from TMEM, B = X_h MN-major, N = 64 per head)
+                // Y_diag = M_h X_h  (A from TMEM, B = X_h MN-major, N = 64 per head)
                 if (!mbar_wait(bar(B_MREADY), j & 1, MASK, abort_flag, prm.status, 27)) break;
-                if (j >= 1 && !mbar_wait(bar(B_RSREADY), (j - 1) & 1, MASK, abort_flag, prm.status, 28)) break;
                 if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 29)) break;
                 SSD_TRACE_PT(kWarpMma, j, 3);
                 tc_fence_after();
                 for (int h = 0; h < 2; ++h)
                     for (int ks = 0; ks < 8; ++ks)
-                        mma_ts(tmem + kColY + 64 * h, tmem + kColG + 16 * ks + 8 * h,
-                               sdesc(aX + h * kTileBytes + ks * 2048, kTileBytes, 1024), id_yd, (j >= 1) || (ks > 0));
+                        mma_ts(tmem + kColYD + 64 * h, tmem + kColG + 16 * ks + 8 * h,
+                               sdesc(aX + h * kTileBytes + ks * 2048, kTileBytes, 1024), id_yd, ks > 0);
                 mma_commit(bar(B_YFULL));
             }
             // drain: every MMA issued above has completed before TMEM is released
             mma_commit(bar(B_DONE));
             mbar_drain(bar(B_DONE), 0, prm.wait_cycles);
         }
-    } else if (warp >= kWarpStore) {
+    } else if (warp == kWarpStore || warp == kWarpStore + 1) {
         // ---------------------------------------------------------- y stores, one warp per head
         const uint32_t MASK = 0xffffffffu;
         const int hs = warp - kWarpStore;
@@ -522,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
         for (int j = 0; j < nblk; ++j) {
             const int st = j & 1;
             const int cm = dir > 0 ? j : nblk - 1 - j;
-            if (!mbar_wait(bar(B_TILE0 + hs), j & 1, MASK, abort_flag, prm.status, 61)) break;
+            if (!mbar_wait(bar(B_TILE00 + 2 * hs + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 61)) break;
             const uint32_t tile = sbase + kOffX + st * kStageBytes + hs * kTileBytes;
             int sec = 0;
             if (prm.bidir) {
@@ -588,144 +636,236 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
         const int r = wq * 32 + lane;              // row in block == TMEM lane
         const int h = h0 + hs;
         const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
-        const float A2 = prm.d[slot].A[h] * kLog2e;   // log2 units: exp(a) = exp2(a * log2 e)
         const float Dh = prm.d[slot].D ? prm.d[slot].D[h] : 0.f;
-        float *cs2 = cs2_s + hs * kBlk, *dts = dt_s + hs * kBlk, *wtab = wtab_s + hs * 4 * kBlk;
         uint8_t *wx_tile = sm + kOffWX + hs * kTileBytes;
         uint8_t *sp_tile = sm + kOffSP + hs * kTileBytes;
-        float *e1_s = reinterpret_cast<float *>(sm + kOffE1);   // [2][128]
-        const uint32_t colS = kColS + 64 * hs + 32 * c, colST = kColST + 64 * hs + 32 * c,
-                       colY = kColY + 64 * hs + 32 * c;
+        const uint32_t colST = kColST + 64 * hs + 32 * c, colYD = kColYD + 64 * hs + 32 * c,
+                       colYO = kColYO + 64 * hs + 32 * c;
 
-        for (int j = 0; j < nblk; ++j) {
-            if (__any_sync(0xffffffffu, *abort_flag)) break;
-            SSD_TRACE_PT(warp, j, 0);
-            const int st = j & 1;
-
-            // x, dt of this block
-            if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 41)) break;
-            SSD_TRACE_PT(warp, j, 1);
-            uint8_t *xt = sm + kOffX + st * kStageBytes + hs * kTileBytes;
-            const __nv_bfloat16 *dtt =
-                reinterpret_cast<const __nv_bfloat16 *>(sm + kOffX + st * kStageBytes + 2 * kTileBytes);
-            const float dtr = __bfloat162float(dtt[r * 8 + (h & 7)]);
-
-            // cumulative A*dt in scan order (prefix over rows forward, suffix over rows reverse):
-            // warp shuffles inside the quarter, and every warp reduces all four quarter totals
-            // itself from the dt tile, so no exchange between warps is needed
-            float s = dtr;
+        // Decay tables of block jj (into buffer jj & 1) from the dt ring.  Thread (r, head hs)
+        // computes the cumulative A dt of its row in scan order (prefix over rows forward, suffix
+        // reverse; log2 units) and writes its share of the row's entries: half c = 0 the mask
+        // tables, half c = 1 the w.x, epilogue and sub-block factors.
+        const float A2 = prm.d[slot].A[h] * kLog2e;   // log2 units: exp(a) = exp2(a * log2 e)
+        auto make_tables = [&](int jj) -> bool {
+            const int sl = jj & 1;
+            if (!mbar_wait(bar(B_DTFULL0 + sl), (jj >> 1) & 1, MASK, abort_flag, prm.status, 51)) return false;
+            // buffer jj & 1 was last read in block jj - 2: every warp has finished its epilogue
+            if (jj >= 2 && !mbar_wait(bar(B_YEMPTY), (jj - 2) & 1, MASK, abort_flag, prm.status, 52)) return false;
+            const __nv_bfloat16 *dtt = reinterpret_cast<const __nv_bfloat16 *>(sm + kOffDT + sl * kDtBytes);
+            const float d = __bfloat162float(dtt[r * 8 + (h & 7)]);
+            float s = d;                                   // inclusive scan inside the quarter
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const float u = dir > 0 ? __shfl_up_sync(0xffffffffu, s, o) : __shfl_down_sync(0xffffffffu, s, o);
+                const float u = dir > 0 ? __shfl_up_sync(MASK, s, o) : __shfl_down_sync(MASK, s, o);
                 if (dir > 0 ? lane >= o : lane + o < 32) s += u;
             }
-            float tot[4], base = 0.f, total = 0.f;
+            float tot[4];
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                float v = __bfloat162float(dtt[(32 * w + lane) * 8 + (h & 7)]);
+            for (int q = 0; q < 4; ++q) {
+                float v = __bfloat162float(dtt[(32 * q + lane) * 8 + (h & 7)]);
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                tot[w] = v;
-                total += v;
-                if (dir > 0 ? w < wq : w > wq) base += v;
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(MASK, v, o);
+                tot[q] = v;
             }
-            // cs (log2 units) at the quarter boundaries: the reference rows of the factorised mask
-            float ref2[4];
-            {
-                float acc = 0.f;
-                if (dir > 0) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_DTEMPTY0 + sl));      // dt slot read: free for block jj + 2
+            // base[q] = sum of the quarters before q in scan order (cs just before quarter q)
+            float base[4], acc = 0.f;
+            if (dir > 0) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) { ref2[q] = A2 * acc; acc += tot[q]; }   // row 32q-1
-                } else {
+                for (int q = 0; q < 4; ++q) { base[q] = acc; acc += tot[q]; }
+            } else {
 #pragma unroll
-                    for (int q = 3; q >= 0; --q) { ref2[q] = A2 * acc; acc += tot[q]; }  // row 32(q+1)
-                }
+                for (int q = 3; q >= 0; --q) { base[q] = acc; acc += tot[q]; }
             }
-            const float c2 = A2 * (base + s);                 // cs_r * log2 e
-            const float cl2 = A2 * total;                     // cs at the block's last scan position
+            const float own_base = wq == 0 ? base[0] : wq == 1 ? base[1] : wq == 2 ? base[2] : base[3];
+            const float own_tot = wq == 0 ? tot[0] : wq == 1 ? tot[1] : wq == 2 ? tot[2] : tot[3];
+            const float c2 = A2 * (own_base + s);
+            const float cl2 = A2 * acc;                    // cs at the block's last scan position
+            float *tb = tab_s + sl * kTabFloats;
             if (c == 0) {
-                // decay tables of this head (written once; both halves compute the same values)
-                cs2[r] = c2;
-                dts[r] = dtr;
-                // column factors of the off-diagonal quarters: W[q][s] = exp(cs_ref(q) - cs_s) dt_s
+                tb[kTabCS + hs * kBlk + r] = c2;
+                tb[kTabDT + hs * kBlk + r] = d;
+                // column factors for the later quarters: W[q2][s] = exp(cs_ref(q2) - cs_s) dt_s
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const bool off = dir > 0 ? wq < q : wq > q;    // this row is a source for quarter q
-                    if (off) wtab[q * kBlk + r] = exp2f(ref2[q] - c2) * dtr;
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    const bool off = dir > 0 ? wq < q2 : wq > q2;
+                    if (off) tb[kTabW + (hs * 4 + q2) * kBlk + r] = ex2_ftz(A2 * base[q2] - c2) * d;
                 }
-                const float ref_own = wq == 0 ? ref2[0] : wq == 1 ? ref2[1] : wq == 2 ? ref2[2] : ref2[3];
-                e1_s[hs * kBlk + r] = exp2f(c2 - ref_own);      // row factor towards the quarter boundary
+                tb[kTabE1 + hs * kBlk + r] = ex2_ftz(c2 - A2 * own_base);   // row factor to the boundary
+            } else {
+                // 16-row sub-block of r: cs just before it and across it, in scan order
+                const float half = __shfl_sync(MASK, s, dir > 0 ? 15 : 16);
+                const bool second = dir > 0 ? lane >= 16 : lane < 16;
+                const float pre2 = A2 * (own_base + (second ? half : 0.f));
+                const float post2 = A2 * (own_base + (second ? own_tot : half));
+                tb[kTabR16 + hs * kBlk + r] = ex2_ftz(c2 - pre2);
+                tb[kTabD16 + hs * kBlk + r] = ex2_ftz(pre2 - c2) * d;
+                tb[kTabO16 + hs * kBlk + r] = ex2_ftz(post2 - c2) * d;
+                // the factorised sub-block is exact while its column factors stay far from
+                // float32 overflow: decay across the sub-block below 2^-120
+                if ((lane & 15) == 0) tb[kTabBig + hs * 8 + (r >> 4)] = (pre2 - post2 > 120.f) ? 1.f : 0.f;
+                tb[kTabWR + hs * kBlk + r] = ex2_ftz(cl2 - c2) * d;
+                tb[kTabER + hs * kBlk + r] = ex2_ftz(c2);
+                if (r == 0) tb[kTabA + hs] = ex2_ftz(cl2);
             }
-            const float wr = exp2f(cl2 - c2) * dtr;           // weight of row r in the block's state
-            const float er = exp2f(c2);                       // decay from the block start to row r
-            const float ablk = exp2f(cl2);                    // decay across the whole block
-            SSD_TRACE_PT(warp, j, 5);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_TABREADY0 + sl));
+            return true;
+        };
 
-            // w (.) x -> wX tile (same swizzled layout as the X tile), this half's 4 chunks
+        // w (.) x of block jj -> wX tile (same swizzled layout as the X tile), this half's 4 chunks
+        auto wx_pass = [&](int jj) -> bool {
+            const int st = jj & 1;
+            if (!mbar_wait(bar(B_TABREADY0 + st), (jj >> 1) & 1, MASK, abort_flag, prm.status, 41)) return false;
+            if (!mbar_wait(bar(B_XFULL0 + st), (jj >> 1) & 1, MASK, abort_flag, prm.status, 42)) return false;
+            // w rounded to bf16 once, then one packed bf16 multiply per pair of x values
+            const float wr = tab_s[st * kTabFloats + kTabWR + hs * kBlk + r];
+            const uint32_t w2 = pack_bf16(wr, wr);
+            const uint8_t *xt = sm + kOffX + st * kStageBytes + hs * kTileBytes;
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq) {
                 const int q = 4 * c + qq;
                 const uint4 v = *reinterpret_cast<const uint4 *>(xt + swz(r, q));
                 uint4 o;
-                o.x = pack_bf16(bf16lo(v.x) * wr, bf16hi(v.x) * wr);
-                o.y = pack_bf16(bf16lo(v.y) * wr, bf16hi(v.y) * wr);
-                o.z = pack_bf16(bf16lo(v.z) * wr, bf16hi(v.z) * wr);
-                o.w = pack_bf16(bf16lo(v.w) * wr, bf16hi(v.w) * wr);
+                o.x = mul_bf16x2(v.x, w2);
+                o.y = mul_bf16x2(v.y, w2);
+                o.z = mul_bf16x2(v.z, w2);
+                o.w = mul_bf16x2(v.w, w2);
                 *reinterpret_cast<uint4 *>(wx_tile + swz(r, q)) = o;
             }
             fence_async_smem();                // w(.)x is read by the tensor core
-            SSD_TRACE_PT(warp, j, 8);
+            __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_WXREADY));
+            return true;
+        };
+
+        // state hand-off into block jj (>= 1): the state MMA of block jj - 1 has left S'
+        // (entering block jj) in TMEM; thread r holds row n = r of this half's 32 columns.
+        // bf16(S') goes to smem for Y_off = C S'^T, and S' is scaled in place by block jj's
+        // decay so that block jj's state MMA accumulates S' <- exp(cs_last) S' + S directly.
+        auto state_pass = [&](int jj) {
+            const float ablk = tab_s[(jj & 1) * kTabFloats + kTabA + hs];
+            tc_fence_after();
+#pragma unroll 1
+            for (int qd = 0; qd < 2; ++qd) {
+                float sv[16];
+                tmem_ld16(tl + colST + 16 * qd, sv);
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    uint4 o;
+                    o.x = pack_bf16(sv[8 * qq + 0], sv[8 * qq + 1]);
+                    o.y = pack_bf16(sv[8 * qq + 2], sv[8 * qq + 3]);
+                    o.z = pack_bf16(sv[8 * qq + 4], sv[8 * qq + 5]);
+                    o.w = pack_bf16(sv[8 * qq + 6], sv[8 * qq + 7]);
+                    *reinterpret_cast<uint4 *>(sp_tile + swz(r, 4 * c + 2 * qd + qq)) = o;
+                }
+                uint32_t w16[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) w16[i] = __float_as_uint(ablk * sv[i]);
+                tmem_st16(tl + colST + 16 * qd, w16);
+            }
+            fence_async_smem();                // SP is read by the tensor core
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_SPREADY));
+        };
+
+        const int jend = (nblk > 0 && make_tables(0)) ? nblk : 0;
+        for (int j = 0; j < jend; ++j) {
+            if (__any_sync(0xffffffffu, *abort_flag)) break;
+            SSD_TRACE_PT(warp, j, 0);
+            const int st = j & 1;
+            const float *tb = tab_s + st * kTabFloats;
+            if (!wx_pass(j)) break;
+            SSD_TRACE_PT(warp, j, 8);
+            if (j >= 1) {
+                if (!mbar_wait(bar(B_STFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 43)) break;
+                SSD_TRACE_PT(warp, j, 6);
+                state_pass(j);
+                SSD_TRACE_PT(warp, j, 7);
+            }
 
             // M_h = G (.) decay (.) dt over the causal triangle, bf16, for both heads.  This
             // warpgroup takes K-steps g and g + 4; the two heads' bf16 results for a K-step
             // replace the 16 float32 G columns they were computed from.
-            if (!mbar_wait(bar(B_GFULL), j & 1, MASK, abort_flag, prm.status, 42)) break;
-            // both heads' decay tables of this block are read below: every warp arrives on this
-            // barrier after its preparation
-            if (!mbar_wait(bar(B_WXREADY), j & 1, MASK, abort_flag, prm.status, 48)) break;
+            if (!mbar_wait(bar(B_GFULL), j & 1, MASK, abort_flag, prm.status, 44)) break;
             SSD_TRACE_PT(warp, j, 9);
             tc_fence_after();
             {
-                const float c2h[2] = {cs2_s[r], cs2_s[kBlk + r]};
-                const float e1h[2] = {e1_s[r], e1_s[kBlk + r]};
+                const float c2h[2] = {tb[kTabCS + r], tb[kTabCS + kBlk + r]};
+                const float e1h[2] = {tb[kTabE1 + r], tb[kTabE1 + kBlk + r]};
 #pragma unroll 1
                 for (int ks = g; ks < 8; ks += 4) {
                     const int sq = ks >> 1;                          // source quarter
                     const bool offd = dir > 0 ? sq < wq : sq > wq;
                     const bool diag = sq == wq;
                     uint32_t m[16];
-                    if (offd || diag) {
+                    if (offd) {
                         float gv[16];
                         tmem_ld16(tl + kColG + 16 * ks, gv);
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
-                            if (offd) {
-                                const float *wrow = wtab_s + (hh * 4 + wq) * kBlk + 16 * ks;
+                            const float *wrow = tb + kTabW + (hh * 4 + wq) * kBlk + 16 * ks;
 #pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    const float4 wv = *reinterpret_cast<const float4 *>(wrow + 4 * i);
-                                    m[8 * hh + 2 * i] = pack_bf16(gv[4 * i] * wv.x * e1h[hh], gv[4 * i + 1] * wv.y * e1h[hh]);
-                                    m[8 * hh + 2 * i + 1] =
-                                        pack_bf16(gv[4 * i + 2] * wv.z * e1h[hh], gv[4 * i + 3] * wv.w * e1h[hh]);
+                            for (int i = 0; i < 4; ++i) {
+                                const float4 wv = *reinterpret_cast<const float4 *>(wrow + 4 * i);
+                                m[8 * hh + 2 * i] = pack_bf16(gv[4 * i] * wv.x * e1h[hh], gv[4 * i + 1] * wv.y * e1h[hh]);
+                                m[8 * hh + 2 * i + 1] =
+                                    pack_bf16(gv[4 * i + 2] * wv.z * e1h[hh], gv[4 * i + 3] * wv.w * e1h[hh]);
+                            }
+                        }
+                    } else if (diag && tb[kTabBig + ks] == 0.f && tb[kTabBig + 8 + ks] == 0.f) {
+                        // diagonal quarter, K-step = 16-row sub-block ks.  Row r's own sub-block:
+                        // exp(cs_r - cs_s) = R16[r] D16[s] for s up to r in scan order; the
+                        // sub-block before it in scan order: R16[r] O16[s]; the one after: 0.
+                        float gv[16];
+                        tmem_ld16(tl + kColG + 16 * ks, gv);
+                        const int kt = r >> 4;
+                        const bool own = kt == ks, prev = kt == ks + dir;
+                        // keep source u (0..15 in the sub-block): u <= bound forward, u >= bound reverse
+                        const int bound = own ? r - 16 * ks : prev ? (dir > 0 ? 15 : 0) : (dir > 0 ? -1 : 16);
+                        bool keep[16];
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) keep[u] = dir > 0 ? u <= bound : u >= bound;
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const float rf = tb[kTabR16 + hh * kBlk + r];
+                            const float *crow = tb + (own ? kTabD16 : kTabO16) + hh * kBlk + 16 * ks;
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const float4 cv = *reinterpret_cast<const float4 *>(crow + 4 * i);
+                                const float cc[4] = {cv.x, cv.y, cv.z, cv.w};
+                                float mv[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) mv[e] = keep[4 * i + e] ? gv[4 * i + e] * cc[e] * rf : 0.f;
+                                m[8 * hh + 2 * i] = pack_bf16(mv[0], mv[1]);
+                                m[8 * hh + 2 * i + 1] = pack_bf16(mv[2], mv[3]);
+                            }
+                        }
+                    } else if (diag) {
+                        // decay across the sub-block too steep for the factorised form: one
+                        // exponential per element
+                        float gv[16];
+                        tmem_ld16(tl + kColG + 16 * ks, gv);
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const float *csrc = tb + kTabCS + hh * kBlk + 16 * ks, *dsrc = tb + kTabDT + hh * kBlk + 16 * ks;
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const float4 cv = *reinterpret_cast<const float4 *>(csrc + 4 * i);
+                                const float4 dv = *reinterpret_cast<const float4 *>(dsrc + 4 * i);
+                                const float cc[4] = {cv.x, cv.y, cv.z, cv.w}, dd[4] = {dv.x, dv.y, dv.z, dv.w};
+                                float mv[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int sidx = 16 * ks + 4 * i + e;
+                                    const bool in = dir > 0 ? sidx <= r : sidx >= r;
+                                    mv[e] = in ? gv[4 * i + e] * ex2_ftz(c2h[hh] - cc[e]) * dd[e] : 0.f;
                                 }
-                            } else {
-                                const float *csrc = cs2_s + hh * kBlk + 16 * ks, *dsrc = dt_s + hh * kBlk + 16 * ks;
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    const float4 cv = *reinterpret_cast<const float4 *>(csrc + 4 * i);
-                                    const float4 dv = *reinterpret_cast<const float4 *>(dsrc + 4 * i);
-                                    const float cc[4] = {cv.x, cv.y, cv.z, cv.w}, dd[4] = {dv.x, dv.y, dv.z, dv.w};
-                                    float mv[4];
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e) {
-                                        const int sidx = 16 * ks + 4 * i + e;
-                                        const bool in = dir > 0 ? sidx <= r : sidx >= r;
-                                        mv[e] = in ? gv[4 * i + e] * exp2f(c2h[hh] - cc[e]) * dd[e] : 0.f;
-                                    }
-                                    m[8 * hh + 2 * i] = pack_bf16(mv[0], mv[1]);
-                                    m[8 * hh + 2 * i + 1] = pack_bf16(mv[2], mv[3]);
-                                }
+                                m[8 * hh + 2 * i] = pack_bf16(mv[0], mv[1]);
+                                m[8 * hh + 2 * i + 1] = pack_bf16(mv[2], mv[3]);
                             }
                         }
                     } else {
@@ -740,76 +880,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             if (lane == 0) mbar_arrive(bar(B_MREADY));
             SSD_TRACE_PT(warp, j, 10);
 
-            // state: S' <- exp(cs_last) S' + S; thread r holds state row n = r (this half's 32
-            // columns), the float32 state lives in TMEM and a bf16 copy goes to smem as the next
-            // block's MMA operand
-            if (!mbar_wait(bar(B_SFULL), j & 1, MASK, abort_flag, prm.status, 43)) break;
+            // next block's decay tables, while the tensor core computes this block's Y_diag
+            if (j + 1 < nblk && !make_tables(j + 1)) break;
             SSD_TRACE_PT(warp, j, 11);
-            // the previous state tile must have been consumed by this block's Y = C S'^T
-            if (j + 1 < nblk && j >= 1 &&
-                !mbar_wait(bar(B_YOFFFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 44))
-                break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int qd = 0; qd < 2; ++qd) {
-                float sv[16], pv[16];
-                if (j > 0) {
-                    tmem_ld16x2(tl + colS + 16 * qd, tl + colST + 16 * qd, sv, pv);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) sv[i] = fmaf(ablk, pv[i], sv[i]);
-                } else {
-                    tmem_ld16(tl + colS + 16 * qd, sv);
-                }
-                uint32_t w16[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) w16[i] = __float_as_uint(sv[i]);
-                tmem_st16(tl + colST + 16 * qd, w16);
-                if (j + 1 < nblk) {
-#pragma unroll
-                    for (int qq = 0; qq < 2; ++qq) {
-                        uint4 o;
-                        o.x = pack_bf16(sv[8 * qq + 0], sv[8 * qq + 1]);
-                        o.y = pack_bf16(sv[8 * qq + 2], sv[8 * qq + 3]);
-                        o.z = pack_bf16(sv[8 * qq + 4], sv[8 * qq + 5]);
-                        o.w = pack_bf16(sv[8 * qq + 6], sv[8 * qq + 7]);
-                        *reinterpret_cast<uint4 *>(sp_tile + swz(r, 4 * c + 2 * qd + qq)) = o;
-                    }
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_SEMPTY));
-            SSD_TRACE_PT(warp, j, 12);
-            if (j + 1 < nblk) {
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_SPREADY));
-            }
-            SSD_TRACE_PT(warp, j, 14);
 
-            // Y (from the incoming state) scaled by exp(cs_r), before the intra-block term is added
-            if (j >= 1) {
-                if (!mbar_wait(bar(B_YOFFFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 45)) break;
-                tc_fence_after();
-                float yv[32];
-                tmem_ld32(tl + colY, yv);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) yv[i] *= er;
-                tmem_st32(tl + colY, yv);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_RSREADY));
-                SSD_TRACE_PT(warp, j, 15);
-            }
-
-            // epilogue: o = Y + D x, bf16, written over this row of the x tile (free once the
-            // intra-block MMA is done); a store warp then writes the tile to y in whole rows
+            // epilogue: o = Y_diag + exp(cs_r) Y_off + D x, bf16, written over this row of the x
+            // tile (free once the intra-block MMA is done); a store warp then writes the tile to y
+            // in whole rows
             if (!mbar_wait(bar(B_YFULL), j & 1, MASK, abort_flag, prm.status, 46)) break;
             SSD_TRACE_PT(warp, j, 16);
             tc_fence_after();
             {
+                uint8_t *xt = sm + kOffX + st * kStageBytes + hs * kTileBytes;
                 float yv[32];
-                tmem_ld32(tl + colY, yv);
+                tmem_ld32(tl + colYD, yv);
+                if (j >= 1) {
+                    // Y_off of the incoming state, scaled by the decay exp(cs_r) up to this row
+                    const float er = tb[kTabER + hs * kBlk + r];
+                    float yo[32];
+                    tmem_ld32(tl + colYO, yo);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) yv[i] = fmaf(er, yo[i], yv[i]);
+                }
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
                     const int q = 4 * c + qq;
@@ -834,7 +926,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(bar(B_YEMPTY));
-                mbar_arrive(bar(B_TILE0 + hs));
+                mbar_arrive(bar(B_TILE00 + 2 * hs + st));
             }
             SSD_TRACE_PT(warp, j, 21);
         }

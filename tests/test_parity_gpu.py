@@ -146,6 +146,26 @@ def test_dt_zero_tensor_core_path(ssd):
         assert torch.equal(y, ref)
 
 
+def test_steep_decay(ssd):
+    """Decays steep enough that a 16-token window falls below 2^-120 (dt = 3, A = -16 on even
+    heads): the tensor-core path's factorised decay mask must switch to its exact form there."""
+    shape = si.Shape(1, 512, 8, 64, 128, 1, "bf16")
+    p = si.make_params(shape, seed=21, with_D=False)
+    q = oracle.params_f64(p)
+    q["dt"][:, 40:56, :] = 3.0          # inside one 16-row sub-block of the first block
+    q["dt"][:, 300:340, :] = 2.0        # across sub-block and quarter boundaries of the third block
+    q["A"][0::2] = -16.0
+    dev = torch.device("cuda")
+    d = {"x": p.x.torch(dev), "dt": torch.from_numpy(q["dt"]).to(dev, torch.bfloat16),
+         "A": torch.from_numpy(q["A"]).to(dev, torch.float32), "B": p.B.torch(dev), "C": p.C.torch(dev), "D": None}
+    for direction in (1, -1):
+        y = ssd.ssd_scan(**d, direction=direction, chunk=256)
+        torch.cuda.synchronize()
+        assert torch.isfinite(y.float()).all()
+        ref = oracle.ssd_scan_f64(q["x"], q["dt"], q["A"], q["B"], q["C"], None, direction)
+        assert oracle.rel_err(_f64(y), ref) <= TOL["bf16"], direction
+
+
 def test_paths_agree(ssd):
     """The tensor-core path (chunk 128) and the SIMT path (chunk 64) on the same inputs."""
     shape = si.Shape(2, 512, 8, 64, 128, 1, "bf16")
