@@ -24,6 +24,7 @@ The JSON line carries, besides the contract keys:
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -54,11 +55,14 @@ def algorithmic_bytes_per_token(shape: si.Shape, directions: int = 2) -> int:
     return directions * per_dir + e * H * P
 
 
-def shard_plan(rank: int, world: int, workload: str) -> dict:
-    """Weak scaling: every rank owns one full batch of independent sequences, drawn with its own seed."""
+def shard_plan(rank: int, world: int, workload: str, batch: int | None = None) -> dict:
+    """Weak scaling: every rank owns one full batch of independent sequences, drawn with its own seed.
+
+    ``batch`` replaces the workload's batch size (a smaller case of the same layer shape, for profiling)."""
     w = si.WORKLOADS[workload]
-    return {"rank": rank, "world": world, "seed": rank, "shape": w["shape"], "chunk": w["chunk"],
-            "tokens": w["shape"].tokens}
+    shape = w["shape"] if batch is None else dataclasses.replace(w["shape"], batch=batch)
+    return {"rank": rank, "world": world, "seed": rank, "shape": shape, "chunk": w["chunk"],
+            "tokens": shape.tokens}
 
 
 def max_over_ranks(value: float, dist) -> float:
@@ -226,7 +230,7 @@ def run_ours(args) -> None:
 
     import bidirectional_mamba_ssd_bidir_b200 as ssd
 
-    plan = shard_plan(rank, world, args.workload)
+    plan = shard_plan(rank, world, args.workload, args.batch)
     shape, chunk = plan["shape"], plan["chunk"]
     pf, pr = si.make_bidir(shape, seed=plan["seed"])
     host = {}
@@ -380,6 +384,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[k for k, v in si.WORKLOADS.items()
                                                                       if v["kind"] == "bidir"])
+    ap.add_argument("--batch", type=int, default=None,
+                    help="replace the workload's batch size (a smaller case of the same shape, for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU work of the oracle baseline sample")
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds for the reference arm's steps")
