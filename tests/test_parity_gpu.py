@@ -189,6 +189,24 @@ def test_deterministic(ssd):
     assert torch.equal(y1, y2)
 
 
+@pytest.mark.parametrize("dims,chunk", [((2, 512, 8, 64, 128, 1), 256), ((2, 256, 4, 32, 64, 1), 64)],
+                         ids=["tensor_core", "simt"])
+def test_output_canaries(ssd, dims, chunk):
+    """The kernels write exactly the output tensor: sentinel words before and after it survive."""
+    shape = si.Shape(*dims, "bf16")
+    pf, pr = si.make_bidir(shape, seed=14)
+    df, dr = _dev(pf), _dev(pr)
+    n, pad = df["x"].numel(), 8192
+    buf = torch.full((n + 2 * pad,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sentinel = buf[:pad].clone()
+    y = buf[pad:pad + n].view(df["x"].shape)
+    ssd.bidir_ssd(df, dr, chunk=chunk, out=y)
+    torch.cuda.synchronize()
+    assert torch.equal(buf[:pad].view(torch.int16), sentinel.view(torch.int16))
+    assert torch.equal(buf[pad + n:].view(torch.int16), sentinel.view(torch.int16))
+    assert torch.isfinite(y.float()).all()
+
+
 def test_empty_batch(ssd):
     shape = si.Shape(0, 256, 4, 64, 128, 1, "bf16")
     x = torch.empty(0, 256, 4, 64, dtype=torch.bfloat16, device="cuda")
