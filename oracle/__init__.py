@@ -20,6 +20,8 @@ Contents
                    ("Bifocal Diffusion Language Models", section 2,
                    mechanism and integration).  s = 0 returns the residual
                    itself, so the model is unchanged at initialisation.
+``ssd_scan_state_f64`` the recurrence with the state carried across the call
+                   (state in, state out), for block-wise decoding.
 ``ssd_chunked_f64`` the chunked (state-passing) form of the same scan, the
                    decomposition the GPU kernels use; pinned against the
                    recurrence for several chunk sizes.
@@ -64,6 +66,10 @@ def load_library(path: str | None = None):
     dp = ctypes.POINTER(ctypes.c_double)
     f.argtypes = [ctypes.c_int] * 6 + [dp] * 6 + [ctypes.c_int, dp, ctypes.c_int]
     f.restype = ctypes.c_int
+    if hasattr(lib, "ssd_oracle_scan_state"):
+        g = lib.ssd_oracle_scan_state
+        g.argtypes = [ctypes.c_int] * 6 + [dp] * 6 + [ctypes.c_int, dp, dp, dp, ctypes.c_int]
+        g.restype = ctypes.c_int
     return lib
 
 
@@ -93,6 +99,36 @@ def ssd_scan_f64(x, dt, A, B, C, D=None, direction=1, nthreads=None, lib=None):
     if rc != 0:
         raise RuntimeError(f"ssd_oracle_scan failed with {rc}")
     return y
+
+
+def ssd_scan_state_f64(x, dt, A, B, C, D=None, direction=1, init_state=None, nthreads=None, lib=None):
+    """The recurrence with the state carried across the call: returns (y, final_state).
+
+    ``init_state`` [b, H, P, N] (None = zero) is the state before the first token in scan order;
+    ``final_state`` is the state after the last one.  Block-wise decoding with cache reuse
+    ("DiffuMamba", technical summary, sections 2 and 4) carries this state from one block
+    to the next."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    dt = np.ascontiguousarray(dt, dtype=np.float64)
+    A = np.ascontiguousarray(A, dtype=np.float64)
+    B = np.ascontiguousarray(B, dtype=np.float64)
+    C = np.ascontiguousarray(C, dtype=np.float64)
+    D = None if D is None else np.ascontiguousarray(D, dtype=np.float64)
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    assert dt.shape == (b, L, H) and A.shape == (H,) and B.shape == (b, L, G, N) and C.shape == B.shape
+    s_in = None if init_state is None else np.ascontiguousarray(init_state, dtype=np.float64)
+    if s_in is not None:
+        assert s_in.shape == (b, H, P, N)
+    y = np.zeros_like(x)
+    s_out = np.zeros((b, H, P, N))
+    lib = lib or load_library()
+    rc = lib.ssd_oracle_scan_state(b, L, H, P, N, G, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                   int(direction), _ptr(s_in), _ptr(y), _ptr(s_out),
+                                   int(nthreads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"ssd_oracle_scan_state failed with {rc}")
+    return y, s_out
 
 
 def bidir_f64(pf: dict, pr: dict, nthreads=None, lib=None):

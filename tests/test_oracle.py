@@ -210,3 +210,80 @@ def test_gate_nonzero():
     out = oracle.r2l_block_f64(p, 0.3, res)
     ref = res + 0.3 * _matrix_form(p, -1).reshape(res.shape)
     assert oracle.rel_err(out, ref) <= 1e-12
+
+
+# ------------------------------------------------------------------ state carried across calls
+
+def _scan_state(p, direction, s0=None):
+    return oracle.ssd_scan_state_f64(p["x"], p["dt"], p["A"], p["B"], p["C"], p.get("D"), direction, s0)
+
+
+def _piece(p, lo, hi):
+    return {k: (v[:, lo:hi] if k in ("x", "dt", "B", "C") else v) for k, v in p.items()}
+
+
+@pytest.mark.parametrize("split", [1, 17, 39])
+def test_state_carry_splits_the_sequence(split):
+    """Scanning in two pieces, the second starting from the first's final state, equals scanning
+    whole: the recurrence sees only S and the current token (both directions; for the reverse
+    the right-hand piece is scanned first)."""
+    rng = np.random.default_rng(11)
+    p = _rand_params(rng, 2, 40, 3, 4, 6, 1)
+    L = 40
+    y_all, s_all = _scan_state(p, 1)
+    assert oracle.rel_err(y_all, _scan(p, 1)) == 0.0
+    y1, s1 = _scan_state(_piece(p, 0, split), 1)
+    y2, s2 = _scan_state(_piece(p, split, L), 1, s1)
+    assert oracle.rel_err(np.concatenate([y1, y2], axis=1), y_all) <= 1e-13
+    assert oracle.rel_err(s2, s_all) <= 1e-13
+    yr_all, sr_all = _scan_state(p, -1)
+    yr2, sr2 = _scan_state(_piece(p, split, L), -1)
+    yr1, sr1 = _scan_state(_piece(p, 0, split), -1, sr2)
+    assert oracle.rel_err(np.concatenate([yr1, yr2], axis=1), yr_all) <= 1e-13
+    assert oracle.rel_err(sr1, sr_all) <= 1e-13
+
+
+def test_state_in_decays_in_closed_form():
+    """x = 0 and a nonzero starting state S0: the state only decays, S_t = exp(A sum_{r<=t} dt_r) S0,
+    so y_t[p] = sum_n C_t[n] S_t[p, n]; the final state is exp(A sum dt) S0."""
+    rng = np.random.default_rng(12)
+    p = _rand_params(rng, 2, 30, 3, 4, 5, 1)
+    p["x"] = np.zeros_like(p["x"])
+    s0 = rng.standard_normal((2, 3, 4, 5))
+    for direction in (1, -1):
+        y, s = _scan_state(p, direction, s0)
+        dts = p["dt"] if direction > 0 else p["dt"][:, ::-1]
+        decay = np.exp(np.cumsum(dts, axis=1) * p["A"][None, None, :])      # [b, L, H] in scan order
+        if direction < 0:
+            decay = decay[:, ::-1]
+        ref = np.einsum("blh,bhpn,bln->blhp", decay, s0, p["C"][:, :, 0])
+        assert oracle.rel_err(y, ref) <= 1e-12
+        total = np.exp(p["A"][None, :] * p["dt"].sum(axis=1))                  # [b, H]
+        assert oracle.rel_err(s, total[:, :, None, None] * s0) <= 1e-12
+
+
+def test_final_state_is_the_decayed_sum_of_inputs():
+    """Final state = sum over tokens s of exp(A * sum of dt after s in scan order) dt_s x_s (outer) B_s,
+    plus the decayed starting state; every decay sum taken term by term."""
+    rng = np.random.default_rng(13)
+    b, L, H, P, N = 1, 12, 2, 3, 4
+    p = _rand_params(rng, b, L, H, P, N, 1)
+    s0 = rng.standard_normal((b, H, P, N))
+    for direction in (1, -1):
+        _, s = _scan_state(p, direction, s0)
+        ref = np.zeros((b, H, P, N))
+        for h in range(H):
+            for t in range(L):
+                after = range(t + 1, L) if direction > 0 else range(0, t)
+                e = math.exp(p["A"][h] * sum(p["dt"][0, r, h] for r in after))
+                ref[0, h] += e * p["dt"][0, t, h] * np.outer(p["x"][0, t, h], p["B"][0, t, 0])
+            ref[0, h] += math.exp(p["A"][h] * sum(p["dt"][0, r, h] for r in range(L))) * s0[0, h]
+        assert oracle.rel_err(s, ref) <= 1e-12
+
+
+def test_empty_sequence_passes_the_state_through():
+    rng = np.random.default_rng(14)
+    p = _rand_params(rng, 2, 5, 3, 4, 5, 1)
+    s0 = rng.standard_normal((2, 3, 4, 5))
+    _, s = _scan_state(_piece(p, 0, 0), 1, s0)
+    assert np.array_equal(s, s0)

@@ -33,6 +33,8 @@ MUTANTS = {
     "dt_head_index_dropped": ("j->dt[((size_t)b * L + t) * H + h]", "j->dt[((size_t)b * L + t) * H]"),
     "output_before_update": ("Sp[n] = decay * Sp[n] + u * Bt[n];\n                acc += Ct[n] * Sp[n];",
                              "acc += Ct[n] * Sp[n];\n                Sp[n] = decay * Sp[n] + u * Bt[n];"),
+    "state_in_ignored": ("if (j->s_in)\n        memcpy", "if (0)\n        memcpy"),
+    "state_slot_head_dropped": ("const size_t soff = ((size_t)b * H + h)", "const size_t soff = ((size_t)b * H)"),
 }
 
 
@@ -71,6 +73,22 @@ def _pins_pass(lib) -> bool:
     a = math.exp(dtv * Av)
     ref = np.array([dtv * xv * (1 - a ** (t + 1)) / (1 - a) for t in range(L)])
     checks.append(np.allclose(scan(pgeo, 1)[0, :, 0, 0], ref, rtol=1e-13))
+    # state carried across a split of the sequence, from a nonzero starting state
+    s0 = rng.standard_normal((2, 4, 3, 5))
+    def scan_state(q, d, s_in):
+        return oracle.ssd_scan_state_f64(q["x"], q["dt"], q["A"], q["B"], q["C"], q.get("D"), d, s_in, lib=lib)
+    piece = lambda lo, hi: {k: (v[:, lo:hi] if k in ("x", "dt", "B", "C") else v) for k, v in p.items()}
+    y_all, s_all = scan_state(p, 1, s0)
+    y1, s1 = scan_state(piece(0, 5), 1, s0)
+    y2, s2 = scan_state(piece(5, 13), 1, s1)
+    checks.append(oracle.rel_err(np.concatenate([y1, y2], axis=1), y_all) <= 1e-12)
+    checks.append(oracle.rel_err(s2, s_all) <= 1e-12)
+    zero_x = dict(p, x=np.zeros_like(p["x"]))
+    y0, _ = scan_state(zero_x, 1, s0)
+    decay = np.exp(np.cumsum(p["dt"], axis=1) * p["A"][None, None, :])
+    g = np.arange(4) // 2
+    ref0 = np.einsum("blh,bhpn,blhn->blhp", decay, s0, p["C"][:, :, g])
+    checks.append(oracle.rel_err(y0, ref0) <= 1e-12)
     return all(bool(c) for c in checks)
 
 
