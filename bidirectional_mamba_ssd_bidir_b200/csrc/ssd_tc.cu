@@ -16,9 +16,9 @@
 //                                      (S' = state entering the block, bf16 copy in smem)
 //   S'    <- exp(cs_last) S'           CUDA cores, in place in TMEM [128,256)
 //   S'    += B^T (w (.) X)             tcgen05, N = 2 heads x 64, accumulates into S'
-//   Y_diag = M_h X_h                   tcgen05, A from TMEM, N = 64    TMEM [256,384)
-//   y      = Y_diag + exp(cs_r) Y_off + D x
-//                                      CUDA cores -> smem tile -> TMA store
+//   Y_diag = D x + M_h X_h             D x stored by the CUDA cores in the w (.) x pass,
+//                                      then tcgen05, A from TMEM, N = 64    TMEM [256,384)
+//   y      = Y_diag + exp(cs_r) Y_off  CUDA cores -> smem tile -> TMA store
 //
 // This is the chunked evaluation of the recurrence S <- exp(dt A) S +
 // dt x (outer) B, y = C.S + D x that the Mamba-2 layers of the DiffuMamba
@@ -317,38 +317,50 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
-// two 16-column loads, one wait
-__device__ __forceinline__ void tmem_ld16x2(uint32_t ta, uint32_t tb, float *va, float *vb) {
-    uint32_t a[16], b[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
-          "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]),
-          "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]),
-          "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15])
-        : "r"(ta), "r"(tb)
-        : "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) { va[i] = __uint_as_float(a[i]); vb[i] = __uint_as_float(b[i]); }
-}
 // TMEM stores: the wait is part of the asm, so the source registers are not reused while
 // the store may still read them and later TMEM reads of these columns see the new values.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
+// store without waiting: the caller issues tmem_wait_st() before the data is consumed
+__device__ __forceinline__ void tmem_st16_nw(uint32_t taddr, const uint32_t *r) {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n\t"
-        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
         "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v) {
-    uint32_t r[32];
+__device__ __forceinline__ void tmem_st16f_nw(uint32_t taddr, const float *v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]),
+        "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// two 32-column loads, one wait
+__device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, float *va, float *vb) {
+    uint32_t a[32], b[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
+          "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]),
+          "=r"(a[16]), "=r"(a[17]), "=r"(a[18]), "=r"(a[19]), "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]),
+          "=r"(a[24]), "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31]),
+          "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]),
+          "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15]),
+          "=r"(b[16]), "=r"(b[17]), "=r"(b[18]), "=r"(b[19]), "=r"(b[20]), "=r"(b[21]), "=r"(b[22]), "=r"(b[23]),
+          "=r"(b[24]), "=r"(b[25]), "=r"(b[26]), "=r"(b[27]), "=r"(b[28]), "=r"(b[29]), "=r"(b[30]), "=r"(b[31])
+        : "r"(ta), "r"(tb)
+        : "memory");
 #pragma unroll
-    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(v[i]);
-    tmem_st16(taddr, r);
-    tmem_st16(taddr + 16, r + 16);
+    for (int i = 0; i < 32; ++i) {
+        va[i] = __uint_as_float(a[i]);
+        vb[i] = __uint_as_float(b[i]);
+    }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -546,7 +558,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 }
                 mma_commit(bar(B_STFULL));
                 mma_commit(bar(B_BCEMPTY));
-                // Y_diag = M_h X_h  (A from TMEM, B = X_h MN-major, N = 64 per head)
+                // Y_diag += M_h X_h  (A from TMEM, B = X_h MN-major, N = 64 per head), on top of
+                // the D x the CUDA-core warps stored there in their w.x pass
                 if (!mbar_wait(bar(B_MREADY), j & 1, MASK, abort_flag, prm.status, 27)) break;
                 if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 29)) break;
                 SSD_TRACE_PT(kWarpMma, j, 3);
@@ -554,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 for (int h = 0; h < 2; ++h)
                     for (int ks = 0; ks < 8; ++ks)
                         mma_ts(tmem + kColYD + 64 * h, tmem + kColG + 16 * ks + 8 * h,
-                               sdesc(aX + h * kTileBytes + ks * 2048, kTileBytes, 1024), id_yd, ks > 0);
+                               sdesc(aX + h * kTileBytes + ks * 2048, kTileBytes, 1024), id_yd, 1);
                 mma_commit(bar(B_YFULL));
             }
             // drain: every MMA issued above has completed before TMEM is released
@@ -725,17 +738,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             const uint32_t w2 = pack_bf16(wr, wr);
             const uint8_t *xt = sm + kOffX + st * kStageBytes + hs * kTileBytes;
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                const int q = 4 * c + qq;
-                const uint4 v = *reinterpret_cast<const uint4 *>(xt + swz(r, q));
-                uint4 o;
-                o.x = mul_bf16x2(v.x, w2);
-                o.y = mul_bf16x2(v.y, w2);
-                o.z = mul_bf16x2(v.z, w2);
-                o.w = mul_bf16x2(v.w, w2);
-                *reinterpret_cast<uint4 *>(wx_tile + swz(r, q)) = o;
+            for (int qh = 0; qh < 2; ++qh) {
+                float dx[16];                  // D x of 16 columns, the starting value of Y_diag
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    const int q = 4 * c + 2 * qh + qq;
+                    const uint4 v = *reinterpret_cast<const uint4 *>(xt + swz(r, q));
+                    uint4 o;
+                    o.x = mul_bf16x2(v.x, w2);
+                    o.y = mul_bf16x2(v.y, w2);
+                    o.z = mul_bf16x2(v.z, w2);
+                    o.w = mul_bf16x2(v.w, w2);
+                    *reinterpret_cast<uint4 *>(wx_tile + swz(r, q)) = o;
+                    const uint32_t xw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        dx[8 * qq + 2 * i] = Dh * bf16lo(xw[i]);
+                        dx[8 * qq + 2 * i + 1] = Dh * bf16hi(xw[i]);
+                    }
+                }
+                tmem_st16f_nw(tl + colYD + 16 * qh, dx);
             }
             fence_async_smem();                // w(.)x is read by the tensor core
+            tmem_wait_st();
+            tc_fence_before();                 // Y_diag's starting value is read by the MMA
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_WXREADY));
             return true;
@@ -761,12 +787,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                     o.w = pack_bf16(sv[8 * qq + 6], sv[8 * qq + 7]);
                     *reinterpret_cast<uint4 *>(sp_tile + swz(r, 4 * c + 2 * qd + qq)) = o;
                 }
-                uint32_t w16[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) w16[i] = __float_as_uint(ablk * sv[i]);
-                tmem_st16(tl + colST + 16 * qd, w16);
+                for (int i = 0; i < 16; ++i) sv[i] *= ablk;
+                tmem_st16f_nw(tl + colST + 16 * qd, sv);
             }
             fence_async_smem();                // SP is read by the tensor core
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_SPREADY));
@@ -872,9 +898,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
 #pragma unroll
                         for (int i = 0; i < 16; ++i) m[i] = 0u;       // outside the causal triangle
                     }
-                    tmem_st16(tl + kColG + 16 * ks, m);
+                    tmem_st16_nw(tl + kColG + 16 * ks, m);
                 }
             }
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_MREADY));
@@ -884,7 +911,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             if (j + 1 < nblk && !make_tables(j + 1)) break;
             SSD_TRACE_PT(warp, j, 11);
 
-            // epilogue: o = Y_diag + exp(cs_r) Y_off + D x, bf16, written over this row of the x
+            // epilogue: o = Y_diag (which started at D x) + exp(cs_r) Y_off, bf16, written over this row of the x
             // tile (free once the intra-block MMA is done); a store warp then writes the tile to y
             // in whole rows
             if (!mbar_wait(bar(B_YFULL), j & 1, MASK, abort_flag, prm.status, 46)) break;
@@ -893,31 +920,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             {
                 uint8_t *xt = sm + kOffX + st * kStageBytes + hs * kTileBytes;
                 float yv[32];
-                tmem_ld32(tl + colYD, yv);
                 if (j >= 1) {
                     // Y_off of the incoming state, scaled by the decay exp(cs_r) up to this row
                     const float er = tb[kTabER + hs * kBlk + r];
                     float yo[32];
-                    tmem_ld32(tl + colYO, yo);
+                    tmem_ld32x2(tl + colYD, tl + colYO, yv, yo);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) yv[i] = fmaf(er, yo[i], yv[i]);
+                } else {
+                    tmem_ld32(tl + colYD, yv);
                 }
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
                     const int q = 4 * c + qq;
-                    const uint4 xv = *reinterpret_cast<const uint4 *>(xt + swz(r, q));
-                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                    float o[8];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        o[2 * i] = fmaf(Dh, bf16lo(xw[i]), yv[8 * qq + 2 * i]);
-                        o[2 * i + 1] = fmaf(Dh, bf16hi(xw[i]), yv[8 * qq + 2 * i + 1]);
-                    }
                     uint4 ov;
-                    ov.x = pack_bf16(o[0], o[1]);
-                    ov.y = pack_bf16(o[2], o[3]);
-                    ov.z = pack_bf16(o[4], o[5]);
-                    ov.w = pack_bf16(o[6], o[7]);
+                    ov.x = pack_bf16(yv[8 * qq + 0], yv[8 * qq + 1]);
+                    ov.y = pack_bf16(yv[8 * qq + 2], yv[8 * qq + 3]);
+                    ov.z = pack_bf16(yv[8 * qq + 4], yv[8 * qq + 5]);
+                    ov.w = pack_bf16(yv[8 * qq + 6], yv[8 * qq + 7]);
                     *reinterpret_cast<uint4 *>(xt + swz(r, q)) = ov;
                 }
             }
