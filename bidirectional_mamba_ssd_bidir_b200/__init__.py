@@ -10,6 +10,7 @@ library has not been built.
 
 Entry points (same names as the C ABI):
   ssd_scan(x, dt, A, B, C, D=None, direction=1, chunk=256)   one direction
+  ssd_scan_state(..., state_in=None)                          one direction, state in and out
   bidir_ssd(fwd, rev, chunk=256)                              y_fwd + flip(scan(flip(.)))
   r2l_block_scan(p, s, residual, chunk=32)                    residual + s * y_rev
   bidir_ssd_noalloc(fwd, rev, out, chunk=256)                 bidir_ssd into a caller-owned `out`,
@@ -22,7 +23,7 @@ import os
 
 import torch
 
-__all__ = ["ssd_scan", "bidir_ssd", "r2l_block_scan", "bidir_ssd_noalloc", "noalloc_status", "workspace_bytes", "path_for",
+__all__ = ["ssd_scan", "ssd_scan_state", "bidir_ssd", "r2l_block_scan", "bidir_ssd_noalloc", "noalloc_status", "workspace_bytes", "path_for",
            "kernel_launches", "workspace_status", "SSDError", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -60,6 +61,8 @@ lib.ssd_kernel_launches.restype = ctypes.c_int
 lib.ssd_scan.argtypes = [_SP, _PP, ctypes.c_int, ctypes.c_int, _VP, _VP, _SZ, _VP]
 lib.ssd_scan.restype = ctypes.c_int
 lib.bidir_ssd.argtypes = [_SP, _PP, _PP, ctypes.c_int, _VP, _VP, _SZ, _VP]
+lib.ssd_scan_state.argtypes = [_SP, _PP, ctypes.c_int, ctypes.c_int, _VP, _VP, _VP, _VP, _SZ, _VP]
+lib.ssd_scan_state.restype = ctypes.c_int
 lib.bidir_ssd.restype = ctypes.c_int
 lib.r2l_block_scan.argtypes = [_SP, _PP, ctypes.c_float, _VP, ctypes.c_int, _VP, _VP, _SZ, _VP]
 lib.r2l_block_scan.restype = ctypes.c_int
@@ -167,6 +170,29 @@ def ssd_scan(x, dt, A, B, C, D=None, direction: int = 1, chunk: int = 256, out=N
     _check(lib.ssd_scan(ctypes.byref(shape), ctypes.byref(prm), int(direction), int(chunk),
                         y.data_ptr(), ws.data_ptr(), nbytes, _stream(x.device)))
     return y
+
+
+def ssd_scan_state(x, dt, A, B, C, D=None, direction: int = 1, chunk: int = 256, state_in=None,
+                   out=None, state_out=None, workspace=None):
+    """One direction with the state carried across the call: returns (y, state_out).
+
+    ``state_in`` (float32 [batch, nheads, headdim, dstate], or None = zero) is the state before
+    the first token in scan order; the returned state is the one after the last token."""
+    shape = _shape_of(x, B)
+    prm = _params(x, dt, A, B, C, D)
+    b, L, H, P = x.shape
+    N = B.shape[3]
+    for name, t in (("state_in", state_in), ("state_out", state_out)):
+        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != (b, H, P, N) or
+                              t.device != x.device or not t.is_contiguous()):
+            raise ValueError(f"{name} must be contiguous float32 of shape {(b, H, P, N)} on {x.device}")
+    y = torch.empty_like(x) if out is None else out
+    so = torch.empty((b, H, P, N), dtype=torch.float32, device=x.device) if state_out is None else state_out
+    ws, nbytes = _workspace(shape, chunk, x.device, workspace)
+    _check(lib.ssd_scan_state(ctypes.byref(shape), ctypes.byref(prm), int(direction), int(chunk),
+                              state_in.data_ptr() if state_in is not None else None, so.data_ptr(),
+                              y.data_ptr(), ws.data_ptr(), nbytes, _stream(x.device)))
+    return y, so
 
 
 def bidir_ssd(fwd: dict, rev: dict, chunk: int = 256, out=None, workspace=None):

@@ -88,10 +88,11 @@ ssd_status check_params(const ssd_params *p, const char *which) {
     return SSD_OK;
 }
 
-// SIMT-path workspace: [status | decays (batch*H*nc floats) | states (batch*H*nc*P*N floats)]
+// SIMT-path workspace: [status | decays (batch*H*nc floats) | states (batch*H*nc*P*N floats)].
+// A single chunk needs the decays and states only when a state crosses the call boundary
+// (ssd_scan_state); the size reported is the larger one.
 size_t simt_ws_bytes(const ssd_shape *s, int chunk) {
     const size_t units = (size_t)s->batch * s->nheads * (s->seqlen / chunk);
-    if (s->seqlen / chunk <= 1) return kStatusBytes;
     return kStatusBytes + round_up(units * sizeof(float)) + round_up(units * s->headdim * s->dstate * sizeof(float));
 }
 
@@ -116,6 +117,8 @@ ssd::ScanArgs make_args(const ssd_shape *s, const ssd_params *p, int dir, int ch
     const size_t units = (size_t)s->batch * s->nheads * a.nc;
     a.decays = reinterpret_cast<float *>(w);
     a.states = reinterpret_cast<float *>(w + round_up(units * sizeof(float)));
+    a.s_in = nullptr;
+    a.s_out = nullptr;
     return a;
 }
 
@@ -136,9 +139,11 @@ ssd_status common_checks(const ssd_shape *s, int chunk, void *out, void *ws, siz
 }
 
 ssd_status run_simt(const ssd_shape *s, const ssd_params *p, int dir, int chunk, void *y, void *ws,
-                    int mode, const void *residual, float gate, cudaStream_t st) {
+                    int mode, const void *residual, float gate, cudaStream_t st,
+                    const float *s_in = nullptr, float *s_out = nullptr) {
     ssd::ScanArgs a = make_args(s, p, dir, chunk, y, ws);
     a.mode = mode; a.residual = residual; a.gate = gate;
+    a.s_in = s_in; a.s_out = s_out;
     cudaError_t e = ssd::launch_simt_scan(a, s->io == SSD_BF16, st);
     return e == cudaSuccess ? SSD_OK : cuda_fail(e, "SIMT scan launch");
 }
@@ -186,6 +191,43 @@ ssd_status ssd_scan(const ssd_shape *shape, const ssd_params *p, int direction, 
         return e == cudaSuccess ? SSD_OK : cuda_fail(e, "tensor-core scan launch");
     }
     return run_simt(shape, p, direction, chunk, y, workspace, ssd::OUT_WRITE, nullptr, 0.f, cs);
+}
+
+ssd_status ssd_scan_state(const ssd_shape *shape, const ssd_params *p, int direction, int chunk,
+                          const float *state_in, float *state_out, void *y, void *workspace,
+                          size_t workspace_bytes, void *stream) {
+    g_err.clear();
+    ssd_status st = check_shape(shape, chunk);
+    if (st != SSD_OK) return st;
+    if (direction != 1 && direction != -1) return fail(SSD_ERR_INVALID_ARG, "direction must be +1 or -1");
+    if ((reinterpret_cast<uintptr_t>(state_in) & 3u) || (reinterpret_cast<uintptr_t>(state_out) & 3u))
+        return fail(SSD_ERR_INVALID_ARG, "states must be 4-byte aligned");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (shape->batch == 0) return SSD_OK;
+    if (shape->seqlen == 0) {
+        // no token: the state passes through unchanged
+        if (!state_out) return SSD_OK;
+        const size_t bytes = (size_t)shape->batch * shape->nheads * shape->headdim * shape->dstate * sizeof(float);
+        cudaError_t e = state_in ? cudaMemcpyAsync(state_out, state_in, bytes, cudaMemcpyDeviceToDevice, cs)
+                                 : cudaMemsetAsync(state_out, 0, bytes, cs);
+        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "state pass-through");
+    }
+    bool empty = false;
+    if ((st = common_checks(shape, chunk, y, workspace, workspace_bytes, &empty)) != SSD_OK) return st;
+    if ((st = check_params(p, "scan")) != SSD_OK) return st;
+    if (choose_path(shape, chunk) == 1) {
+        ssd::TcArgs t = ssd::make_tc_args(shape->batch, shape->seqlen, shape->nheads, chunk,
+                                          static_cast<char *>(workspace) + kStatusBytes,
+                                          static_cast<int *>(workspace));
+        t.wait_cycles = wait_cycles_now();
+        t.fault = g_fault.load();
+        t.s_in = state_in;
+        t.s_out = state_out;
+        ssd::tc_set_direction(t, 0, direction, p->x, p->dt, p->A, p->B, p->C, p->D);
+        cudaError_t e = ssd::launch_tc(t, /*bidir=*/false, y, cs);
+        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "tensor-core scan launch");
+    }
+    return run_simt(shape, p, direction, chunk, y, workspace, ssd::OUT_WRITE, nullptr, 0.f, cs, state_in, state_out);
 }
 
 ssd_status bidir_ssd(const ssd_shape *shape, const ssd_params *fwd, const ssd_params *rev, int chunk, void *y,

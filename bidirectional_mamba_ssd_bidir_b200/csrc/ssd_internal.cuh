@@ -31,6 +31,8 @@ struct ScanArgs {
     int mode;
     float *states;           // [batch][H][nc][P][N] chunk states -> incoming states
     float *decays;           // [batch][H][nc] chunk decay exp(cs_last)
+    const float *s_in;       // [batch][H][P][N] state before the first scanned token, or null (zero)
+    float *s_out;            // [batch][H][P][N] state after the last scanned token, or null
 };
 
 // token index in memory for scan position k

@@ -11,7 +11,7 @@
 //     from state   y_off[k]  = exp(cs_k) C_k . Sin_c
 // in three launches: chunk states (all chunks in parallel), the sequential
 // pass over chunks, and the outputs (all chunks in parallel).  A single-chunk
-// sequence skips the first two.
+// sequence skips the first two unless a state enters or leaves the call.
 #include "ssd_internal.cuh"
 
 namespace ssd {
@@ -106,8 +106,9 @@ __global__ void __launch_bounds__(kThreads) k_state_pass(ScanArgs a) {
     constexpr int E = P * N / kThreads;
     const int h = blockIdx.x, b = blockIdx.y;
     float run[E];
+    const size_t sbase = ((size_t)b * a.H + h) * P * N;     // [b][h] slot of s_in / s_out
 #pragma unroll
-    for (int j = 0; j < E; ++j) run[j] = 0.f;
+    for (int j = 0; j < E; ++j) run[j] = a.s_in ? a.s_in[sbase + threadIdx.x + kThreads * j] : 0.f;
     const size_t base = ((size_t)b * a.H + h) * a.nc;
     for (int c = 0; c < a.nc; ++c) {
         float *S = a.states + (base + c) * P * N;
@@ -119,6 +120,10 @@ __global__ void __launch_bounds__(kThreads) k_state_pass(ScanArgs a) {
             S[e] = run[j];                       // state entering chunk c
             run[j] = fmaf(dc, run[j], sc);
         }
+    }
+    if (a.s_out) {
+#pragma unroll
+        for (int j = 0; j < E; ++j) a.s_out[sbase + threadIdx.x + kThreads * j] = run[j];
     }
 }
 
@@ -226,7 +231,8 @@ __global__ void __launch_bounds__(kThreads) k_chunk_output(ScanArgs a, int have_
 
 template <typename T, int P, int N>
 cudaError_t launch_typed(const ScanArgs &a, cudaStream_t st) {
-    const bool multi = a.nc > 1;
+    // the state kernels run whenever a state crosses a chunk or the call boundary
+    const bool multi = a.nc > 1 || a.s_in || a.s_out;
     const size_t sm_state = sizeof(float) * (2 * a.Q + kSTile * P + kSTile * N);
     const size_t sm_out = sizeof(float) * (2 * a.Q + kRows * N + (multi ? P * (N + 1) : 0) +
                                            kSTile * (N + 1) + kSTile * P + kRows * kSTile);

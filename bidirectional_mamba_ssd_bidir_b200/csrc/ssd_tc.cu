@@ -169,6 +169,8 @@ struct TcParams {
     unsigned long long epoch;
     long long wait_cycles;              // bound of every device-side wait
     int fault;                          // test hook: 1 = the first direction never publishes its part
+    const float *s_in;                  // single direction: [batch][H][P][N] state entering the scan, or null
+    float *s_out;                       // single direction: [batch][H][P][N] state leaving the scan, or null
 };
 
 struct TcMaps {
@@ -416,7 +418,10 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 
 // ------------------------------------------------------------------ the kernel
 
-__global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ TcMaps maps, TcParams prm) {
+// kState: the state may enter and leave the call (single-direction scan with a carried state);
+// the instantiation without it is the one the bidirectional mixer and plain scans run.
+template <bool kState>
+__global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ TcMaps maps, const __grid_constant__ TcParams prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -433,6 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
     const int b = unit / npairs, hp = unit % npairs;
     const int h0 = 2 * hp;
     const int nblk = prm.nblk, L = prm.L;
+    const int has_in = kState && prm.s_in != nullptr;   // a state enters the scan (single direction)
     const CUtensorMap *map_x = &maps.x[slot], *map_dt = &maps.dt[slot], *map_b = &maps.b[slot],
                       *map_c = &maps.c[slot];
 
@@ -533,12 +539,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                     mma_ss(tmem + kColG, sdesc(aC + off, 16, 1024), sdesc(aB + off, 16, 1024), id_g, ks > 0);
                 }
                 mma_commit(bar(B_GFULL));
-                if (j >= 1) {
+                if (j >= 1 || has_in) {
                     // Y_off = C S'^T of the state entering this block (M = rows, N = (head, p), K = n);
                     // SP holds bf16(S') and the float32 state has been scaled by this block's decay
-                    if (!mbar_wait(bar(B_SPREADY), (j - 1) & 1, MASK, abort_flag, prm.status, 23)) break;
+                    if (!mbar_wait(bar(B_SPREADY), (j - 1 + has_in) & 1, MASK, abort_flag, prm.status, 23)) break;
                     // the previous block's epilogue has read both Y accumulators
-                    if (!mbar_wait(bar(B_YEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 24)) break;
+                    if (j >= 1 && !mbar_wait(bar(B_YEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 24)) break;
                     SSD_TRACE_PT(kWarpMma, j, 1);
                     tc_fence_after();
                     for (int ks = 0; ks < 8; ++ks) {
@@ -554,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = ks * 2048;
                     mma_ss(tmem + kColST, sdesc(aB + off, kTileBytes, 1024), sdesc(aWX + off, kTileBytes, 1024), id_s,
-                           (j > 0) || (ks > 0));
+                           (j > 0) || has_in || (ks > 0));
                 }
                 mma_commit(bar(B_STFULL));
                 mma_commit(bar(B_BCEMPTY));
@@ -771,6 +777,37 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
         // (entering block jj) in TMEM; thread r holds row n = r of this half's 32 columns.
         // bf16(S') goes to smem for Y_off = C S'^T, and S' is scaled in place by block jj's
         // decay so that block jj's state MMA accumulates S' <- exp(cs_last) S' + S directly.
+        // state entering the scan (single direction with a carried state): S' of this row
+        // (n = r) and half is read from global memory, a bf16 copy goes to smem for block 0's
+        // Y_off and S' is scaled in place by block 0's decay, as the hand-off does between blocks
+        const size_t sslot = ((size_t)b * prm.H + h) * kP * kN;   // [b][h] slot of s_in / s_out
+        auto init_pass = [&]() {
+            const float ablk = tab_s[kTabA + hs];
+#pragma unroll 1
+            for (int qd = 0; qd < 2; ++qd) {
+                float sv[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sv[i] = prm.s_in[sslot + (size_t)(32 * c + 16 * qd + i) * kN + r];
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    uint4 o;
+                    o.x = pack_bf16(sv[8 * qq + 0], sv[8 * qq + 1]);
+                    o.y = pack_bf16(sv[8 * qq + 2], sv[8 * qq + 3]);
+                    o.z = pack_bf16(sv[8 * qq + 4], sv[8 * qq + 5]);
+                    o.w = pack_bf16(sv[8 * qq + 6], sv[8 * qq + 7]);
+                    *reinterpret_cast<uint4 *>(sp_tile + swz(r, 4 * c + 2 * qd + qq)) = o;
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sv[i] *= ablk;
+                tmem_st16f_nw(tl + colST + 16 * qd, sv);
+            }
+            fence_async_smem();                // SP is read by the tensor core
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_SPREADY));
+        };
+
         auto state_pass = [&](int jj) {
             const float ablk = tab_s[(jj & 1) * kTabFloats + kTabA + hs];
             tc_fence_after();
@@ -811,6 +848,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 SSD_TRACE_PT(warp, j, 6);
                 state_pass(j);
                 SSD_TRACE_PT(warp, j, 7);
+            } else if (has_in) {
+                init_pass();
             }
 
             // M_h = G (.) decay (.) dt over the causal triangle, bf16, for both heads.  This
@@ -920,7 +959,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             {
                 uint8_t *xt = sm + kOffX + st * kStageBytes + hs * kTileBytes;
                 float yv[32];
-                if (j >= 1) {
+                if (j >= 1 || has_in) {
                     // Y_off of the incoming state, scaled by the decay exp(cs_r) up to this row
                     const float er = tb[kTabER + hs * kBlk + r];
                     float yo[32];
@@ -949,6 +988,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 mbar_arrive(bar(B_TILE00 + 2 * hs + st));
             }
             SSD_TRACE_PT(warp, j, 21);
+            if (kState && j + 1 == nblk && prm.s_out) {
+                // state leaving the scan: S' after the last block's state MMA, row n = r
+                if (!mbar_wait(bar(B_STFULL), j & 1, MASK, abort_flag, prm.status, 49)) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int qd = 0; qd < 2; ++qd) {
+                    float sv[16];
+                    tmem_ld16(tl + colST + 16 * qd, sv);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) prm.s_out[sslot + (size_t)(32 * c + 16 * qd + i) * kN + r] = sv[i];
+                }
+            }
         }
     }
 
@@ -1043,7 +1094,9 @@ cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(k_ssd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+        attr_err = cudaFuncSetAttribute(k_ssd_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(k_ssd_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
     const int ndir = bidir ? 2 : 1;
@@ -1072,8 +1125,13 @@ cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
     p.epoch = next_epoch();
     p.wait_cycles = t.wait_cycles;
     p.fault = t.fault;
+    p.s_in = bidir ? nullptr : t.s_in;
+    p.s_out = bidir ? nullptr : t.s_out;
     const int grid = t.batch * (t.H / 2) * ndir;
-    k_ssd_tc<<<grid, kThreads, kSmemBytes, st>>>(maps, p);
+    if (p.s_in || p.s_out)
+        k_ssd_tc<true><<<grid, kThreads, kSmemBytes, st>>>(maps, p);
+    else
+        k_ssd_tc<false><<<grid, kThreads, kSmemBytes, st>>>(maps, p);
     return cudaGetLastError();
 }
 

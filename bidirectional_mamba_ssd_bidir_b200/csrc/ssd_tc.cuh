@@ -19,6 +19,8 @@ struct TcArgs {
     int *status;       // device status word
     long long wait_cycles;   // bound of every device-side wait, in SM clock cycles
     int fault;               // test hook (0 = none)
+    const float *s_in;       // single direction only: [batch][H][P][N] state entering the scan, or null
+    float *s_out;            // single direction only: [batch][H][P][N] state leaving the scan, or null
 };
 
 bool tc_supported(bool bf16, int batch, int L, int H, int P, int N, int G, int chunk);

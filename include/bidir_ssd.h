@@ -100,6 +100,25 @@ size_t ssd_workspace_bytes(const ssd_shape *shape, int chunk);
 ssd_status ssd_scan(const ssd_shape *shape, const ssd_params *p, int direction, int chunk,
                     void *y, void *workspace, size_t workspace_bytes, void *stream);
 
+/* ssd_scan with the state carried across the call boundary, for block-wise
+ * decoding: the DiffuMamba page (technical summary, section 2, training and
+ * inference: block diffusion with cache reuse; section 4, block caching)
+ * reuses what precedes a block, and for a Mamba layer that is this state.
+ *
+ * state_in  [batch][nheads][headdim][dstate] float32: the state S before the
+ *           first token in scan order (the token at t = 0 forward, t = L-1
+ *           reverse); NULL = zero, which makes the call ssd_scan.
+ * state_out [batch][nheads][headdim][dstate] float32: receives S after the
+ *           last token in scan order; NULL = not wanted.
+ * Both are device pointers, 4-byte aligned; state_in and state_out may be the
+ * same buffer.  Scanning a sequence in pieces, each piece starting from the
+ * previous piece's state_out, gives the y and final state of the whole
+ * sequence up to rounding.  seqlen = 0 copies state_in to state_out (or zeroes
+ * it).  Same layouts, workspace and errors as ssd_scan. */
+ssd_status ssd_scan_state(const ssd_shape *shape, const ssd_params *p, int direction, int chunk,
+                          const float *state_in, float *state_out, void *y,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
 /* The DiffuMamba bidirectional mixer ("DiffuMamba", technical summary,
  * section 2: a forward and a reverse Mamba layer, independent of each other,
  * for a symmetric context): y = scan(fwd, +1) + scan(rev, -1), the two
