@@ -20,6 +20,8 @@ Contents
                    ("Bifocal Diffusion Language Models", section 2,
                    mechanism and integration).  s = 0 returns the residual
                    itself, so the model is unchanged at initialisation.
+``ssd_scan_bwd_f64`` the gradients of the scan (reverse-mode, position by
+                   position), for training the layers that run it.
 ``ssd_scan_state_f64`` the recurrence with the state carried across the call
                    (state in, state out), for block-wise decoding.
 ``ssd_chunked_f64`` the chunked (state-passing) form of the same scan, the
@@ -66,6 +68,10 @@ def load_library(path: str | None = None):
     dp = ctypes.POINTER(ctypes.c_double)
     f.argtypes = [ctypes.c_int] * 6 + [dp] * 6 + [ctypes.c_int, dp, ctypes.c_int]
     f.restype = ctypes.c_int
+    if hasattr(lib, "ssd_oracle_scan_bwd"):
+        k = lib.ssd_oracle_scan_bwd
+        k.argtypes = [ctypes.c_int] * 6 + [dp] * 6 + [ctypes.c_int, dp] + [dp] * 6 + [ctypes.c_int]
+        k.restype = ctypes.c_int
     if hasattr(lib, "ssd_oracle_scan_state"):
         g = lib.ssd_oracle_scan_state
         g.argtypes = [ctypes.c_int] * 6 + [dp] * 6 + [ctypes.c_int, dp, dp, dp, ctypes.c_int]
@@ -129,6 +135,32 @@ def ssd_scan_state_f64(x, dt, A, B, C, D=None, direction=1, init_state=None, nth
     if rc != 0:
         raise RuntimeError(f"ssd_oracle_scan_state failed with {rc}")
     return y, s_out
+
+
+def ssd_scan_bwd_f64(x, dt, A, B, C, D, direction, gy, nthreads=None, lib=None):
+    """Gradients of L = sum(gy * y) for the scan from a zero state: dict with x, dt, A, B, C, D.
+
+    The reverse-mode derivative of the recurrence, taken position by position
+    (oracle header); D's entry is None when D is None."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    dt = np.ascontiguousarray(dt, dtype=np.float64)
+    A = np.ascontiguousarray(A, dtype=np.float64)
+    B = np.ascontiguousarray(B, dtype=np.float64)
+    C = np.ascontiguousarray(C, dtype=np.float64)
+    D = None if D is None else np.ascontiguousarray(D, dtype=np.float64)
+    gy = np.ascontiguousarray(gy, dtype=np.float64)
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    assert gy.shape == x.shape
+    g = {"x": np.zeros_like(x), "dt": np.zeros_like(dt), "A": np.zeros(H), "B": np.zeros_like(B),
+         "C": np.zeros_like(C), "D": None if D is None else np.zeros(H)}
+    lib = lib or load_library()
+    rc = lib.ssd_oracle_scan_bwd(b, L, H, P, N, G, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                 int(direction), _ptr(gy), _ptr(g["x"]), _ptr(g["dt"]), _ptr(g["A"]),
+                                 _ptr(g["B"]), _ptr(g["C"]), _ptr(g["D"]), int(nthreads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"ssd_oracle_scan_bwd failed with {rc}")
+    return g
 
 
 def bidir_f64(pf: dict, pr: dict, nthreads=None, lib=None):

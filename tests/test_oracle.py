@@ -287,3 +287,66 @@ def test_empty_sequence_passes_the_state_through():
     s0 = rng.standard_normal((2, 3, 4, 5))
     _, s = _scan_state(_piece(p, 0, 0), 1, s0)
     assert np.array_equal(s, s0)
+
+
+# ------------------------------------------------------------------ gradients
+
+def _loss(p, direction, gy):
+    return float(np.sum(gy * _scan(p, direction)))
+
+
+def _grads(p, direction, gy):
+    return oracle.ssd_scan_bwd_f64(p["x"], p["dt"], p["A"], p["B"], p["C"], p.get("D"), direction, gy)
+
+
+@pytest.mark.parametrize("direction", [1, -1])
+@pytest.mark.parametrize("G", [1, 2])
+def test_gradients_match_central_differences(direction, G):
+    """Every gradient entry against a central difference of L = sum(gy * y) computed with the forward
+    recurrence, on a small problem (L = 11 crosses no checkpoint; the second case is grouped)."""
+    rng = np.random.default_rng(21 + G)
+    p = _rand_params(rng, 2, 11, 4, 3, 4, G)
+    gy = rng.standard_normal(p["x"].shape)
+    g = _grads(p, direction, gy)
+    eps = 1e-6
+    for name in ("x", "dt", "A", "B", "C", "D"):
+        base = p[name]
+        idx = list(np.ndindex(base.shape))
+        pick = [idx[i] for i in rng.choice(len(idx), size=min(12, len(idx)), replace=False)]
+        for ix in pick:
+            q = {k: (v.copy() if v is not None else None) for k, v in p.items()}
+            q[name][ix] += eps
+            lp = _loss(q, direction, gy)
+            q[name][ix] -= 2 * eps
+            lm = _loss(q, direction, gy)
+            fd = (lp - lm) / (2 * eps)
+            assert abs(fd - g[name][ix]) <= 1e-6 * max(1.0, abs(fd)), (name, ix, fd, g[name][ix])
+
+
+def test_gradients_are_exact_for_the_linear_inputs():
+    """y is linear in x, and y - D x is linear in B and in C, so L = sum(gy * y) equals the gradient's
+    inner product with the input exactly: <gx, x> = L, <gB, B> = <gC, C> = L - <gy, D x>, and
+    gD = sum_t <gy_t, x_t>.  Long enough (L = 150) to cross the checkpoint segments."""
+    rng = np.random.default_rng(31)
+    p = _rand_params(rng, 2, 150, 3, 4, 5, 1)
+    gy = rng.standard_normal(p["x"].shape)
+    for direction in (1, -1):
+        g = _grads(p, direction, gy)
+        L_ = _loss(p, direction, gy)
+        Ldx = float(np.sum(gy * p["D"][None, None, :, None] * p["x"]))
+        assert abs(np.sum(g["x"] * p["x"]) - L_) <= 1e-10 * max(1.0, abs(L_))
+        assert abs(np.sum(g["B"] * p["B"]) - (L_ - Ldx)) <= 1e-10 * max(1.0, abs(L_))
+        assert abs(np.sum(g["C"] * p["C"]) - (L_ - Ldx)) <= 1e-10 * max(1.0, abs(L_))
+        np.testing.assert_allclose(g["D"], np.einsum("blhp,blhp->h", gy, p["x"]), rtol=1e-12)
+
+
+def test_gradients_reverse_is_flip_of_forward():
+    rng = np.random.default_rng(41)
+    p = _rand_params(rng, 1, 70, 2, 3, 4, 1)
+    gy = rng.standard_normal(p["x"].shape)
+    flip = {k: (v[:, ::-1].copy() if k in ("x", "dt", "B", "C") else v) for k, v in p.items()}
+    gr = _grads(p, -1, gy)
+    gf = _grads(flip, 1, gy[:, ::-1].copy())
+    for name in ("x", "dt", "B", "C"):
+        np.testing.assert_allclose(gr[name], gf[name][:, ::-1], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(gr["A"], gf["A"], rtol=1e-12)

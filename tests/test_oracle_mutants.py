@@ -35,6 +35,9 @@ MUTANTS = {
                              "acc += Ct[n] * Sp[n];\n                Sp[n] = decay * Sp[n] + u * Bt[n];"),
     "state_in_ignored": ("if (j->s_in)\n        memcpy", "if (0)\n        memcpy"),
     "state_slot_head_dropped": ("const size_t soff = ((size_t)b * H + h)", "const size_t soff = ((size_t)b * H)"),
+    "bwd_adjoint_not_decayed": ("G[i] *= a;", "G[i] *= 1.0;"),
+    "bwd_dt_gradient_misses_decay_term": ("gxb + a_h * a * q", "gxb"),
+    "bwd_B_gradient_without_dt": ("gBt[n] += dt * acc;", "gBt[n] += acc;"),
 }
 
 
@@ -89,6 +92,20 @@ def _pins_pass(lib) -> bool:
     g = np.arange(4) // 2
     ref0 = np.einsum("blh,bhpn,blhn->blhp", decay, s0, p["C"][:, :, g])
     checks.append(oracle.rel_err(y0, ref0) <= 1e-12)
+    # gradients: exact inner-product identities for x and B, a central difference for dt
+    gy = rng.standard_normal(p["x"].shape)
+    for d in (1, -1):
+        g = oracle.ssd_scan_bwd_f64(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], d, gy, lib=lib)
+        L_ = float(np.sum(gy * scan(p, d)))
+        Ldx = float(np.sum(gy * p["D"][None, None, :, None] * p["x"]))
+        checks.append(abs(np.sum(g["x"] * p["x"]) - L_) <= 1e-10 * max(1.0, abs(L_)))
+        checks.append(abs(np.sum(g["B"] * p["B"]) - (L_ - Ldx)) <= 1e-10 * max(1.0, abs(L_)))
+        q = {k: (v.copy() if v is not None else None) for k, v in p.items()}
+        q["dt"][0, 4, 1] += 1e-6
+        lp = float(np.sum(gy * scan(q, d)))
+        q["dt"][0, 4, 1] -= 2e-6
+        lm = float(np.sum(gy * scan(q, d)))
+        checks.append(abs((lp - lm) / 2e-6 - g["dt"][0, 4, 1]) <= 1e-6 * max(1.0, abs(lp - lm) / 2e-6))
     return all(bool(c) for c in checks)
 
 
