@@ -106,7 +106,7 @@ constexpr uint32_t kTabFloats = kTabA + 4;
 constexpr uint32_t kOffTab = kOffSP + 2 * kTileBytes;   // 2 buffers
 constexpr uint32_t kOffDT = (kOffTab + 2 * kTabFloats * 4 + 127) / 128 * 128;   // dt ring, 2 slots
 constexpr uint32_t kOffBar = kOffDT + 2 * kDtBytes;
-constexpr uint32_t kNumBars = 24;
+constexpr uint32_t kNumBars = 25;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
 static_assert(kStageBytes % 1024 == 0, "x tiles must stay 1024-byte aligned");
@@ -120,7 +120,7 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 enum Bar {
     B_XFULL0 = 0, B_XFULL1, B_XEMPTY0, B_XEMPTY1, B_BCFULL, B_BCEMPTY, B_GFULL, B_WXREADY, B_SPREADY, B_STFULL,
     B_MREADY, B_YFULL, B_YEMPTY, B_DONE, B_TILE00, B_TILE01, B_TILE10, B_TILE11, B_TABREADY0, B_TABREADY1,
-    B_DTFULL0, B_DTFULL1, B_DTEMPTY0, B_DTEMPTY1
+    B_DTFULL0, B_DTFULL1, B_DTEMPTY0, B_DTEMPTY1, B_YFULLH0
 };
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -570,10 +570,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 29)) break;
                 SSD_TRACE_PT(kWarpMma, j, 3);
                 tc_fence_after();
-                for (int h = 0; h < 2; ++h)
+                for (int h = 0; h < 2; ++h) {
                     for (int ks = 0; ks < 8; ++ks)
                         mma_ts(tmem + kColYD + 64 * h, tmem + kColG + 16 * ks + 8 * h,
                                sdesc(aX + h * kTileBytes + ks * 2048, kTileBytes, 1024), id_yd, 1);
+                    // head 0's warps can start their epilogue while head 1's MMAs run
+                    if (h == 0) mma_commit(bar(B_YFULLH0));
+                }
                 mma_commit(bar(B_YFULL));
             }
             // drain: every MMA issued above has completed before TMEM is released
@@ -953,7 +956,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             // epilogue: o = Y_diag (which started at D x) + exp(cs_r) Y_off, bf16, written over this row of the x
             // tile (free once the intra-block MMA is done); a store warp then writes the tile to y
             // in whole rows
-            if (!mbar_wait(bar(B_YFULL), j & 1, MASK, abort_flag, prm.status, 46)) break;
+            if (!mbar_wait(bar(hs == 0 ? B_YFULLH0 : B_YFULL), j & 1, MASK, abort_flag, prm.status, 46)) break;
             SSD_TRACE_PT(warp, j, 16);
             tc_fence_after();
             {
