@@ -339,6 +339,55 @@ def run_ours(args) -> None:
 
 # ------------------------------------------------------------------ reference arm (the oracle)
 
+def run_bwd(args) -> None:
+    """Gradients of the bidirectional mixer (both directions, the same dL/dy), one GPU, device-timed."""
+    import torch
+    import bidirectional_mamba_ssd_bidir_b200 as ssd
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    plan = shard_plan(0, 1, args.workload, args.batch)
+    shape, chunk = plan["shape"], plan["chunk"]
+    pf, pr = si.make_bidir(shape, seed=0)
+    fwd = {k: getattr(pf, k).torch(dev) for k in ("x", "dt", "A", "B", "C", "D")}
+    rev = {k: getattr(pr, k).torch(dev) for k in ("x", "dt", "A", "B", "C", "D")}
+    gy = torch.randn(fwd["x"].shape, device=dev).to(fwd["x"].dtype)
+    dims = (shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate, shape.ngroups)
+    s_ = ssd._Shape(*dims, ssd.SSD_BF16 if shape.io == "bf16" else ssd.SSD_F32)
+    ws = torch.empty(int(ssd.lib.ssd_bwd_workspace_bytes(ssd.ctypes.byref(s_), chunk)), dtype=torch.uint8, device=dev)
+
+    def step():
+        ssd.ssd_scan_bwd(**fwd, gy=gy, direction=1, chunk=chunk, workspace=ws)
+        ssd.ssd_scan_bwd(**rev, gy=gy, direction=-1, chunk=chunk, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    with ClockSampler(0) as clk:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / args.steps
+    e = 2 if shape.io == "bf16" else 4
+    H, P, N, G = shape.nheads, shape.headdim, shape.dstate, shape.ngroups
+    # per token and direction: read x, dt, B, C, gy; write float32 dx, ddt, dB, dC
+    bpt = 2 * (e * (2 * H * P + H + 2 * G * N) + 4 * (H * P + H + 2 * G * N))
+    peaks = measured_peaks()
+    achieved = bpt * plan["tokens"] / (ms / 1e3) / 1e9
+    line = {"metric": "bidirectional SSD scan gradients tokens/s (both directions)", "op": "bwd",
+            "value": plan["tokens"] / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "f32",
+            "data": "synthetic", "config": {"workload": args.workload, "global_batch": shape.batch,
+                                             "seq_len": shape.seqlen, "chunk": chunk, "path": "simt"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "bytes_per_token": bpt},
+            "gpu_launches": 2 * 5 * args.steps, "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args) -> None:
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -386,6 +435,8 @@ def main(argv=None):
                                                                       if v["kind"] == "bidir"])
     ap.add_argument("--batch", type=int, default=None,
                     help="replace the workload's batch size (a smaller case of the same shape, for profiling)")
+    ap.add_argument("--op", choices=["fwd", "bwd"], default="fwd",
+                    help="bwd: time the gradients of both directions instead (an extra line, one GPU)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU work of the oracle baseline sample")
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds for the reference arm's steps")
@@ -394,6 +445,8 @@ def main(argv=None):
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.op == "bwd":
+        run_bwd(args)
     else:
         run_ours(args)
 

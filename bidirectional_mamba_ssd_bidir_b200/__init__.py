@@ -11,6 +11,7 @@ library has not been built.
 Entry points (same names as the C ABI):
   ssd_scan(x, dt, A, B, C, D=None, direction=1, chunk=256)   one direction
   ssd_scan_state(..., state_in=None)                          one direction, state in and out
+  ssd_scan_bwd(x, dt, A, B, C, D, gy, direction, chunk)       gradients of one direction
   bidir_ssd(fwd, rev, chunk=256)                              y_fwd + flip(scan(flip(.)))
   r2l_block_scan(p, s, residual, chunk=32)                    residual + s * y_rev
   bidir_ssd_noalloc(fwd, rev, out, chunk=256)                 bidir_ssd into a caller-owned `out`,
@@ -23,7 +24,7 @@ import os
 
 import torch
 
-__all__ = ["ssd_scan", "ssd_scan_state", "bidir_ssd", "r2l_block_scan", "bidir_ssd_noalloc", "noalloc_status", "workspace_bytes", "path_for",
+__all__ = ["ssd_scan", "ssd_scan_state", "ssd_scan_bwd", "bidir_ssd", "r2l_block_scan", "bidir_ssd_noalloc", "noalloc_status", "workspace_bytes", "path_for",
            "kernel_launches", "workspace_status", "SSDError", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -63,6 +64,10 @@ lib.ssd_scan.restype = ctypes.c_int
 lib.bidir_ssd.argtypes = [_SP, _PP, _PP, ctypes.c_int, _VP, _VP, _SZ, _VP]
 lib.ssd_scan_state.argtypes = [_SP, _PP, ctypes.c_int, ctypes.c_int, _VP, _VP, _VP, _VP, _SZ, _VP]
 lib.ssd_scan_state.restype = ctypes.c_int
+lib.ssd_bwd_workspace_bytes.argtypes = [_SP, ctypes.c_int]
+lib.ssd_bwd_workspace_bytes.restype = _SZ
+lib.ssd_scan_bwd.argtypes = [_SP, _PP, ctypes.c_int, ctypes.c_int, _VP] + [_VP] * 6 + [_VP, _SZ, _VP]
+lib.ssd_scan_bwd.restype = ctypes.c_int
 lib.bidir_ssd.restype = ctypes.c_int
 lib.r2l_block_scan.argtypes = [_SP, _PP, ctypes.c_float, _VP, ctypes.c_int, _VP, _VP, _SZ, _VP]
 lib.r2l_block_scan.restype = ctypes.c_int
@@ -193,6 +198,27 @@ def ssd_scan_state(x, dt, A, B, C, D=None, direction: int = 1, chunk: int = 256,
                               state_in.data_ptr() if state_in is not None else None, so.data_ptr(),
                               y.data_ptr(), ws.data_ptr(), nbytes, _stream(x.device)))
     return y, so
+
+
+def ssd_scan_bwd(x, dt, A, B, C, D, gy, direction: int = 1, chunk: int = 256, workspace=None) -> dict:
+    """Gradients of ssd_scan for dL/dy = gy: dict with float32 x, dt, A, B, C and D (None if D is None)."""
+    shape = _shape_of(x, B)
+    prm = _params(x, dt, A, B, C, D)
+    if gy.shape != x.shape or gy.dtype != x.dtype or gy.device != x.device or not gy.is_contiguous():
+        raise ValueError(f"gy must be a contiguous {x.dtype} tensor of shape {tuple(x.shape)} on {x.device}")
+    dev = x.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = {"x": torch.empty(x.shape, **f32), "dt": torch.empty(dt.shape, **f32), "A": torch.empty(A.shape, **f32),
+         "B": torch.empty(B.shape, **f32), "C": torch.empty(C.shape, **f32),
+         "D": torch.empty(A.shape, **f32) if D is not None else None}
+    need = int(lib.ssd_bwd_workspace_bytes(ctypes.byref(shape), int(chunk)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    ptr = lambda t: t.data_ptr() if t is not None else None
+    _check(lib.ssd_scan_bwd(ctypes.byref(shape), ctypes.byref(prm), int(direction), int(chunk), gy.data_ptr(),
+                            ptr(g["x"]), ptr(g["dt"]), ptr(g["A"]), ptr(g["B"]), ptr(g["C"]), ptr(g["D"]),
+                            workspace.data_ptr(), workspace.numel(), _stream(dev)))
+    return g
 
 
 def bidir_ssd(fwd: dict, rev: dict, chunk: int = 256, out=None, workspace=None):

@@ -230,6 +230,62 @@ ssd_status ssd_scan_state(const ssd_shape *shape, const ssd_params *p, int direc
     return run_simt(shape, p, direction, chunk, y, workspace, ssd::OUT_WRITE, nullptr, 0.f, cs, state_in, state_out);
 }
 
+size_t ssd_bwd_workspace_bytes(const ssd_shape *shape, int chunk) {
+    if (check_shape(shape, chunk) != SSD_OK) return 0;
+    const int Q = chunk < 64 ? chunk : 64;
+    const size_t nc = (size_t)shape->seqlen / Q, bh = (size_t)shape->batch * shape->nheads;
+    const size_t PN = (size_t)shape->headdim * shape->dstate, tokh = (size_t)shape->batch * shape->seqlen * shape->nheads;
+    return kStatusBytes + 2 * round_up(bh * nc * PN * sizeof(float)) + 2 * round_up(bh * nc * sizeof(float)) +
+           2 * round_up(tokh * shape->dstate * sizeof(float)) + 2 * round_up(tokh * sizeof(float)) +
+           2 * round_up(bh * sizeof(float));
+}
+
+ssd_status ssd_scan_bwd(const ssd_shape *shape, const ssd_params *p, int direction, int chunk, const void *gy,
+                        float *gx, float *gdt, float *gA, float *gB, float *gC, float *gD, void *workspace,
+                        size_t workspace_bytes, void *stream) {
+    g_err.clear();
+    ssd_status st = check_shape(shape, chunk);
+    if (st != SSD_OK) return st;
+    if (direction != 1 && direction != -1) return fail(SSD_ERR_INVALID_ARG, "direction must be +1 or -1");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (!gA) return fail(SSD_ERR_INVALID_ARG, "gA must be non-NULL");
+    const bool empty = shape->batch == 0 || shape->seqlen == 0;
+    if (empty) {
+        // no token: dA and dD are zero
+        cudaError_t e = cudaMemsetAsync(gA, 0, sizeof(float) * shape->nheads, cs);
+        if (e == cudaSuccess && gD) e = cudaMemsetAsync(gD, 0, sizeof(float) * shape->nheads, cs);
+        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "empty gradient clear");
+    }
+    if ((st = check_params(p, "scan")) != SSD_OK) return st;
+    if (!aligned16(gy)) return fail(SSD_ERR_INVALID_ARG, "gy must be non-NULL and 16-byte aligned");
+    if (!gx || !gdt || !gB || !gC) return fail(SSD_ERR_INVALID_ARG, "gx, gdt, gB and gC must be non-NULL");
+    if (gD && !p->D) return fail(SSD_ERR_INVALID_ARG, "gD requested but D is NULL");
+    const size_t need = ssd_bwd_workspace_bytes(shape, chunk);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)))
+        return fail(SSD_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+    if (workspace_bytes < need) return fail(SSD_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+    ssd::BwdArgs a{};
+    a.batch = shape->batch; a.L = shape->seqlen; a.H = shape->nheads; a.P = shape->headdim; a.N = shape->dstate;
+    a.G = shape->ngroups; a.Q = chunk < 64 ? chunk : 64; a.nc = shape->seqlen / a.Q; a.dir = direction;
+    a.x = p->x; a.dt = p->dt; a.B = p->B; a.C = p->C; a.gy = gy; a.A = p->A; a.D = p->D;
+    a.gx = gx; a.gdt = gdt; a.gA = gA; a.gB = gB; a.gC = gC; a.gD = gD;
+    const size_t nc = a.nc, bh = (size_t)a.batch * a.H, PN = (size_t)a.P * a.N, tokh = (size_t)a.batch * a.L * a.H;
+    char *w = static_cast<char *>(workspace) + kStatusBytes;
+    auto take = [&](size_t bytes) { float *f = reinterpret_cast<float *>(w); w += round_up(bytes); return f; };
+    a.sf = take(bh * nc * PN * sizeof(float));
+    a.sg = take(bh * nc * PN * sizeof(float));
+    a.dec = take(bh * nc * sizeof(float));
+    a.gxd = take(bh * nc * sizeof(float));
+    a.gBh = take(tokh * a.N * sizeof(float));
+    a.gCh = take(tokh * a.N * sizeof(float));
+    a.gcs = take(tokh * sizeof(float));
+    a.u = take(tokh * sizeof(float));
+    a.gAp = take(bh * sizeof(float));
+    a.gDp = take(bh * sizeof(float));
+    cudaError_t e = ssd::launch_simt_bwd(a, shape->io == SSD_BF16, cs);
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, "scan gradient launch");
+}
+
 ssd_status bidir_ssd(const ssd_shape *shape, const ssd_params *fwd, const ssd_params *rev, int chunk, void *y,
                      void *workspace, size_t workspace_bytes, void *stream) {
     g_err.clear();

@@ -49,8 +49,27 @@ template <> __device__ __forceinline__ void stf<__nv_bfloat16>(__nv_bfloat16 *p,
     p[i] = __float2bfloat16_rn(v);
 }
 
+// Gradients of one direction of the scan (ssd_bwd.cu).  Inputs in the io
+// dtype, gradients and every intermediate in float32.
+struct BwdArgs {
+    int batch, L, H, P, N, G, Q, nc;
+    int dir;
+    const void *x, *dt, *B, *C, *gy;
+    const float *A, *D;      // D may be null
+    float *gx, *gdt, *gA, *gB, *gC, *gD;   // gD may be null
+    // workspace
+    float *sf;               // [batch][H][nc][P][N] chunk states -> state entering each chunk
+    float *sg;               // [batch][H][nc][P][N] adjoint chunk terms -> adjoint entering from the right
+    float *dec;              // [batch][H][nc] decay across each chunk
+    float *gBh, *gCh;        // [batch][L][H][N] per-head parts of dB and dC
+    float *gcs, *u;          // [batch][L][H] dL/dcs and <G_k, x_k B_k^T> per token
+    float *gxd;              // [batch][H][nc] per-chunk sum of <gy, x>
+    float *gAp, *gDp;        // [batch][H] per-sequence parts of dA and dD
+};
+
 // Launchers (defined in the kernel translation units).  All return the
 // cudaError_t of the launch.
 cudaError_t launch_simt_scan(const ScanArgs &a, bool bf16, cudaStream_t st);
+cudaError_t launch_simt_bwd(const BwdArgs &a, bool bf16, cudaStream_t st);
 
 }  // namespace ssd

@@ -119,6 +119,26 @@ ssd_status ssd_scan_state(const ssd_shape *shape, const ssd_params *p, int direc
                           const float *state_in, float *state_out, void *y,
                           void *workspace, size_t workspace_bytes, void *stream);
 
+/* Gradients of ssd_scan (zero starting state), for training the layers that
+ * run it (the DiffuMamba page, technical summary, section 2, trains the Mamba
+ * backbone).  Given gy = dL/dy ([batch][seqlen][nheads][headdim], io dtype)
+ * it writes, all float32 device arrays:
+ *     gx  [batch][seqlen][nheads][headdim]      dL/dx
+ *     gdt [batch][seqlen][nheads]               dL/ddt
+ *     gA  [nheads]                              dL/dA, summed over the batch
+ *     gB  [batch][seqlen][ngroups][dstate]      dL/dB, summed over the heads of a group
+ *     gC  [batch][seqlen][ngroups][dstate]      dL/dC, likewise
+ *     gD  [nheads] or NULL                      dL/dD (NULL when p->D is NULL)
+ * The bidirectional mixer's gradients are the two directions' gradients for
+ * the same gy (y is their sum).  Runs on the CUDA cores in float32, chunked
+ * like the forward scan (at most 64 positions per chunk).  workspace must be
+ * 256-byte aligned and hold ssd_bwd_workspace_bytes(shape, chunk) bytes.  Errors
+ * as for ssd_scan. */
+size_t ssd_bwd_workspace_bytes(const ssd_shape *shape, int chunk);
+ssd_status ssd_scan_bwd(const ssd_shape *shape, const ssd_params *p, int direction, int chunk,
+                        const void *gy, float *gx, float *gdt, float *gA, float *gB, float *gC,
+                        float *gD, void *workspace, size_t workspace_bytes, void *stream);
+
 /* The DiffuMamba bidirectional mixer ("DiffuMamba", technical summary,
  * section 2: a forward and a reverse Mamba layer, independent of each other,
  * for a symmetric context): y = scan(fwd, +1) + scan(rev, -1), the two
