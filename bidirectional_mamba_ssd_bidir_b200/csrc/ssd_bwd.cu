@@ -150,36 +150,41 @@ template <typename T, int P, int N>
 __global__ void __launch_bounds__(kT) k_bwd_chunk(BwdArgs a) {
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int Q = a.Q, g = h / (a.H / a.G);
+    // rows of x, gy (stride P + 1), B, C (stride N + 1) and of the entering state and adjoint
+    // (stride N + 1) are padded by one word, so that a warp reading one column across rows hits
+    // 32 different banks
+    constexpr int SP = P + 1, SN = N + 1;
     extern __shared__ float sm[];
-    float *cs = sm, *dts = cs + 64, *xs = dts + 64, *gys = xs + Q * P, *bs = gys + Q * P, *cc = bs + Q * N;
-    float *CB = cc + Q * N, *XG = CB + Q * Q, *Lm = XG + Q * Q, *Sin = Lm + Q * Q, *Gin = Sin + P * N;
-    float *red = Gin + P * N;    // [3][64]: u, <gy, y - D x>, <gy, x> per position
+    float *cs = sm, *dts = cs + 64, *xs = dts + 64, *gys = xs + Q * SP, *bs = gys + Q * SP, *cc = bs + Q * SN;
+    float *CB = cc + Q * SN, *XG = CB + Q * Q, *Lm = XG + Q * Q, *Sin = Lm + Q * Q, *Gin = Sin + P * SN;
+    float *red = Gin + P * SN;   // [3][64]: u, <gy, y - D x>, <gy, x> per position
     bwd_cumsum<T>(a, b, h, c, cs, dts);
     const float cl = cs[Q - 1];
     for (int i = threadIdx.x; i < Q * P; i += kT) {
         const int k = i / P, p = i % P;
         const size_t xi = (((size_t)b * a.L + tok(c * Q + k, a.L, a.dir)) * a.H + h) * P + p;
-        xs[i] = ldf<T>((const T *)a.x, xi);
-        gys[i] = ldf<T>((const T *)a.gy, xi);
+        xs[k * SP + p] = ldf<T>((const T *)a.x, xi);
+        gys[k * SP + p] = ldf<T>((const T *)a.gy, xi);
     }
     for (int i = threadIdx.x; i < Q * N; i += kT) {
         const int k = i / N, n = i % N;
         const size_t bi = (((size_t)b * a.L + tok(c * Q + k, a.L, a.dir)) * a.G + g) * N + n;
-        bs[i] = ldf<T>((const T *)a.B, bi);
-        cc[i] = ldf<T>((const T *)a.C, bi);
+        bs[k * SN + n] = ldf<T>((const T *)a.B, bi);
+        cc[k * SN + n] = ldf<T>((const T *)a.C, bi);
     }
     const size_t sbase = (((size_t)b * a.H + h) * a.nc + c) * P * N;
     for (int i = threadIdx.x; i < P * N; i += kT) {
-        Sin[i] = a.sf[sbase + i];
-        Gin[i] = a.sg[sbase + i];
+        const int p = i / N, n = i % N;
+        Sin[p * SN + n] = a.sf[sbase + i];
+        Gin[p * SN + n] = a.sg[sbase + i];
     }
     for (int i = threadIdx.x; i < 3 * 64; i += kT) red[i] = 0.f;
     __syncthreads();
     for (int i = threadIdx.x; i < Q * Q; i += kT) {
         const int k = i / Q, s = i % Q;
         float cb = 0.f, xg = 0.f;
-        for (int n = 0; n < N; ++n) cb = fmaf(cc[k * N + n], bs[s * N + n], cb);
-        for (int p = 0; p < P; ++p) xg = fmaf(xs[k * P + p], gys[s * P + p], xg);
+        for (int n = 0; n < N; ++n) cb = fmaf(cc[k * SN + n], bs[s * SN + n], cb);
+        for (int p = 0; p < P; ++p) xg = fmaf(xs[k * SP + p], gys[s * SP + p], xg);
         CB[i] = cb;
         XG[i] = xg;
         Lm[i] = s <= k ? expf(cs[k] - cs[s]) : 0.f;
@@ -190,32 +195,32 @@ __global__ void __launch_bounds__(kT) k_bwd_chunk(BwdArgs a) {
     for (int i = threadIdx.x; i < Q * P; i += kT) {
         const int k = i / P, p = i % P;
         float yv = 0.f, gb = 0.f;
-        for (int s = 0; s <= k; ++s) yv = fmaf(CB[k * Q + s] * Lm[k * Q + s] * dts[s], xs[s * P + p], yv);
-        for (int s = k; s < Q; ++s) gb = fmaf(CB[s * Q + k] * Lm[s * Q + k], gys[s * P + p], gb);
+        for (int s = 0; s <= k; ++s) yv = fmaf(CB[k * Q + s] * Lm[k * Q + s] * dts[s], xs[s * SP + p], yv);
+        for (int s = k; s < Q; ++s) gb = fmaf(CB[s * Q + k] * Lm[s * Q + k], gys[s * SP + p], gb);
         float yo = 0.f, go = 0.f;
         for (int n = 0; n < N; ++n) {
-            yo = fmaf(cc[k * N + n], Sin[p * N + n], yo);
-            go = fmaf(Gin[p * N + n], bs[k * N + n], go);
+            yo = fmaf(cc[k * SN + n], Sin[p * SN + n], yo);
+            go = fmaf(Gin[p * SN + n], bs[k * SN + n], go);
         }
         yv = fmaf(expf(cs[k]), yo, yv);
         gb = fmaf(expf(cl - cs[k]), go, gb);
         const float dh = a.D ? a.D[h] : 0.f;
         const int t = tok(c * Q + k, a.L, a.dir);
-        a.gx[(((size_t)b * a.L + t) * a.H + h) * P + p] = fmaf(dts[k], gb, dh * gys[k * P + p]);
-        atomicAdd(&red[k], xs[k * P + p] * gb);
-        atomicAdd(&red[64 + k], gys[k * P + p] * yv);
-        atomicAdd(&red[128 + k], gys[k * P + p] * xs[k * P + p]);
+        a.gx[(((size_t)b * a.L + t) * a.H + h) * P + p] = fmaf(dts[k], gb, dh * gys[k * SP + p]);
+        atomicAdd(&red[k], xs[k * SP + p] * gb);
+        atomicAdd(&red[64 + k], gys[k * SP + p] * yv);
+        atomicAdd(&red[128 + k], gys[k * SP + p] * xs[k * SP + p]);
     }
     // outputs over (k, n): this head's parts of dB and dC
     for (int i = threadIdx.x; i < Q * N; i += kT) {
         const int k = i / N, n = i % N;
         float gbv = 0.f, gcv = 0.f;
-        for (int s = k; s < Q; ++s) gbv = fmaf(XG[k * Q + s] * Lm[s * Q + k], cc[s * N + n], gbv);
-        for (int s = 0; s <= k; ++s) gcv = fmaf(XG[s * Q + k] * Lm[k * Q + s] * dts[s], bs[s * N + n], gcv);
+        for (int s = k; s < Q; ++s) gbv = fmaf(XG[k * Q + s] * Lm[s * Q + k], cc[s * SN + n], gbv);
+        for (int s = 0; s <= k; ++s) gcv = fmaf(XG[s * Q + k] * Lm[k * Q + s] * dts[s], bs[s * SN + n], gcv);
         float bo = 0.f, co = 0.f;
         for (int p = 0; p < P; ++p) {
-            bo = fmaf(Gin[p * N + n], xs[k * P + p], bo);
-            co = fmaf(Sin[p * N + n], gys[k * P + p], co);
+            bo = fmaf(Gin[p * SN + n], xs[k * SP + p], bo);
+            co = fmaf(Sin[p * SN + n], gys[k * SP + p], co);
         }
         gbv = dts[k] * fmaf(expf(cl - cs[k]), bo, gbv);
         gcv = fmaf(expf(cs[k]), co, gcv);
@@ -330,7 +335,7 @@ template <typename T, int P, int N>
 cudaError_t bwd_typed(const BwdArgs &a, cudaStream_t st) {
     const int Q = a.Q;
     const size_t sm1 = sizeof(float) * (128 + 2 * Q * P + 2 * Q * N);
-    const size_t sm3 = sizeof(float) * (128 + 2 * Q * P + 2 * Q * N + 3 * Q * Q + 2 * P * N + 3 * 64);
+    const size_t sm3 = sizeof(float) * (128 + 2 * Q * (P + 1) + 2 * Q * (N + 1) + 3 * Q * Q + 2 * P * (N + 1) + 3 * 64);
     cudaError_t e = cudaFuncSetAttribute(k_bwd_chunk_sums<T, P, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sm1);
     if (e != cudaSuccess) return e;

@@ -1093,15 +1093,21 @@ extern "C" int ssd_debug_trace(unsigned long long *out, int n) {
 }
 #endif
 
+// The shared-memory opt-in is a per-device setting: done once for each device the kernel runs on.
+std::atomic<uint64_t> g_attr_done{0};
+
 cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
+    int dev = 0;
+    cudaError_t attr_err = cudaGetDevice(&dev);
+    if (attr_err != cudaSuccess) return attr_err;
+    const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+    if (!bit || !(g_attr_done.load(std::memory_order_acquire) & bit)) {
         attr_err = cudaFuncSetAttribute(k_ssd_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
         if (attr_err == cudaSuccess)
             attr_err = cudaFuncSetAttribute(k_ssd_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    });
-    if (attr_err != cudaSuccess) return attr_err;
+        if (attr_err != cudaSuccess) return attr_err;
+        g_attr_done.fetch_or(bit, std::memory_order_release);
+    }
     const int ndir = bidir ? 2 : 1;
     const uint64_t rows = (uint64_t)t.batch * t.L;
     TcMaps maps;
