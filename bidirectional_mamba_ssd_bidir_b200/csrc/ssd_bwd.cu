@@ -35,11 +35,13 @@ namespace ssd {
 namespace {
 
 constexpr int kT = 256;       // threads per CTA
+constexpr int kTC = 512;      // threads per CTA of the per-chunk gradient kernel (more warps hide its
+                              // shared-memory latency; one CTA per SM fits its shared memory)
 
 // Inclusive prefix sum of A*dt over one chunk in scan order (cs[]), and dt (dts[]).
 template <typename T>
 __device__ void bwd_cumsum(const BwdArgs &a, int b, int h, int c, float *cs, float *dts) {
-    __shared__ float wt[kT / 32];
+    __shared__ float wt[kTC / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     float v = 0.f;
     if (tid < a.Q) {
@@ -108,37 +110,63 @@ __global__ void __launch_bounds__(kT) k_bwd_chunk_sums(BwdArgs a) {
 }
 
 // Step 2: state entering each chunk (forward pass over chunks) and adjoint entering each chunk
-// from the right (reverse pass), both in place.
+// from the right (reverse pass), both in place.  A (batch, head) pair's P x N entries are split
+// over gridDim.z CTAs of kPassE entries per thread; each chunk's values are loaded before any
+// of them is overwritten, so the loads of one chunk overlap.
+constexpr int kPassE = 2;
 template <int P, int N>
 __global__ void __launch_bounds__(kT) k_bwd_pass(BwdArgs a) {
-    constexpr int E = P * N / kT;
     const int h = blockIdx.x, b = blockIdx.y;
+    const int e0 = blockIdx.z * kT * kPassE + threadIdx.x;
     const size_t base = ((size_t)b * a.H + h) * a.nc;
-    float run[E];
+    float run[kPassE], v[kPassE];
 #pragma unroll
-    for (int j = 0; j < E; ++j) run[j] = 0.f;
+    for (int j = 0; j < kPassE; ++j) run[j] = 0.f;
     for (int c = 0; c < a.nc; ++c) {
         float *S = a.sf + (base + c) * P * N;
         const float dc = a.dec[base + c];
 #pragma unroll
-        for (int j = 0; j < E; ++j) {
-            const int e = threadIdx.x + kT * j;
-            const float v = S[e];
-            S[e] = run[j];
-            run[j] = fmaf(dc, run[j], v);
+        for (int j = 0; j < kPassE; ++j) v[j] = S[e0 + kT * j];
+#pragma unroll
+        for (int j = 0; j < kPassE; ++j) {
+            S[e0 + kT * j] = run[j];
+            run[j] = fmaf(dc, run[j], v[j]);
         }
     }
 #pragma unroll
-    for (int j = 0; j < E; ++j) run[j] = 0.f;
+    for (int j = 0; j < kPassE; ++j) run[j] = 0.f;
     for (int c = a.nc - 1; c >= 0; --c) {
         float *Z = a.sg + (base + c) * P * N;
         const float dc = a.dec[base + c];
 #pragma unroll
-        for (int j = 0; j < E; ++j) {
-            const int e = threadIdx.x + kT * j;
+        for (int j = 0; j < kPassE; ++j) v[j] = Z[e0 + kT * j];
+#pragma unroll
+        for (int j = 0; j < kPassE; ++j) {
+            Z[e0 + kT * j] = run[j];
+            run[j] = fmaf(dc, run[j], v[j]);
+        }
+    }
+}
+
+// Step 2 for small states (P N < kT kPassE): one entry per thread or fewer.
+template <int P, int N>
+__global__ void __launch_bounds__(kT) k_bwd_pass_small(BwdArgs a) {
+    const int h = blockIdx.x, b = blockIdx.y;
+    const size_t base = ((size_t)b * a.H + h) * a.nc;
+    for (int e = threadIdx.x; e < P * N; e += kT) {
+        float run = 0.f;
+        for (int c = 0; c < a.nc; ++c) {
+            float *S = a.sf + (base + c) * P * N;
+            const float v = S[e];
+            S[e] = run;
+            run = fmaf(a.dec[base + c], run, v);
+        }
+        run = 0.f;
+        for (int c = a.nc - 1; c >= 0; --c) {
+            float *Z = a.sg + (base + c) * P * N;
             const float v = Z[e];
-            Z[e] = run[j];
-            run[j] = fmaf(dc, run[j], v);
+            Z[e] = run;
+            run = fmaf(a.dec[base + c], run, v);
         }
     }
 }
@@ -147,7 +175,7 @@ __global__ void __launch_bounds__(kT) k_bwd_pass(BwdArgs a) {
 // CB[k][s] = C_k . B_s, XG[k][s] = x_k . gy_s and Lm[k][s] = exp(cs_k - cs_s) (s <= k, else 0);
 // the entering state Sin and the entering adjoint Gin carry everything outside the chunk.
 template <typename T, int P, int N>
-__global__ void __launch_bounds__(kT) k_bwd_chunk(BwdArgs a) {
+__global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int Q = a.Q, g = h / (a.H / a.G);
     // rows of x, gy (stride P + 1), B, C (stride N + 1) and of the entering state and adjoint
@@ -160,27 +188,27 @@ __global__ void __launch_bounds__(kT) k_bwd_chunk(BwdArgs a) {
     float *red = Gin + P * SN;   // [3][64]: u, <gy, y - D x>, <gy, x> per position
     bwd_cumsum<T>(a, b, h, c, cs, dts);
     const float cl = cs[Q - 1];
-    for (int i = threadIdx.x; i < Q * P; i += kT) {
+    for (int i = threadIdx.x; i < Q * P; i += kTC) {
         const int k = i / P, p = i % P;
         const size_t xi = (((size_t)b * a.L + tok(c * Q + k, a.L, a.dir)) * a.H + h) * P + p;
         xs[k * SP + p] = ldf<T>((const T *)a.x, xi);
         gys[k * SP + p] = ldf<T>((const T *)a.gy, xi);
     }
-    for (int i = threadIdx.x; i < Q * N; i += kT) {
+    for (int i = threadIdx.x; i < Q * N; i += kTC) {
         const int k = i / N, n = i % N;
         const size_t bi = (((size_t)b * a.L + tok(c * Q + k, a.L, a.dir)) * a.G + g) * N + n;
         bs[k * SN + n] = ldf<T>((const T *)a.B, bi);
         cc[k * SN + n] = ldf<T>((const T *)a.C, bi);
     }
     const size_t sbase = (((size_t)b * a.H + h) * a.nc + c) * P * N;
-    for (int i = threadIdx.x; i < P * N; i += kT) {
+    for (int i = threadIdx.x; i < P * N; i += kTC) {
         const int p = i / N, n = i % N;
         Sin[p * SN + n] = a.sf[sbase + i];
         Gin[p * SN + n] = a.sg[sbase + i];
     }
-    for (int i = threadIdx.x; i < 3 * 64; i += kT) red[i] = 0.f;
+    for (int i = threadIdx.x; i < 3 * 64; i += kTC) red[i] = 0.f;
     __syncthreads();
-    for (int i = threadIdx.x; i < Q * Q; i += kT) {
+    for (int i = threadIdx.x; i < Q * Q; i += kTC) {
         const int k = i / Q, s = i % Q;
         float cb = 0.f, xg = 0.f;
         for (int n = 0; n < N; ++n) cb = fmaf(cc[k * SN + n], bs[s * SN + n], cb);
@@ -191,46 +219,93 @@ __global__ void __launch_bounds__(kT) k_bwd_chunk(BwdArgs a) {
     }
     __syncthreads();
 
-    // outputs over (k, p): y - D x (recomputed), G_k B_k, dx
-    for (int i = threadIdx.x; i < Q * P; i += kT) {
-        const int k = i / P, p = i % P;
-        float yv = 0.f, gb = 0.f;
-        for (int s = 0; s <= k; ++s) yv = fmaf(CB[k * Q + s] * Lm[k * Q + s] * dts[s], xs[s * SP + p], yv);
-        for (int s = k; s < Q; ++s) gb = fmaf(CB[s * Q + k] * Lm[s * Q + k], gys[s * SP + p], gb);
-        float yo = 0.f, go = 0.f;
+    // outputs over (k, p): y - D x (recomputed), G_k B_k, dx.  A thread takes one position k and
+    // four columns p0 + kGP j, so the pair terms of k (read once per s) serve four outputs.
+    constexpr int kGP = P / 4;                      // threads per position
+    const float dh = a.D ? a.D[h] : 0.f;
+    for (int i = threadIdx.x; i < Q * kGP; i += kTC) {
+        const int k = i / kGP, p0 = i % kGP;
+        float yv[4] = {0.f, 0.f, 0.f, 0.f}, gb[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int s = 0; s <= k; ++s) {
+            const float m = CB[k * Q + s] * Lm[k * Q + s] * dts[s];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) yv[j] = fmaf(m, xs[s * SP + p0 + kGP * j], yv[j]);
+        }
+        for (int s = k; s < Q; ++s) {
+            const float m = CB[s * Q + k] * Lm[s * Q + k];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) gb[j] = fmaf(m, gys[s * SP + p0 + kGP * j], gb[j]);
+        }
+        float yo[4] = {0.f, 0.f, 0.f, 0.f}, go[4] = {0.f, 0.f, 0.f, 0.f};
         for (int n = 0; n < N; ++n) {
-            yo = fmaf(cc[k * SN + n], Sin[p * SN + n], yo);
-            go = fmaf(Gin[p * SN + n], bs[k * SN + n], go);
+            const float cv = cc[k * SN + n], bv = bs[k * SN + n];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                yo[j] = fmaf(cv, Sin[(p0 + kGP * j) * SN + n], yo[j]);
+                go[j] = fmaf(bv, Gin[(p0 + kGP * j) * SN + n], go[j]);
+            }
         }
-        yv = fmaf(expf(cs[k]), yo, yv);
-        gb = fmaf(expf(cl - cs[k]), go, gb);
-        const float dh = a.D ? a.D[h] : 0.f;
+        const float ek = expf(cs[k]), el = expf(cl - cs[k]);
         const int t = tok(c * Q + k, a.L, a.dir);
-        a.gx[(((size_t)b * a.L + t) * a.H + h) * P + p] = fmaf(dts[k], gb, dh * gys[k * SP + p]);
-        atomicAdd(&red[k], xs[k * SP + p] * gb);
-        atomicAdd(&red[64 + k], gys[k * SP + p] * yv);
-        atomicAdd(&red[128 + k], gys[k * SP + p] * xs[k * SP + p]);
+        float r0 = 0.f, r1 = 0.f, r2 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int p = p0 + kGP * j;
+            const float y_ = fmaf(ek, yo[j], yv[j]), g_ = fmaf(el, go[j], gb[j]);
+            const float xv = xs[k * SP + p], gv = gys[k * SP + p];
+            a.gx[(((size_t)b * a.L + t) * a.H + h) * P + p] = fmaf(dts[k], g_, dh * gv);
+            r0 = fmaf(xv, g_, r0);
+            r1 = fmaf(gv, y_, r1);
+            r2 = fmaf(gv, xv, r2);
+        }
+        // the kGP consecutive lanes that share position k reduce their terms; one adds them
+#pragma unroll
+        for (int o = kGP / 2; o > 0; o >>= 1) {
+            r0 += __shfl_xor_sync(0xffffffffu, r0, o);
+            r1 += __shfl_xor_sync(0xffffffffu, r1, o);
+            r2 += __shfl_xor_sync(0xffffffffu, r2, o);
+        }
+        if ((threadIdx.x & (kGP - 1)) == 0) {
+            atomicAdd(&red[k], r0);
+            atomicAdd(&red[64 + k], r1);
+            atomicAdd(&red[128 + k], r2);
+        }
     }
-    // outputs over (k, n): this head's parts of dB and dC
-    for (int i = threadIdx.x; i < Q * N; i += kT) {
-        const int k = i / N, n = i % N;
-        float gbv = 0.f, gcv = 0.f;
-        for (int s = k; s < Q; ++s) gbv = fmaf(XG[k * Q + s] * Lm[s * Q + k], cc[s * SN + n], gbv);
-        for (int s = 0; s <= k; ++s) gcv = fmaf(XG[s * Q + k] * Lm[k * Q + s] * dts[s], bs[s * SN + n], gcv);
-        float bo = 0.f, co = 0.f;
-        for (int p = 0; p < P; ++p) {
-            bo = fmaf(Gin[p * SN + n], xs[k * SP + p], bo);
-            co = fmaf(Sin[p * SN + n], gys[k * SP + p], co);
+    // outputs over (k, n): this head's parts of dB and dC, four columns n0 + kGN j per thread
+    constexpr int kGN = N / 4;
+    for (int i = threadIdx.x; i < Q * kGN; i += kTC) {
+        const int k = i / kGN, n0 = i % kGN;
+        float gbv[4] = {0.f, 0.f, 0.f, 0.f}, gcv[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int s = k; s < Q; ++s) {
+            const float m = XG[k * Q + s] * Lm[s * Q + k];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) gbv[j] = fmaf(m, cc[s * SN + n0 + kGN * j], gbv[j]);
         }
-        gbv = dts[k] * fmaf(expf(cl - cs[k]), bo, gbv);
-        gcv = fmaf(expf(cs[k]), co, gcv);
+        for (int s = 0; s <= k; ++s) {
+            const float m = XG[s * Q + k] * Lm[k * Q + s] * dts[s];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) gcv[j] = fmaf(m, bs[s * SN + n0 + kGN * j], gcv[j]);
+        }
+        float bo[4] = {0.f, 0.f, 0.f, 0.f}, co[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int p = 0; p < P; ++p) {
+            const float xv = xs[k * SP + p], gv = gys[k * SP + p];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                bo[j] = fmaf(Gin[p * SN + n0 + kGN * j], xv, bo[j]);
+                co[j] = fmaf(Sin[p * SN + n0 + kGN * j], gv, co[j]);
+            }
+        }
+        const float ek = expf(cs[k]), el = expf(cl - cs[k]);
         const int t = tok(c * Q + k, a.L, a.dir);
-        const size_t oi = (((size_t)b * a.L + t) * a.H + h) * N + n;
-        a.gBh[oi] = gbv;
-        a.gCh[oi] = gcv;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const size_t oi = (((size_t)b * a.L + t) * a.H + h) * N + n0 + kGN * j;
+            a.gBh[oi] = dts[k] * fmaf(el, bo[j], gbv[j]);
+            a.gCh[oi] = fmaf(ek, co[j], gcv[j]);
+        }
     }
     __syncthreads();
-    for (int k = threadIdx.x; k < Q; k += kT) {
+    for (int k = threadIdx.x; k < Q; k += kTC) {
         const int t = tok(c * Q + k, a.L, a.dir);
         const size_t ti = ((size_t)b * a.L + t) * a.H + h;
         a.u[ti] = red[k];
@@ -343,9 +418,14 @@ cudaError_t bwd_typed(const BwdArgs &a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     k_bwd_chunk_sums<T, P, N><<<dim3(a.nc, a.H, a.batch), kT, sm1, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_bwd_pass<P, N><<<dim3(a.H, a.batch), kT, 0, st>>>(a);
+    static_assert(P * N % (kT * kPassE) == 0 || P * N < kT * kPassE, "pass slicing");
+    if constexpr (P * N >= kT * kPassE) {
+        k_bwd_pass<P, N><<<dim3(a.H, a.batch, P * N / (kT * kPassE)), kT, 0, st>>>(a);
+    } else {
+        k_bwd_pass_small<P, N><<<dim3(a.H, a.batch), kT, 0, st>>>(a);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_bwd_chunk<T, P, N><<<dim3(a.nc, a.H, a.batch), kT, sm3, st>>>(a);
+    k_bwd_chunk<T, P, N><<<dim3(a.nc, a.H, a.batch), kTC, sm3, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     k_bwd_dt<T><<<dim3(a.H, a.batch), kT, 0, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
