@@ -136,11 +136,11 @@ def measured_peaks() -> dict:
 
 
 def _kernel_source_hash() -> str:
+    """Hash of the tensor-core kernel's sources: a traffic record is valid only for the kernel it measured."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bidirectional_mamba_ssd_bidir_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in ("ssd_tc.cu", "ssd_tc.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
