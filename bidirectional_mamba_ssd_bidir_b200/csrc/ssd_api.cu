@@ -259,6 +259,7 @@ ssd_status ssd_scan_bwd(const ssd_shape *shape, const ssd_params *p, int directi
     if ((st = check_params(p, "scan")) != SSD_OK) return st;
     if (!aligned16(gy)) return fail(SSD_ERR_INVALID_ARG, "gy must be non-NULL and 16-byte aligned");
     if (!gx || !gdt || !gB || !gC) return fail(SSD_ERR_INVALID_ARG, "gx, gdt, gB and gC must be non-NULL");
+    if (!aligned16(gx)) return fail(SSD_ERR_INVALID_ARG, "gx must be 16-byte aligned");
     if (gD && !p->D) return fail(SSD_ERR_INVALID_ARG, "gD requested but D is NULL");
     const size_t need = ssd_bwd_workspace_bytes(shape, chunk);
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)))

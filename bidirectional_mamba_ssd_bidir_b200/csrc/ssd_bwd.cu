@@ -38,6 +38,51 @@ constexpr int kT = 256;       // threads per CTA
 constexpr int kTC = 512;      // threads per CTA of the per-chunk gradient kernel (more warps hide its
                               // shared-memory latency; one CTA per SM fits its shared memory)
 
+// Eight consecutive values of a 16-byte aligned row, as float.
+template <typename T> __device__ __forceinline__ void ld8(const T *p, float (&v)[8]);
+template <> __device__ __forceinline__ void ld8<float>(const float *p, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4 *>(p), b = *reinterpret_cast<const float4 *>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+template <> __device__ __forceinline__ void ld8<__nv_bfloat16>(const __nv_bfloat16 *p, float (&v)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// Eight floats to a 16-byte aligned shared-memory address.
+__device__ __forceinline__ void st8(float *d, const float (&v)[8]) {
+    *reinterpret_cast<float4 *>(d) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4 *>(d + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// Rows 0 .. Q-1 of two [token][W] arrays that share their row addresses (x and gy, or B and C)
+// for one chunk, eight values per unit.  Every unit of this thread is loaded before any is
+// handed to op(k, w0, va, vb), so that the loads are in flight together.
+template <typename T, int W, int NT, typename RowOff, typename Op>
+__device__ __forceinline__ void load_rows2(int Q, const T *ga, const T *gb, RowOff rowoff, Op op) {
+    constexpr int WU = W / 8, MAXU = (64 * WU + NT - 1) / NT;
+    float va[MAXU][8], vb[MAXU][8];
+#pragma unroll
+    for (int u = 0; u < MAXU; ++u) {
+        const int i = threadIdx.x + NT * u;
+        if (i < Q * WU) {
+            const size_t o = rowoff(i / WU) + 8 * (i % WU);
+            ld8<T>(ga + o, va[u]);
+            ld8<T>(gb + o, vb[u]);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < MAXU; ++u) {
+        const int i = threadIdx.x + NT * u;
+        if (i < Q * WU) op(i / WU, 8 * (i % WU), va[u], vb[u]);
+    }
+}
+
 // Inclusive prefix sum of A*dt over one chunk in scan order (cs[]), and dt (dts[]).
 template <typename T>
 __device__ void bwd_cumsum(const BwdArgs &a, int b, int h, int c, float *cs, float *dts) {
@@ -70,80 +115,113 @@ __global__ void __launch_bounds__(kT) k_bwd_chunk_sums(BwdArgs a) {
     constexpr int E = P * N / kT;
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int Q = a.Q, g = h / (a.H / a.G);
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     float *cs = sm, *dts = cs + 64, *xw = dts + 64, *gw = xw + Q * P, *bs = gw + Q * P, *cc = bs + Q * N;
+    auto xrow = [&](int k) { return (((size_t)b * a.L + tok(c * Q + k, a.L, a.dir)) * a.H + h) * P; };
+    auto brow = [&](int k) { return (((size_t)b * a.L + tok(c * Q + k, a.L, a.dir)) * a.G + g) * N; };
+    load_rows2<T, N, kT>(Q, (const T *)a.B, (const T *)a.C, brow,
+                         [&](int k, int n, const float (&vb)[8], const float (&vc)[8]) {
+                             st8(bs + k * N + n, vb);
+                             st8(cc + k * N + n, vc);
+                         });
     bwd_cumsum<T>(a, b, h, c, cs, dts);
     const float cl = cs[Q - 1];
-    for (int i = threadIdx.x; i < Q * P; i += kT) {
-        const int k = i / P, p = i % P;
-        const size_t xi = (((size_t)b * a.L + tok(c * Q + k, a.L, a.dir)) * a.H + h) * P + p;
-        xw[i] = expf(cl - cs[k]) * dts[k] * ldf<T>((const T *)a.x, xi);
-        gw[i] = expf(cs[k]) * ldf<T>((const T *)a.gy, xi);
-    }
-    for (int i = threadIdx.x; i < Q * N; i += kT) {
-        const int k = i / N, n = i % N;
-        const size_t bi = (((size_t)b * a.L + tok(c * Q + k, a.L, a.dir)) * a.G + g) * N + n;
-        bs[i] = ldf<T>((const T *)a.B, bi);
-        cc[i] = ldf<T>((const T *)a.C, bi);
-    }
+    load_rows2<T, P, kT>(Q, (const T *)a.x, (const T *)a.gy, xrow,
+                         [&](int k, int p, const float (&vx)[8], const float (&vg)[8]) {
+                             const float wx = expf(cl - cs[k]) * dts[k], wg = expf(cs[k]);
+                             float ox[8], og[8];
+#pragma unroll
+                             for (int e = 0; e < 8; ++e) {
+                                 ox[e] = wx * vx[e];
+                                 og[e] = wg * vg[e];
+                             }
+                             st8(xw + k * P + p, ox);
+                             st8(gw + k * P + p, og);
+                         });
     __syncthreads();
+    // thread: column n and E consecutive rows p0 .. p0 + E - 1, so that the row weights of one k
+    // are read as whole vectors (the same for every lane of a warp when N >= 32)
     float sf[E], sg[E];
 #pragma unroll
     for (int j = 0; j < E; ++j) sf[j] = sg[j] = 0.f;
-    const int n = threadIdx.x % N;
+    const int n = threadIdx.x % N, p0 = (threadIdx.x / N) * E;
+#pragma unroll 2
     for (int k = 0; k < Q; ++k) {
         const float bv = bs[k * N + n], cv = cc[k * N + n];
+        if constexpr (E % 4 == 0) {
 #pragma unroll
-        for (int j = 0; j < E; ++j) {
-            const int p = (threadIdx.x + kT * j) / N;
-            sf[j] = fmaf(xw[k * P + p], bv, sf[j]);
-            sg[j] = fmaf(gw[k * P + p], cv, sg[j]);
+            for (int j = 0; j < E; j += 4) {
+                const float4 xv = *reinterpret_cast<const float4 *>(xw + k * P + p0 + j);
+                const float4 gv = *reinterpret_cast<const float4 *>(gw + k * P + p0 + j);
+                sf[j] = fmaf(xv.x, bv, sf[j]); sf[j + 1] = fmaf(xv.y, bv, sf[j + 1]);
+                sf[j + 2] = fmaf(xv.z, bv, sf[j + 2]); sf[j + 3] = fmaf(xv.w, bv, sf[j + 3]);
+                sg[j] = fmaf(gv.x, cv, sg[j]); sg[j + 1] = fmaf(gv.y, cv, sg[j + 1]);
+                sg[j + 2] = fmaf(gv.z, cv, sg[j + 2]); sg[j + 3] = fmaf(gv.w, cv, sg[j + 3]);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < E; ++j) {
+                sf[j] = fmaf(xw[k * P + p0 + j], bv, sf[j]);
+                sg[j] = fmaf(gw[k * P + p0 + j], cv, sg[j]);
+            }
         }
     }
     const size_t base = (((size_t)b * a.H + h) * a.nc + c) * P * N;
 #pragma unroll
     for (int j = 0; j < E; ++j) {
-        a.sf[base + threadIdx.x + kT * j] = sf[j];
-        a.sg[base + threadIdx.x + kT * j] = sg[j];
+        a.sf[base + (size_t)(p0 + j) * N + n] = sf[j];
+        a.sg[base + (size_t)(p0 + j) * N + n] = sg[j];
     }
     if (threadIdx.x == 0) a.dec[((size_t)b * a.H + h) * a.nc + c] = expf(cl);
 }
 
 // Step 2: state entering each chunk (forward pass over chunks) and adjoint entering each chunk
 // from the right (reverse pass), both in place.  A (batch, head) pair's P x N entries are split
-// over gridDim.z CTAs of kPassE entries per thread; each chunk's values are loaded before any
-// of them is overwritten, so the loads of one chunk overlap.
+// over gridDim.z CTAs of kPassE entries per thread.  The values of kPassU chunks are loaded
+// before any of them is overwritten, so that their loads are in flight together; the chain of
+// multiply-adds then runs on registers.
 constexpr int kPassE = 2;
+constexpr int kPassU = 8;
 template <int P, int N>
 __global__ void __launch_bounds__(kT) k_bwd_pass(BwdArgs a) {
     const int h = blockIdx.x, b = blockIdx.y;
     const int e0 = blockIdx.z * kT * kPassE + threadIdx.x;
     const size_t base = ((size_t)b * a.H + h) * a.nc;
-    float run[kPassE], v[kPassE];
+    for (int dirn = 0; dirn < 2; ++dirn) {
+        // dirn 0: states S (a.sf), chunks in increasing order; dirn 1: adjoints (a.sg), decreasing
+        float *arr = dirn == 0 ? a.sf : a.sg;
+        float run[kPassE];
 #pragma unroll
-    for (int j = 0; j < kPassE; ++j) run[j] = 0.f;
-    for (int c = 0; c < a.nc; ++c) {
-        float *S = a.sf + (base + c) * P * N;
-        const float dc = a.dec[base + c];
+        for (int j = 0; j < kPassE; ++j) run[j] = 0.f;
+        for (int c0 = 0; c0 < a.nc; c0 += kPassU) {
+            float v[kPassU][kPassE], dc[kPassU];
 #pragma unroll
-        for (int j = 0; j < kPassE; ++j) v[j] = S[e0 + kT * j];
+            for (int u = 0; u < kPassU; ++u) {
+                const int i = c0 + u;
+                const int c = dirn == 0 ? i : a.nc - 1 - i;
+                dc[u] = 0.f;
 #pragma unroll
-        for (int j = 0; j < kPassE; ++j) {
-            S[e0 + kT * j] = run[j];
-            run[j] = fmaf(dc, run[j], v[j]);
-        }
-    }
+                for (int j = 0; j < kPassE; ++j) v[u][j] = 0.f;
+                if (i < a.nc) {
+                    const float *S = arr + (base + c) * P * N;
+                    dc[u] = a.dec[base + c];
 #pragma unroll
-    for (int j = 0; j < kPassE; ++j) run[j] = 0.f;
-    for (int c = a.nc - 1; c >= 0; --c) {
-        float *Z = a.sg + (base + c) * P * N;
-        const float dc = a.dec[base + c];
+                    for (int j = 0; j < kPassE; ++j) v[u][j] = S[e0 + kT * j];
+                }
+            }
 #pragma unroll
-        for (int j = 0; j < kPassE; ++j) v[j] = Z[e0 + kT * j];
+            for (int u = 0; u < kPassU; ++u) {
+                const int i = c0 + u;
+                if (i < a.nc) {
+                    const int c = dirn == 0 ? i : a.nc - 1 - i;
+                    float *S = arr + (base + c) * P * N;
 #pragma unroll
-        for (int j = 0; j < kPassE; ++j) {
-            Z[e0 + kT * j] = run[j];
-            run[j] = fmaf(dc, run[j], v[j]);
+                    for (int j = 0; j < kPassE; ++j) {
+                        S[e0 + kT * j] = run[j];
+                        run[j] = fmaf(dc[u], run[j], v[u][j]);
+                    }
+                }
+            }
         }
     }
 }
@@ -172,146 +250,257 @@ __global__ void __launch_bounds__(kT) k_bwd_pass_small(BwdArgs a) {
 }
 
 // Step 3: every per-position gradient of one chunk.  Pair terms (k, s) inside the chunk use
-// CB[k][s] = C_k . B_s, XG[k][s] = x_k . gy_s and Lm[k][s] = exp(cs_k - cs_s) (s <= k, else 0);
-// the entering state Sin and the entering adjoint Gin carry everything outside the chunk.
+// E[k][s] = (C_k . B_s) exp(cs_k - cs_s) for s <= k (else 0) and
+// F[k][s] = (x_k . gy_s) exp(cs_s - cs_k) for s >= k (else 0); the entering state Sin and the
+// entering adjoint Gin carry everything outside the chunk.  Every product below is a small
+// matrix product evaluated in register tiles (one k and 8 columns, or 2 k and 8 columns per
+// thread), so that each shared-memory load feeds several multiply-adds.
+constexpr int kQm = 64;        // largest chunk of the gradient kernels
+constexpr int kSQ = kQm + 1;   // row stride of E and F (odd: column reads hit distinct banks)
+
+template <int P, int N>
+struct ChunkSmem {
+    static constexpr int SX = P + 4;   // rows of x, gy (16-byte aligned, 4 banks apart)
+    static constexpr int SB = N + 4;   // rows of B, C and of Sin, Gin in [p][n] order
+    static constexpr int kS = (N * SX > P * SB) ? N * SX : P * SB;   // one of Sin, Gin, either order
+    static constexpr int kCs = 0, kDt = 64, kRed = 128, kX = 320, kGy = kX + kQm * SX, kB = kGy + kQm * SX,
+                         kC = kB + kQm * SB, kS0 = kC + kQm * SB, kS1 = kS0 + kS, kE = kS1 + kS, kF = kE + kQm * kSQ,
+                         kFloats = kF + kQm * kSQ;
+};
+
+__device__ __forceinline__ void fma8(float (&acc)[8], float m, const float *v) {
+    const float4 a = *reinterpret_cast<const float4 *>(v), b = *reinterpret_cast<const float4 *>(v + 4);
+    acc[0] = fmaf(m, a.x, acc[0]); acc[1] = fmaf(m, a.y, acc[1]); acc[2] = fmaf(m, a.z, acc[2]);
+    acc[3] = fmaf(m, a.w, acc[3]); acc[4] = fmaf(m, b.x, acc[4]); acc[5] = fmaf(m, b.y, acc[5]);
+    acc[6] = fmaf(m, b.z, acc[6]); acc[7] = fmaf(m, b.w, acc[7]);
+}
+
 template <typename T, int P, int N>
 __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
+    using L_ = ChunkSmem<P, N>;
+    constexpr int SX = L_::SX, SB = L_::SB;
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int Q = a.Q, g = h / (a.H / a.G);
-    // rows of x, gy (stride P + 1), B, C (stride N + 1) and of the entering state and adjoint
-    // (stride N + 1) are padded by one word, so that a warp reading one column across rows hits
-    // 32 different banks
-    constexpr int SP = P + 1, SN = N + 1;
-    extern __shared__ float sm[];
-    float *cs = sm, *dts = cs + 64, *xs = dts + 64, *gys = xs + Q * SP, *bs = gys + Q * SP, *cc = bs + Q * SN;
-    float *CB = cc + Q * SN, *XG = CB + Q * Q, *Lm = XG + Q * Q, *Sin = Lm + Q * Q, *Gin = Sin + P * SN;
-    float *red = Gin + P * SN;   // [3][64]: u, <gy, y - D x>, <gy, x> per position
+    const int tid = threadIdx.x;
+    extern __shared__ __align__(16) float sm[];
+    float *cs = sm + L_::kCs, *dts = sm + L_::kDt, *red = sm + L_::kRed;   // red: [3][64] u, <gy, y - D x>, <gy, x>
+    float *xs = sm + L_::kX, *gys = sm + L_::kGy, *bs = sm + L_::kB, *cc = sm + L_::kC;
+    float *S0 = sm + L_::kS0, *S1 = sm + L_::kS1, *E = sm + L_::kE, *F = sm + L_::kF;
+    auto xrow = [&](int k) { return (((size_t)b * a.L + tok(c * Q + k, a.L, a.dir)) * a.H + h) * P; };
+    auto brow = [&](int k) { return (((size_t)b * a.L + tok(c * Q + k, a.L, a.dir)) * a.G + g) * N; };
+    load_rows2<T, N, kTC>(Q, (const T *)a.B, (const T *)a.C, brow,
+                          [&](int k, int n, const float (&vb)[8], const float (&vc)[8]) {
+                              st8(bs + k * SB + n, vb);
+                              st8(cc + k * SB + n, vc);
+                          });
+    load_rows2<T, P, kTC>(Q, (const T *)a.x, (const T *)a.gy, xrow,
+                          [&](int k, int p, const float (&vx)[8], const float (&vg)[8]) {
+                              st8(xs + k * SX + p, vx);
+                              st8(gys + k * SX + p, vg);
+                          });
     bwd_cumsum<T>(a, b, h, c, cs, dts);
     const float cl = cs[Q - 1];
-    for (int i = threadIdx.x; i < Q * P; i += kTC) {
-        const int k = i / P, p = i % P;
-        const size_t xi = (((size_t)b * a.L + tok(c * Q + k, a.L, a.dir)) * a.H + h) * P + p;
-        xs[k * SP + p] = ldf<T>((const T *)a.x, xi);
-        gys[k * SP + p] = ldf<T>((const T *)a.gy, xi);
-    }
-    for (int i = threadIdx.x; i < Q * N; i += kTC) {
-        const int k = i / N, n = i % N;
-        const size_t bi = (((size_t)b * a.L + tok(c * Q + k, a.L, a.dir)) * a.G + g) * N + n;
-        bs[k * SN + n] = ldf<T>((const T *)a.B, bi);
-        cc[k * SN + n] = ldf<T>((const T *)a.C, bi);
-    }
+    // the entering state and adjoint in [n][p] order for the (k, p) outputs: a lane reads four
+    // n of one p, and the lanes of a warp take consecutive p, so the stores hit distinct banks
     const size_t sbase = (((size_t)b * a.H + h) * a.nc + c) * P * N;
-    for (int i = threadIdx.x; i < P * N; i += kTC) {
-        const int p = i / N, n = i % N;
-        Sin[p * SN + n] = a.sf[sbase + i];
-        Gin[p * SN + n] = a.sg[sbase + i];
+    constexpr int kSU = (P * N / 4 + kTC - 1) / kTC;
+    {
+        float4 sv[kSU], gv[kSU];
+#pragma unroll
+        for (int u = 0; u < kSU; ++u) {
+            const int i = tid + kTC * u;
+            if (i < P * (N / 4)) {
+                const int p = i % P, n = 4 * (i / P);
+                sv[u] = *reinterpret_cast<const float4 *>(a.sf + sbase + (size_t)p * N + n);
+                gv[u] = *reinterpret_cast<const float4 *>(a.sg + sbase + (size_t)p * N + n);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kSU; ++u) {
+            const int i = tid + kTC * u;
+            if (i < P * (N / 4)) {
+                const int p = i % P, n = 4 * (i / P);
+                S0[n * SX + p] = sv[u].x; S0[(n + 1) * SX + p] = sv[u].y;
+                S0[(n + 2) * SX + p] = sv[u].z; S0[(n + 3) * SX + p] = sv[u].w;
+                S1[n * SX + p] = gv[u].x; S1[(n + 1) * SX + p] = gv[u].y;
+                S1[(n + 2) * SX + p] = gv[u].z; S1[(n + 3) * SX + p] = gv[u].w;
+            }
+        }
     }
-    for (int i = threadIdx.x; i < 3 * 64; i += kTC) red[i] = 0.f;
+    for (int i = tid; i < 3 * 64; i += kTC) red[i] = 0.f;
     __syncthreads();
-    for (int i = threadIdx.x; i < Q * Q; i += kTC) {
-        const int k = i / Q, s = i % Q;
-        float cb = 0.f, xg = 0.f;
-        for (int n = 0; n < N; ++n) cb = fmaf(cc[k * SN + n], bs[s * SN + n], cb);
-        for (int p = 0; p < P; ++p) xg = fmaf(xs[k * SP + p], gys[s * SP + p], xg);
-        CB[i] = cb;
-        XG[i] = xg;
-        Lm[i] = s <= k ? expf(cs[k] - cs[s]) : 0.f;
+
+    // E (threads 0..255) and F (threads 256..511), 4 x 4 tiles.  For Q = 64 a warp covers
+    // 32 k x 16 s with k = k0 + 8i, s = s0 + 4j, so the scalar loads of one instruction fall in
+    // distinct banks.
+    {
+        const bool second = tid >= kTC / 2;
+        const int t = tid & (kTC / 2 - 1);
+        const int qt = Q / 4;
+        if (t < qt * qt) {
+            int k0, kst, s0, sst;
+            if (Q == kQm) {
+                const int w = t >> 5, l = t & 31;
+                k0 = 32 * (w & 1) + (l & 7); kst = 8; s0 = 16 * (w >> 1) + (l >> 3); sst = 4;
+            } else {
+                k0 = 4 * (t % qt); kst = 1; s0 = 4 * (t / qt); sst = 1;
+            }
+            float acc[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+            const float *ra = second ? xs : cc, *rb = second ? gys : bs;
+            const int st = second ? SX : SB, K = second ? P : N;
+#pragma unroll 4
+            for (int kk = 0; kk < K; ++kk) {
+                float av[4], bv[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) av[i] = ra[(k0 + kst * i) * st + kk];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) bv[j] = rb[(s0 + sst * j) * st + kk];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int k = k0 + kst * i, s = s0 + sst * j;
+                    if (!second) E[k * kSQ + s] = s <= k ? acc[i][j] * expf(cs[k] - cs[s]) : 0.f;
+                    else F[k * kSQ + s] = s >= k ? acc[i][j] * expf(cs[s] - cs[k]) : 0.f;
+                }
+        }
     }
     __syncthreads();
 
-    // outputs over (k, p): y - D x (recomputed), G_k B_k, dx.  A thread takes one position k and
-    // four columns p0 + kGP j, so the pair terms of k (read once per s) serve four outputs.
-    constexpr int kGP = P / 4;                      // threads per position
+    // outputs over (k, p): y - D x (recomputed), the adjoint times B, dx.  Thread: one k and
+    // columns p0 .. p0 + 7; the PG threads of one k are consecutive lanes.
+    constexpr int PG = P / 8;
     const float dh = a.D ? a.D[h] : 0.f;
-    for (int i = threadIdx.x; i < Q * kGP; i += kTC) {
-        const int k = i / kGP, p0 = i % kGP;
-        float yv[4] = {0.f, 0.f, 0.f, 0.f}, gb[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int s = 0; s <= k; ++s) {
-            const float m = CB[k * Q + s] * Lm[k * Q + s] * dts[s];
+    for (int t = tid; t < Q * PG; t += kTC) {
+        const int k = t / PG, p0 = 8 * (t % PG);
+        float yv[8], gb[8], yo[8], go[8];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) yv[j] = fmaf(m, xs[s * SP + p0 + kGP * j], yv[j]);
-        }
-        for (int s = k; s < Q; ++s) {
-            const float m = CB[s * Q + k] * Lm[s * Q + k];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) gb[j] = fmaf(m, gys[s * SP + p0 + kGP * j], gb[j]);
-        }
-        float yo[4] = {0.f, 0.f, 0.f, 0.f}, go[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < 8; ++j) yv[j] = gb[j] = yo[j] = go[j] = 0.f;
+        for (int s = 0; s <= k; ++s) fma8(yv, E[k * kSQ + s] * dts[s], xs + s * SX + p0);
+        for (int s = k; s < Q; ++s) fma8(gb, E[s * kSQ + k], gys + s * SX + p0);
+#pragma unroll 2
         for (int n = 0; n < N; ++n) {
-            const float cv = cc[k * SN + n], bv = bs[k * SN + n];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                yo[j] = fmaf(cv, Sin[(p0 + kGP * j) * SN + n], yo[j]);
-                go[j] = fmaf(bv, Gin[(p0 + kGP * j) * SN + n], go[j]);
-            }
+            fma8(yo, cc[k * SB + n], S0 + n * SX + p0);
+            fma8(go, bs[k * SB + n], S1 + n * SX + p0);
         }
         const float ek = expf(cs[k]), el = expf(cl - cs[k]);
-        const int t = tok(c * Q + k, a.L, a.dir);
-        float r0 = 0.f, r1 = 0.f, r2 = 0.f;
+        const int tk = tok(c * Q + k, a.L, a.dir);
+        float r0 = 0.f, r1 = 0.f, r2 = 0.f, gxo[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int p = p0 + kGP * j;
+        for (int j = 0; j < 8; ++j) {
             const float y_ = fmaf(ek, yo[j], yv[j]), g_ = fmaf(el, go[j], gb[j]);
-            const float xv = xs[k * SP + p], gv = gys[k * SP + p];
-            a.gx[(((size_t)b * a.L + t) * a.H + h) * P + p] = fmaf(dts[k], g_, dh * gv);
+            const float xv = xs[k * SX + p0 + j], gv = gys[k * SX + p0 + j];
+            gxo[j] = fmaf(dts[k], g_, dh * gv);
             r0 = fmaf(xv, g_, r0);
             r1 = fmaf(gv, y_, r1);
             r2 = fmaf(gv, xv, r2);
         }
-        // the kGP consecutive lanes that share position k reduce their terms; one adds them
+        float *gxp = a.gx + (((size_t)b * a.L + tk) * a.H + h) * P + p0;
+        *reinterpret_cast<float4 *>(gxp) = make_float4(gxo[0], gxo[1], gxo[2], gxo[3]);
+        *reinterpret_cast<float4 *>(gxp + 4) = make_float4(gxo[4], gxo[5], gxo[6], gxo[7]);
+        // Q PG is a multiple of 32, so whole warps take part in the shuffles
 #pragma unroll
-        for (int o = kGP / 2; o > 0; o >>= 1) {
+        for (int o = PG / 2; o > 0; o >>= 1) {
             r0 += __shfl_xor_sync(0xffffffffu, r0, o);
             r1 += __shfl_xor_sync(0xffffffffu, r1, o);
             r2 += __shfl_xor_sync(0xffffffffu, r2, o);
         }
-        if ((threadIdx.x & (kGP - 1)) == 0) {
-            atomicAdd(&red[k], r0);
-            atomicAdd(&red[64 + k], r1);
-            atomicAdd(&red[128 + k], r2);
-        }
-    }
-    // outputs over (k, n): this head's parts of dB and dC, four columns n0 + kGN j per thread
-    constexpr int kGN = N / 4;
-    for (int i = threadIdx.x; i < Q * kGN; i += kTC) {
-        const int k = i / kGN, n0 = i % kGN;
-        float gbv[4] = {0.f, 0.f, 0.f, 0.f}, gcv[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int s = k; s < Q; ++s) {
-            const float m = XG[k * Q + s] * Lm[s * Q + k];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) gbv[j] = fmaf(m, cc[s * SN + n0 + kGN * j], gbv[j]);
-        }
-        for (int s = 0; s <= k; ++s) {
-            const float m = XG[s * Q + k] * Lm[k * Q + s] * dts[s];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) gcv[j] = fmaf(m, bs[s * SN + n0 + kGN * j], gcv[j]);
-        }
-        float bo[4] = {0.f, 0.f, 0.f, 0.f}, co[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int p = 0; p < P; ++p) {
-            const float xv = xs[k * SP + p], gv = gys[k * SP + p];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                bo[j] = fmaf(Gin[p * SN + n0 + kGN * j], xv, bo[j]);
-                co[j] = fmaf(Sin[p * SN + n0 + kGN * j], gv, co[j]);
-            }
-        }
-        const float ek = expf(cs[k]), el = expf(cl - cs[k]);
-        const int t = tok(c * Q + k, a.L, a.dir);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const size_t oi = (((size_t)b * a.L + t) * a.H + h) * N + n0 + kGN * j;
-            a.gBh[oi] = dts[k] * fmaf(el, bo[j], gbv[j]);
-            a.gCh[oi] = fmaf(ek, co[j], gcv[j]);
+        if ((t & (PG - 1)) == 0) {
+            red[k] = r0;
+            red[64 + k] = r1;
+            red[128 + k] = r2;
         }
     }
     __syncthreads();
-    for (int k = threadIdx.x; k < Q; k += kTC) {
-        const int t = tok(c * Q + k, a.L, a.dir);
-        const size_t ti = ((size_t)b * a.L + t) * a.H + h;
+    // the entering state and adjoint again, now in [p][n] order for the (k, n) outputs
+    {
+        float4 sv[kSU], gv[kSU];
+#pragma unroll
+        for (int u = 0; u < kSU; ++u) {
+            const int i = tid + kTC * u;
+            if (i < P * (N / 4)) {
+                sv[u] = *reinterpret_cast<const float4 *>(a.sf + sbase + 4 * (size_t)i);
+                gv[u] = *reinterpret_cast<const float4 *>(a.sg + sbase + 4 * (size_t)i);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kSU; ++u) {
+            const int i = tid + kTC * u;
+            if (i < P * (N / 4)) {
+                const int p = i / (N / 4), n = 4 * (i % (N / 4));
+                *reinterpret_cast<float4 *>(S0 + p * SB + n) = sv[u];
+                *reinterpret_cast<float4 *>(S1 + p * SB + n) = gv[u];
+            }
+        }
+    }
+    __syncthreads();
+
+    // outputs over (k, n): this head's parts of dB and dC.  Thread: rows k0, k0 + 1 and
+    // columns n0 .. n0 + 7.
+    constexpr int NG = N / 8;
+    for (int t = tid; t < (Q / 2) * NG; t += kTC) {
+        const int k0 = 2 * (t / NG), n0 = 8 * (t % NG);
+        float gbv0[8], gbv1[8], gcv0[8], gcv1[8], bo0[8], bo1[8], co0[8], co1[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            gbv0[j] = gbv1[j] = gcv0[j] = gcv1[j] = bo0[j] = bo1[j] = co0[j] = co1[j] = 0.f;
+        // sum over s >= k of F[k][s] C_s (F[k0 + 1][k0] is 0)
+        for (int s = k0; s < Q; ++s) {
+            const float *cv = cc + s * SB + n0;
+            fma8(gbv0, F[k0 * kSQ + s], cv);
+            fma8(gbv1, F[(k0 + 1) * kSQ + s], cv);
+        }
+        // sum over s <= k of F[s][k] dt_s B_s (F[k0 + 1][k0] is 0)
+        for (int s = 0; s <= k0 + 1; ++s) {
+            const float d = dts[s];
+            const float *bv = bs + s * SB + n0;
+            fma8(gcv0, F[s * kSQ + k0] * d, bv);
+            fma8(gcv1, F[s * kSQ + k0 + 1] * d, bv);
+        }
+#pragma unroll 2
+        for (int p = 0; p < P; ++p) {
+            const float *gi = S1 + p * SB + n0, *si = S0 + p * SB + n0;
+            fma8(bo0, xs[k0 * SX + p], gi);
+            fma8(bo1, xs[(k0 + 1) * SX + p], gi);
+            fma8(co0, gys[k0 * SX + p], si);
+            fma8(co1, gys[(k0 + 1) * SX + p], si);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            const int k = k0 + kk;
+            const float ek = expf(cs[k]), el = expf(cl - cs[k]), dk = dts[k];
+            const float *bo = kk ? bo1 : bo0, *gbv = kk ? gbv1 : gbv0, *co = kk ? co1 : co0, *gcv = kk ? gcv1 : gcv0;
+            float ob[8], oc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                ob[j] = dk * fmaf(el, bo[j], gbv[j]);
+                oc[j] = fmaf(ek, co[j], gcv[j]);
+            }
+            const int tk = tok(c * Q + k, a.L, a.dir);
+            const size_t oi = (((size_t)b * a.L + tk) * a.H + h) * N + n0;
+            *reinterpret_cast<float4 *>(a.gBh + oi) = make_float4(ob[0], ob[1], ob[2], ob[3]);
+            *reinterpret_cast<float4 *>(a.gBh + oi + 4) = make_float4(ob[4], ob[5], ob[6], ob[7]);
+            *reinterpret_cast<float4 *>(a.gCh + oi) = make_float4(oc[0], oc[1], oc[2], oc[3]);
+            *reinterpret_cast<float4 *>(a.gCh + oi + 4) = make_float4(oc[4], oc[5], oc[6], oc[7]);
+        }
+    }
+    __syncthreads();
+    for (int k = tid; k < Q; k += kTC) {
+        const int tk = tok(c * Q + k, a.L, a.dir);
+        const size_t ti = ((size_t)b * a.L + tk) * a.H + h;
         a.u[ti] = red[k];
         a.gcs[ti] = red[64 + k] - dts[k] * red[k];
     }
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
         float sx = 0.f;
         for (int k = 0; k < Q; ++k) sx += red[128 + k];
         a.gxd[((size_t)b * a.H + h) * a.nc + c] = sx;
@@ -410,7 +599,7 @@ template <typename T, int P, int N>
 cudaError_t bwd_typed(const BwdArgs &a, cudaStream_t st) {
     const int Q = a.Q;
     const size_t sm1 = sizeof(float) * (128 + 2 * Q * P + 2 * Q * N);
-    const size_t sm3 = sizeof(float) * (128 + 2 * Q * (P + 1) + 2 * Q * (N + 1) + 3 * Q * Q + 2 * P * (N + 1) + 3 * 64);
+    const size_t sm3 = sizeof(float) * ChunkSmem<P, N>::kFloats;
     cudaError_t e = cudaFuncSetAttribute(k_bwd_chunk_sums<T, P, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sm1);
     if (e != cudaSuccess) return e;

@@ -131,9 +131,9 @@ ssd_status ssd_scan_state(const ssd_shape *shape, const ssd_params *p, int direc
  *     gD  [nheads] or NULL                      dL/dD (NULL when p->D is NULL)
  * The bidirectional mixer's gradients are the two directions' gradients for
  * the same gy (y is their sum).  Runs on the CUDA cores in float32, chunked
- * like the forward scan (at most 64 positions per chunk).  workspace must be
- * 256-byte aligned and hold ssd_bwd_workspace_bytes(shape, chunk) bytes.  Errors
- * as for ssd_scan. */
+ * like the forward scan (at most 64 positions per chunk).  gy and gx must be
+ * 16-byte aligned; workspace must be 256-byte aligned and hold
+ * ssd_bwd_workspace_bytes(shape, chunk) bytes.  Errors as for ssd_scan. */
 size_t ssd_bwd_workspace_bytes(const ssd_shape *shape, int chunk);
 ssd_status ssd_scan_bwd(const ssd_shape *shape, const ssd_params *p, int direction, int chunk,
                         const void *gy, float *gx, float *gdt, float *gA, float *gB, float *gC,

@@ -24,6 +24,8 @@ CASES = [
     (si.Shape(2, 256, 4, 64, 128, 1, "bf16"), 256),     # 4 chunks of 64
     (si.Shape(2, 192, 4, 32, 64, 2, "bf16"), 64),       # two groups
     (si.Shape(1, 1024, 2, 64, 128, 1, "bf16"), 128),    # 16 chunks
+    (si.Shape(1, 128, 2, 64, 16, 1, "f32"), 32),         # wide x, narrow state, 32-position chunks
+    (si.Shape(1, 48, 2, 32, 128, 1, "bf16"), 16),        # 16-position chunks, wide state
 ]
 
 
