@@ -252,9 +252,11 @@ __global__ void __launch_bounds__(kT) k_bwd_pass_small(BwdArgs a) {
 // Step 3: every per-position gradient of one chunk.  Pair terms (k, s) inside the chunk use
 // E[k][s] = (C_k . B_s) exp(cs_k - cs_s) for s <= k (else 0) and
 // F[k][s] = (x_k . gy_s) exp(cs_s - cs_k) for s >= k (else 0); the entering state Sin and the
-// entering adjoint Gin carry everything outside the chunk.  Every product below is a small
-// matrix product evaluated in register tiles (one k and 8 columns, or 2 k and 8 columns per
-// thread), so that each shared-memory load feeds several multiply-adds.
+// entering adjoint Gin carry everything outside the chunk.  The forward output is not
+// recomputed: <gy_k, y_k - D x_k> = exp(cs_k) C_k . (Sin gy_k) + sum_{s<=k} E[k][s] dt_s x_s . gy_k,
+// whose first part falls out of the dC products.  Every product below is a small matrix product
+// evaluated in register tiles (one k and 8 columns, or 4 k and 8 columns per thread), so that
+// each shared-memory load feeds several multiply-adds.
 constexpr int kQm = 64;        // largest chunk of the gradient kernels
 constexpr int kSQ = kQm + 1;   // row stride of E and F (odd: column reads hit distinct banks)
 
@@ -300,8 +302,9 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
                           });
     bwd_cumsum<T>(a, b, h, c, cs, dts);
     const float cl = cs[Q - 1];
-    // the entering state and adjoint in [n][p] order for the (k, p) outputs: a lane reads four
-    // n of one p, and the lanes of a warp take consecutive p, so the stores hit distinct banks
+    // the entering adjoint in [n][p] order for the (k, p) outputs (a lane reads four n of one p,
+    // and the lanes of a warp take consecutive p, so the stores hit distinct banks); the
+    // entering state in [p][n] order for the (k, n) outputs
     const size_t sbase = (((size_t)b * a.H + h) * a.nc + c) * P * N;
     constexpr int kSU = (P * N / 4 + kTC - 1) / kTC;
     {
@@ -311,8 +314,8 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
             const int i = tid + kTC * u;
             if (i < P * (N / 4)) {
                 const int p = i % P, n = 4 * (i / P);
-                sv[u] = *reinterpret_cast<const float4 *>(a.sf + sbase + (size_t)p * N + n);
                 gv[u] = *reinterpret_cast<const float4 *>(a.sg + sbase + (size_t)p * N + n);
+                sv[u] = *reinterpret_cast<const float4 *>(a.sf + sbase + 4 * (size_t)i);
             }
         }
 #pragma unroll
@@ -320,10 +323,10 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
             const int i = tid + kTC * u;
             if (i < P * (N / 4)) {
                 const int p = i % P, n = 4 * (i / P);
-                S0[n * SX + p] = sv[u].x; S0[(n + 1) * SX + p] = sv[u].y;
-                S0[(n + 2) * SX + p] = sv[u].z; S0[(n + 3) * SX + p] = sv[u].w;
-                S1[n * SX + p] = gv[u].x; S1[(n + 1) * SX + p] = gv[u].y;
-                S1[(n + 2) * SX + p] = gv[u].z; S1[(n + 3) * SX + p] = gv[u].w;
+                S0[n * SX + p] = gv[u].x; S0[(n + 1) * SX + p] = gv[u].y;
+                S0[(n + 2) * SX + p] = gv[u].z; S0[(n + 3) * SX + p] = gv[u].w;
+                const int p2 = i / (N / 4), n2 = 4 * (i % (N / 4));
+                *reinterpret_cast<float4 *>(S1 + p2 * SB + n2) = sv[u];
             }
         }
     }
@@ -376,121 +379,147 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
     }
     __syncthreads();
 
-    // outputs over (k, p): y - D x (recomputed), the adjoint times B, dx.  Thread: one k and
-    // columns p0 .. p0 + 7; the PG threads of one k are consecutive lanes.
+    // <gy_k, y_k - D x_k> without y: its intra-chunk part is sum_{s <= k} E[k][s] dt_s (x_s . gy_k)
+    // with x_s . gy_k = F[s][k] exp(cs_s - cs_k) (the entering-state part is added with the dC
+    // products below), and <gy_k, x_k> = F[k][k].  Eight lanes per position.
+    {
+        const int k = tid >> 3, sl = tid & 7;
+        float acc = 0.f;
+        if (k < Q) {
+            for (int s = sl; s <= k; s += 8) {
+                const float d = cs[s] - cs[k];           // >= 0; F[s][k] carries exp(-d)
+                if (d < 80.f) acc = fmaf(E[k * kSQ + s] * dts[s], F[s * kSQ + k] * expf(d), acc);
+            }
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        if (k < Q && sl == 0) {
+            red[64 + k] = acc;
+            red[128 + k] = F[k * kSQ + k];
+        }
+    }
+
+    // outputs over (k, p): the adjoint times B (its entering part and the chunk's own part) and
+    // dx.  Thread: one k and columns p0 .. p0 + 7; the PG threads of one k are consecutive lanes.
     constexpr int PG = P / 8;
     const float dh = a.D ? a.D[h] : 0.f;
     for (int t = tid; t < Q * PG; t += kTC) {
         const int k = t / PG, p0 = 8 * (t % PG);
-        float yv[8], gb[8], yo[8], go[8];
+        float gb[8], go[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) yv[j] = gb[j] = yo[j] = go[j] = 0.f;
-        for (int s = 0; s <= k; ++s) fma8(yv, E[k * kSQ + s] * dts[s], xs + s * SX + p0);
+        for (int j = 0; j < 8; ++j) gb[j] = go[j] = 0.f;
         for (int s = k; s < Q; ++s) fma8(gb, E[s * kSQ + k], gys + s * SX + p0);
-#pragma unroll 2
-        for (int n = 0; n < N; ++n) {
-            fma8(yo, cc[k * SB + n], S0 + n * SX + p0);
-            fma8(go, bs[k * SB + n], S1 + n * SX + p0);
-        }
-        const float ek = expf(cs[k]), el = expf(cl - cs[k]);
+#pragma unroll 4
+        for (int n = 0; n < N; ++n) fma8(go, bs[k * SB + n], S0 + n * SX + p0);
+        const float el = expf(cl - cs[k]);
         const int tk = tok(c * Q + k, a.L, a.dir);
-        float r0 = 0.f, r1 = 0.f, r2 = 0.f, gxo[8];
+        float r0 = 0.f, gxo[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const float y_ = fmaf(ek, yo[j], yv[j]), g_ = fmaf(el, go[j], gb[j]);
-            const float xv = xs[k * SX + p0 + j], gv = gys[k * SX + p0 + j];
-            gxo[j] = fmaf(dts[k], g_, dh * gv);
-            r0 = fmaf(xv, g_, r0);
-            r1 = fmaf(gv, y_, r1);
-            r2 = fmaf(gv, xv, r2);
+            const float g_ = fmaf(el, go[j], gb[j]);
+            gxo[j] = fmaf(dts[k], g_, dh * gys[k * SX + p0 + j]);
+            r0 = fmaf(xs[k * SX + p0 + j], g_, r0);
         }
         float *gxp = a.gx + (((size_t)b * a.L + tk) * a.H + h) * P + p0;
         *reinterpret_cast<float4 *>(gxp) = make_float4(gxo[0], gxo[1], gxo[2], gxo[3]);
         *reinterpret_cast<float4 *>(gxp + 4) = make_float4(gxo[4], gxo[5], gxo[6], gxo[7]);
         // Q PG is a multiple of 32, so whole warps take part in the shuffles
 #pragma unroll
-        for (int o = PG / 2; o > 0; o >>= 1) {
-            r0 += __shfl_xor_sync(0xffffffffu, r0, o);
-            r1 += __shfl_xor_sync(0xffffffffu, r1, o);
-            r2 += __shfl_xor_sync(0xffffffffu, r2, o);
-        }
-        if ((t & (PG - 1)) == 0) {
-            red[k] = r0;
-            red[64 + k] = r1;
-            red[128 + k] = r2;
-        }
+        for (int o = PG / 2; o > 0; o >>= 1) r0 += __shfl_xor_sync(0xffffffffu, r0, o);
+        if ((t & (PG - 1)) == 0) red[k] = r0;
     }
     __syncthreads();
-    // the entering state and adjoint again, now in [p][n] order for the (k, n) outputs
+    // the entering adjoint again, now in [p][n] order
     {
-        float4 sv[kSU], gv[kSU];
+        float4 gv[kSU];
 #pragma unroll
         for (int u = 0; u < kSU; ++u) {
             const int i = tid + kTC * u;
-            if (i < P * (N / 4)) {
-                sv[u] = *reinterpret_cast<const float4 *>(a.sf + sbase + 4 * (size_t)i);
-                gv[u] = *reinterpret_cast<const float4 *>(a.sg + sbase + 4 * (size_t)i);
-            }
+            if (i < P * (N / 4)) gv[u] = *reinterpret_cast<const float4 *>(a.sg + sbase + 4 * (size_t)i);
         }
 #pragma unroll
         for (int u = 0; u < kSU; ++u) {
             const int i = tid + kTC * u;
-            if (i < P * (N / 4)) {
-                const int p = i / (N / 4), n = 4 * (i % (N / 4));
-                *reinterpret_cast<float4 *>(S0 + p * SB + n) = sv[u];
-                *reinterpret_cast<float4 *>(S1 + p * SB + n) = gv[u];
-            }
+            if (i < P * (N / 4)) *reinterpret_cast<float4 *>(S0 + (i / (N / 4)) * SB + 4 * (i % (N / 4))) = gv[u];
         }
     }
     __syncthreads();
 
-    // outputs over (k, n): this head's parts of dB and dC.  Thread: rows k0, k0 + 1 and
-    // columns n0 .. n0 + 7.
+    // outputs over (k, n): this head's parts of dB (threads 0 .. kTC/2 - 1) and of dC (the
+    // rest).  Thread: rows k0 .. k0 + 3 and columns n0 .. n0 + 7; the NG threads of one row
+    // quad are consecutive lanes.
     constexpr int NG = N / 8;
-    for (int t = tid; t < (Q / 2) * NG; t += kTC) {
-        const int k0 = 2 * (t / NG), n0 = 8 * (t % NG);
-        float gbv0[8], gbv1[8], gcv0[8], gcv1[8], bo0[8], bo1[8], co0[8], co1[8];
+    {
+        const bool second = tid >= kTC / 2;            // uniform per warp
+        const int t = tid & (kTC / 2 - 1);
+        const bool active = t < (Q / 4) * NG;
+        const int k0 = 4 * (t / NG), n0 = 8 * (t % NG);
+        float acc[4][8], pro[4][8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            gbv0[j] = gbv1[j] = gcv0[j] = gcv1[j] = bo0[j] = bo1[j] = co0[j] = co1[j] = 0.f;
-        // sum over s >= k of F[k][s] C_s (F[k0 + 1][k0] is 0)
-        for (int s = k0; s < Q; ++s) {
-            const float *cv = cc + s * SB + n0;
-            fma8(gbv0, F[k0 * kSQ + s], cv);
-            fma8(gbv1, F[(k0 + 1) * kSQ + s], cv);
-        }
-        // sum over s <= k of F[s][k] dt_s B_s (F[k0 + 1][k0] is 0)
-        for (int s = 0; s <= k0 + 1; ++s) {
-            const float d = dts[s];
-            const float *bv = bs + s * SB + n0;
-            fma8(gcv0, F[s * kSQ + k0] * d, bv);
-            fma8(gcv1, F[s * kSQ + k0 + 1] * d, bv);
-        }
-#pragma unroll 2
-        for (int p = 0; p < P; ++p) {
-            const float *gi = S1 + p * SB + n0, *si = S0 + p * SB + n0;
-            fma8(bo0, xs[k0 * SX + p], gi);
-            fma8(bo1, xs[(k0 + 1) * SX + p], gi);
-            fma8(co0, gys[k0 * SX + p], si);
-            fma8(co1, gys[(k0 + 1) * SX + p], si);
-        }
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-            const int k = k0 + kk;
-            const float ek = expf(cs[k]), el = expf(cl - cs[k]), dk = dts[k];
-            const float *bo = kk ? bo1 : bo0, *gbv = kk ? gbv1 : gbv0, *co = kk ? co1 : co0, *gcv = kk ? gcv1 : gcv0;
-            float ob[8], oc[8];
+            for (int j = 0; j < 8; ++j) acc[i][j] = pro[i][j] = 0.f;
+        if (active && !second) {
+            // sum over s >= k of F[k][s] C_s (F[k][s] = 0 for s < k); x_k . Gin
+            for (int s = k0; s < Q; ++s) {
+                const float *cv = cc + s * SB + n0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                ob[j] = dk * fmaf(el, bo[j], gbv[j]);
-                oc[j] = fmaf(ek, co[j], gcv[j]);
+                for (int i = 0; i < 4; ++i) fma8(acc[i], F[(k0 + i) * kSQ + s], cv);
             }
-            const int tk = tok(c * Q + k, a.L, a.dir);
-            const size_t oi = (((size_t)b * a.L + tk) * a.H + h) * N + n0;
-            *reinterpret_cast<float4 *>(a.gBh + oi) = make_float4(ob[0], ob[1], ob[2], ob[3]);
-            *reinterpret_cast<float4 *>(a.gBh + oi + 4) = make_float4(ob[4], ob[5], ob[6], ob[7]);
-            *reinterpret_cast<float4 *>(a.gCh + oi) = make_float4(oc[0], oc[1], oc[2], oc[3]);
-            *reinterpret_cast<float4 *>(a.gCh + oi + 4) = make_float4(oc[4], oc[5], oc[6], oc[7]);
+#pragma unroll 2
+            for (int p = 0; p < P; ++p) {
+                const float *gi = S0 + p * SB + n0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) fma8(pro[i], xs[(k0 + i) * SX + p], gi);
+            }
+        } else if (active) {
+            // sum over s <= k of F[s][k] dt_s B_s (F[s][k] = 0 for s > k); gy_k . Sin
+            for (int s = 0; s <= k0 + 3; ++s) {
+                const float d = dts[s];
+                const float *bv = bs + s * SB + n0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) fma8(acc[i], F[s * kSQ + k0 + i] * d, bv);
+            }
+#pragma unroll 2
+            for (int p = 0; p < P; ++p) {
+                const float *si = S1 + p * SB + n0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) fma8(pro[i], gys[(k0 + i) * SX + p], si);
+            }
+        }
+        float rpart[4] = {0.f, 0.f, 0.f, 0.f};
+        if (active) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int k = k0 + i;
+                const float ek = expf(cs[k]), el = expf(cl - cs[k]), dk = dts[k];
+                float o[8];
+                if (!second) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) o[j] = dk * fmaf(el, pro[i][j], acc[i][j]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        o[j] = fmaf(ek, pro[i][j], acc[i][j]);
+                        rpart[i] = fmaf(cc[k * SB + n0 + j], pro[i][j], rpart[i]);   // C_k . (Sin gy_k)
+                    }
+                    rpart[i] *= ek;
+                }
+                const int tk = tok(c * Q + k, a.L, a.dir);
+                float *op = (second ? a.gCh : a.gBh) + (((size_t)b * a.L + tk) * a.H + h) * N + n0;
+                *reinterpret_cast<float4 *>(op) = make_float4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<float4 *>(op + 4) = make_float4(o[4], o[5], o[6], o[7]);
+            }
+        }
+        if (second) {
+#pragma unroll
+            for (int o = NG / 2; o > 0; o >>= 1)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) rpart[i] += __shfl_xor_sync(0xffffffffu, rpart[i], o);
+            if (active && (t & (NG - 1)) == 0)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) red[64 + k0 + i] += rpart[i];
         }
     }
     __syncthreads();
