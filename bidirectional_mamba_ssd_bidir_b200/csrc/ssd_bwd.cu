@@ -255,8 +255,8 @@ __global__ void __launch_bounds__(kT) k_bwd_pass_small(BwdArgs a) {
 // entering adjoint Gin carry everything outside the chunk.  The forward output is not
 // recomputed: <gy_k, y_k - D x_k> = exp(cs_k) C_k . (Sin gy_k) + sum_{s<=k} E[k][s] dt_s x_s . gy_k,
 // whose first part falls out of the dC products.  Every product below is a small matrix product
-// evaluated in register tiles (one k and 8 columns, or 4 k and 8 columns per thread), so that
-// each shared-memory load feeds several multiply-adds.
+// evaluated in register tiles (2 or 4 k and 8 columns per thread), so that each shared-memory
+// load feeds several multiply-adds.
 constexpr int kQm = 64;        // largest chunk of the gradient kernels
 constexpr int kSQ = kQm + 1;   // row stride of E and F (odd: column reads hit distinct banks)
 
@@ -264,7 +264,9 @@ template <int P, int N>
 struct ChunkSmem {
     static constexpr int SX = P + 4;   // rows of x, gy (16-byte aligned, 4 banks apart)
     static constexpr int SB = N + 4;   // rows of B, C and of Sin, Gin in [p][n] order
-    static constexpr int kS = (N * SX > P * SB) ? N * SX : P * SB;   // one of Sin, Gin, either order
+    // one of Sin, Gin in either order; also the [k][p] hand-off of the two CTA halves
+    static constexpr int kS2 = (N * SX > P * SB) ? N * SX : P * SB;
+    static constexpr int kS = kS2 > kQm * P ? kS2 : kQm * P;
     static constexpr int kCs = 0, kDt = 64, kRed = 128, kX = 320, kGy = kX + kQm * SX, kB = kGy + kQm * SX,
                          kC = kB + kQm * SB, kS0 = kC + kQm * SB, kS1 = kS0 + kS, kE = kS1 + kS, kF = kE + kQm * kSQ,
                          kFloats = kF + kQm * kSQ;
@@ -302,20 +304,18 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
                           });
     bwd_cumsum<T>(a, b, h, c, cs, dts);
     const float cl = cs[Q - 1];
-    // the entering adjoint in [n][p] order for the (k, p) outputs (a lane reads four n of one p,
-    // and the lanes of a warp take consecutive p, so the stores hit distinct banks); the
-    // entering state in [p][n] order for the (k, n) outputs
+    // the entering adjoint in [n][p] order for the (k, p) outputs: a lane reads four n of one p,
+    // and the lanes of a warp take consecutive p, so the stores hit distinct banks
     const size_t sbase = (((size_t)b * a.H + h) * a.nc + c) * P * N;
     constexpr int kSU = (P * N / 4 + kTC - 1) / kTC;
     {
-        float4 sv[kSU], gv[kSU];
+        float4 gv[kSU];
 #pragma unroll
         for (int u = 0; u < kSU; ++u) {
             const int i = tid + kTC * u;
             if (i < P * (N / 4)) {
                 const int p = i % P, n = 4 * (i / P);
                 gv[u] = *reinterpret_cast<const float4 *>(a.sg + sbase + (size_t)p * N + n);
-                sv[u] = *reinterpret_cast<const float4 *>(a.sf + sbase + 4 * (size_t)i);
             }
         }
 #pragma unroll
@@ -325,8 +325,6 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
                 const int p = i % P, n = 4 * (i / P);
                 S0[n * SX + p] = gv[u].x; S0[(n + 1) * SX + p] = gv[u].y;
                 S0[(n + 2) * SX + p] = gv[u].z; S0[(n + 3) * SX + p] = gv[u].w;
-                const int p2 = i / (N / 4), n2 = 4 * (i % (N / 4));
-                *reinterpret_cast<float4 *>(S1 + p2 * SB + n2) = sv[u];
             }
         }
     }
@@ -401,47 +399,100 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
     }
 
     // outputs over (k, p): the adjoint times B (its entering part and the chunk's own part) and
-    // dx.  Thread: one k and columns p0 .. p0 + 7; the PG threads of one k are consecutive lanes.
+    // dx.  Thread: rows k0, k0 + 1 and columns p0 .. p0 + 7.  The two halves of the CTA take
+    // alternate s of the chunk's own part and one half each of the state index n of the entering
+    // part; the second half hands its sums to the first through the entering state's buffer
+    // (not loaded yet).  The PG threads of one row pair are consecutive lanes.
     constexpr int PG = P / 8;
-    const float dh = a.D ? a.D[h] : 0.f;
-    for (int t = tid; t < Q * PG; t += kTC) {
-        const int k = t / PG, p0 = 8 * (t % PG);
-        float gb[8], go[8];
+    {
+        const float dh = a.D ? a.D[h] : 0.f;
+        const int half = tid >= kTC / 2;               // uniform per warp
+        const int t = tid & (kTC / 2 - 1);
+        const bool active = t < (Q / 2) * PG;
+        const int k0 = 2 * (t / PG), p0 = 8 * (t % PG);
+        float *xch = S1;                               // [k][p], Q P floats
+        float g0[8], g1[8];
+        if (active) {
+            float gb0[8], gb1[8], go0[8], go1[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) gb[j] = go[j] = 0.f;
-        for (int s = k; s < Q; ++s) fma8(gb, E[s * kSQ + k], gys + s * SX + p0);
+            for (int j = 0; j < 8; ++j) gb0[j] = gb1[j] = go0[j] = go1[j] = 0.f;
+            // E[k0][k0 + 1] is 0
+            for (int s = k0 + half; s < Q; s += 2) {
+                const float *v = gys + s * SX + p0;
+                fma8(gb0, E[s * kSQ + k0], v);
+                fma8(gb1, E[s * kSQ + k0 + 1], v);
+            }
+            const int n1 = half * (N / 2);
 #pragma unroll 4
-        for (int n = 0; n < N; ++n) fma8(go, bs[k * SB + n], S0 + n * SX + p0);
-        const float el = expf(cl - cs[k]);
-        const int tk = tok(c * Q + k, a.L, a.dir);
-        float r0 = 0.f, gxo[8];
+            for (int n = n1; n < n1 + N / 2; ++n) {
+                const float *v = S0 + n * SX + p0;
+                fma8(go0, bs[k0 * SB + n], v);
+                fma8(go1, bs[(k0 + 1) * SB + n], v);
+            }
+            const float el0 = expf(cl - cs[k0]), el1 = expf(cl - cs[k0 + 1]);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float g_ = fmaf(el, go[j], gb[j]);
-            gxo[j] = fmaf(dts[k], g_, dh * gys[k * SX + p0 + j]);
-            r0 = fmaf(xs[k * SX + p0 + j], g_, r0);
+            for (int j = 0; j < 8; ++j) {
+                g0[j] = fmaf(el0, go0[j], gb0[j]);
+                g1[j] = fmaf(el1, go1[j], gb1[j]);
+            }
+            if (half) {
+                st8(xch + k0 * P + p0, g0);
+                st8(xch + (k0 + 1) * P + p0, g1);
+            }
         }
-        float *gxp = a.gx + (((size_t)b * a.L + tk) * a.H + h) * P + p0;
-        *reinterpret_cast<float4 *>(gxp) = make_float4(gxo[0], gxo[1], gxo[2], gxo[3]);
-        *reinterpret_cast<float4 *>(gxp + 4) = make_float4(gxo[4], gxo[5], gxo[6], gxo[7]);
-        // Q PG is a multiple of 32, so whole warps take part in the shuffles
+        __syncthreads();
+        if (!half) {
+            float r0a = 0.f, r0b = 0.f;
+            if (active) {
 #pragma unroll
-        for (int o = PG / 2; o > 0; o >>= 1) r0 += __shfl_xor_sync(0xffffffffu, r0, o);
-        if ((t & (PG - 1)) == 0) red[k] = r0;
+                for (int kk = 0; kk < 2; ++kk) {
+                    const int k = k0 + kk;
+                    const float *gk = kk ? g1 : g0;
+                    float gxo[8], r0 = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float g_ = gk[j] + xch[k * P + p0 + j];
+                        gxo[j] = fmaf(dts[k], g_, dh * gys[k * SX + p0 + j]);
+                        r0 = fmaf(xs[k * SX + p0 + j], g_, r0);
+                    }
+                    if (kk) r0b = r0; else r0a = r0;
+                    const int tk = tok(c * Q + k, a.L, a.dir);
+                    float *gxp = a.gx + (((size_t)b * a.L + tk) * a.H + h) * P + p0;
+                    *reinterpret_cast<float4 *>(gxp) = make_float4(gxo[0], gxo[1], gxo[2], gxo[3]);
+                    *reinterpret_cast<float4 *>(gxp + 4) = make_float4(gxo[4], gxo[5], gxo[6], gxo[7]);
+                }
+            }
+#pragma unroll
+            for (int o = PG / 2; o > 0; o >>= 1) {
+                r0a += __shfl_xor_sync(0xffffffffu, r0a, o);
+                r0b += __shfl_xor_sync(0xffffffffu, r0b, o);
+            }
+            if (active && (t & (PG - 1)) == 0) {
+                red[k0] = r0a;
+                red[k0 + 1] = r0b;
+            }
+        }
     }
     __syncthreads();
-    // the entering adjoint again, now in [p][n] order
+    // the entering adjoint again, now in [p][n] order, and the entering state in [p][n] order
     {
-        float4 gv[kSU];
+        float4 gv[kSU], sv[kSU];
 #pragma unroll
         for (int u = 0; u < kSU; ++u) {
             const int i = tid + kTC * u;
-            if (i < P * (N / 4)) gv[u] = *reinterpret_cast<const float4 *>(a.sg + sbase + 4 * (size_t)i);
+            if (i < P * (N / 4)) {
+                gv[u] = *reinterpret_cast<const float4 *>(a.sg + sbase + 4 * (size_t)i);
+                sv[u] = *reinterpret_cast<const float4 *>(a.sf + sbase + 4 * (size_t)i);
+            }
         }
 #pragma unroll
         for (int u = 0; u < kSU; ++u) {
             const int i = tid + kTC * u;
-            if (i < P * (N / 4)) *reinterpret_cast<float4 *>(S0 + (i / (N / 4)) * SB + 4 * (i % (N / 4))) = gv[u];
+            if (i < P * (N / 4)) {
+                const int o = (i / (N / 4)) * SB + 4 * (i % (N / 4));
+                *reinterpret_cast<float4 *>(S0 + o) = gv[u];
+                *reinterpret_cast<float4 *>(S1 + o) = sv[u];
+            }
         }
     }
     __syncthreads();
