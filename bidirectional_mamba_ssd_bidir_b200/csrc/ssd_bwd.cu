@@ -38,6 +38,13 @@ constexpr int kT = 256;       // threads per CTA
 constexpr int kTC = 512;      // threads per CTA of the per-chunk gradient kernel (more warps hide its
                               // shared-memory latency; one CTA per SM fits its shared memory)
 
+// Offset of the P x N chunk state (or adjoint) of (b, h, chunk c) in a.sf / a.sg.  The heads of
+// one chunk are neighbours, so the state passes, which walk all heads chunk by chunk, touch one
+// contiguous range at a time instead of addresses a power of two apart.
+__device__ __forceinline__ size_t chunk_slot(const BwdArgs &a, int b, int h, int c, int PN) {
+    return (((size_t)b * a.nc + c) * a.H + h) * (size_t)PN;
+}
+
 // Eight consecutive values of a 16-byte aligned row, as float.
 template <typename T> __device__ __forceinline__ void ld8(const T *p, float (&v)[8]);
 template <> __device__ __forceinline__ void ld8<float>(const float *p, float (&v)[8]) {
@@ -54,10 +61,11 @@ template <> __device__ __forceinline__ void ld8<__nv_bfloat16>(const __nv_bfloat
     }
 }
 
-// Eight floats to a 16-byte aligned shared-memory address.
+// Eight floats to two 16-byte aligned addresses HALF apart (HALF = 4: eight consecutive).
+template <int HALF = 4>
 __device__ __forceinline__ void st8(float *d, const float (&v)[8]) {
     *reinterpret_cast<float4 *>(d) = make_float4(v[0], v[1], v[2], v[3]);
-    *reinterpret_cast<float4 *>(d + 4) = make_float4(v[4], v[5], v[6], v[7]);
+    *reinterpret_cast<float4 *>(d + HALF) = make_float4(v[4], v[5], v[6], v[7]);
 }
 
 // Rows 0 .. Q-1 of two [token][W] arrays that share their row addresses (x and gy, or B and C)
@@ -139,38 +147,76 @@ __global__ void __launch_bounds__(kT) k_bwd_chunk_sums(BwdArgs a) {
                              st8(gw + k * P + p, og);
                          });
     __syncthreads();
-    // thread: column n and E consecutive rows p0 .. p0 + E - 1, so that the row weights of one k
-    // are read as whole vectors (the same for every lane of a warp when N >= 32)
-    float sf[E], sg[E];
+    const size_t base = chunk_slot(a, b, h, c, P * N);
+    if constexpr (E == 32 && N == 4 * 32 && P == 8 * (kT / 32)) {
+        // 4 columns x 8 rows of each sum per thread: lane = column quad n0, warp = row octet p0.
+        // B and C rows are read as whole-warp vectors, the row weights as broadcasts.
+        const int n0 = 4 * (threadIdx.x & 31), p0 = 8 * (threadIdx.x >> 5);
+        float sf[8][4], sg[8][4];
 #pragma unroll
-    for (int j = 0; j < E; ++j) sf[j] = sg[j] = 0.f;
-    const int n = threadIdx.x % N, p0 = (threadIdx.x / N) * E;
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sf[i][j] = sg[i][j] = 0.f;
 #pragma unroll 2
-    for (int k = 0; k < Q; ++k) {
-        const float bv = bs[k * N + n], cv = cc[k * N + n];
-        if constexpr (E % 4 == 0) {
+        for (int k = 0; k < Q; ++k) {
+            const float4 bv = *reinterpret_cast<const float4 *>(bs + k * N + n0);
+            const float4 cv = *reinterpret_cast<const float4 *>(cc + k * N + n0);
+            const float b4[4] = {bv.x, bv.y, bv.z, bv.w}, c4[4] = {cv.x, cv.y, cv.z, cv.w};
+            float xv[8], gv[8];
+            const float4 x0 = *reinterpret_cast<const float4 *>(xw + k * P + p0);
+            const float4 x1 = *reinterpret_cast<const float4 *>(xw + k * P + p0 + 4);
+            const float4 g0 = *reinterpret_cast<const float4 *>(gw + k * P + p0);
+            const float4 g1 = *reinterpret_cast<const float4 *>(gw + k * P + p0 + 4);
+            xv[0] = x0.x; xv[1] = x0.y; xv[2] = x0.z; xv[3] = x0.w; xv[4] = x1.x; xv[5] = x1.y; xv[6] = x1.z; xv[7] = x1.w;
+            gv[0] = g0.x; gv[1] = g0.y; gv[2] = g0.z; gv[3] = g0.w; gv[4] = g1.x; gv[5] = g1.y; gv[6] = g1.z; gv[7] = g1.w;
 #pragma unroll
-            for (int j = 0; j < E; j += 4) {
-                const float4 xv = *reinterpret_cast<const float4 *>(xw + k * P + p0 + j);
-                const float4 gv = *reinterpret_cast<const float4 *>(gw + k * P + p0 + j);
-                sf[j] = fmaf(xv.x, bv, sf[j]); sf[j + 1] = fmaf(xv.y, bv, sf[j + 1]);
-                sf[j + 2] = fmaf(xv.z, bv, sf[j + 2]); sf[j + 3] = fmaf(xv.w, bv, sf[j + 3]);
-                sg[j] = fmaf(gv.x, cv, sg[j]); sg[j + 1] = fmaf(gv.y, cv, sg[j + 1]);
-                sg[j + 2] = fmaf(gv.z, cv, sg[j + 2]); sg[j + 3] = fmaf(gv.w, cv, sg[j + 3]);
-            }
-        } else {
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int j = 0; j < E; ++j) {
-                sf[j] = fmaf(xw[k * P + p0 + j], bv, sf[j]);
-                sg[j] = fmaf(gw[k * P + p0 + j], cv, sg[j]);
+                for (int j = 0; j < 4; ++j) {
+                    sf[i][j] = fmaf(xv[i], b4[j], sf[i][j]);
+                    sg[i][j] = fmaf(gv[i], c4[j], sg[i][j]);
+                }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            *reinterpret_cast<float4 *>(a.sf + base + (size_t)(p0 + i) * N + n0) =
+                make_float4(sf[i][0], sf[i][1], sf[i][2], sf[i][3]);
+            *reinterpret_cast<float4 *>(a.sg + base + (size_t)(p0 + i) * N + n0) =
+                make_float4(sg[i][0], sg[i][1], sg[i][2], sg[i][3]);
+        }
+    } else {
+        // thread: column n and E consecutive rows p0 .. p0 + E - 1, so that the row weights of one k
+        // are read as whole vectors (the same for every lane of a warp when N >= 32)
+        float sf[E], sg[E];
+#pragma unroll
+        for (int j = 0; j < E; ++j) sf[j] = sg[j] = 0.f;
+        const int n = threadIdx.x % N, p0 = (threadIdx.x / N) * E;
+#pragma unroll 2
+        for (int k = 0; k < Q; ++k) {
+            const float bv = bs[k * N + n], cv = cc[k * N + n];
+            if constexpr (E % 4 == 0) {
+#pragma unroll
+                for (int j = 0; j < E; j += 4) {
+                    const float4 xv = *reinterpret_cast<const float4 *>(xw + k * P + p0 + j);
+                    const float4 gv = *reinterpret_cast<const float4 *>(gw + k * P + p0 + j);
+                    sf[j] = fmaf(xv.x, bv, sf[j]); sf[j + 1] = fmaf(xv.y, bv, sf[j + 1]);
+                    sf[j + 2] = fmaf(xv.z, bv, sf[j + 2]); sf[j + 3] = fmaf(xv.w, bv, sf[j + 3]);
+                    sg[j] = fmaf(gv.x, cv, sg[j]); sg[j + 1] = fmaf(gv.y, cv, sg[j + 1]);
+                    sg[j + 2] = fmaf(gv.z, cv, sg[j + 2]); sg[j + 3] = fmaf(gv.w, cv, sg[j + 3]);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < E; ++j) {
+                    sf[j] = fmaf(xw[k * P + p0 + j], bv, sf[j]);
+                    sg[j] = fmaf(gw[k * P + p0 + j], cv, sg[j]);
+                }
             }
         }
-    }
-    const size_t base = (((size_t)b * a.H + h) * a.nc + c) * P * N;
 #pragma unroll
-    for (int j = 0; j < E; ++j) {
-        a.sf[base + (size_t)(p0 + j) * N + n] = sf[j];
-        a.sg[base + (size_t)(p0 + j) * N + n] = sg[j];
+        for (int j = 0; j < E; ++j) {
+            a.sf[base + (size_t)(p0 + j) * N + n] = sf[j];
+            a.sg[base + (size_t)(p0 + j) * N + n] = sg[j];
+        }
     }
     if (threadIdx.x == 0) a.dec[((size_t)b * a.H + h) * a.nc + c] = expf(cl);
 }
@@ -203,7 +249,7 @@ __global__ void __launch_bounds__(kT) k_bwd_pass(BwdArgs a) {
 #pragma unroll
                 for (int j = 0; j < kPassE; ++j) v[u][j] = 0.f;
                 if (i < a.nc) {
-                    const float *S = arr + (base + c) * P * N;
+                    const float *S = arr + chunk_slot(a, b, h, c, P * N);
                     dc[u] = a.dec[base + c];
 #pragma unroll
                     for (int j = 0; j < kPassE; ++j) v[u][j] = S[e0 + kT * j];
@@ -214,7 +260,7 @@ __global__ void __launch_bounds__(kT) k_bwd_pass(BwdArgs a) {
                 const int i = c0 + u;
                 if (i < a.nc) {
                     const int c = dirn == 0 ? i : a.nc - 1 - i;
-                    float *S = arr + (base + c) * P * N;
+                    float *S = arr + chunk_slot(a, b, h, c, P * N);
 #pragma unroll
                     for (int j = 0; j < kPassE; ++j) {
                         S[e0 + kT * j] = run[j];
@@ -234,14 +280,14 @@ __global__ void __launch_bounds__(kT) k_bwd_pass_small(BwdArgs a) {
     for (int e = threadIdx.x; e < P * N; e += kT) {
         float run = 0.f;
         for (int c = 0; c < a.nc; ++c) {
-            float *S = a.sf + (base + c) * P * N;
+            float *S = a.sf + chunk_slot(a, b, h, c, P * N);
             const float v = S[e];
             S[e] = run;
             run = fmaf(a.dec[base + c], run, v);
         }
         run = 0.f;
         for (int c = a.nc - 1; c >= 0; --c) {
-            float *Z = a.sg + (base + c) * P * N;
+            float *Z = a.sg + chunk_slot(a, b, h, c, P * N);
             const float v = Z[e];
             Z[e] = run;
             run = fmaf(a.dec[base + c], run, v);
@@ -272,8 +318,12 @@ struct ChunkSmem {
                          kFloats = kF + kQm * kSQ;
 };
 
+// acc[j] += m v[col(j)] over a thread's eight columns col(j) = (j & 3) + (j >> 2) HALF: two groups
+// of four, HALF apart.  The lanes of a warp take consecutive groups of four, so each 16-byte
+// load of a warp reads one contiguous run of the row (no bank conflicts).
+template <int HALF>
 __device__ __forceinline__ void fma8(float (&acc)[8], float m, const float *v) {
-    const float4 a = *reinterpret_cast<const float4 *>(v), b = *reinterpret_cast<const float4 *>(v + 4);
+    const float4 a = *reinterpret_cast<const float4 *>(v), b = *reinterpret_cast<const float4 *>(v + HALF);
     acc[0] = fmaf(m, a.x, acc[0]); acc[1] = fmaf(m, a.y, acc[1]); acc[2] = fmaf(m, a.z, acc[2]);
     acc[3] = fmaf(m, a.w, acc[3]); acc[4] = fmaf(m, b.x, acc[4]); acc[5] = fmaf(m, b.y, acc[5]);
     acc[6] = fmaf(m, b.z, acc[6]); acc[7] = fmaf(m, b.w, acc[7]);
@@ -306,7 +356,7 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
     const float cl = cs[Q - 1];
     // the entering adjoint in [n][p] order for the (k, p) outputs: a lane reads four n of one p,
     // and the lanes of a warp take consecutive p, so the stores hit distinct banks
-    const size_t sbase = (((size_t)b * a.H + h) * a.nc + c) * P * N;
+    const size_t sbase = chunk_slot(a, b, h, c, P * N);
     constexpr int kSU = (P * N / 4 + kTC - 1) / kTC;
     {
         float4 gv[kSU];
@@ -399,7 +449,7 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
     }
 
     // outputs over (k, p): the adjoint times B (its entering part and the chunk's own part) and
-    // dx.  Thread: rows k0, k0 + 1 and columns p0 .. p0 + 7.  The two halves of the CTA take
+    // dx.  Thread: rows k0, k0 + 1 and columns p0 + (j & 3) + (j >> 2) P/2.  The two halves of the CTA take
     // alternate s of the chunk's own part and one half each of the state index n of the entering
     // part; the second half hands its sums to the first through the entering state's buffer
     // (not loaded yet).  The PG threads of one row pair are consecutive lanes.
@@ -409,7 +459,8 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
         const int half = tid >= kTC / 2;               // uniform per warp
         const int t = tid & (kTC / 2 - 1);
         const bool active = t < (Q / 2) * PG;
-        const int k0 = 2 * (t / PG), p0 = 8 * (t % PG);
+        constexpr int HP = P / 2;
+        const int k0 = 2 * (t / PG), p0 = 4 * (t % PG);
         float *xch = S1;                               // [k][p], Q P floats
         float g0[8], g1[8];
         if (active) {
@@ -419,15 +470,15 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
             // E[k0][k0 + 1] is 0
             for (int s = k0 + half; s < Q; s += 2) {
                 const float *v = gys + s * SX + p0;
-                fma8(gb0, E[s * kSQ + k0], v);
-                fma8(gb1, E[s * kSQ + k0 + 1], v);
+                fma8<HP>(gb0, E[s * kSQ + k0], v);
+                fma8<HP>(gb1, E[s * kSQ + k0 + 1], v);
             }
             const int n1 = half * (N / 2);
 #pragma unroll 4
             for (int n = n1; n < n1 + N / 2; ++n) {
                 const float *v = S0 + n * SX + p0;
-                fma8(go0, bs[k0 * SB + n], v);
-                fma8(go1, bs[(k0 + 1) * SB + n], v);
+                fma8<HP>(go0, bs[k0 * SB + n], v);
+                fma8<HP>(go1, bs[(k0 + 1) * SB + n], v);
             }
             const float el0 = expf(cl - cs[k0]), el1 = expf(cl - cs[k0 + 1]);
 #pragma unroll
@@ -436,8 +487,8 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
                 g1[j] = fmaf(el1, go1[j], gb1[j]);
             }
             if (half) {
-                st8(xch + k0 * P + p0, g0);
-                st8(xch + (k0 + 1) * P + p0, g1);
+                st8<HP>(xch + k0 * P + p0, g0);
+                st8<HP>(xch + (k0 + 1) * P + p0, g1);
             }
         }
         __syncthreads();
@@ -451,15 +502,16 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
                     float gxo[8], r0 = 0.f;
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const float g_ = gk[j] + xch[k * P + p0 + j];
-                        gxo[j] = fmaf(dts[k], g_, dh * gys[k * SX + p0 + j]);
-                        r0 = fmaf(xs[k * SX + p0 + j], g_, r0);
+                        const int pj = p0 + (j & 3) + (j >> 2) * HP;
+                        const float g_ = gk[j] + xch[k * P + pj];
+                        gxo[j] = fmaf(dts[k], g_, dh * gys[k * SX + pj]);
+                        r0 = fmaf(xs[k * SX + pj], g_, r0);
                     }
                     if (kk) r0b = r0; else r0a = r0;
                     const int tk = tok(c * Q + k, a.L, a.dir);
                     float *gxp = a.gx + (((size_t)b * a.L + tk) * a.H + h) * P + p0;
                     *reinterpret_cast<float4 *>(gxp) = make_float4(gxo[0], gxo[1], gxo[2], gxo[3]);
-                    *reinterpret_cast<float4 *>(gxp + 4) = make_float4(gxo[4], gxo[5], gxo[6], gxo[7]);
+                    *reinterpret_cast<float4 *>(gxp + HP) = make_float4(gxo[4], gxo[5], gxo[6], gxo[7]);
                 }
             }
 #pragma unroll
@@ -498,14 +550,15 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
     __syncthreads();
 
     // outputs over (k, n): this head's parts of dB (threads 0 .. kTC/2 - 1) and of dC (the
-    // rest).  Thread: rows k0 .. k0 + 3 and columns n0 .. n0 + 7; the NG threads of one row
-    // quad are consecutive lanes.
+    // rest).  Thread: rows k0 .. k0 + 3 and columns n0 + (j & 3) + (j >> 2) N/2; the NG threads
+    // of one row quad are consecutive lanes.
     constexpr int NG = N / 8;
     {
         const bool second = tid >= kTC / 2;            // uniform per warp
         const int t = tid & (kTC / 2 - 1);
         const bool active = t < (Q / 4) * NG;
-        const int k0 = 4 * (t / NG), n0 = 8 * (t % NG);
+        constexpr int HN = N / 2;
+        const int k0 = 4 * (t / NG), n0 = 4 * (t % NG);
         float acc[4][8], pro[4][8];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -516,13 +569,13 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
             for (int s = k0; s < Q; ++s) {
                 const float *cv = cc + s * SB + n0;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) fma8(acc[i], F[(k0 + i) * kSQ + s], cv);
+                for (int i = 0; i < 4; ++i) fma8<HN>(acc[i], F[(k0 + i) * kSQ + s], cv);
             }
 #pragma unroll 2
             for (int p = 0; p < P; ++p) {
                 const float *gi = S0 + p * SB + n0;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) fma8(pro[i], xs[(k0 + i) * SX + p], gi);
+                for (int i = 0; i < 4; ++i) fma8<HN>(pro[i], xs[(k0 + i) * SX + p], gi);
             }
         } else if (active) {
             // sum over s <= k of F[s][k] dt_s B_s (F[s][k] = 0 for s > k); gy_k . Sin
@@ -530,13 +583,13 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
                 const float d = dts[s];
                 const float *bv = bs + s * SB + n0;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) fma8(acc[i], F[s * kSQ + k0 + i] * d, bv);
+                for (int i = 0; i < 4; ++i) fma8<HN>(acc[i], F[s * kSQ + k0 + i] * d, bv);
             }
 #pragma unroll 2
             for (int p = 0; p < P; ++p) {
                 const float *si = S1 + p * SB + n0;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) fma8(pro[i], gys[(k0 + i) * SX + p], si);
+                for (int i = 0; i < 4; ++i) fma8<HN>(pro[i], gys[(k0 + i) * SX + p], si);
             }
         }
         float rpart[4] = {0.f, 0.f, 0.f, 0.f};
@@ -553,14 +606,14 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         o[j] = fmaf(ek, pro[i][j], acc[i][j]);
-                        rpart[i] = fmaf(cc[k * SB + n0 + j], pro[i][j], rpart[i]);   // C_k . (Sin gy_k)
+                        rpart[i] = fmaf(cc[k * SB + n0 + (j & 3) + (j >> 2) * HN], pro[i][j], rpart[i]);   // C_k . (Sin gy_k)
                     }
                     rpart[i] *= ek;
                 }
                 const int tk = tok(c * Q + k, a.L, a.dir);
                 float *op = (second ? a.gCh : a.gBh) + (((size_t)b * a.L + tk) * a.H + h) * N + n0;
                 *reinterpret_cast<float4 *>(op) = make_float4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<float4 *>(op + 4) = make_float4(o[4], o[5], o[6], o[7]);
+                *reinterpret_cast<float4 *>(op + HN) = make_float4(o[4], o[5], o[6], o[7]);
             }
         }
         if (second) {
