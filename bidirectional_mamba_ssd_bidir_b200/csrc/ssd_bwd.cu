@@ -382,8 +382,8 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
     __syncthreads();
 
     // E (threads 0..255) and F (threads 256..511), 4 x 4 tiles.  For Q = 64 a warp covers
-    // 32 k x 16 s with k = k0 + 8i, s = s0 + 4j, so the scalar loads of one instruction fall in
-    // distinct banks.
+    // 32 k x 16 s with k = k0 + 8i, s = s0 + 4j, so the rows read by one instruction are
+    // consecutive and their 16-byte pieces fall in distinct banks.
     {
         const bool second = tid >= kTC / 2;
         const int t = tid & (kTC / 2 - 1);
@@ -403,17 +403,23 @@ __global__ void __launch_bounds__(kTC) k_bwd_chunk(BwdArgs a) {
                 for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
             const float *ra = second ? xs : cc, *rb = second ? gys : bs;
             const int st = second ? SX : SB, K = second ? P : N;
-#pragma unroll 4
-            for (int kk = 0; kk < K; ++kk) {
-                float av[4], bv[4];
+            // four K steps per iteration: each row is read as one 16-byte vector
+#pragma unroll 2
+            for (int kk = 0; kk < K; kk += 4) {
+                float4 av[4], bv[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) av[i] = ra[(k0 + kst * i) * st + kk];
+                for (int i = 0; i < 4; ++i) av[i] = *reinterpret_cast<const float4 *>(ra + (k0 + kst * i) * st + kk);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) bv[j] = rb[(s0 + sst * j) * st + kk];
+                for (int j = 0; j < 4; ++j) bv[j] = *reinterpret_cast<const float4 *>(rb + (s0 + sst * j) * st + kk);
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+                    for (int j = 0; j < 4; ++j) {
+                        acc[i][j] = fmaf(av[i].x, bv[j].x, acc[i][j]);
+                        acc[i][j] = fmaf(av[i].y, bv[j].y, acc[i][j]);
+                        acc[i][j] = fmaf(av[i].z, bv[j].z, acc[i][j]);
+                        acc[i][j] = fmaf(av[i].w, bv[j].w, acc[i][j]);
+                    }
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i)
