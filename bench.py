@@ -373,18 +373,31 @@ def run_bwd(args) -> None:
     ms = start.elapsed_time(end) / args.steps
     e = 2 if shape.io == "bf16" else 4
     H, P, N, G = shape.nheads, shape.headdim, shape.dstate, shape.ngroups
+    Q = min(chunk, 64)
     # per token and direction: read x, dt, B, C, gy; write float32 dx, ddt, dB, dC
     bpt = 2 * (e * (2 * H * P + H + 2 * G * N) + 4 * (H * P + H + 2 * G * N))
-    peaks = measured_peaks()
-    achieved = bpt * plan["tokens"] / (ms / 1e3) / 1e9
+    # float32 multiply-adds of the chunked gradient per token, head and direction: chunk state and
+    # adjoint sums 2PN; pair matrices C.B^T and x.gy^T Q(N + P); the adjoint times B, entering
+    # part PN and causal in-chunk part QP/2; dB and dC, entering parts 2PN and causal in-chunk
+    # parts 2 QN/2
+    macs = 5 * P * N + 2 * Q * N + 1.5 * Q * P
+    fpt = 2 * 2 * H * macs                       # flops per token, both directions
+    clocks = clk.summary()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    mhz = clocks.get("sm_max_mhz") or 1965
+    peak_tf = sms * 128 * 2 * mhz * 1e6 / 1e12   # float32 FMA lanes per SM, 2 flops each
+    achieved = fpt * plan["tokens"] / (ms / 1e3) / 1e12
     line = {"metric": "bidirectional SSD scan gradients tokens/s (both directions)", "op": "bwd",
             "value": plan["tokens"] / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "f32",
             "data": "synthetic", "config": {"workload": args.workload, "global_batch": shape.batch,
                                              "seq_len": shape.seqlen, "chunk": chunk, "path": "simt"},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "bytes_per_token": bpt},
-            "gpu_launches": 2 * 5 * args.steps, "clocks": clk.summary()}
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": achieved / peak_tf, "flops_per_token": fpt,
+                         "peak_source": f"derived: {sms} SMs x 128 float32 lanes x 2 flops x {mhz} MHz",
+                         "hbm_bytes_per_token": bpt,
+                         "hbm_gbs": bpt * plan["tokens"] / (ms / 1e3) / 1e9},
+            "gpu_launches": 2 * 5 * args.steps, "clocks": clocks}
     print(json.dumps(line), flush=True)
 
 
