@@ -223,52 +223,58 @@ __global__ void __launch_bounds__(kT) k_bwd_chunk_sums(BwdArgs a) {
 
 // Step 2: state entering each chunk (forward pass over chunks) and adjoint entering each chunk
 // from the right (reverse pass), both in place.  A (batch, head) pair's P x N entries are split
-// over gridDim.z CTAs of kPassE entries per thread.  The values of kPassU chunks are loaded
-// before any of them is overwritten, so that their loads are in flight together; the chain of
-// multiply-adds then runs on registers.
-constexpr int kPassE = 2;
-constexpr int kPassU = 8;
+// over gridDim.z CTAs; a thread owns four neighbouring entries.  The dependent chain over the
+// chunks reads its inputs from a ring of kRing chunks in shared memory that asynchronous copies
+// fill ahead of it, so that kRing - 1 chunks' loads are always in flight.
+constexpr int kPassE = 4;
+constexpr int kRing = 12;      // 12 chunks x 256 threads x 16 B = 48 KB of static shared memory
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory"); }
+
 template <int P, int N>
 __global__ void __launch_bounds__(kT) k_bwd_pass(BwdArgs a) {
+    __shared__ __align__(16) float4 ring[kRing][kT];
     const int h = blockIdx.x, b = blockIdx.y;
-    const int e0 = blockIdx.z * kT * kPassE + threadIdx.x;
-    const size_t base = ((size_t)b * a.H + h) * a.nc;
+    const int e = kPassE * (blockIdx.z * kT + threadIdx.x);
+    const size_t dbase = ((size_t)b * a.H + h) * a.nc;
     for (int dirn = 0; dirn < 2; ++dirn) {
         // dirn 0: states S (a.sf), chunks in increasing order; dirn 1: adjoints (a.sg), decreasing
         float *arr = dirn == 0 ? a.sf : a.sg;
-        float run[kPassE];
+        auto chunk_of = [&](int i) { return dirn == 0 ? i : a.nc - 1 - i; };
+        // one commit group per chunk index (empty past the last chunk), into ring slot i % kRing
+        auto issue = [&](int i, int slot) {
+            if (i < a.nc) cp_async16(&ring[slot][threadIdx.x], arr + chunk_slot(a, b, h, chunk_of(i), P * N) + e);
+            cp_async_commit();
+        };
 #pragma unroll
-        for (int j = 0; j < kPassE; ++j) run[j] = 0.f;
-        for (int c0 = 0; c0 < a.nc; c0 += kPassU) {
-            float v[kPassU][kPassE], dc[kPassU];
+        for (int u = 0; u < kRing - 1; ++u) issue(u, u);
+        float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i0 = 0; i0 < a.nc; i0 += kRing) {
+            float dcb[kRing];
 #pragma unroll
-            for (int u = 0; u < kPassU; ++u) {
-                const int i = c0 + u;
-                const int c = dirn == 0 ? i : a.nc - 1 - i;
-                dc[u] = 0.f;
+            for (int u = 0; u < kRing; ++u) dcb[u] = i0 + u < a.nc ? a.dec[dbase + chunk_of(i0 + u)] : 0.f;
 #pragma unroll
-                for (int j = 0; j < kPassE; ++j) v[u][j] = 0.f;
-                if (i < a.nc) {
-                    const float *S = arr + chunk_slot(a, b, h, c, P * N);
-                    dc[u] = a.dec[base + c];
-#pragma unroll
-                    for (int j = 0; j < kPassE; ++j) v[u][j] = S[e0 + kT * j];
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kPassU; ++u) {
-                const int i = c0 + u;
-                if (i < a.nc) {
-                    const int c = dirn == 0 ? i : a.nc - 1 - i;
-                    float *S = arr + chunk_slot(a, b, h, c, P * N);
-#pragma unroll
-                    for (int j = 0; j < kPassE; ++j) {
-                        S[e0 + kT * j] = run[j];
-                        run[j] = fmaf(dc[u], run[j], v[u][j]);
-                    }
-                }
+            for (int u = 0; u < kRing; ++u) {
+                const int i = i0 + u;
+                if (i >= a.nc) break;
+                issue(i + kRing - 1, (u + kRing - 1) % kRing);
+                cp_async_wait<kRing - 1>();              // chunk i has landed in slot u
+                const float4 v = ring[u][threadIdx.x];
+                *reinterpret_cast<float4 *>(arr + chunk_slot(a, b, h, chunk_of(i), P * N) + e) = r;
+                r.x = fmaf(dcb[u], r.x, v.x);
+                r.y = fmaf(dcb[u], r.y, v.y);
+                r.z = fmaf(dcb[u], r.z, v.z);
+                r.w = fmaf(dcb[u], r.w, v.w);
             }
         }
+        cp_async_wait<0>();                              // the ring is reused by the next pass
     }
 }
 
