@@ -45,6 +45,20 @@ def test_library_exports_every_declared_symbol():
     assert set(names) <= exported
 
 
+def test_tracing_code_only_in_the_tracing_build():
+    """The product library exports no trace readers; the tracing build exports them and every ABI symbol."""
+    out = subprocess.run(["nm", "-D", "--defined-only", ssd.library_path], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert not {"ssd_debug_trace", "ssd_debug_cta_times"} & exported
+    trace_path = os.path.join(os.path.dirname(ssd.library_path), "libbidirssd_trace.so")
+    if not os.path.exists(trace_path):
+        pytest.skip("tracing build not compiled")
+    out = subprocess.run(["nm", "-D", "--defined-only", trace_path], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert {"ssd_debug_trace", "ssd_debug_cta_times"} <= exported
+    assert set(_declared_functions()) <= exported
+
+
 def _shape(b=1, L=64, H=2, P=16, N=16, G=1, io=1):
     return ssd._Shape(b, L, H, P, N, G, io)
 

@@ -1,0 +1,39 @@
+"""The tracing build of the tensor-core kernel (phase_trace.py).
+
+Its output must equal the product library's bit for bit.  Its per-phase
+stamps must come in program order: within a block, the MMA warp issues G,
+Y_off, the state product and Y_diag in that order, and each CUDA-core warp
+passes its phase boundaries in order.  Every CTA must have recorded a start
+before its end.
+"""
+import pytest
+import torch
+
+import ssd_inputs as si
+
+pytestmark = pytest.mark.gpu
+
+
+def test_trace_build_matches_product_and_orders_phases():
+    import bidirectional_mamba_ssd_bidir_b200 as ssd
+    from bidirectional_mamba_ssd_bidir_b200 import phase_trace as pt
+
+    shape = si.Shape(2, 2048, 8, 64, 128, 1, "bf16")        # 16 blocks per sequence, 16 CTAs
+    pf, pr = si.make_bidir(shape, seed=3)
+    dev = lambda p: {k: getattr(p, k).torch("cuda") for k in ("x", "dt", "A", "B", "C", "D")}
+    f, r = dev(pf), dev(pr)
+    y_ref = ssd.bidir_ssd(f, r, chunk=256)
+    y, ph, ctas = pt.run(f, r, chunk=256)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_ref)
+    order = [k for k, _ in pt.COMPUTE_POINTS]
+    for j in range(1, pt.N_BLOCKS):
+        m = ph[pt.WARP_MMA, j, :4]                           # G, Y_off, state, Y_diag
+        assert m[0] <= m[1] <= m[2] <= m[3], (j, m)
+        assert ph[pt.WARP_MMA, j, 0] > ph[pt.WARP_MMA, j - 1, 3]
+        for w in range(16):
+            seq = [ph[w, j, k] for k in order]
+            assert all(a <= b for a, b in zip(seq, seq[1:])), (j, w, seq)
+    assert len(ctas) == 2 * shape.batch * shape.nheads // 2
+    assert (ctas[:, 1] > ctas[:, 0]).all()
+    assert "block 3: period" in pt.summary(ph)
