@@ -242,7 +242,7 @@ def run_ours(args) -> None:
     rev = {k: devt["r" + k] for k in ("x", "dt", "A", "B", "C", "D")}
     y = torch.empty_like(fwd["x"])
     dims = (shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate, shape.ngroups)
-    ws = torch.empty(max(256, ssd.workspace_bytes(dims, fwd["x"].dtype, chunk)), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(max(256, ssd.workspace_bytes(dims, fwd["x"].dtype, chunk)), dtype=torch.uint8, device=dev)
     path = ssd.path_for(dims, fwd["x"].dtype, chunk)
     launches_per_step = ssd.kernel_launches(dims, fwd["x"].dtype, chunk, "bidir")
     stream = torch.cuda.current_stream(dev)
@@ -353,7 +353,7 @@ def run_bwd(args) -> None:
     gy = torch.randn(fwd["x"].shape, device=dev).to(fwd["x"].dtype)
     dims = (shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate, shape.ngroups)
     s_ = ssd._Shape(*dims, ssd.SSD_BF16 if shape.io == "bf16" else ssd.SSD_F32)
-    ws = torch.empty(int(ssd.lib.ssd_bwd_workspace_bytes(ssd.ctypes.byref(s_), chunk)), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(int(ssd.lib.ssd_bwd_workspace_bytes(ssd.ctypes.byref(s_), chunk)), dtype=torch.uint8, device=dev)
 
     def step():
         ssd.ssd_scan_bwd(**fwd, gy=gy, direction=1, chunk=chunk, workspace=ws)

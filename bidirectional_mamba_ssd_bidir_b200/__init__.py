@@ -162,7 +162,9 @@ def kernel_launches(shape: tuple, io: torch.dtype, chunk: int, op: str) -> int:
 def _workspace(shape: _Shape, chunk: int, dev, workspace):
     need = int(lib.ssd_workspace_bytes(ctypes.byref(shape), int(chunk)))
     if workspace is None:
+        # only the status word (the first 256 bytes) must start at zero
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        workspace[:256].zero_()
     return workspace, workspace.numel() * workspace.element_size()
 
 
@@ -214,6 +216,7 @@ def ssd_scan_bwd(x, dt, A, B, C, D, gy, direction: int = 1, chunk: int = 256, wo
     need = int(lib.ssd_bwd_workspace_bytes(ctypes.byref(shape), int(chunk)))
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        workspace[:256].zero_()
     ptr = lambda t: t.data_ptr() if t is not None else None
     _check(lib.ssd_scan_bwd(ctypes.byref(shape), ctypes.byref(prm), int(direction), int(chunk), gy.data_ptr(),
                             ptr(g["x"]), ptr(g["dt"]), ptr(g["A"]), ptr(g["B"]), ptr(g["C"]), ptr(g["D"]),

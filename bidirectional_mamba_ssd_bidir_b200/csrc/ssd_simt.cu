@@ -49,6 +49,13 @@ __device__ void chunk_cumsum(const ScanArgs &a, const T *dt, int b, int h, int c
     __syncthreads();
 }
 
+// Offset of the P x N state of (b, h, chunk c) in a.states.  The heads of one chunk are
+// neighbours, so the state pass, which walks all heads chunk by chunk, touches one contiguous
+// range at a time.
+__device__ __forceinline__ size_t state_slot(const ScanArgs &a, int b, int h, int c, int PN) {
+    return (((size_t)b * a.nc + c) * a.H + h) * (size_t)PN;
+}
+
 template <typename T, int P, int N>
 __global__ void __launch_bounds__(kThreads) k_chunk_state(ScanArgs a) {
     constexpr int E = P * N / kThreads;
@@ -95,35 +102,78 @@ __global__ void __launch_bounds__(kThreads) k_chunk_state(ScanArgs a) {
         }
         __syncthreads();
     }
-    float *S = a.states + (((size_t)b * a.H + h) * a.nc + c) * P * N;
+    float *S = a.states + state_slot(a, b, h, c, P * N);
 #pragma unroll
     for (int j = 0; j < E; ++j) S[threadIdx.x + kThreads * j] = acc[j];
     if (threadIdx.x == 0) a.decays[((size_t)b * a.H + h) * a.nc + c] = expf(cl);
 }
 
+// The sequential pass over chunks.  A (batch, head)'s P x N entries are split over gridDim.z
+// CTAs, kSE neighbouring entries per thread.  The dependent chain reads its inputs from a ring
+// of kSRing chunks in shared memory that asynchronous copies fill ahead of it, so that
+// kSRing - 1 chunks' loads are always in flight.
+constexpr int kSRing = 12;
+
+template <int E>
+__device__ __forceinline__ void cp_async_e(float *dst, const float *src) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    if constexpr (E == 4) {
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+    } else {
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(src) : "memory");
+    }
+}
+
+template <int P, int N>
+struct StatePassShape {
+    static constexpr int kE = (P * N >= 4 * kThreads) ? 4 : 1;   // entries per thread
+    static constexpr int kSlices = (P * N + kThreads * kE - 1) / (kThreads * kE);
+};
+
 template <int P, int N>
 __global__ void __launch_bounds__(kThreads) k_state_pass(ScanArgs a) {
-    constexpr int E = P * N / kThreads;
+    constexpr int E = StatePassShape<P, N>::kE;
+    __shared__ __align__(16) float ring[kSRing][kThreads * E];
     const int h = blockIdx.x, b = blockIdx.y;
-    float run[E];
+    const int e = E * (blockIdx.z * kThreads + threadIdx.x);   // this thread's first entry
+    const bool mine = e < P * N;
     const size_t sbase = ((size_t)b * a.H + h) * P * N;     // [b][h] slot of s_in / s_out
+    const size_t dbase = ((size_t)b * a.H + h) * a.nc;
+    float run[E];
 #pragma unroll
-    for (int j = 0; j < E; ++j) run[j] = a.s_in ? a.s_in[sbase + threadIdx.x + kThreads * j] : 0.f;
-    const size_t base = ((size_t)b * a.H + h) * a.nc;
-    for (int c = 0; c < a.nc; ++c) {
-        float *S = a.states + (base + c) * P * N;
-        const float dc = a.decays[base + c];
+    for (int j = 0; j < E; ++j) run[j] = (a.s_in && mine) ? a.s_in[sbase + e + j] : 0.f;
+    // one commit group per chunk (empty past the last chunk), into ring slot c % kSRing
+    auto issue = [&](int c, int slot) {
+        if (c < a.nc && mine) cp_async_e<E>(&ring[slot][threadIdx.x * E], a.states + state_slot(a, b, h, c, P * N) + e);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
 #pragma unroll
-        for (int j = 0; j < E; ++j) {
-            const int e = threadIdx.x + kThreads * j;
-            const float sc = S[e];
-            S[e] = run[j];                       // state entering chunk c
-            run[j] = fmaf(dc, run[j], sc);
+    for (int u = 0; u < kSRing - 1; ++u) issue(u, u);
+    for (int c0 = 0; c0 < a.nc; c0 += kSRing) {
+        float dcb[kSRing];
+#pragma unroll
+        for (int u = 0; u < kSRing; ++u) dcb[u] = c0 + u < a.nc ? a.decays[dbase + c0 + u] : 0.f;
+#pragma unroll
+        for (int u = 0; u < kSRing; ++u) {
+            const int c = c0 + u;
+            if (c >= a.nc) break;
+            issue(c + kSRing - 1, (u + kSRing - 1) % kSRing);
+            asm volatile("cp.async.wait_group %0;" ::"n"(kSRing - 1) : "memory");   // chunk c has landed
+            if (mine) {
+                float *S = a.states + state_slot(a, b, h, c, P * N) + e;
+#pragma unroll
+                for (int j = 0; j < E; ++j) {
+                    const float sc = ring[u][threadIdx.x * E + j];
+                    S[j] = run[j];                   // state entering chunk c
+                    run[j] = fmaf(dcb[u], run[j], sc);
+                }
+            }
         }
     }
-    if (a.s_out) {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    if (a.s_out && mine) {
 #pragma unroll
-        for (int j = 0; j < E; ++j) a.s_out[sbase + threadIdx.x + kThreads * j] = run[j];
+        for (int j = 0; j < E; ++j) a.s_out[sbase + e + j] = run[j];
     }
 }
 
@@ -147,7 +197,7 @@ __global__ void __launch_bounds__(kThreads) k_chunk_output(ScanArgs a, int have_
         Cs[i] = ldf<T>(Cm, (((size_t)b * a.L + t) * a.G + g) * N + n);
     }
     if (have_state) {
-        const float *S = a.states + (((size_t)b * a.H + h) * a.nc + c) * P * N;
+        const float *S = a.states + state_slot(a, b, h, c, P * N);
         for (int i = threadIdx.x; i < P * N; i += kThreads) Sin[(i / N) * NP + (i % N)] = S[i];
     }
     __syncthreads();
@@ -242,7 +292,7 @@ cudaError_t launch_typed(const ScanArgs &a, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         k_chunk_state<T, P, N><<<dim3(a.nc, a.H, a.batch), kThreads, sm_state, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        k_state_pass<P, N><<<dim3(a.H, a.batch), kThreads, 0, st>>>(a);
+        k_state_pass<P, N><<<dim3(a.H, a.batch, StatePassShape<P, N>::kSlices), kThreads, 0, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     e = cudaFuncSetAttribute(k_chunk_output<T, P, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_out);

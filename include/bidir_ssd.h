@@ -36,9 +36,11 @@
  * Workspace.  Some paths keep scratch data in global memory (chunk states,
  * direction hand-off flags, the device status word).  Query its size with
  * ssd_workspace_bytes() for the exact shape and chunk and pass a device
- * buffer of at least that size; its contents need no initialisation and are
- * not meaningful after the call.  Calls that share a workspace must not run
- * concurrently.
+ * buffer of at least that size.  Its first 256 bytes hold the status word:
+ * they must be zero before the workspace's first use.  Calls write them only
+ * to record a device-side timeout, and ssd_workspace_status() clears them.
+ * The rest needs no initialisation and is not meaningful after the call.
+ * Calls that share a workspace must not run concurrently.
  *
  * Errors.  Every entry point returns an ssd_status; no exception or abort
  * crosses the ABI.  Arguments are checked on the host before anything is

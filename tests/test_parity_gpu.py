@@ -263,3 +263,55 @@ def test_r2l_block_parity(ssd, chunk):
         torch.cuda.synchronize()
         ref2 = oracle.r2l_block_f64(oracle.params_f64(q), gate, np.zeros(zero.shape))
         assert oracle.rel_err(_f64(o2), ref2) <= TOL["bf16"]
+
+
+def test_homogeneous_in_x_bitwise_tensor_core(ssd):
+    """y is linear in x.  Doubling x doubles every bf16 operand and float32 partial sum exactly,
+    so on the tensor-core path y(2x) is 2 y(x) bit for bit, in both directions and for the sum."""
+    shape = si.Shape(2, 512, 8, 64, 128, 1, "bf16")
+    pf, pr = si.make_bidir(shape, seed=12)
+    df, dr = _dev(pf), _dev(pr)
+    df2, dr2 = dict(df, x=df["x"] * 2), dict(dr, x=dr["x"] * 2)
+    for d in (1, -1):
+        p, p2 = (df, df2) if d > 0 else (dr, dr2)
+        y, y2 = ssd.ssd_scan(**p, direction=d, chunk=256), ssd.ssd_scan(**p2, direction=d, chunk=256)
+        torch.cuda.synchronize()
+        assert torch.equal(y2, y * 2)
+    yb, yb2 = ssd.bidir_ssd(df, dr, chunk=256), ssd.bidir_ssd(df2, dr2, chunk=256)
+    torch.cuda.synchronize()
+    assert torch.equal(yb2, yb * 2)
+
+
+def test_additive_in_x_float32(ssd):
+    """y(a x1 + b x2) = a y(x1) + b y(x2) for fixed dt, A, B, C, D, on the float32 path."""
+    shape = si.Shape(1, 256, 4, 32, 64, 1, "f32")
+    p1 = _dev(si.make_params(shape, seed=13))
+    x2 = _dev(si.make_params(shape, seed=14))["x"]
+    a, b = 0.75, -1.5
+    for d in (1, -1):
+        y1 = ssd.ssd_scan(**p1, direction=d, chunk=64)
+        y2 = ssd.ssd_scan(**dict(p1, x=x2), direction=d, chunk=64)
+        y3 = ssd.ssd_scan(**dict(p1, x=a * p1["x"] + b * x2), direction=d, chunk=64)
+        torch.cuda.synchronize()
+        ref = a * y1.double() + b * y2.double()
+        assert torch.max(torch.abs(y3.double() - ref)).item() <= 1e-5 * torch.max(torch.abs(ref)).item()
+
+
+@pytest.mark.parametrize("dims,chunk", [((2, 1024, 8, 64, 128, 1), 256), ((1, 256, 4, 32, 64, 1), 64)])
+def test_workspace_needs_only_its_status_word_zeroed(ssd, dims, chunk):
+    """Apart from the status word (first 256 bytes), a workspace may hold anything before a call:
+    the hand-off flags are epoch-tagged and the chunk states are written before they are read."""
+    shape = si.Shape(*dims, "bf16")
+    pf, pr = si.make_bidir(shape, seed=15)
+    df, dr = _dev(pf), _dev(pr)
+    n = ssd.workspace_bytes(dims, torch.bfloat16, chunk)
+    clean = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    y_ref = ssd.bidir_ssd(df, dr, chunk=chunk, workspace=clean)
+    for fill in (0xFF, 0xA5):
+        ws = torch.full((n,), fill, dtype=torch.uint8, device="cuda")
+        ws[:256] = 0
+        for _ in range(2):
+            y = ssd.bidir_ssd(df, dr, chunk=chunk, workspace=ws)
+            torch.cuda.synchronize()
+            ssd.workspace_status(ws)
+            assert torch.equal(y, y_ref)
