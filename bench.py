@@ -1,6 +1,7 @@
 """Benchmark: bidirectional SSD scan throughput (tokens/s) at the DiffuMamba ~1.3B layer shape.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+                    [--op fwd|bwd] [--batch B]
 
 One step is one full bidirectional scan call (forward + reverse + sum) over a
 batch of synthetic seeded inputs already resident in HBM.  The default
@@ -20,6 +21,9 @@ The JSON line carries, besides the contract keys:
                 inside the timed region
   clocks        SM clocks and throttle reasons sampled during the timed region
 ``--impl reference`` times the oracle alone (the CPU reference arm).
+``--op bwd`` times the gradients of both directions (its own JSON line, with
+a roofline against the float32 ALU peak).  ``--batch`` replaces the batch
+size, for small ncu captures.
 """
 from __future__ import annotations
 
