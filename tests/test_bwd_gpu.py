@@ -77,3 +77,37 @@ def test_bidirectional_gradient_is_the_sum_of_directions(ssd):
     rr = oracle.ssd_scan_bwd_f64(q["x"], q["dt"], q["A"], q["B"], q["C"], q["D"], -1, g64)
     got = (gf["x"] + gr["x"]).double().cpu().numpy()
     assert oracle.rel_err(got, rf["x"] + rr["x"]) <= TOL["bf16"]
+
+
+def test_empty_inputs_give_zero_parameter_gradients(ssd):
+    """No token: dA and dD are zero (dx, ddt, dB, dC are empty)."""
+    for b, L in ((0, 256), (2, 0)):
+        x = torch.empty(b, L, 4, 64, dtype=torch.bfloat16, device="cuda")
+        dt = torch.empty(b, L, 4, dtype=torch.bfloat16, device="cuda")
+        B = torch.empty(b, L, 1, 128, dtype=torch.bfloat16, device="cuda")
+        A = -torch.ones(4, device="cuda")
+        D = torch.ones(4, device="cuda")
+        g = ssd.ssd_scan_bwd(x, dt, A, B, B, D, torch.empty_like(x), direction=1, chunk=256)
+        torch.cuda.synchronize()
+        assert torch.equal(g["A"], torch.zeros(4, device="cuda"))
+        assert torch.equal(g["D"], torch.zeros(4, device="cuda"))
+        assert g["x"].numel() == 0 and g["B"].numel() == 0
+
+
+def test_gradients_at_the_bench_layer_shape(ssd):
+    """The 1.3B layer shape at L = 8192 (one sequence of the bench workload), forward direction,
+    every gradient against the oracle's adjoint over the whole sequence (about half a minute of
+    single-threaded oracle; the reverse direction is covered at smaller sizes)."""
+    direction = 1
+    shape = si.Shape(1, 8192, 64, 64, 128, 1, "bf16")
+    p = si.make_params(shape, seed=43)
+    d = {k: getattr(p, k).torch("cuda") for k in ("x", "dt", "A", "B", "C", "D")}
+    gy = torch.randn(d["x"].shape, device="cuda", generator=torch.Generator("cuda").manual_seed(5)).to(torch.bfloat16)
+    g = ssd.ssd_scan_bwd(**d, gy=gy, direction=direction, chunk=256)
+    torch.cuda.synchronize()
+    q = oracle.params_f64(p)
+    ref = oracle.ssd_scan_bwd_f64(q["x"], q["dt"], q["A"], q["B"], q["C"], q["D"], direction,
+                                  gy.double().cpu().numpy())
+    for name in ("x", "dt", "A", "B", "C", "D"):
+        err = oracle.rel_err(g[name].double().cpu().numpy(), ref[name])
+        assert err <= TOL["bf16"], (name, err)
