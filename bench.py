@@ -140,11 +140,17 @@ def measured_peaks() -> dict:
 
 
 def _kernel_source_hash() -> str:
-    """Hash of the tensor-core kernel's sources: a traffic record is valid only for the kernel it measured."""
+    """Hash of the tensor-core kernel's sources: a traffic record is valid only for the kernel it measured.
+
+    Comments and whitespace are left out, so that editing a comment keeps the record of an
+    unchanged kernel."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bidirectional_mamba_ssd_bidir_b200", "csrc")
     for f in ("ssd_tc.cu", "ssd_tc.cuh"):
-        h.update(open(os.path.join(csrc, f), "rb").read())
+        text = open(os.path.join(csrc, f), encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

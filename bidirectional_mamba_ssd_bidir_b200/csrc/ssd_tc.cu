@@ -125,8 +125,9 @@ enum Bar {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Optional phase timeline for profiling builds (-DSSD_TRACE): %globaltimer
-// stamps of CTA 0, first kTraceBlocks blocks, per warp and phase.
+// Optional phase timeline for the tracing build (-DSSD_TRACE): SM-clock stamps
+// of CTA 0, first kTraceBlocks blocks, per warp and phase; and every CTA's
+// start and end on the global timer, with its SM.
 #ifdef SSD_TRACE
 constexpr int kTraceWarps = 20, kTraceBlocks = 8, kTracePts = 24;
 __device__ unsigned long long g_trace[kTraceWarps][kTraceBlocks][kTracePts];
