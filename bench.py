@@ -147,11 +147,15 @@ def _kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bidirectional_mamba_ssd_bidir_b200", "csrc")
     for f in ("ssd_tc.cu", "ssd_tc.cuh"):
-        text = open(os.path.join(csrc, f), encoding="utf-8").read()
-        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
-        text = re.sub(r"//[^\n]*", " ", text)
-        h.update(" ".join(text.split()).encode())
+        h.update(_code_only(open(os.path.join(csrc, f), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
+
+
+def _code_only(text: str) -> str:
+    """C/CUDA source without its comments, whitespace runs collapsed to one space."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
 
 
 def profiled_traffic(kernel: str, workload: str):

@@ -70,3 +70,15 @@ def test_algorithmic_bytes_per_token():
     shape = si.WORKLOADS[bench.DEFAULT_WORKLOAD]["shape"]
     # per direction: x 64*64*2 + dt 64*2 + B,C 2*128*2; y 64*64*2 written once
     assert bench.algorithmic_bytes_per_token(shape) == 2 * (8192 + 128 + 512) + 8192 == 25856
+
+
+def test_traffic_record_survives_comment_edits_only():
+    """The ncu traffic record is keyed on the kernel's code: comments and layout do not change
+    the key, any code change does."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    src = "int f(int a) { // doubles\n  return 2 * a; /* the\n  result */ }\n"
+    assert bench._code_only(src) == bench._code_only("int f(int a) {\n\n    return 2 * a;   }  // other words")
+    assert bench._code_only(src) != bench._code_only(src.replace("2 * a", "3 * a"))
+    assert bench.profiled_traffic("ssd_bidir_tc", "diffumamba_1p3b_L8192") is not None
