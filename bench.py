@@ -140,14 +140,20 @@ def measured_peaks() -> dict:
 
 
 def _kernel_source_hash() -> str:
-    """Hash of the tensor-core kernel's sources: a traffic record is valid only for the kernel it measured.
+    """Hash of the tensor-core kernels' sources and build flags: a traffic record is valid only for
+    the kernel it measured.
 
     Comments and whitespace are left out, so that editing a comment keeps the record of an
-    unchanged kernel."""
+    unchanged kernel; the nvcc architecture and flags are part of the key."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "bidirectional_mamba_ssd_bidir_b200", "csrc")
-    for f in ("ssd_tc.cu", "ssd_tc.cuh"):
-        h.update(_code_only(open(os.path.join(csrc, f), encoding="utf-8").read()).encode())
+    pkg = os.path.join(ROOT, "bidirectional_mamba_ssd_bidir_b200")
+    for f in ("ssd_tcs.cu", "ssd_tc.cu", "ssd_tc.cuh", "ssd_tc_common.cuh"):
+        h.update(_code_only(open(os.path.join(pkg, "csrc", f), encoding="utf-8").read()).encode())
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_ssd_build_flags", os.path.join(pkg, "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    h.update(" ".join(mod.ARCH + mod.FLAGS).encode())
     return h.hexdigest()[:16]
 
 
@@ -158,9 +164,9 @@ def _code_only(text: str) -> str:
     return " ".join(text.split())
 
 
-def profiled_traffic(kernel: str, workload: str):
+def profiled_traffic(kernel: str, workload: str, prof: str | None = None):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on the current kernel source."""
-    prof = os.path.join(ROOT, "profiles")
+    prof = prof or os.path.join(ROOT, "profiles")
     if not os.path.isdir(prof):
         return None
     src_hash = _kernel_source_hash()

@@ -24,7 +24,7 @@ import os
 
 import torch
 
-__all__ = ["ssd_scan", "ssd_scan_state", "ssd_scan_bwd", "bidir_ssd", "r2l_block_scan", "bidir_ssd_noalloc", "noalloc_status", "workspace_bytes", "path_for",
+__all__ = ["ssd_scan", "ssd_scan_state", "ssd_scan_bwd", "bidir_ssd", "r2l_block_scan", "bidir_ssd_noalloc", "noalloc_status", "NoallocArea", "workspace_bytes", "path_for",
            "kernel_launches", "workspace_status", "SSDError", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -258,7 +258,16 @@ def workspace_status(workspace) -> None:
     _check(lib.ssd_workspace_status(workspace.data_ptr(), workspace.numel(), _stream(dev)))
 
 
-def bidir_ssd_noalloc(fwd: dict, rev: dict, out, chunk: int = 256) -> int:
+class NoallocArea(int):
+    """Device address of the no-allocation scratch's status area, with the device the call ran on."""
+
+    def __new__(cls, address: int, device: int):
+        obj = super().__new__(cls, address)
+        obj.device = device
+        return obj
+
+
+def bidir_ssd_noalloc(fwd: dict, rev: dict, out, chunk: int = 256) -> NoallocArea:
     """``bidir_ssd`` for callers that cannot allocate device memory at the call.
 
     Writes y into ``out`` (preallocated, contiguous, shaped like ``fwd["x"]``).
@@ -266,8 +275,8 @@ def bidir_ssd_noalloc(fwd: dict, rev: dict, out, chunk: int = 256) -> int:
     neither this function nor the library allocates anything; shapes whose
     scratch exceeds that array raise SSDError (unsupported shape).  Calls
     that overlap on the GPU share the array and race: order them on one
-    stream.  Returns the device address of the scratch's status area, for
-    ``noalloc_status``.
+    stream.  Returns the device address of the scratch's status area (with the
+    device it lives on), for ``noalloc_status``.
     """
     shape = _shape_of(fwd["x"], fwd["B"])
     if tuple(rev["x"].shape) != tuple(fwd["x"].shape) or tuple(rev["B"].shape) != tuple(fwd["B"].shape):
@@ -278,12 +287,18 @@ def bidir_ssd_noalloc(fwd: dict, rev: dict, out, chunk: int = 256) -> int:
     pf = _params(x, fwd["dt"], fwd["A"], fwd["B"], fwd["C"], fwd.get("D"))
     pr = _params(rev["x"], rev["dt"], rev["A"], rev["B"], rev["C"], rev.get("D"))
     area = ctypes.c_void_p()
-    _check(lib.bidir_ssd_noalloc(ctypes.byref(shape), ctypes.byref(pf), ctypes.byref(pr), int(chunk),
-                                 out.data_ptr(), _stream(x.device), ctypes.byref(area)))
-    return int(area.value or 0)
+    dev = x.device.index if x.device.index is not None else torch.cuda.current_device()
+    with torch.cuda.device(dev):
+        _check(lib.bidir_ssd_noalloc(ctypes.byref(shape), ctypes.byref(pf), ctypes.byref(pr), int(chunk),
+                                     out.data_ptr(), _stream(x.device), ctypes.byref(area)))
+    return NoallocArea(int(area.value or 0), dev)
 
 
-def noalloc_status(area: int, device=None) -> None:
-    """Raise SSDError if a bounded device-side wait gave up in the last ``bidir_ssd_noalloc`` call."""
+def noalloc_status(area: NoallocArea) -> None:
+    """Raise SSDError if a bounded device-side wait gave up in the ``bidir_ssd_noalloc`` call that
+    returned ``area`` (read on that call's device, whatever device is current now)."""
+    if not isinstance(area, NoallocArea):
+        raise TypeError("pass the value bidir_ssd_noalloc returned (it carries the device of the call)")
     if area:
-        _check(lib.ssd_workspace_status(area, 256, _stream(device or torch.cuda.current_device())))
+        with torch.cuda.device(area.device):
+            _check(lib.ssd_workspace_status(int(area), 256, _stream(torch.device("cuda", area.device))))

@@ -386,21 +386,16 @@ namespace {
 // cleared again at every call.
 __device__ __align__(256) unsigned char g_noalloc_scratch[SSD_NOALLOC_MAX_SCRATCH_BYTES];
 
-// Its device address, per device, looked up by the first call on that device.
-std::atomic<void *> g_noalloc_ptr[64];
-
+// Its device address in the current device's context.  Looked up on every call
+// (cudaGetSymbolAddress allocates nothing): a cached address would go stale if
+// the context were destroyed (cudaDeviceReset) and the library's module loaded
+// again at another address, or if the caller switched to another context on the
+// same device.  A host-side reference to the array itself is never a device address.
 ssd_status noalloc_scratch(void **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-    if (dev < 0 || dev >= 64) return fail(SSD_ERR_UNSUPPORTED, "device ordinal %d above 63", dev);
-    void *ptr = g_noalloc_ptr[dev].load(std::memory_order_acquire);
-    if (!ptr) {
-        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the scratch array");
-        if (!ptr) return fail(SSD_ERR_CUDA, "cudaGetSymbolAddress returned NULL");
-        g_noalloc_ptr[dev].store(ptr, std::memory_order_release);
-    }
+    void *ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the scratch array");
+    if (!ptr) return fail(SSD_ERR_CUDA, "cudaGetSymbolAddress returned NULL");
     *out = ptr;
     return SSD_OK;
 }

@@ -66,6 +66,7 @@
 #include <mutex>
 
 #include "ssd_tc.cuh"
+#include "ssd_tc_common.cuh"
 
 namespace ssd {
 namespace {
@@ -107,8 +108,8 @@ constexpr uint32_t kOffTab = kOffSP + 2 * kTileBytes;   // 2 buffers
 constexpr uint32_t kOffDT = (kOffTab + 2 * kTabFloats * 4 + 127) / 128 * 128;   // dt ring, 2 slots
 constexpr uint32_t kOffBar = kOffDT + 2 * kDtBytes;
 constexpr uint32_t kNumBars = 25;
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
-constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag, wait limit, steep flag
+constexpr uint32_t kSmemBytes = kOffMisc + 32 + 1024;  // + alignment slack
 static_assert(kStageBytes % 1024 == 0, "x tiles must stay 1024-byte aligned");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
@@ -125,37 +126,10 @@ enum Bar {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Optional phase timeline for the tracing build (-DSSD_TRACE): SM-clock stamps
-// of CTA 0, first kTraceBlocks blocks, per warp and phase; and every CTA's
-// start and end on the global timer, with its SM.
-#ifdef SSD_TRACE
-constexpr int kTraceWarps = 20, kTraceBlocks = 8, kTracePts = 24;
-__device__ unsigned long long g_trace[kTraceWarps][kTraceBlocks][kTracePts];
-__device__ __forceinline__ void trace_pt(int w, int j, int k) {
-    if (blockIdx.x == 0 && j < kTraceBlocks && (threadIdx.x & 31) == 0) {
-        g_trace[w][j][k] = (unsigned long long)clock64();   // SM cycles: exact within the CTA
-    }
-}
-#define SSD_TRACE_PT(w, j, k) trace_pt(w, j, k)
-__device__ unsigned long long g_cta_time[4096][3];     // start, end, SM id
-#define SSD_TRACE_CTA(k)                                                              \
-    do {                                                                              \
-        if (threadIdx.x == 0 && blockIdx.x < 4096) {                                  \
-            unsigned long long t_;                                                    \
-            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                    \
-            g_cta_time[blockIdx.x][k] = t_;                                           \
-            unsigned smid_;                                                           \
-            asm volatile("mov.u32 %0, %%smid;" : "=r"(smid_));                        \
-            g_cta_time[blockIdx.x][2] = smid_;                                        \
-        }                                                                             \
-    } while (0)
-#else
-#define SSD_TRACE_CTA(k) ((void)0)
-#define SSD_TRACE_PT(w, j, k) ((void)0)
-#endif
 
 struct TcDirParams {
     const float *A, *D;
+    const __nv_bfloat16 *dt;
 };
 
 struct TcParams {
@@ -172,250 +146,14 @@ struct TcParams {
     int fault;                          // test hook: 1 = the first direction never publishes its part
     const float *s_in;                  // single direction: [batch][H][P][N] state entering the scan, or null
     float *s_out;                       // single direction: [batch][H][P][N] state leaving the scan, or null
+    // Non-null: run only the chains the shared-score kernel left to this one.  A CTA then
+    // returns at once unless *deferred == epoch and its own chain fails the same steep test.
+    const unsigned long long *deferred;
 };
 
 struct TcMaps {
     CUtensorMap x[2], dt[2], b[2], c[2], y;
 };
-
-// ------------------------------------------------------------------ PTX helpers
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-#ifdef SSD_EXP_TESTWAIT
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-#else
-    // the suspend-time hint lets a waiting warp sleep until the phase completes (or 1 us passes)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(1000u)
-        : "memory");
-#endif
-    return ok != 0;
-}
-
-// Slow path of mbar_wait: polls until the phase completes, the CTA aborts or
-// the time limit passes (then raises the abort flag and the status word).
-__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *status,
-                                            int code) {
-    const long long t0 = clock64();
-    const long long limit = *reinterpret_cast<volatile long long *>(abort_flag + 1);
-    while (true) {
-        if (mbar_try(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (clock64() - t0 > limit) {
-            *abort_flag = 1;
-            atomicExch(status, code);
-            return false;
-        }
-    }
-}
-
-// Bounded wait on phase `parity` by the lanes in `mask` (all of them call it).
-// Returns false if the phase did not complete in time or the CTA aborted; the
-// result is the same for every lane in `mask`.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t mask, volatile int *abort_flag,
-                                          int *status, int code) {
-    bool ok = mbar_try(bar, parity);
-    if (__all_sync(mask, ok)) return true;
-    if (!ok) ok = mbar_wait_slow(bar, parity, abort_flag, status, code);
-    return __all_sync(mask, ok);
-}
-
-// Bounded wait that ignores the abort flag: used on the way out to let
-// copies already in flight land before the CTA releases its shared memory.
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, long long limit) {
-    const long long t0 = clock64();
-    while (!mbar_try(bar, parity) && clock64() - t0 < limit) {
-    }
-}
-
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
-        : "memory");
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 "version 1").
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-    return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// Instruction descriptor: f32 accumulate, bf16 A and B, M = 128.
-__host__ __device__ constexpr uint32_t idesc(int n, int a_mn_major, int b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
-           ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-        "l"(a), "l"(b), "r"(id), "r"(acc));
-}
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t id, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-        "r"(a_tmem), "l"(b), "r"(id), "r"(acc));
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-// TMEM loads complete asynchronously: the wait is part of the same asm statement,
-// so no instruction that uses the loaded registers can be scheduled before it.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr)
-        : "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-// TMEM stores: the wait is part of the asm, so the source registers are not reused while
-// the store may still read them and later TMEM reads of these columns see the new values.
-// store without waiting: the caller issues tmem_wait_st() before the data is consumed
-__device__ __forceinline__ void tmem_st16_nw(uint32_t taddr, const uint32_t *r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-            taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_st16f_nw(uint32_t taddr, const float *v) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-            taddr),
-        "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]),
-        "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15])
-        : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-// two 32-column loads, one wait
-__device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, float *va, float *vb) {
-    uint32_t a[32], b[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
-          "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]),
-          "=r"(a[16]), "=r"(a[17]), "=r"(a[18]), "=r"(a[19]), "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]),
-          "=r"(a[24]), "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31]),
-          "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]),
-          "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15]),
-          "=r"(b[16]), "=r"(b[17]), "=r"(b[18]), "=r"(b[19]), "=r"(b[20]), "=r"(b[21]), "=r"(b[22]), "=r"(b[23]),
-          "=r"(b[24]), "=r"(b[25]), "=r"(b[26]), "=r"(b[27]), "=r"(b[28]), "=r"(b[29]), "=r"(b[30]), "=r"(b[31])
-        : "r"(ta), "r"(tb)
-        : "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        va[i] = __uint_as_float(a[i]);
-        vb[i] = __uint_as_float(b[i]);
-    }
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // .x = lo (low 16 bits), .y = hi
-    return *reinterpret_cast<uint32_t *>(&v);
-}
-__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
-// 2^x by the PTX ex2.approx.ftz instruction (relative error about 2^-22; results below
-// 2^-126 flush to zero, far below what a bf16 output resolves)
-__device__ __forceinline__ float ex2_ftz(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-// (lo, hi) bf16 pair times a bf16 scalar, one packed multiply rounded to nearest even
-__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t v, uint32_t w2) {
-    uint32_t o;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(o) : "r"(v), "r"(w2));
-    return o;
-}
-__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
-
-// byte offset of 16-byte chunk q of row r in a [rows][64] bf16 tile with 128-byte swizzle
-__device__ __forceinline__ uint32_t swz(int r, int q) { return (uint32_t)(r * 128 + ((q ^ (r & 7)) << 4)); }
-
-
-// ------------------------------------------------------------------ global-memory hand-off helpers
-
-__device__ __forceinline__ void st_release(unsigned long long *p, unsigned long long v) {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ unsigned long long ld_acquire(const unsigned long long *p) {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int c0, int c1) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(src), "r"(c0), "r"(c1)
-                 : "memory");
-}
-__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, uint32_t src, int c0, int c1) {
-    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(src), "r"(c0), "r"(c1)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ------------------------------------------------------------------ the kernel
 
@@ -443,6 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
     const CUtensorMap *map_x = &maps.x[slot], *map_dt = &maps.dt[slot], *map_b = &maps.b[slot],
                       *map_c = &maps.c[slot];
 
+    if (prm.deferred != nullptr) {
+        if (*reinterpret_cast<const volatile unsigned long long *>(prm.deferred) != prm.epoch) return;
+        if (!chain_is_steep(prm.d[slot].dt, prm.d[slot].A, b, L, prm.H, h0, threadIdx.x, kThreads,
+                            reinterpret_cast<int *>(sm + kOffMisc + 16)))
+            return;
+    }
+
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         *reinterpret_cast<volatile long long *>(abort_flag + 1) = prm.wait_cycles;
@@ -464,7 +209,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    SSD_TRACE_CTA(0);
 
     if (warp == kWarpTma) {
         // ---------------------------------------------------------- TMA producer
@@ -493,7 +237,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 const int row = b * L + cm * kBlk;
                 const int st = j & 1;
                 if (j >= 2 && !mbar_wait(bar(B_XEMPTY0 + st), ((j >> 1) - 1) & 1, MASK, abort_flag, prm.status, 11)) break;
-                SSD_TRACE_PT(kWarpTma, j, 0);
                 const uint32_t stage = sbase + kOffX + st * kStageBytes;
                 mbar_expect_tx(bar(B_XFULL0 + st), kStageBytes);
                 for (int h = 0; h < 2; ++h)
@@ -501,7 +244,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 x_issued = j + 1;
                 if (j + 1 < nblk && !load_dt(j + 1)) break;
                 if (j >= 1 && !mbar_wait(bar(B_BCEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 12)) break;
-                SSD_TRACE_PT(kWarpTma, j, 1);
                 mbar_expect_tx(bar(B_BCFULL), 4 * kTileBytes);
                 for (int q = 0; q < 2; ++q) {
                     tma_load_2d(sbase + kOffB + q * kTileBytes, map_b, q * 64, row, bar(B_BCFULL));
@@ -533,7 +275,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 if (!mbar_wait(bar(B_BCFULL), j & 1, MASK, abort_flag, prm.status, 21)) break;
                 // the previous block's M (read by its intra-block MMA) occupies the G columns
                 if (j >= 1 && !mbar_wait(bar(B_YFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 22)) break;
-                SSD_TRACE_PT(kWarpMma, j, 0);
                 tc_fence_after();
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = (ks >> 2) * kTileBytes + (ks & 3) * 32;
@@ -546,7 +287,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                     if (!mbar_wait(bar(B_SPREADY), (j - 1 + has_in) & 1, MASK, abort_flag, prm.status, 23)) break;
                     // the previous block's epilogue has read both Y accumulators
                     if (j >= 1 && !mbar_wait(bar(B_YEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 24)) break;
-                    SSD_TRACE_PT(kWarpMma, j, 1);
                     tc_fence_after();
                     for (int ks = 0; ks < 8; ++ks) {
                         const uint32_t offc = (ks >> 2) * kTileBytes + (ks & 3) * 32;
@@ -556,7 +296,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 }
                 // S'^T (+)= B^T (w x)  (M = n, N = (head, p), K = rows); both operands MN-major
                 if (!mbar_wait(bar(B_WXREADY), j & 1, MASK, abort_flag, prm.status, 25)) break;
-                SSD_TRACE_PT(kWarpMma, j, 2);
                 tc_fence_after();
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t off = ks * 2048;
@@ -569,7 +308,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 // the D x the CUDA-core warps stored there in their w.x pass
                 if (!mbar_wait(bar(B_MREADY), j & 1, MASK, abort_flag, prm.status, 27)) break;
                 if (!mbar_wait(bar(B_XFULL0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 29)) break;
-                SSD_TRACE_PT(kWarpMma, j, 3);
                 tc_fence_after();
                 for (int h = 0; h < 2; ++h) {
                     for (int ks = 0; ks < 8; ++ks)
@@ -842,16 +580,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
         const int jend = (nblk > 0 && make_tables(0)) ? nblk : 0;
         for (int j = 0; j < jend; ++j) {
             if (__any_sync(0xffffffffu, *abort_flag)) break;
-            SSD_TRACE_PT(warp, j, 0);
             const int st = j & 1;
             const float *tb = tab_s + st * kTabFloats;
             if (!wx_pass(j)) break;
-            SSD_TRACE_PT(warp, j, 8);
             if (j >= 1) {
                 if (!mbar_wait(bar(B_STFULL), (j - 1) & 1, MASK, abort_flag, prm.status, 43)) break;
-                SSD_TRACE_PT(warp, j, 6);
                 state_pass(j);
-                SSD_TRACE_PT(warp, j, 7);
             } else if (has_in) {
                 init_pass();
             }
@@ -860,7 +594,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             // warpgroup takes K-steps g and g + 4; the two heads' bf16 results for a K-step
             // replace the 16 float32 G columns they were computed from.
             if (!mbar_wait(bar(B_GFULL), j & 1, MASK, abort_flag, prm.status, 44)) break;
-            SSD_TRACE_PT(warp, j, 9);
             tc_fence_after();
             {
                 const float c2h[2] = {tb[kTabCS + r], tb[kTabCS + kBlk + r]};
@@ -948,17 +681,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_MREADY));
-            SSD_TRACE_PT(warp, j, 10);
 
             // next block's decay tables, while the tensor core computes this block's Y_diag
             if (j + 1 < nblk && !make_tables(j + 1)) break;
-            SSD_TRACE_PT(warp, j, 11);
 
             // epilogue: o = Y_diag (which started at D x) + exp(cs_r) Y_off, bf16, written over this row of the x
             // tile (free once the intra-block MMA is done); a store warp then writes the tile to y
             // in whole rows
             if (!mbar_wait(bar(hs == 0 ? B_YFULLH0 : B_YFULL), j & 1, MASK, abort_flag, prm.status, 46)) break;
-            SSD_TRACE_PT(warp, j, 16);
             tc_fence_after();
             {
                 uint8_t *xt = sm + kOffX + st * kStageBytes + hs * kTileBytes;
@@ -991,7 +721,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 mbar_arrive(bar(B_YEMPTY));
                 mbar_arrive(bar(B_TILE00 + 2 * hs + st));
             }
-            SSD_TRACE_PT(warp, j, 21);
             if (kState && j + 1 == nblk && prm.s_out) {
                 // state leaving the scan: S' after the last block's state MMA, row n = r
                 if (!mbar_wait(bar(B_STFULL), j & 1, MASK, abort_flag, prm.status, 49)) break;
@@ -1009,7 +738,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
 
     tc_fence_before();
     __syncthreads();
-    SSD_TRACE_CTA(1);
     if (warp == kWarpMma) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
@@ -1017,36 +745,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
 }
 
 // ------------------------------------------------------------------ host side
-
-using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled get_encode() {
-    static EncodeTiled fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiled>(p);
-    });
-    return fn;
-}
-
-// [rows][cols] bf16 matrix, row-major; box [128 rows][box_cols columns]
-bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t cols, uint32_t box_cols, bool swizzle) {
-    EncodeTiled enc = get_encode();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {box_cols, (cuuint32_t)kBlk};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 unsigned long long next_epoch() {
     // distinct per call in this process; the random start keeps a fresh workspace's
@@ -1065,8 +763,9 @@ bool tc_supported(bool bf16, int batch, int L, int H, int P, int N, int G, int c
 }
 
 size_t tc_workspace_bytes(int batch, int L, int H, int) {
-    // epoch-tagged ticket and ready words per (batch, head, block)
-    return 2 * sizeof(unsigned long long) * (size_t)batch * H * (L / kBlk);
+    // epoch-tagged ticket and ready words per (batch, head, block), then the epoch-tagged
+    // word that tells the exact kernel some chain was left to it
+    return 2 * sizeof(unsigned long long) * (size_t)batch * H * (L / kBlk) + sizeof(unsigned long long);
 }
 
 TcArgs make_tc_args(int batch, int L, int H, int chunk, void *ws, int *status) {
@@ -1080,35 +779,26 @@ void tc_set_direction(TcArgs &t, int slot, int dir, const void *x, const void *d
     t.d[slot] = TcDir{x, dt, B, C, A, D, dir};
 }
 
-int tc_launches(bool) { return 1; }
+// Every call runs the shared-score kernel and then the exact kernel for the chains it left
+// (which returns at once when there are none).
+int tc_launches(bool) { return 2; }
 
-#ifdef SSD_TRACE
-extern "C" int ssd_debug_cta_times(unsigned long long *out, int n) {
-    if (n < 4096 * 3) return -1;
-    return cudaMemcpyFromSymbol(out, g_cta_time, sizeof(unsigned long long) * 4096 * 3) == cudaSuccess ? 4096 : -2;
-}
-extern "C" int ssd_debug_trace(unsigned long long *out, int n) {
-    const int total = kTraceWarps * kTraceBlocks * kTracePts;
-    if (n < total) return -1;
-    return cudaMemcpyFromSymbol(out, g_trace, sizeof(unsigned long long) * total) == cudaSuccess ? total : -2;
-}
-#endif
 
-// The shared-memory opt-in is a per-device setting: done once for each device the kernel runs on.
-std::atomic<uint64_t> g_attr_done{0};
 
 cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
-    int dev = 0;
-    cudaError_t attr_err = cudaGetDevice(&dev);
+    const size_t nflags = (size_t)t.batch * t.H * (t.L / kBlk);
+    unsigned long long *ticket = static_cast<unsigned long long *>(t.ws);
+    unsigned long long *ready = ticket + nflags;
+    unsigned long long *deferred = ready + nflags;
+    const unsigned long long epoch = next_epoch();
+    const bool with_state = !bidir && (t.s_in || t.s_out);
+    cudaError_t e = launch_tcs(t, bidir, y, ticket, ready, deferred, epoch, st);
+    if (e != cudaSuccess) return e;
+    // The shared-memory opt-in belongs to the kernel in the current context: set on every launch.
+    cudaError_t attr_err =
+        cudaFuncSetAttribute(with_state ? k_ssd_tc<true> : k_ssd_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes);
     if (attr_err != cudaSuccess) return attr_err;
-    const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
-    if (!bit || !(g_attr_done.load(std::memory_order_acquire) & bit)) {
-        attr_err = cudaFuncSetAttribute(k_ssd_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(k_ssd_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-        if (attr_err != cudaSuccess) return attr_err;
-        g_attr_done.fetch_or(bit, std::memory_order_release);
-    }
     const int ndir = bidir ? 2 : 1;
     const uint64_t rows = (uint64_t)t.batch * t.L;
     TcMaps maps;
@@ -1122,6 +812,7 @@ cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
             return cudaErrorInvalidValue;
         p.d[s].A = d.A;
         p.d[s].D = d.D;
+        p.d[s].dt = static_cast<const __nv_bfloat16 *>(d.dt);
     }
     if (!make_map(&maps.y, y, rows, (uint64_t)t.H * kP, 64, true)) return cudaErrorInvalidValue;
     p.batch = t.batch; p.L = t.L; p.H = t.H; p.nblk = t.L / kBlk;
@@ -1129,10 +820,10 @@ cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
     p.dir_single = t.d[0].dir;
     p.y = static_cast<__nv_bfloat16 *>(y);
     p.status = t.status;
-    const size_t nflags = (size_t)t.batch * t.H * p.nblk;
-    p.ticket = static_cast<unsigned long long *>(t.ws);
-    p.ready = p.ticket + nflags;
-    p.epoch = next_epoch();
+    p.ticket = ticket;
+    p.ready = ready;
+    p.deferred = deferred;
+    p.epoch = epoch;
     p.wait_cycles = t.wait_cycles;
     p.fault = t.fault;
     p.s_in = bidir ? nullptr : t.s_in;

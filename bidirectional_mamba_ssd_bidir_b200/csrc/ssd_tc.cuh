@@ -30,5 +30,9 @@ void tc_set_direction(TcArgs &t, int slot, int dir, const void *x, const void *d
                       const void *B, const void *C, const float *D);
 int tc_launches(bool bidir);
 cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st);
+// the shared-score kernel (ssd_tcs.cu); launch_tc runs it first for calls without a carried state
+cudaError_t launch_tcs(const TcArgs &t, bool bidir, void *y, unsigned long long *ticket, unsigned long long *ready,
+                       unsigned long long *deferred, unsigned long long epoch, cudaStream_t st);
+size_t tcs_smem_bytes();
 
 }  // namespace ssd

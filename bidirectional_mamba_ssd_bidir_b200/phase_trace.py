@@ -7,11 +7,12 @@ The tracing build (``libbidirssd_trace.so``: the same sources compiled with
   at its phase boundaries: points 0..23 per (warp, block).
 * For every CTA, its start and end on the global timer (ns) and its SM.
 
-This module builds that library on demand and runs one bidirectional call
+The kernel traced is the shared-score kernel (ssd_tcs.cu), the one that runs
+every chain whose decay it can factorise.  This module builds that library on demand and runs one bidirectional call
 through it.  The marshalling is the package's own and the call is the same
 C ABI entry point, so the output equals the product library's bit for bit.
 It returns the stamps; ``summary`` prints when each phase of a block ended,
-relative to the MMA warp's issue of that block's score product G = C B^T.
+relative to the issue of that block's score product G = C B^T (MMA stream A).
 
 The product library carries none of this code.  Tracing changes the timing
 a little (one store per warp per point).
@@ -28,14 +29,19 @@ from . import build as _build
 
 N_WARPS, N_BLOCKS, N_POINTS = 20, 8, 24
 N_CTA_SLOTS = 4096
-WARP_TMA, WARP_MMA = 16, 17
+WARP_MMA_A, WARP_MMA_B = 17, 19
+WARP_MMA = WARP_MMA_A
 
 # the points each role records, in program order within a block
-COMPUTE_POINTS = [(0, "block start"), (8, "w.x tile and D x written"), (6, "state product of the last block done"),
-                  (7, "state hand-off done"), (9, "scores G ready"), (10, "decay mask M written"),
-                  (11, "next block's tables built"), (16, "Y_diag and Y_off ready"), (21, "epilogue done")]
-MMA_POINTS = [(0, "G issued"), (1, "Y_off issued"), (2, "state product issued"), (3, "Y_diag issued")]
-TMA_POINTS = [(0, "x stage free, x loads issued"), (1, "B/C buffer free, B/C loads issued")]
+COMPUTE_POINTS = [(0, "block start"), (1, "scores G ready"), (2, "masked scores Gc written"),
+                  (3, "tables two blocks ahead built"), (4, "state product done"), (5, "state hand-off done"),
+                  (6, "next block's cX and Y start written"), (7, "Y ready"), (8, "epilogue done")]
+# (warp, point): stream A (warp 17) issues G and the state product, stream B (warp 19) Y_off and Y_diag
+MMA_POINTS = [(17, 0, "G issued"), (19, 1, "Y_off issued"), (17, 2, "state product issued"), (19, 3, "Y_diag issued")]
+# (warp, point, name) of the load and hand-off warps
+LOAD_POINTS = [(16, 0, "x stage free, x loads issued"), (16, 1, "B buffer free, B loads issued"),
+               (16, 2, "C buffer free, C loads issued"), (18, 0, "y tiles written, store issued"),
+               (18, 1, "stored (first parts published)")]
 
 _trace_lib = None
 
@@ -96,10 +102,10 @@ def summary(phases: np.ndarray, clock_mhz: float = 1965.0, blocks=(3, 4, 5, 6)) 
         ref = phases[WARP_MMA, j, 0]
         nxt = phases[WARP_MMA, j + 1, 0] if j + 1 < N_BLOCKS else np.nan
         lines.append(f"block {j}: period {(nxt - ref) / clock_mhz:.3f} us")
-        for k, name in MMA_POINTS:
-            lines.append(f"  mma      {name:40s} {(phases[WARP_MMA, j, k] - ref) / clock_mhz:8.3f}")
-        for k, name in TMA_POINTS:
-            lines.append(f"  tma      {name:40s} {(phases[WARP_TMA, j, k] - ref) / clock_mhz:8.3f}")
+        for w, k, name in MMA_POINTS:
+            lines.append(f"  mma {w:2d}   {name:40s} {(phases[w, j, k] - ref) / clock_mhz:8.3f}")
+        for w, k, name in LOAD_POINTS:
+            lines.append(f"  warp {w:2d}  {name:40s} {(phases[w, j, k] - ref) / clock_mhz:8.3f}")
         for k, name in COMPUTE_POINTS:
             v = (phases[:16, j, k] - ref) / clock_mhz
             if np.all(np.isnan(v)):
@@ -109,4 +115,4 @@ def summary(phases: np.ndarray, clock_mhz: float = 1965.0, blocks=(3, 4, 5, 6)) 
     return "\n".join(lines)
 
 
-__all__ = ["library", "run", "summary", "COMPUTE_POINTS", "MMA_POINTS", "TMA_POINTS"]
+__all__ = ["library", "run", "summary", "COMPUTE_POINTS", "MMA_POINTS", "LOAD_POINTS"]

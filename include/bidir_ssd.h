@@ -180,9 +180,11 @@ ssd_status r2l_block_scan(const ssd_shape *shape, const ssd_params *p, float s,
  * the part of the scratch that must start at zero (the status word and the
  * forward/reverse hand-off flags).
  *
- * The first call on a device (with that device current) looks up the
- * array's device address once; make that first call before any stream
- * capture.  All calls on one device share the one array: two calls whose
+ * Every call looks up the array's address in the current device's context
+ * (cudaGetSymbolAddress, which allocates nothing), so it stays right after a
+ * cudaDeviceReset or in another context.  The first call on a device also
+ * makes the CUDA runtime load this library's kernels there: make that first
+ * call before any stream capture.  All calls on one device share the one array: two calls whose
  * work overlaps on the GPU (different streams, no ordering between them) race
  * on it and give wrong results.  Order them on one stream, or with events.
  *

@@ -81,4 +81,17 @@ def test_traffic_record_survives_comment_edits_only():
     src = "int f(int a) { // doubles\n  return 2 * a; /* the\n  result */ }\n"
     assert bench._code_only(src) == bench._code_only("int f(int a) {\n\n    return 2 * a;   }  // other words")
     assert bench._code_only(src) != bench._code_only(src.replace("2 * a", "3 * a"))
-    assert bench.profiled_traffic("ssd_bidir_tc", "diffumamba_1p3b_L8192") is not None
+
+
+def test_traffic_record_is_keyed_on_the_current_kernel(tmp_path):
+    """A record whose key is the current sources' hash is found; one with another key is not."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    key = bench._kernel_source_hash()
+    (tmp_path / "a.md").write_text(
+        f"traffic-record: kernel=k workload=w source={key} bytes_per_launch=123\n")
+    (tmp_path / "b.md").write_text("traffic-record: kernel=k2 workload=w source=0000000000000000 bytes_per_launch=9\n")
+    assert bench.profiled_traffic("k", "w", str(tmp_path)) == 123
+    assert bench.profiled_traffic("k2", "w", str(tmp_path)) is None
+    assert bench.profiled_traffic("k", "other", str(tmp_path)) is None

@@ -1,9 +1,10 @@
 """The tracing build of the tensor-core kernel (phase_trace.py).
 
 Its output must equal the product library's bit for bit.  Its per-phase
-stamps must come in program order: within a block, the MMA warp issues G,
-Y_off, the state product and Y_diag in that order, and each CUDA-core warp
-passes its phase boundaries in order.  Every CTA must have recorded a start
+stamps must come in program order: within a block, MMA stream A issues G
+before the state product and stream B Y_off before Y_diag; G waits for the
+previous block's Y_diag; each CUDA-core warp passes its phase boundaries in
+order.  Every CTA must have recorded a start
 before its end.
 """
 import pytest
@@ -27,10 +28,11 @@ def test_trace_build_matches_product_and_orders_phases():
     torch.cuda.synchronize()
     assert torch.equal(y, y_ref)
     order = [k for k, _ in pt.COMPUTE_POINTS]
+    A, Bw = pt.WARP_MMA_A, pt.WARP_MMA_B
     for j in range(1, pt.N_BLOCKS):
-        m = ph[pt.WARP_MMA, j, :4]                           # G, Y_off, state, Y_diag
-        assert m[0] <= m[1] <= m[2] <= m[3], (j, m)
-        assert ph[pt.WARP_MMA, j, 0] > ph[pt.WARP_MMA, j - 1, 3]
+        assert ph[A, j, 0] <= ph[A, j, 2], j                 # stream A: G, then the state product
+        assert ph[Bw, j, 1] <= ph[Bw, j, 3], j               # stream B: Y_off, then Y_diag
+        assert ph[A, j, 0] > ph[Bw, j - 1, 3]                # G waits for the previous block's Y_diag
         for w in range(16):
             seq = [ph[w, j, k] for k in order]
             assert all(a <= b for a, b in zip(seq, seq[1:])), (j, w, seq)

@@ -70,18 +70,128 @@ def test_matches_workspace_entry_point_twice(ssd, dims, chunk):
     assert oracle.rel_err(out[0:1, :, 0:1].double().cpu().numpy(), ref) <= 2e-2
 
 
-def test_allocates_nothing_through_torch(ssd):
+def test_allocates_nothing(ssd):
     dims, chunk = (1, 512, 8, 64, 128, 1), 256
     pf, pr = si.make_bidir(si.Shape(*dims, "bf16"), seed=5)
     f, r = _dev(pf), _dev(pr)
     out = torch.empty_like(f["x"])
-    ssd.bidir_ssd_noalloc(f, r, out, chunk=chunk)      # first call on this device: looks up the scratch
+    ssd.bidir_ssd_noalloc(f, r, out, chunk=chunk)      # first call on this device: loads the kernels
     torch.cuda.synchronize()
     before = (torch.cuda.memory_allocated(), torch.cuda.memory_reserved())
+    free_before = torch.cuda.mem_get_info()[0]          # cudaMemGetInfo: sees any cudaMalloc, not only torch's
     area = ssd.bidir_ssd_noalloc(f, r, out, chunk=chunk)
     torch.cuda.synchronize()
+    free_after = torch.cuda.mem_get_info()[0]
     assert (torch.cuda.memory_allocated(), torch.cuda.memory_reserved()) == before
+    # device allocations come in pages of at least 2 MiB: any allocation would show
+    assert free_before - free_after < (2 << 20), (free_before, free_after)
     ssd.noalloc_status(area)
+
+
+# Runs without torch: two driver-API contexts on the same device, one after the other, each
+# with its own buffers.  In each, the no-allocation call must match bidir_ssd with a workspace:
+# the scratch's address is the one in the context current at the call, not a leftover from the
+# first context (whose memory is gone once that context is destroyed).
+_TWO_CONTEXTS = r"""
+import ctypes, sys
+import numpy as np
+root = sys.argv[1]
+sys.path.insert(0, root)
+import ssd_inputs as si
+
+cu = ctypes.CDLL("libcuda.so.1")
+U64, VP = ctypes.c_uint64, ctypes.c_void_p
+cu.cuCtxCreate_v2.argtypes = [ctypes.POINTER(VP), ctypes.c_uint, ctypes.c_int]
+cu.cuCtxDestroy_v2.argtypes = [VP]
+cu.cuMemAlloc_v2.argtypes = [ctypes.POINTER(U64), ctypes.c_size_t]
+cu.cuMemFree_v2.argtypes = [U64]
+cu.cuMemcpyHtoD_v2.argtypes = [U64, VP, ctypes.c_size_t]
+cu.cuMemcpyDtoH_v2.argtypes = [VP, U64, ctypes.c_size_t]
+cu.cuMemsetD8_v2.argtypes = [U64, ctypes.c_ubyte, ctypes.c_size_t]
+
+def ck(rc, what):
+    if rc != 0:
+        raise SystemExit(f"{what} returned {rc}")
+
+ck(cu.cuInit(0), "cuInit")
+dev = ctypes.c_int()
+ck(cu.cuDeviceGet(ctypes.byref(dev), 0), "cuDeviceGet")
+
+lib = ctypes.CDLL(root + "/bidirectional_mamba_ssd_bidir_b200/libbidirssd.so")
+class Shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("batch", "seqlen", "nheads", "headdim", "dstate", "ngroups", "io")]
+class Params(ctypes.Structure):
+    _fields_ = [(n, VP) for n in ("x", "dt", "A", "B", "C", "D")]
+PS, PP = ctypes.POINTER(Shape), ctypes.POINTER(Params)
+lib.ssd_workspace_bytes.argtypes = [PS, ctypes.c_int]
+lib.ssd_workspace_bytes.restype = ctypes.c_size_t
+lib.bidir_ssd.argtypes = [PS, PP, PP, ctypes.c_int, VP, VP, ctypes.c_size_t, VP]
+lib.bidir_ssd_noalloc.argtypes = [PS, PP, PP, ctypes.c_int, VP, VP, ctypes.POINTER(VP)]
+lib.ssd_workspace_status.argtypes = [VP, ctypes.c_size_t, VP]
+lib.ssd_last_error.restype = ctypes.c_char_p
+
+dims, chunk = (2, 384, 8, 64, 128, 1), 128
+pf, pr = si.make_bidir(si.Shape(*dims, "bf16"), seed=17)
+sh = Shape(*dims, 0)
+ny = dims[0] * dims[1] * dims[2] * dims[3]
+
+def one_context():
+    ctx = VP()
+    ck(cu.cuCtxCreate_v2(ctypes.byref(ctx), 0, dev.value), "cuCtxCreate")      # now current
+    bufs = []
+    def alloc(n):
+        p = U64()
+        ck(cu.cuMemAlloc_v2(ctypes.byref(p), n), "cuMemAlloc")
+        bufs.append(p.value)
+        return p.value
+    def up(stored):
+        a = np.ascontiguousarray(stored.data)
+        p = alloc(a.nbytes)
+        ck(cu.cuMemcpyHtoD_v2(p, a.ctypes.data, a.nbytes), "cuMemcpyHtoD")
+        return p
+    f = Params(*(up(getattr(pf, k)) for k in ("x", "dt", "A", "B", "C", "D")))
+    r = Params(*(up(getattr(pr, k)) for k in ("x", "dt", "A", "B", "C", "D")))
+    y_ws, y_na = alloc(2 * ny), alloc(2 * ny)
+    nws = lib.ssd_workspace_bytes(ctypes.byref(sh), chunk)
+    ws = alloc(nws)
+    ck(cu.cuMemsetD8_v2(ws, 0, nws), "cuMemsetD8")
+    if lib.bidir_ssd(ctypes.byref(sh), ctypes.byref(f), ctypes.byref(r), chunk, y_ws, ws, nws, None) != 0:
+        raise SystemExit("bidir_ssd: " + lib.ssd_last_error().decode())
+    area = VP()
+    if lib.bidir_ssd_noalloc(ctypes.byref(sh), ctypes.byref(f), ctypes.byref(r), chunk, y_na, None,
+                             ctypes.byref(area)) != 0:
+        raise SystemExit("bidir_ssd_noalloc: " + lib.ssd_last_error().decode())
+    ck(cu.cuCtxSynchronize(), "cuCtxSynchronize")
+    for w in (ws, area.value):
+        if lib.ssd_workspace_status(w, 256, None) != 0:
+            raise SystemExit("status: " + lib.ssd_last_error().decode())
+    out = []
+    for y in (y_ws, y_na):
+        h = np.empty(ny, np.uint16)
+        ck(cu.cuMemcpyDtoH_v2(h.ctypes.data, y, 2 * ny), "cuMemcpyDtoH")
+        out.append(si.bf16_bits_to_f32(h).astype(np.float64))
+    for p in bufs:
+        ck(cu.cuMemFree_v2(p), "cuMemFree")
+    ck(cu.cuCtxDestroy_v2(ctx), "cuCtxDestroy")
+    return out
+
+rel = lambda a, b: float(np.abs(a - b).max() / np.abs(b).max())
+(a_ws, a_na), (b_ws, b_na) = one_context(), one_context()
+errs = [rel(a_na, a_ws), rel(b_na, b_ws), rel(b_ws, a_ws)]
+print("errs", errs)
+assert all(np.isfinite(v).all() for v in (a_ws, a_na, b_ws, b_na))
+assert max(errs) <= 1e-2, errs
+print("TWO_CONTEXTS_OK")
+"""
+
+
+def test_scratch_address_follows_the_current_context():
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _TWO_CONTEXTS, root], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and "TWO_CONTEXTS_OK" in r.stdout, r.stdout[-2000:] + r.stderr[-2000:]
 
 
 def test_refuses_shapes_beyond_the_scratch(ssd):
