@@ -43,19 +43,20 @@
 //
 // Bidirectional mixer in one launch: the CTAs of the forward and reverse
 // scans of a head pair are neighbours in the grid.  For every output block of
-// the head pair, an epoch-tagged ticket, taken when the block's scores are issued,
-// makes one direction first: it stores its part of y and publishes an
-// epoch-tagged ready word; the other, second, adds its part once that word is
-// published, with a TMA bf16 reduce-add (performed in L2).  The first never
-// waits, so the hand-off cannot deadlock whatever the residency.
+// the head pair, an epoch-tagged ticket makes one direction first: it stores
+// its part of y and publishes an epoch-tagged ready word; the other, second,
+// adds its part once that word is published, with a TMA bf16 reduce-add
+// (performed in L2).  The first never waits, so the hand-off cannot deadlock
+// whatever the residency.
 //
 // Warp roles (640 threads): warps 0-15 are the CUDA-core warps (warp w: TMEM
 // lane quarter w & 3, column group w >> 2 of 32 columns; the head of a column
-// group is (w >> 2) >> 1); warp 16 issues the TMA loads and L2 prefetches; warps
-// 17 and 19 issue the MMAs, two independent streams (17 also owns TMEM); warp 18
-// takes the forward/reverse tickets, stores y (TMA) and publishes first parts.
-// The CUDA-core warps never wait for global memory or for the other direction.
-// Every wait is
+// group is (w >> 2) >> 1); warp 16 issues the x, C and dt loads and builds the
+// decay tables; warps 17 and 19 issue the MMAs, two independent streams (17
+// also owns TMEM); warp 18
+// takes the forward/reverse tickets, stores y (TMA), publishes first parts and
+// loads B into each buffer as soon as its y tile has been read.  The CUDA-core
+// warps never wait for global memory or for the other direction.  Every wait is
 // bounded; a wait that runs out records SSD_ERR_TIMEOUT in the status word and
 // the CTA winds down without touching more data.
 #include <cuda.h>
@@ -88,20 +89,19 @@ constexpr uint32_t kOffX = 0;                           // 2 stages: x, scaled i
 constexpr uint32_t kOffB = kOffX + 2 * kPairBytes;      // 2 buffers: B (n halves), then the y tile (heads)
 constexpr uint32_t kOffC = kOffB + 2 * kPairBytes;      // C (n halves)
 constexpr uint32_t kOffS = kOffC + kPairBytes;          // bf16 scaled state, rows = n, one tile per head
-constexpr uint32_t kOffTab = kOffS + kPairBytes;        // 4 table buffers (block j in buffer j & 3)
+constexpr uint32_t kOffTab = kOffS + kPairBytes;        // 3 table buffers (block j in buffer j % 3)
 // one table buffer (floats): row factor r, column factor c = e dt, prestore factor e D (per head
 // and row, memory order), and per head the mid-point m and kappa exponent (log2 units)
 constexpr uint32_t kTabR = 0, kTabCF = 2 * kBlk, kTabDR = 4 * kBlk, kTabM2 = 6 * kBlk, kTabK2 = 6 * kBlk + 2;
 constexpr uint32_t kTabFloats = 6 * kBlk + 8;
-constexpr uint32_t kOffDT = (kOffTab + 4 * kTabFloats * 4 + 127) / 128 * 128;   // dt ring, 3 slots
+constexpr uint32_t kOffDT = (kOffTab + 3 * kTabFloats * 4 + 127) / 128 * 128;   // dt ring, 3 slots
 constexpr uint32_t kOffBar = kOffDT + 3 * kDtBytes;
 
 enum Bar {
-    B_XFULL0 = 0, B_XFULL1, B_XEMPTY0, B_XEMPTY1, B_BFULL0, B_BFULL1, B_BFREE0, B_BFREE1, B_CFULL, B_CEMPTY,
+    B_XFULL0 = 0, B_XFULL1, B_XEMPTY0, B_XEMPTY1, B_BFULL0, B_BFULL1, B_CFULL, B_CEMPTY,
     B_DTFULL0, B_DTFULL1, B_DTFULL2, B_GFULL, B_GCREADY, B_CXREADY0,
     B_CXREADY1, B_STFULL, B_SREADY, B_YOFFDONE, B_YFULL, B_YEMPTY, B_TABREADY0, B_TABREADY1, B_TABREADY2,
-    B_TABREADY3,
-    B_TILE0, B_TILE1, B_DONEA, B_DONEB, kNumBars
+    B_TABFREE0, B_TABFREE1, B_TABFREE2, B_TILE0, B_TILE1, B_DONEA, B_DONEB, kNumBars
 };
 // misc: tmem base, abort flag, wait limit, steep flag
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
@@ -127,6 +127,15 @@ __device__ __forceinline__ void trace_pt(int w, int j, int k) {
     }
 }
 #define SSD_TRACE_PT(w, j, k) trace_pt(w, j, k)
+// per-block timeline of CTAs 0 and 1 (the two directions of the first head pair), every block:
+// 0 G issued, 1 y store issued, 2 y tiles read (B buffer free), 3 B load issued
+constexpr int kTraceAllBlocks = 1024;
+__device__ unsigned long long g_blk[2][kTraceAllBlocks][4];
+#define SSD_TRACE_BLK(j, k)                                                                   \
+    do {                                                                                      \
+        if (blockIdx.x < 2 && (j) < kTraceAllBlocks && (threadIdx.x & 31) == 0)               \
+            g_blk[blockIdx.x][j][k] = (unsigned long long)clock64();                          \
+    } while (0)
 __device__ unsigned long long g_cta_time[4096][3];     // start, end, SM id
 #define SSD_TRACE_CTA(k)                                                              \
     do {                                                                              \
@@ -142,6 +151,7 @@ __device__ unsigned long long g_cta_time[4096][3];     // start, end, SM id
 #else
 #define SSD_TRACE_CTA(k) ((void)0)
 #define SSD_TRACE_PT(w, j, k) ((void)0)
+#define SSD_TRACE_BLK(j, k) ((void)0)
 #endif
 
 struct TcsDirParams {
@@ -179,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);   // limit at +8
     int *steep_flag = reinterpret_cast<int *>(sm + kOffMisc + 16);
-    float *tab_s = reinterpret_cast<float *>(sm + kOffTab);         // [4 buffers][kTabFloats]
+    float *tab_s = reinterpret_cast<float *>(sm + kOffTab);         // [3 buffers][kTabFloats]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int npairs = prm.H / 2;
@@ -203,11 +213,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
         *abort_flag = 0;
         *reinterpret_cast<volatile long long *>(abort_flag + 1) = prm.wait_cycles;
         for (int i = 0; i < (int)kNumBars; ++i) {
-            // arrivals: 16 = one per CUDA-core warp, 8 = one per table warp or per warp of a
-            // head, 1 = one thread or one MMA commit (TMA completions count bytes)
+            // arrivals: 16 = one per CUDA-core warp, 1 = one thread or one MMA commit (TMA
+            // completions count bytes)
             uint32_t cnt = 1;
             if (i == B_GCREADY || i == B_CXREADY0 || i == B_CXREADY1 || i == B_SREADY || i == B_YEMPTY) cnt = 16;
-            if (i == B_TILE0 || i == B_TILE1) cnt = 16;
+            if (i == B_TILE0 || i == B_TILE1 || (i >= B_TABFREE0 && i <= B_TABFREE2)) cnt = 16;
             // read by both MMA streams: a commit from each
             if (i == B_XEMPTY0 || i == B_XEMPTY1 || i == B_CEMPTY) cnt = 2;
             mbar_init(bar(i), cnt);
@@ -226,12 +236,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
 
     auto row_of = [&](int jj) { return b * L + (dir > 0 ? jj : nblk - 1 - jj) * kBlk; };
     if (warp == kWarpLoad) {
-        // ---------------------------------------------------------- TMA loads, L2 prefetch, tables
-        // Lane 0 issues all loads in the order their buffers free up: x of block j+1 once block
-        // j-1's products have read its stage, B of block j once block j-2's y tile (staged in the
-        // B buffer) has been stored, C once block j-1's products have read it, dt three blocks
-        // ahead; and prefetches x, B and C of block j+3 into L2.  The whole warp then builds the
-        // decay tables of block j+2 (the CUDA-core warps never wait for them).
+        // ---------------------------------------------------------- TMA loads, tables
+        // Lane 0 issues the loads as their buffers free up: x of block j once block j-2's
+        // products have read its stage, C once block j-1's products have read it, dt three
+        // blocks ahead of the tables.  (B is loaded by the store warp, into the buffer its y
+        // store has just read.)  No L2 prefetches: measured, they cost more copy-engine time
+        // than they save in load latency.
+        // The whole warp builds the decay tables (the CUDA-core warps never compute them).
         const uint32_t MASK = 0xffffffffu;
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map_x)) : "memory");
@@ -239,9 +250,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map_b)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map_c)) : "memory");
         }
-        int x_issued = 0, b_issued = 0, c_issued = 0, dt_issued = 0;
-        // dt of block jj into slot jj % 3: its tables are built at iteration jj-2, before the slot
-        // is loaded again (iteration jj), in this warp's program order
+        int x_issued = 0, c_issued = 0, dt_issued = 0;
+        // dt of block jj into slot jj % 3, loaded once the tables of block jj-3 (the slot's
+        // previous content) have been built, in this warp's program order
         auto load_dt = [&](int jj) {
             const int sl = jj % 3;
             if (lane == 0) {
@@ -250,40 +261,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
             }
             dt_issued = jj + 1;
         };
-        auto prefetch = [&](int jj) {
-            if (lane == 0) {
-                const int row = row_of(jj);
-                tma_prefetch_2d(map_x, h0 * kP, row);
-                tma_prefetch_2d(map_x, (h0 + 1) * kP, row);
-                for (int q = 0; q < 2; ++q) {
-                    tma_prefetch_2d(map_b, q * 64, row);
-                    tma_prefetch_2d(map_c, q * 64, row);
-                }
-            }
-        };
-        // x of block jj into stage jj & 1, once block jj-2's products have read that stage
-        auto load_x = [&](int jj) -> bool {
-            const int sx = jj & 1;
-            if (jj >= 2 && !mbar_wait(bar(B_XEMPTY0 + sx), ((jj >> 1) - 1) & 1, MASK, abort_flag, prm.status, 11))
-                return false;
-            SSD_TRACE_PT(kWarpLoad, jj, 0);
-            if (lane == 0) {
-                mbar_expect_tx(bar(B_XFULL0 + sx), kPairBytes);
-                for (int h = 0; h < 2; ++h)
-                    tma_load_2d(sbase + kOffX + sx * kPairBytes + h * kTileBytes, map_x, (h0 + h) * kP, row_of(jj),
-                                bar(B_XFULL0 + sx));
-            }
-            x_issued = jj + 1;
-            return true;
-        };
-        // Tables of block jj (buffer jj & 3), both heads: lane l takes scan positions 4l..4l+3
+        // Tables of block jj (buffer jj % 3), both heads: lane l takes scan positions 4l..4l+3
         // (memory rows k forward, 127 - k reverse), forms the inclusive cumulative A dt in scan
         // order (its own four, then a warp scan), the block's mid-point m and the factors.
         auto build_tables = [&](int jj) -> bool {
             const int sl = jj % 3;
             if (!mbar_wait(bar(B_DTFULL0 + sl), (jj / 3) & 1, MASK, abort_flag, prm.status, 51)) return false;
             const uint8_t *dtt = sm + kOffDT + sl * kDtBytes;      // [128 rows][8 heads] bf16
-            float *tb = tab_s + (jj & 3) * kTabFloats;
+            float *tb = tab_s + (jj % 3) * kTabFloats;
             const int hc = h0 & 7;                                  // column of head h0 (h0 + 1 next to it)
             int rows[4];
             uint32_t dpair[4];                                      // (head h0, head h0 + 1) dt of each row
@@ -335,53 +320,79 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                 return false;
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_TABREADY0 + (jj & 3)));
+            if (lane == 0) mbar_arrive(bar(B_TABREADY0 + jj % 3));
             return true;
         };
-        bool ok = true;
+        // Three independent in-order streams, served by readiness (C first: it gates the next
+        // block's scores; then x, the tables with dt).  Each buffer's wait condition is a parity
+        // test on a barrier that is at most one phase away from the awaited one, since its
+        // stream issues in block order.
         for (int jj = 0; jj < 3 && jj < nblk; ++jj) load_dt(jj);
-        for (int jj = 0; jj < 3 && jj < nblk; ++jj) prefetch(jj);
-        if (nblk > 0) ok = load_x(0);
-        for (int jj = 0; jj < 2 && jj < nblk && ok; ++jj) ok = build_tables(jj);
-        for (int j = 0; j < nblk && ok; ++j) {
-            const int st = j & 1;
-            const int row = row_of(j);
-            if (j + 3 < nblk) prefetch(j + 3);
-            // x runs one block ahead of B and C: its stage frees on an MMA completion, while the B
-            // buffer waits for a y store
-            if (j + 1 < nblk && !load_x(j + 1)) break;
-            // B: buffer st is free once block j-2's y tile, staged there after its products had
-            // read B, has been read by its TMA store
-            if (j >= 2 && !mbar_wait(bar(B_BFREE0 + st), ((j >> 1) - 1) & 1, MASK, abort_flag, prm.status, 12))
+        int tb_built = 0;
+        long long t_idle = clock64();
+        const long long limit = *reinterpret_cast<volatile long long *>(abort_flag + 1);
+        while (c_issued < nblk || x_issued < nblk || tb_built < nblk) {
+            if (*abort_flag) break;
+            uint32_t ready = 0;
+            if (lane == 0) {
+                if (c_issued < nblk && (c_issued == 0 || mbar_test(bar(B_CEMPTY), (c_issued - 1) & 1)))
+                    ready |= 1u;
+                if (x_issued < nblk &&
+                    (x_issued < 2 || mbar_test(bar(B_XEMPTY0 + (x_issued & 1)), ((x_issued >> 1) - 1) & 1)))
+                    ready |= 4u;
+                // tables of block t go to buffer t % 3, free once every CUDA-core warp has read
+                // block t-3's tables for the last time (its epilogue, B_TABFREE)
+                if (tb_built < nblk &&
+                    (tb_built < 3 || mbar_test(bar(B_TABFREE0 + tb_built % 3), ((tb_built - 3) / 3) & 1)) &&
+                    mbar_test(bar(B_DTFULL0 + tb_built % 3), (tb_built / 3) & 1))
+                    ready |= 8u;
+            }
+            ready = __shfl_sync(MASK, ready, 0);
+            if (ready & 1u) {
+                const int j = c_issued;
+                SSD_TRACE_PT(kWarpLoad, j, 2);
+                if (lane == 0) {
+                    mbar_expect_tx(bar(B_CFULL), kPairBytes);
+                    for (int q = 0; q < 2; ++q)
+                        tma_load_2d(sbase + kOffC + q * kTileBytes, map_c, q * 64, row_of(j), bar(B_CFULL));
+                }
+                c_issued = j + 1;
+            }
+            if (ready & 4u) {
+                const int j = x_issued, sx = j & 1;
+                SSD_TRACE_PT(kWarpLoad, j, 0);
+                if (lane == 0) {
+                    mbar_expect_tx(bar(B_XFULL0 + sx), kPairBytes);
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_2d(sbase + kOffX + sx * kPairBytes + h * kTileBytes, map_x, (h0 + h) * kP,
+                                    row_of(j), bar(B_XFULL0 + sx));
+                }
+                x_issued = j + 1;
+            }
+            if (ready & 8u) {
+                if (!build_tables(tb_built)) break;
+                SSD_TRACE_PT(kWarpLoad, tb_built, 3);
+                ++tb_built;
+                // dt slot (t + 3) % 3 held the block whose tables were just built
+                if (dt_issued < nblk) load_dt(dt_issued);
+            }
+            if (ready) {
+                t_idle = clock64();
+            } else if (clock64() - t_idle > limit) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    atomicExch(prm.status, 13);
+                }
                 break;
-            SSD_TRACE_PT(kWarpLoad, j, 1);
-            if (lane == 0) {
-                mbar_expect_tx(bar(B_BFULL0 + st), kPairBytes);
-                for (int q = 0; q < 2; ++q)
-                    tma_load_2d(sbase + kOffB + st * kPairBytes + q * kTileBytes, map_b, q * 64, row,
-                                bar(B_BFULL0 + st));
+            } else {
+                __nanosleep(32);
             }
-            b_issued = j + 1;
-            // C: free once block j-1's scores and Y_off (the two MMA streams) have read it
-            if (j >= 1 && !mbar_wait(bar(B_CEMPTY), (j - 1) & 1, MASK, abort_flag, prm.status, 14)) break;
-            SSD_TRACE_PT(kWarpLoad, j, 2);
-            if (lane == 0) {
-                mbar_expect_tx(bar(B_CFULL), kPairBytes);
-                for (int q = 0; q < 2; ++q)
-                    tma_load_2d(sbase + kOffC + q * kTileBytes, map_c, q * 64, row, bar(B_CFULL));
-            }
-            c_issued = j + 1;
-            if (j + 3 < nblk) load_dt(j + 3);
-            // tables of block j+2 into buffer (j+2) & 3, last read for block j-2: every CUDA-core
-            // warp has finished block j-2's epilogue, since its y tile has been stored (B_BFREE)
-            if (j + 2 < nblk && !(ok = build_tables(j + 2))) break;
         }
+        __syncwarp();
         if (*abort_flag && lane == 0) {
             // let copies still in flight land before the CTA exits
             for (int jj = x_issued - 1; jj >= 0 && jj >= x_issued - 2; --jj)
                 mbar_drain(bar(B_XFULL0 + (jj & 1)), (jj >> 1) & 1, prm.wait_cycles);
-            for (int jj = b_issued - 1; jj >= 0 && jj >= b_issued - 2; --jj)
-                mbar_drain(bar(B_BFULL0 + (jj & 1)), (jj >> 1) & 1, prm.wait_cycles);
             if (c_issued > 0) mbar_drain(bar(B_CFULL), (c_issued - 1) & 1, prm.wait_cycles);
             for (int jj = dt_issued - 1; jj >= 0 && jj >= dt_issued - 3; --jj)
                 mbar_drain(bar(B_DTFULL0 + jj % 3), (jj / 3) & 1, prm.wait_cycles);
@@ -430,6 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                 mma_commit_w(bar(B_GFULL));
                 mma_commit_w(bar(B_CEMPTY));
                 SSD_TRACE_PT(kWarpMmaA, j, 0);
+                SSD_TRACE_BLK(j, 0);
                 // S (+)= B^T (cX): M = n, N = (head, p), K = rows; both operands MN-major.  The
                 // state was scaled in place for this block (B_SREADY); cX is ready (B_CXREADY).
                 if (!mbar_wait(bar(B_CXREADY0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 25)) break;
@@ -478,18 +490,40 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
         if (lane == 0) mbar_drain(done, 0, prm.wait_cycles);
         __syncwarp();
     } else if (warp == kWarpStore) {
-        // ---------------------------------------------------------- tickets and y stores
+        // ---------------------------------------------------------- tickets, y stores, B loads
         // Per block (scan order): take the head pair's ticket; if the other direction took it
         // first, wait until its part is published.  Then, once the CUDA-core warps have written
         // both heads' y tiles into the block's B buffer: first direction, TMA store; second,
-        // TMA bf16 reduce-add (in L2) onto the published part.  When the tiles have been read the
-        // buffer goes back to the B loads.  A first part is published as soon as its own writes
-        // have completed.  One ticket covers both heads, so the directions agree on the order of
-        // whole blocks; a direction only waits on a block the other has claimed, whose
-        // publication depends on nothing this direction still has to do.
+        // TMA bf16 reduce-add (in L2) onto the published part.  As soon as the tiles have been
+        // read, B of block j+2 is loaded into the buffer.  A first part is published once its
+        // writes have completed, checked after the next block's store is issued; before this
+        // direction waits on a block the other direction took, it publishes what it has
+        // pending.  So a publication depends on nothing the other direction still has to do,
+        // and the two cannot wait on each other.  One ticket covers both heads.
         if (lane == 0) {
             const uint32_t MASK = 1u;
-            for (int j = 0; j < nblk; ++j) {
+            int b_issued = 0;
+            auto load_b = [&](int jj) {
+                const int sb = jj & 1;
+                SSD_TRACE_PT(kWarpLoad, jj, 1);
+                SSD_TRACE_BLK(jj, 3);
+                mbar_expect_tx(bar(B_BFULL0 + sb), kPairBytes);
+                for (int q = 0; q < 2; ++q)
+                    tma_load_2d(sbase + kOffB + sb * kPairBytes + q * kTileBytes, map_b, q * 64, row_of(jj),
+                                bar(B_BFULL0 + sb));
+                b_issued = jj + 1;
+            };
+            int pend = -1;                  // block stored first whose part is not yet published
+            size_t pend_slot = 0;
+            auto publish = [&]() {          // call once the block's writes have completed
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                if (prm.fault != 1) st_release(prm.ready + pend_slot, prm.epoch);
+                SSD_TRACE_PT(kWarpStore, pend, 1);
+                pend = -1;
+            };
+            for (int jj = 0; jj < 2 && jj < nblk; ++jj) load_b(jj);
+            bool ok = true;
+            for (int j = 0; j < nblk && ok; ++j) {
                 const int st = j & 1;
                 const int cm = dir > 0 ? j : nblk - 1 - j;
                 const size_t pair_slot = ((size_t)b * prm.H + h0) * nblk + cm;
@@ -497,9 +531,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                 if (prm.bidir) {
                     sec = atomicExch(prm.ticket + pair_slot, prm.epoch) == prm.epoch;
                     if (sec) {
+                        if (pend >= 0) {
+                            bulk_wait0();
+                            publish();
+                        }
                         const unsigned long long *rp = prm.ready + pair_slot;
                         const long long t0 = clock64();
-                        bool ok = true;
                         while (ld_acquire(rp) != prm.epoch) {
                             if (*abort_flag) { ok = false; break; }
                             if (clock64() - t0 > prm.wait_cycles) {
@@ -515,6 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                 }
                 if (!mbar_wait(bar(B_TILE0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 61)) break;
                 SSD_TRACE_PT(kWarpStore, j, 0);
+                SSD_TRACE_BLK(j, 1);
                 const uint32_t tile = sbase + kOffB + st * kPairBytes;
                 if (!sec) {
                     for (int hs = 0; hs < 2; ++hs)
@@ -526,16 +564,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                 }
                 bulk_commit();
                 bulk_wait_read0();                        // the tiles may be overwritten from here on
-                mbar_arrive(bar(B_BFREE0 + st));
-                if (prm.bidir && !sec) {
-                    bulk_wait0();                         // this part of y is in global memory
-                    asm volatile("fence.proxy.async.global;" ::: "memory");
-                    if (prm.fault != 1) st_release(prm.ready + pair_slot, prm.epoch);
+                SSD_TRACE_PT(kWarpStore, j, 2);
+                SSD_TRACE_BLK(j, 2);
+                if (j + 2 < nblk) load_b(j + 2);
+                if (pend >= 0) {
+                    bulk_wait1();                         // every store group but this block's is done
+                    publish();
                 }
-                SSD_TRACE_PT(kWarpStore, j, 1);
+                if (prm.bidir && !sec) {
+                    pend = j;
+                    pend_slot = pair_slot;
+                }
             }
             bulk_wait0();                                 // every store has landed before the CTA exits
+            if (ok && pend >= 0 && !*abort_flag) publish();
+            if (*abort_flag) {
+                for (int jj = b_issued - 1; jj >= 0 && jj >= b_issued - 2; --jj)
+                    mbar_drain(bar(B_BFULL0 + (jj & 1)), (jj >> 1) & 1, prm.wait_cycles);
+            }
         }
+        __syncwarp();
     } else {
         // ---------------------------------------------------------- CUDA-core work
         const uint32_t MASK = 0xffffffffu;
@@ -549,8 +597,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
         // cX of block jj (rows scaled in place by c, this group's 4 chunks of its row) and the
         // starting value D x / r of its Y accumulator
         auto cx_pass = [&](int jj) -> bool {
-            const int st = jj & 1, sl = jj & 3;
-            if (!mbar_wait(bar(B_TABREADY0 + sl), (jj >> 2) & 1, MASK, abort_flag, prm.status, 41)) return false;
+            const int st = jj & 1, sl = jj % 3;
+            if (!mbar_wait(bar(B_TABREADY0 + sl), (jj / 3) & 1, MASK, abort_flag, prm.status, 41)) return false;
             if (!mbar_wait(bar(B_XFULL0 + st), (jj >> 1) & 1, MASK, abort_flag, prm.status, 42)) return false;
             // Y buffer st was last read by block jj-2's epilogue
             if (jj >= 2 && !mbar_wait(bar(B_YEMPTY), (jj - 2) & 1, MASK, abort_flag, prm.status, 43)) return false;
@@ -591,13 +639,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
             if (all || diag) {
                 float gv[32];
                 tmem_ld32(tl + kColG + 32 * g, gv);
-                if (diag) {
-#pragma unroll
-                    for (int u = 0; u < 32; ++u)
-                        if (dir > 0 ? u > lane : u < lane) gv[u] = 0.f;
-                }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) m[i] = pack_bf16(gv[2 * i], gv[2 * i + 1]);
+                if (diag) {
+                    // keep sources u <= lane (forward) or u >= lane (reverse): bit u of keep.
+                    // Applied to the packed words with integer masks, without branches.
+                    const uint32_t low = lane == 31 ? 0xffffffffu : (2u << lane) - 1u;
+                    const uint32_t keep = dir > 0 ? low : ~((1u << lane) - 1u);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const uint32_t k2 = keep >> (2 * i);
+                        m[i] &= ((k2 & 1u) * 0xffffu) | (((k2 >> 1) & 1u) * 0xffff0000u);
+                    }
+                }
             } else {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) m[i] = 0u;
@@ -614,10 +668,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
         // by e^{m_jn} kappa_{jn-1} in place, and its bf16 copy (rows = n) is the B operand of the
         // next Y_off.  k2p = kappa exponent of block jn-1.
         auto state_pass = [&](int jn, float k2p) -> bool {
-            if (!mbar_wait(bar(B_TABREADY0 + (jn & 3)), (jn >> 2) & 1, MASK, abort_flag, prm.status, 48)) return false;
+            if (!mbar_wait(bar(B_TABREADY0 + jn % 3), (jn / 3) & 1, MASK, abort_flag, prm.status, 48)) return false;
             // the bf16 copy is read by Y_off of block jn-1 (stream B commits B_YOFFDONE every block)
             if (!mbar_wait(bar(B_YOFFDONE), (jn - 1) & 1, MASK, abort_flag, prm.status, 50)) return false;
-            const float m2n = tab_s[(jn & 3) * kTabFloats + kTabM2 + hs];
+            const float m2n = tab_s[(jn % 3) * kTabFloats + kTabM2 + hs];
             const float l2 = m2n + k2p;
             float sv[32];
             tmem_ld32(tl + kColS + 32 * g, sv);
@@ -683,7 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
         for (int j = 0; j < nblk && ok; ++j) {
             if (__any_sync(0xffffffffu, *abort_flag)) break;
             SSD_TRACE_PT(warp, j, 0);
-            const int st = j & 1, sl = j & 3;
+            const int st = j & 1, sl = j % 3;
             // (1) mask this block's scores
             if (!mbar_wait(bar(B_GFULL), j & 1, MASK, abort_flag, prm.status, 44)) break;
             SSD_TRACE_PT(warp, j, 1);
@@ -714,8 +768,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                 for (int i = 0; i < 32; ++i) prm.s_out[sslot + (size_t)(32 * ch + i) * kN + r] = sv[i] * f;
             }
             // (4) epilogue: y = r Y_j in bf16 into this block's B buffer, which G and the state
-            // product have consumed (the state product's completion was awaited in (4), or here for
-            // the last block); the store warp writes the tiles to y
+            // product have consumed (the state product's completion was awaited in (2), or here
+            // for the last block); the store warp writes the tiles to y
             if (j + 1 == nblk && !prm.s_out && !mbar_wait(bar(B_STFULL), j & 1, MASK, abort_flag, prm.status, 49))
                 break;
             if (!mbar_wait(bar(B_YFULL), j & 1, MASK, abort_flag, prm.status, 46)) break;
@@ -740,7 +794,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(bar(B_YEMPTY));
+                mbar_arrive(bar(B_YEMPTY));            // the Y accumulator has been read
+                mbar_arrive(bar(B_TABFREE0 + sl));     // and the block's tables, for the last time
                 mbar_arrive(bar(B_TILE0 + st));
             }
             SSD_TRACE_PT(warp, j, 8);
@@ -764,6 +819,11 @@ size_t tcs_smem_bytes() { return kSmemBytes; }
 extern "C" int ssd_debug_cta_times(unsigned long long *out, int n) {
     if (n < 4096 * 3) return -1;
     return cudaMemcpyFromSymbol(out, g_cta_time, sizeof(unsigned long long) * 4096 * 3) == cudaSuccess ? 4096 : -2;
+}
+extern "C" int ssd_debug_blocks(unsigned long long *out, int n) {
+    const int total = 2 * kTraceAllBlocks * 4;
+    if (n < total) return -1;
+    return cudaMemcpyFromSymbol(out, g_blk, sizeof(unsigned long long) * total) == cudaSuccess ? total : -2;
 }
 extern "C" int ssd_debug_trace(unsigned long long *out, int n) {
     const int total = kTraceWarps * kTraceBlocks * kTracePts;

@@ -39,9 +39,13 @@ COMPUTE_POINTS = [(0, "block start"), (1, "scores G ready"), (2, "masked scores 
 # (warp, point): stream A (warp 17) issues G and the state product, stream B (warp 19) Y_off and Y_diag
 MMA_POINTS = [(17, 0, "G issued"), (19, 1, "Y_off issued"), (17, 2, "state product issued"), (19, 3, "Y_diag issued")]
 # (warp, point, name) of the load and hand-off warps
-LOAD_POINTS = [(16, 0, "x stage free, x loads issued"), (16, 1, "B buffer free, B loads issued"),
-               (16, 2, "C buffer free, C loads issued"), (18, 0, "y tiles written, store issued"),
-               (18, 1, "stored (first parts published)")]
+LOAD_POINTS = [(16, 0, "x stage free, x loads issued"), (16, 1, "B loads issued (store warp)"),
+               (16, 2, "C buffer free, C loads issued"), (16, 3, "decay tables built"),
+               (18, 0, "y tiles written, store issued"), (18, 2, "y tiles read"),
+               (18, 1, "first part published")]
+# per-block timeline of CTAs 0 and 1, every block (see block_times)
+BLOCK_POINTS = ["G issued", "y store issued", "y tiles read", "B load issued"]
+N_ALL_BLOCKS = 1024
 
 _trace_lib = None
 
@@ -57,6 +61,8 @@ def library(force_build: bool = False) -> ctypes.CDLL:
             getattr(t, name).restype = getattr(_lib, name).restype
         t.ssd_debug_trace.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int]
         t.ssd_debug_trace.restype = ctypes.c_int
+        t.ssd_debug_blocks.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int]
+        t.ssd_debug_blocks.restype = ctypes.c_int
         t.ssd_debug_cta_times.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int]
         t.ssd_debug_cta_times.restype = ctypes.c_int
         _trace_lib = t
@@ -95,6 +101,18 @@ def run(fwd: dict, rev: dict, chunk: int = 256):
     return y, phases, ctas
 
 
+def block_times() -> np.ndarray:
+    """Per-block timeline of CTAs 0 and 1 of the last traced call: float64 [cta][block][point]
+    of SM cycles (points in ``BLOCK_POINTS``), NaN where nothing was recorded."""
+    n = 2 * N_ALL_BLOCKS * len(BLOCK_POINTS)
+    buf = (ctypes.c_ulonglong * n)()
+    if library().ssd_debug_blocks(buf, n) != n:
+        raise RuntimeError("could not read the block timeline")
+    out = np.array(buf[:], dtype=np.float64).reshape(2, N_ALL_BLOCKS, len(BLOCK_POINTS))
+    out[out == 0] = np.nan
+    return out
+
+
 def summary(phases: np.ndarray, clock_mhz: float = 1965.0, blocks=(3, 4, 5, 6)) -> str:
     """Per block: when each phase ended, in microseconds after the MMA warp issued that block's G."""
     lines = []
@@ -115,4 +133,5 @@ def summary(phases: np.ndarray, clock_mhz: float = 1965.0, blocks=(3, 4, 5, 6)) 
     return "\n".join(lines)
 
 
-__all__ = ["library", "run", "summary", "COMPUTE_POINTS", "MMA_POINTS", "LOAD_POINTS"]
+__all__ = ["library", "run", "summary", "block_times", "COMPUTE_POINTS", "MMA_POINTS", "LOAD_POINTS",
+           "BLOCK_POINTS"]
