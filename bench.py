@@ -1,7 +1,7 @@
 """Benchmark: bidirectional SSD scan throughput (tokens/s) at the DiffuMamba ~1.3B layer shape.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
-                    [--op fwd|bwd] [--batch B]
+                    [--op fwd|bwd] [--batch B] [--dry-run]
 
 One step is one full bidirectional scan call (forward + reverse + sum) over a
 batch of synthetic seeded inputs already resident in HBM.  The default
@@ -21,6 +21,11 @@ The JSON line carries, besides the contract keys:
                 inside the timed region
   clocks        SM clocks and throttle reasons sampled during the timed region
 ``--impl reference`` times the oracle alone (the CPU reference arm).
+``--gpus N`` outside torchrun starts N rank processes itself (127.0.0.1
+rendezvous); ``--dry-run`` runs only the host logic of the ranks (gloo
+process group, shards, MAX reduction), without a GPU.
+``--workload r2l_block_L32`` times the R2L sidecar decode: one step is 256
+back-to-back denoising-step calls on fresh inputs, reported per call.
 ``--op bwd`` times the gradients of both directions (its own JSON line, with
 a roofline against the float32 ALU peak).  ``--batch`` replaces the batch
 size, for small ncu captures.
@@ -358,7 +363,8 @@ def run_ours(args) -> None:
         achieved = alg_bytes / (per_launch_ms / 1e3) / 1e9
         kernel = "ssd_bidir_tc" if path == 1 else "simt_call(6 kernels)"
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "metric": METRIC if args.workload == DEFAULT_WORKLOAD else f"bidirectional SSD scan tokens/s, {args.workload}",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if shape.io == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": args.workload, "global_batch": shape.batch * world, "seq_len": shape.seqlen,
@@ -383,6 +389,171 @@ def run_ours(args) -> None:
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_r2l(args) -> None:
+    """R2L sidecar decode: 256 denoising steps back to back, each a fresh block of inputs.
+
+    One bench step is the 256 calls; the metric is microseconds per denoising-step call (lower
+    is better).  Every call's inputs are generated up front and resident on the device."""
+    import torch
+    import torch.distributed as dist
+    import bidirectional_mamba_ssd_bidir_b200 as ssd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    w = si.WORKLOADS[args.workload]
+    shape, chunk, nsteps = w["shape"], w["chunk"], w["steps"]
+    if args.batch is not None:
+        shape = dataclasses.replace(shape, batch=args.batch)
+    seed = rank
+    host, dev_in, gates = [], [], []
+    for st in range(nsteps):
+        p = si.make_params(shape, seed=seed, offset=si.STEP_STRIDE * st + si.REV_OFFSET)
+        h = {k: getattr(p, k).torch().pin_memory() for k in ("x", "dt", "A", "B", "C", "D")}
+        h["res"] = si.make_residual(shape, seed=seed, step=st).torch().pin_memory()
+        host.append(h)
+        dev_in.append({k: v.to(dev, non_blocking=True) for k, v in h.items()})
+        gates.append(si.make_gate(seed, st))
+    outs = [torch.empty_like(d["res"]) for d in dev_in]
+    dims = (shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate, shape.ngroups)
+    ws = torch.zeros(max(256, ssd.workspace_bytes(dims, torch.bfloat16, chunk)), dtype=torch.uint8, device=dev)
+    path = ssd.path_for(dims, torch.bfloat16, chunk)
+    per_call = ssd.kernel_launches(dims, torch.bfloat16, chunk, "r2l")
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize()
+
+    def one_pass():
+        for st in range(nsteps):
+            d = dev_in[st]
+            ssd.r2l_block_scan(d, gates[st], d["res"], chunk=chunk, out=outs[st], workspace=ws)
+
+    for _ in range(args.warmup):
+        one_pass()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    with ClockSampler(local) as clk:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(args.steps):
+            one_pass()
+        end.record(stream)
+        torch.cuda.synchronize()
+    ssd.workspace_status(ws)
+    total_ms = max_over_ranks(start.elapsed_time(end), dist)
+    us_per_call = total_ms * 1e3 / (args.steps * nsteps)
+
+    # end to end: each call's inputs copied in from pinned host memory and its output copied back,
+    # in order on one stream (a decode loop needs each step's output before the next step)
+    outs_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs[:2]]
+    h2d = sum(v.numel() * v.element_size() for v in host[0].values())
+    d2h = outs[0].numel() * outs[0].element_size()
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for st in range(nsteps):
+        d = dev_in[st]
+        for k, v in host[st].items():
+            d[k].copy_(v, non_blocking=True)
+        ssd.r2l_block_scan(d, gates[st], d["res"], chunk=chunk, out=outs[st], workspace=ws)
+        outs_h[st % 2].copy_(outs[st], non_blocking=True)
+    e2.record(stream)
+    torch.cuda.synchronize()
+    e2e_us = max_over_ranks(s2.elapsed_time(e2), dist) * 1e3 / nsteps
+
+    if rank == 0:
+        peaks = measured_peaks()
+        bpt = algorithmic_bytes_per_token(shape, directions=1) + 2 * shape.nheads * shape.headdim  # + residual
+        alg_bytes = bpt * shape.tokens
+        achieved = alg_bytes / (us_per_call / 1e6) / 1e9
+        line = {
+            "metric": "R2L sidecar block scan, microseconds per denoising step (256 steps back to back)",
+            "value": us_per_call, "unit": "us", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "global_batch": shape.batch * world, "seq_len": shape.seqlen,
+                       "nheads": shape.nheads, "headdim": shape.headdim, "dstate": shape.dstate, "chunk": chunk,
+                       "calls_per_step": nsteps, "parallelism": f"dp{world} (independent decodes)",
+                       "path": "tcgen05" if path == 1 else "simt",
+                       "l2": "inputs of all 256 calls resident, no flush (a decode loop's inputs are hot)"},
+            "roofline": {"bound": "hbm", "kernel": "r2l_call", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes_per_launch": alg_bytes, "bytes_per_token": bpt,
+                         "launch_us": us_per_call, "peak_source": peaks["source"] + " hbm_gbs",
+                         "note": "latency-bound: a few MB per call; per-call launch latency dominates"},
+            "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": nsteps, "overlap": "none: each call's copies and call in order on one stream"},
+            "gpu_launches": per_call * nsteps * args.steps,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            cores = oracle.default_threads()
+            n = 0
+            t0 = time.perf_counter()
+            while time.perf_counter() - t0 < min(args.cpu_seconds, 10.0) and n < nsteps:
+                p = si.make_params(shape, seed=seed, offset=si.STEP_STRIDE * n + si.REV_OFFSET)
+                oracle.r2l_block_f64(oracle.params_f64(p), gates[n],
+                                     si.make_residual(shape, seed=seed, step=n).f64())
+                n += 1
+            cpu_us = (time.perf_counter() - t0) * 1e6 / n
+            line["cpu_baseline"] = {"value": cpu_us, "unit": "us", "cores": cores, "kind": "oracle",
+                                    "sample": f"float64 r2l block, the first {n} of {nsteps} steps, whole block "
+                                              "(input generation included)"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_dry(args) -> None:
+    """Host logic of a multi-rank run, without a GPU: gloo process group, each rank's shard,
+    and the MAX reduction of a per-rank time (rank r reports 1 + r: the slowest sets the line)."""
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("gloo", timeout=timedelta(seconds=60))
+    plan = shard_plan(rank, world, args.workload, args.batch)
+    t = max_over_ranks(1.0 + rank, dist if world > 1 else None)
+    mine = (rank, plan["seed"], plan["tokens"])
+    ranks = [mine]
+    if world > 1:
+        ranks = [None] * world
+        dist.all_gather_object(ranks, mine)
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "n_ranks": world, "ranks": ranks, "max_time": t,
+                          "tokens_all": sum(r[2] for r in ranks)}), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def _rank_entry(index: int, world: int, port: int, argv: list) -> None:
+    os.environ.update(RANK=str(index), LOCAL_RANK=str(index), WORLD_SIZE=str(world), LOCAL_WORLD_SIZE=str(world),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    main(argv)
+
+
+def spawn_ranks(n: int, argv: list) -> None:
+    """Start n rank processes (one per GPU), as torchrun would, and wait for them."""
+    import torch.multiprocessing as mp
+    mp.start_processes(_rank_entry, args=(n, _free_port(), list(argv)), nprocs=n, start_method="spawn", join=True)
 
 
 # ------------------------------------------------------------------ reference arm (the oracle)
@@ -458,6 +629,31 @@ def run_reference(args) -> None:
     shape = w["shape"]
     import oracle
     cores = oracle.default_threads()
+    if w["kind"] == "r2l":
+        # the R2L decode: the float64 block per denoising step, inputs generated before the clock
+        nsteps = w["steps"]
+        per_step = max(1, min(nsteps, 16))
+        steps_in = [(oracle.params_f64(si.make_params(shape, seed=0, offset=si.STEP_STRIDE * st + si.REV_OFFSET)),
+                     si.make_gate(0, st), si.make_residual(shape, seed=0, step=st).f64()) for st in range(per_step)]
+        for _ in range(args.warmup):
+            oracle.r2l_block_f64(*steps_in[0])
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            for q, g, r in steps_in:
+                oracle.r2l_block_f64(q, g, r)
+        us = (time.perf_counter() - t0) * 1e6 / (args.steps * per_step)
+        sample = f"float64 r2l block, the first {per_step} of {nsteps} denoising steps per bench step"
+        line = {"metric": "R2L sidecar block scan, microseconds per denoising step (256 steps back to back)",
+                "value": us, "unit": "us", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": us * nsteps / 1e3, "higher_is_better": False, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+                "config": {"workload": args.workload, "global_batch": shape.batch, "seq_len": shape.seqlen,
+                           "nheads": shape.nheads, "headdim": shape.headdim, "dstate": shape.dstate,
+                           "chunk": w["chunk"], "calls_per_step": nsteps, "parallelism": "host cores"},
+                "cpu_baseline": {"value": us, "unit": "us", "cores": cores, "kind": "oracle", "sample": sample},
+                "e2e": {"value": us, "unit": "us", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
     # size each step so that warmup + steps stay within ~args.ref_budget seconds
     per_step_budget = max(0.05, args.ref_budget / max(1, args.steps + args.warmup))
     probe, _, _ = time_oracle(shape, 0, min(cores, shape.nheads), seqlen=min(shape.seqlen, 1024))
@@ -492,8 +688,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=[k for k, v in si.WORKLOADS.items()
-                                                                      if v["kind"] == "bidir"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(si.WORKLOADS))
     ap.add_argument("--batch", type=int, default=None,
                     help="replace the workload's batch size (a smaller case of the same shape, for profiling)")
     ap.add_argument("--op", choices=["fwd", "bwd"], default="fwd",
@@ -501,13 +696,23 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU work of the oracle baseline sample")
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds for the reference arm's steps")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="host logic of the ranks only (gloo group, shards, MAX reduction), no GPU")
+    argv = sys.argv[1:] if argv is None else list(argv)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        spawn_ranks(args.gpus, argv)
+        return
+    if args.dry_run:
+        run_dry(args)
+    elif args.impl == "reference":
         run_reference(args)
     elif args.op == "bwd":
         run_bwd(args)
+    elif si.WORKLOADS[args.workload]["kind"] == "r2l":
+        run_r2l(args)
     else:
         run_ours(args)
 

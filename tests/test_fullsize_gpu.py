@@ -63,10 +63,16 @@ def test_fullsize_sampled(ssd, name):
 
 
 def test_r2l_workload_all_steps(ssd):
-    """The R2L sidecar decode workload: 256 denoising steps, fresh seeded inputs per step."""
+    """The R2L sidecar decode workload: 256 denoising steps, fresh seeded inputs per step.
+
+    Each step is checked twice: the full output (residual + gate * reverse scan), and the scan
+    alone (zero residual and no D), where the SSD term is the whole output and cannot hide
+    behind the residual."""
     w = si.WORKLOADS["r2l_block_L32"]
     shape, chunk = w["shape"], w["chunk"]
-    worst = 0.0
+    zero = torch.zeros(shape.batch, shape.seqlen, shape.nheads * shape.headdim, dtype=torch.bfloat16, device="cuda")
+    zero64 = np.zeros(zero.shape)
+    worst = worst_ssd = 0.0
     for step in range(w["steps"]):
         p = si.make_params(shape, seed=0, offset=si.STEP_STRIDE * step + si.REV_OFFSET)
         res = si.make_residual(shape, seed=0, step=step)
@@ -74,4 +80,12 @@ def test_r2l_workload_all_steps(ssd):
         out = ssd.r2l_block_scan(_dev(p), gate, res.torch("cuda"), chunk=chunk)
         ref = oracle.r2l_block_f64(oracle.params_f64(p), gate, res.f64())
         worst = max(worst, oracle.rel_err(out.double().cpu().numpy(), ref))
+        q = si.make_params(shape, seed=0, offset=si.STEP_STRIDE * step + si.REV_OFFSET, with_D=False)
+        o2 = ssd.r2l_block_scan(_dev(q, False), gate, zero, chunk=chunk)
+        ref2 = oracle.r2l_block_f64(oracle.params_f64(q), gate, zero64)
+        if gate != 0:
+            worst_ssd = max(worst_ssd, oracle.rel_err(o2.double().cpu().numpy(), ref2))
+        else:
+            assert not o2.any(), f"step {step}: gate 0 must give the zero residual back"
     assert worst <= 2e-2
+    assert worst_ssd <= 2e-2

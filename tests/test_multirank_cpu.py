@@ -95,3 +95,26 @@ def test_traffic_record_is_keyed_on_the_current_kernel(tmp_path):
     assert bench.profiled_traffic("k", "w", str(tmp_path)) == 123
     assert bench.profiled_traffic("k2", "w", str(tmp_path)) is None
     assert bench.profiled_traffic("k", "other", str(tmp_path)) is None
+
+
+def test_bench_gpus_flag_spawns_ranks():
+    """``bench.py --gpus 2`` outside torchrun starts two rank processes itself.  The dry run goes
+    through the same spawn path and process-group setup on gloo: two ranks, their own seeds,
+    the same per-rank work, and the slowest rank's time in the line."""
+    import json
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dry-run",
+                        "--warmup", "3"], capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout                     # rank 0 alone prints
+    out = json.loads(lines[0])
+    assert out["n_ranks"] == 2
+    ranks = sorted(tuple(x) for x in out["ranks"])
+    assert [x[0] for x in ranks] == [0, 1]
+    assert ranks[0][1] != ranks[1][1]                    # independent sequences per rank
+    assert ranks[0][2] == ranks[1][2]                    # the same work per rank: weak scaling
+    assert out["max_time"] == 2.0                        # rank 1 reports 2.0, the slowest
+    assert out["tokens_all"] == 2 * ranks[0][2]

@@ -43,26 +43,32 @@ def _bidir_case(ssd, shape, chunk, with_D, seed=0):
 
 
 SHAPES = [
-    # (batch, L, H, P, N, G, io), chunk
-    (si.Shape(1, 64, 2, 16, 16, 1, "f32"), 16),            # the tiny float32 workload
-    (si.Shape(2, 512, 8, 64, 128, 1, "bf16"), 256),        # layer shape, tensor-core path, 4 blocks
-    (si.Shape(1, 128, 8, 64, 128, 1, "bf16"), 128),        # tensor-core path, a single block
-    (si.Shape(3, 384, 16, 64, 128, 1, "bf16"), 128),       # tensor-core path, odd block count, 8 head pairs
-    (si.Shape(1, 1280, 24, 64, 128, 1, "bf16"), 256),      # tensor-core path, 10 blocks, 12 head pairs
-    (si.Shape(1, 768, 6, 64, 128, 1, "bf16"), 256),        # SIMT path (6 heads), odd chunk count
-    (si.Shape(3, 384, 4, 64, 128, 1, "bf16"), 128),        # SIMT path, 3 chunks of 128
-    (si.Shape(2, 256, 4, 32, 64, 1, "bf16"), 64),
-    (si.Shape(1, 256, 4, 16, 16, 1, "bf16"), 16),
-    (si.Shape(2, 192, 4, 64, 64, 2, "bf16"), 64),          # two groups
-    (si.Shape(1, 96, 3, 16, 32, 1, "f32"), 32),
-    (si.Shape(2, 256, 2, 64, 128, 1, "f32"), 128),
+    # (batch, L, H, P, N, G, io), chunk, path the call must take (1 tensor core, 0 SIMT)
+    (si.Shape(1, 64, 2, 16, 16, 1, "f32"), 16, 0),            # the tiny float32 workload
+    (si.Shape(2, 512, 8, 64, 128, 1, "bf16"), 256, 1),        # layer shape, tensor-core path, 4 blocks
+    (si.Shape(1, 128, 8, 64, 128, 1, "bf16"), 128, 1),        # tensor-core path, a single block
+    (si.Shape(3, 384, 16, 64, 128, 1, "bf16"), 128, 1),       # tensor-core path, odd block count, 8 head pairs
+    (si.Shape(1, 1280, 24, 64, 128, 1, "bf16"), 256, 1),      # tensor-core path, 10 blocks, 12 head pairs
+    (si.Shape(1, 768, 6, 64, 128, 1, "bf16"), 256, 0),        # SIMT path (6 heads), odd chunk count
+    (si.Shape(3, 384, 4, 64, 128, 1, "bf16"), 128, 0),        # SIMT path, 3 chunks of 128
+    (si.Shape(2, 256, 4, 32, 64, 1, "bf16"), 64, 0),
+    (si.Shape(1, 256, 4, 16, 16, 1, "bf16"), 16, 0),
+    (si.Shape(2, 192, 4, 64, 64, 2, "bf16"), 64, 0),          # two groups
+    (si.Shape(1, 96, 3, 16, 32, 1, "f32"), 32, 0),
+    (si.Shape(2, 256, 2, 64, 128, 1, "f32"), 128, 0),
 ]
 
 
-@pytest.mark.parametrize("shape,chunk", SHAPES, ids=lambda v: str(v) if isinstance(v, int) else
+def _dims(shape):
+    return (shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate, shape.ngroups)
+
+
+@pytest.mark.parametrize("shape,chunk,path", SHAPES, ids=lambda v: str(v) if isinstance(v, int) else
                          f"b{v.batch}L{v.seqlen}H{v.nheads}P{v.headdim}N{v.dstate}G{v.ngroups}{v.io}")
 @pytest.mark.parametrize("with_D", [True, False], ids=["full", "ssd_only"])
-def test_bidir_parity(ssd, shape, chunk, with_D):
+def test_bidir_parity(ssd, shape, chunk, path, with_D):
+    io = torch.bfloat16 if shape.io == "bf16" else torch.float32
+    assert ssd.path_for(_dims(shape), io, chunk) == path
     err = _bidir_case(ssd, shape, chunk, with_D)
     assert err <= TOL[shape.io], f"rel err {err:.3e}"
 

@@ -25,12 +25,19 @@ pytestmark = pytest.mark.gpu
 TOL = {"bf16": 2e-2, "f32": 1e-4}
 
 CASES = [
-    # shape, chunk, split points (token indices)
-    (si.Shape(2, 512, 8, 64, 128, 1, "bf16"), 256, [256]),          # tensor-core path, block-aligned
-    (si.Shape(1, 768, 8, 64, 128, 1, "bf16"), 128, [128, 512]),     # tensor-core path, three pieces
-    (si.Shape(2, 96, 4, 32, 64, 1, "bf16"), 32, [32, 64]),          # SIMT, single-chunk pieces
-    (si.Shape(1, 64, 2, 16, 16, 1, "f32"), 16, [16]),               # SIMT float32
+    # shape, chunk, split points (token indices), path of the whole-sequence call (1 tensor core,
+    # 0 SIMT)
+    (si.Shape(2, 512, 8, 64, 128, 1, "bf16"), 256, [256], 1),          # tensor-core path, block-aligned
+    (si.Shape(1, 768, 8, 64, 128, 1, "bf16"), 128, [128, 512], 1),     # tensor-core path, three pieces
+    (si.Shape(2, 96, 4, 32, 64, 1, "bf16"), 32, [32, 64], 0),          # SIMT, single-chunk pieces
+    (si.Shape(1, 64, 2, 16, 16, 1, "f32"), 16, [16], 0),               # SIMT float32
 ]
+
+
+def _path(ssd, shape, chunk, lo=0, hi=None):
+    io = torch.bfloat16 if shape.io == "bf16" else torch.float32
+    n = shape.seqlen if hi is None else hi - lo
+    return ssd.path_for((shape.batch, n, shape.nheads, shape.headdim, shape.dstate, shape.ngroups), io, chunk)
 
 
 @pytest.fixture(scope="module")
@@ -56,9 +63,10 @@ def _oracle(q, direction, s0=None):
     return oracle.ssd_scan_state_f64(q["x"], q["dt"], q["A"], q["B"], q["C"], q.get("D"), direction, s0)
 
 
-@pytest.mark.parametrize("shape,chunk,splits", CASES, ids=_ids)
+@pytest.mark.parametrize("shape,chunk,splits,path", CASES, ids=_ids)
 @pytest.mark.parametrize("direction", [1, -1])
-def test_pieces_carry_the_state(ssd, shape, chunk, splits, direction):
+def test_pieces_carry_the_state(ssd, shape, chunk, splits, path, direction):
+    assert _path(ssd, shape, chunk) == path
     p = si.make_params(shape, seed=31, with_D=False)
     dev = torch.device("cuda")
     d = {k: getattr(p, k).torch(dev) for k in ("x", "dt", "A", "B", "C")}
@@ -72,6 +80,7 @@ def test_pieces_carry_the_state(ssd, shape, chunk, splits, direction):
     state = None
     ys = {}
     for lo, hi in pieces:
+        assert _path(ssd, shape, chunk, lo, hi) == path       # every piece takes the same path
         y, state = ssd.ssd_scan_state(**_dev_piece(d, lo, hi), direction=direction, chunk=chunk, state_in=state)
         ys[lo] = y
     torch.cuda.synchronize()
@@ -80,9 +89,10 @@ def test_pieces_carry_the_state(ssd, shape, chunk, splits, direction):
     assert oracle.rel_err(state.double().cpu().numpy(), s_ref) <= TOL[shape.io]
 
 
-@pytest.mark.parametrize("shape,chunk,splits", CASES, ids=_ids)
+@pytest.mark.parametrize("shape,chunk,splits,path", CASES, ids=_ids)
 @pytest.mark.parametrize("direction", [1, -1])
-def test_scan_from_a_given_state(ssd, shape, chunk, splits, direction):
+def test_scan_from_a_given_state(ssd, shape, chunk, splits, path, direction):
+    assert _path(ssd, shape, chunk) == path
     p = si.make_params(shape, seed=32, with_D=True)
     dev = torch.device("cuda")
     d = {k: getattr(p, k).torch(dev) for k in ("x", "dt", "A", "B", "C", "D")}
@@ -101,6 +111,7 @@ def test_scan_from_a_given_state(ssd, shape, chunk, splits, direction):
 
 def test_no_state_in_matches_ssd_scan(ssd):
     shape = si.Shape(2, 512, 8, 64, 128, 1, "bf16")
+    assert _path(ssd, shape, 256) == 1
     p = si.make_params(shape, seed=33)
     d = {k: getattr(p, k).torch("cuda") for k in ("x", "dt", "A", "B", "C", "D")}
     for direction in (1, -1):

@@ -39,12 +39,14 @@ def _rel(a, b):
     return ((a.float() - b.float()).abs().max() / b.float().abs().max().clamp_min(1e-30)).item()
 
 
-@pytest.mark.parametrize("dims,chunk", [
-    ((2, 1024, 8, 64, 128, 1), 256),     # tensor-core path, 8 blocks of 128 rows per sequence
-    ((1, 384, 4, 64, 128, 1), 128),      # tensor-core path, 3 blocks
-    ((2, 96, 4, 32, 64, 1), 32),         # SIMT path (headdim 32), three chunks
+@pytest.mark.parametrize("dims,chunk,path", [
+    ((2, 1024, 8, 64, 128, 1), 256, 1),     # tensor-core path, 8 blocks of 128 rows per sequence
+    ((1, 384, 8, 64, 128, 1), 128, 1),      # tensor-core path, 3 blocks
+    ((1, 384, 4, 64, 128, 1), 128, 0),      # SIMT path (4 heads), 3 chunks
+    ((2, 96, 4, 32, 64, 1), 32, 0),         # SIMT path (headdim 32), three chunks
 ])
-def test_matches_workspace_entry_point_twice(ssd, dims, chunk):
+def test_matches_workspace_entry_point_twice(ssd, dims, chunk, path):
+    assert ssd.path_for(dims, torch.bfloat16, chunk) == path
     shape = si.Shape(*dims, "bf16")
     pf, pr = si.make_bidir(shape, seed=11)
     f, r = _dev(pf), _dev(pr)
@@ -72,6 +74,7 @@ def test_matches_workspace_entry_point_twice(ssd, dims, chunk):
 
 def test_allocates_nothing(ssd):
     dims, chunk = (1, 512, 8, 64, 128, 1), 256
+    assert ssd.path_for(dims, torch.bfloat16, chunk) == 1
     pf, pr = si.make_bidir(si.Shape(*dims, "bf16"), seed=5)
     f, r = _dev(pf), _dev(pr)
     out = torch.empty_like(f["x"])
