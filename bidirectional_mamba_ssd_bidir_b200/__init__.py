@@ -25,7 +25,7 @@ import os
 import torch
 
 __all__ = ["ssd_scan", "ssd_scan_state", "ssd_scan_bwd", "bidir_ssd", "r2l_block_scan", "bidir_ssd_noalloc", "noalloc_status", "NoallocArea", "workspace_bytes", "path_for",
-           "kernel_launches", "workspace_status", "SSDError", "library_path", "lib"]
+           "segments_for", "kernel_launches", "workspace_status", "SSDError", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libbidirssd.so")
@@ -59,6 +59,8 @@ lib.ssd_path_for.argtypes = [_SP, ctypes.c_int]
 lib.ssd_path_for.restype = ctypes.c_int
 lib.ssd_kernel_launches.argtypes = [_SP, ctypes.c_int, ctypes.c_int]
 lib.ssd_kernel_launches.restype = ctypes.c_int
+lib.ssd_segments_for.argtypes = [_SP, ctypes.c_int]
+lib.ssd_segments_for.restype = ctypes.c_int
 lib.ssd_scan.argtypes = [_SP, _PP, ctypes.c_int, ctypes.c_int, _VP, _VP, _SZ, _VP]
 lib.ssd_scan.restype = ctypes.c_int
 lib.bidir_ssd.argtypes = [_SP, _PP, _PP, ctypes.c_int, _VP, _VP, _SZ, _VP]
@@ -151,6 +153,12 @@ def path_for(shape: tuple, io: torch.dtype, chunk: int) -> int:
     """1 = tensor-core path, 0 = SIMT path, -1 = refused."""
     s = _Shape(*shape, SSD_BF16 if io == torch.bfloat16 else SSD_F32)
     return int(lib.ssd_path_for(ctypes.byref(s), int(chunk)))
+
+
+def segments_for(shape: tuple, io: torch.dtype, chunk: int) -> int:
+    """Segments per sequence on the tensor-core path (1 = none), 0 on the SIMT path, -1 = refused."""
+    s = _Shape(*shape, SSD_BF16 if io == torch.bfloat16 else SSD_F32)
+    return int(lib.ssd_segments_for(ctypes.byref(s), int(chunk)))
 
 
 def kernel_launches(shape: tuple, io: torch.dtype, chunk: int, op: str) -> int:

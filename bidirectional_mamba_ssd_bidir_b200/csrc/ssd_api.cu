@@ -101,9 +101,15 @@ int choose_path(const ssd_shape *s, int chunk) {
                              s->ngroups, chunk) ? 1 : 0;
 }
 
-size_t path_ws_bytes(const ssd_shape *s, int chunk) {
+// Segments per sequence on the tensor-core path (1 when segmenting is not allowed).
+int tc_nseg(const ssd_shape *s, bool segments) {
+    return segments ? ssd::tc_segments(s->batch, s->seqlen, s->nheads) : 1;
+}
+
+size_t path_ws_bytes(const ssd_shape *s, int chunk, bool segments = true) {
     if (choose_path(s, chunk) == 1)
-        return kStatusBytes + round_up(ssd::tc_workspace_bytes(s->batch, s->seqlen, s->nheads, chunk));
+        return kStatusBytes +
+               round_up(ssd::tc_workspace_bytes(s->batch, s->seqlen, s->nheads, chunk, tc_nseg(s, segments)));
     return simt_ws_bytes(s, chunk);
 }
 
@@ -125,13 +131,14 @@ ssd::ScanArgs make_args(const ssd_shape *s, const ssd_params *p, int dir, int ch
 // Validates the shape and, for a non-empty problem, the output and workspace.
 // *empty is set when there is nothing to compute (batch or seqlen zero): the
 // call then succeeds without looking at any pointer.
-ssd_status common_checks(const ssd_shape *s, int chunk, void *out, void *ws, size_t ws_bytes, bool *empty) {
+ssd_status common_checks(const ssd_shape *s, int chunk, void *out, void *ws, size_t ws_bytes, bool *empty,
+                         bool segments = true) {
     ssd_status st = check_shape(s, chunk);
     if (st != SSD_OK) return st;
     *empty = s->batch == 0 || s->seqlen == 0;
     if (*empty) return SSD_OK;
     if (!aligned16(out)) return fail(SSD_ERR_INVALID_ARG, "output must be non-NULL and 16-byte aligned");
-    const size_t need = path_ws_bytes(s, chunk);
+    const size_t need = path_ws_bytes(s, chunk, segments);
     if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)))
         return fail(SSD_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
     if (ws_bytes < need) return fail(SSD_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", ws_bytes, need);
@@ -148,6 +155,34 @@ ssd_status run_simt(const ssd_shape *s, const ssd_params *p, int dir, int chunk,
     return e == cudaSuccess ? SSD_OK : cuda_fail(e, "SIMT scan launch");
 }
 
+// The bidirectional mixer; `segments` lets the tensor-core path cut sequences into segments
+// (the no-allocation entry point keeps one CTA per sequence: its scratch is fixed).
+ssd_status bidir_run(const ssd_shape *shape, const ssd_params *fwd, const ssd_params *rev, int chunk, void *y,
+                     void *workspace, size_t workspace_bytes, void *stream, bool segments) {
+    g_err.clear();
+    bool empty = false;
+    ssd_status st = common_checks(shape, chunk, y, workspace, workspace_bytes, &empty, segments);
+    if (st != SSD_OK || empty) return st;
+    if ((st = check_params(fwd, "forward")) != SSD_OK) return st;
+    if ((st = check_params(rev, "reverse")) != SSD_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (choose_path(shape, chunk) == 1) {
+        ssd::TcArgs t = ssd::make_tc_args(shape->batch, shape->seqlen, shape->nheads, chunk,
+                                          static_cast<char *>(workspace) + kStatusBytes,
+                                          static_cast<int *>(workspace));
+        t.wait_cycles = wait_cycles_now();
+        t.fault = g_fault.load();
+        t.nseg = tc_nseg(shape, segments);
+        ssd::tc_set_direction(t, 0, 1, fwd->x, fwd->dt, fwd->A, fwd->B, fwd->C, fwd->D);
+        ssd::tc_set_direction(t, 1, -1, rev->x, rev->dt, rev->A, rev->B, rev->C, rev->D);
+        cudaError_t e = ssd::launch_tc(t, /*bidir=*/true, y, cs);
+        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "tensor-core bidirectional launch");
+    }
+    st = run_simt(shape, fwd, 1, chunk, y, workspace, ssd::OUT_WRITE, nullptr, 0.f, cs);
+    if (st != SSD_OK) return st;
+    return run_simt(shape, rev, -1, chunk, y, workspace, ssd::OUT_ACCUM, nullptr, 0.f, cs);
+}
+
 }  // namespace
 
 extern "C" {
@@ -162,11 +197,16 @@ int ssd_path_for(const ssd_shape *shape, int chunk) {
     return choose_path(shape, chunk);
 }
 
+int ssd_segments_for(const ssd_shape *shape, int chunk) {
+    if (check_shape(shape, chunk) != SSD_OK) return -1;
+    return choose_path(shape, chunk) == 1 ? tc_nseg(shape, true) : 0;
+}
+
 int ssd_kernel_launches(const ssd_shape *shape, int chunk, int op) {
     if (check_shape(shape, chunk) != SSD_OK || op < 0 || op > 2) return -1;
     if (shape->batch == 0 || shape->seqlen == 0) return 0;
     const int dirs = op == 1 ? 2 : 1;
-    if (op != 2 && choose_path(shape, chunk) == 1) return ssd::tc_launches(op == 1);
+    if (op != 2 && choose_path(shape, chunk) == 1) return ssd::tc_launches(op == 1, tc_nseg(shape, true));
     return dirs * (shape->seqlen / chunk > 1 ? 3 : 1);
 }
 
@@ -289,27 +329,7 @@ ssd_status ssd_scan_bwd(const ssd_shape *shape, const ssd_params *p, int directi
 
 ssd_status bidir_ssd(const ssd_shape *shape, const ssd_params *fwd, const ssd_params *rev, int chunk, void *y,
                      void *workspace, size_t workspace_bytes, void *stream) {
-    g_err.clear();
-    bool empty = false;
-    ssd_status st = common_checks(shape, chunk, y, workspace, workspace_bytes, &empty);
-    if (st != SSD_OK || empty) return st;
-    if ((st = check_params(fwd, "forward")) != SSD_OK) return st;
-    if ((st = check_params(rev, "reverse")) != SSD_OK) return st;
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (choose_path(shape, chunk) == 1) {
-        ssd::TcArgs t = ssd::make_tc_args(shape->batch, shape->seqlen, shape->nheads, chunk,
-                                          static_cast<char *>(workspace) + kStatusBytes,
-                                          static_cast<int *>(workspace));
-        t.wait_cycles = wait_cycles_now();
-        t.fault = g_fault.load();
-        ssd::tc_set_direction(t, 0, 1, fwd->x, fwd->dt, fwd->A, fwd->B, fwd->C, fwd->D);
-        ssd::tc_set_direction(t, 1, -1, rev->x, rev->dt, rev->A, rev->B, rev->C, rev->D);
-        cudaError_t e = ssd::launch_tc(t, /*bidir=*/true, y, cs);
-        return e == cudaSuccess ? SSD_OK : cuda_fail(e, "tensor-core bidirectional launch");
-    }
-    st = run_simt(shape, fwd, 1, chunk, y, workspace, ssd::OUT_WRITE, nullptr, 0.f, cs);
-    if (st != SSD_OK) return st;
-    return run_simt(shape, rev, -1, chunk, y, workspace, ssd::OUT_ACCUM, nullptr, 0.f, cs);
+    return bidir_run(shape, fwd, rev, chunk, y, workspace, workspace_bytes, stream, true);
 }
 
 ssd_status r2l_block_scan(const ssd_shape *shape, const ssd_params *p, float s, const void *residual, int chunk,
@@ -411,7 +431,7 @@ ssd_status bidir_ssd_noalloc(const ssd_shape *shape, const ssd_params *fwd, cons
     ssd_status st = check_shape(shape, chunk);
     if (st != SSD_OK) return st;
     if (shape->batch == 0 || shape->seqlen == 0) return SSD_OK;
-    const size_t need = path_ws_bytes(shape, chunk);
+    const size_t need = path_ws_bytes(shape, chunk, /*segments=*/false);
     if (need > (size_t)SSD_NOALLOC_MAX_SCRATCH_BYTES)
         return fail(SSD_ERR_UNSUPPORTED,
                     "this shape needs %zu bytes of scratch, more than the %zu the no-allocation entry point "
@@ -423,7 +443,7 @@ ssd_status bidir_ssd_noalloc(const ssd_shape *shape, const ssd_params *fwd, cons
     const size_t clear = choose_path(shape, chunk) == 1 ? need : kStatusBytes;
     cudaError_t e = cudaMemsetAsync(ws, 0, clear, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "scratch clear");
-    st = bidir_ssd(shape, fwd, rev, chunk, y, ws, (size_t)SSD_NOALLOC_MAX_SCRATCH_BYTES, stream);
+    st = bidir_run(shape, fwd, rev, chunk, y, ws, (size_t)SSD_NOALLOC_MAX_SCRATCH_BYTES, stream, false);
     if (st == SSD_OK && status_area) *status_area = ws;
     return st;
 }

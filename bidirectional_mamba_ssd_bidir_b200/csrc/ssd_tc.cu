@@ -762,15 +762,57 @@ bool tc_supported(bool bf16, int batch, int L, int H, int P, int N, int G, int c
            L % kBlk == 0 && (long long)batch * L <= (1ll << 31) - 1 && get_encode() != nullptr;
 }
 
-size_t tc_workspace_bytes(int batch, int L, int H, int) {
-    // epoch-tagged ticket and ready words per (batch, head, block), then the epoch-tagged
-    // word that tells the exact kernel some chain was left to it
-    return 2 * sizeof(unsigned long long) * (size_t)batch * H * (L / kBlk) + sizeof(unsigned long long);
+int tc_segments(int batch, int L, int H) {
+    // CTAs of a bidirectional call without segments: one per (batch row, head pair, direction)
+    constexpr int kTargetCtas = 148;                  // one wave on a B200
+    const long long units = (long long)batch * H;
+    const int nblk = L / kBlk;
+    if (units <= 0 || nblk < 4) return 1;
+    long long k = kTargetCtas / units;
+    if (k > nblk / 2) k = nblk / 2;
+    if (k > 16) k = 16;
+    if (k < 2) return 1;
+    // no empty segment: the count that the segment length implies
+    const int sb = (nblk + (int)k - 1) / (int)k;
+    return (nblk + sb - 1) / sb;
 }
+
+int tc_segment_blocks(int L, int nseg) {
+    const int nblk = L / kBlk;
+    return nseg > 1 ? (nblk + nseg - 1) / nseg : nblk;
+}
+
+namespace {
+size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+// Workspace: epoch-tagged ticket and ready words per (batch, head, block), the epoch-tagged
+// word that tells the exact kernel some chain was left to it; with segments, the steep marks,
+// the per-segment decays and local end states.
+struct TcLayout {
+    size_t ticket, ready, deferred, steep, ldec, sloc, total;
+};
+TcLayout tc_layout(int batch, int L, int H, int nseg) {
+    TcLayout o{};
+    const size_t nflags = (size_t)batch * H * (L / kBlk);
+    o.ticket = 0;
+    o.ready = nflags * 8;
+    o.deferred = 2 * nflags * 8;
+    o.total = round256(o.deferred + 8);
+    if (nseg > 1) {
+        o.steep = o.total;
+        o.ldec = round256(o.steep + (size_t)batch * (H / 2) * 2 * 8);
+        o.sloc = round256(o.ldec + (size_t)batch * H * 2 * nseg * 4);
+        o.total = round256(o.sloc + (size_t)batch * H * 2 * nseg * kP * kN * 4);
+    }
+    return o;
+}
+}  // namespace
+
+size_t tc_workspace_bytes(int batch, int L, int H, int, int nseg) { return tc_layout(batch, L, H, nseg).total; }
 
 TcArgs make_tc_args(int batch, int L, int H, int chunk, void *ws, int *status) {
     TcArgs t{};
     t.batch = batch; t.L = L; t.H = H; t.chunk = chunk; t.ws = ws; t.status = status;
+    t.nseg = tc_segments(batch, L, H);
     return t;
 }
 
@@ -780,19 +822,30 @@ void tc_set_direction(TcArgs &t, int slot, int dir, const void *x, const void *d
 }
 
 // Every call runs the shared-score kernel and then the exact kernel for the chains it left
-// (which returns at once when there are none).
-int tc_launches(bool) { return 2; }
+// (which returns at once when there are none); a segmented call runs the segment-state kernel
+// first.
+int tc_launches(bool, int nseg) { return nseg > 1 ? 3 : 2; }
 
 
 
 cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
-    const size_t nflags = (size_t)t.batch * t.H * (t.L / kBlk);
-    unsigned long long *ticket = static_cast<unsigned long long *>(t.ws);
-    unsigned long long *ready = ticket + nflags;
-    unsigned long long *deferred = ready + nflags;
+    const int nseg = t.nseg > 1 ? t.nseg : 1;
+    const TcLayout lo = tc_layout(t.batch, t.L, t.H, nseg);
+    char *ws = static_cast<char *>(t.ws);
+    unsigned long long *ticket = reinterpret_cast<unsigned long long *>(ws + lo.ticket);
+    unsigned long long *ready = reinterpret_cast<unsigned long long *>(ws + lo.ready);
+    unsigned long long *deferred = reinterpret_cast<unsigned long long *>(ws + lo.deferred);
+    SegScratch sc{};
+    if (nseg > 1) {
+        sc.sloc = reinterpret_cast<float *>(ws + lo.sloc);
+        sc.ldec = reinterpret_cast<float *>(ws + lo.ldec);
+        sc.steep = reinterpret_cast<unsigned long long *>(ws + lo.steep);
+    }
     const unsigned long long epoch = next_epoch();
     const bool with_state = !bidir && (t.s_in || t.s_out);
-    cudaError_t e = launch_tcs(t, bidir, y, ticket, ready, deferred, epoch, st);
+    cudaError_t e = cudaSuccess;
+    if (nseg > 1 && (e = launch_segstate(t, bidir, sc, epoch, st)) != cudaSuccess) return e;
+    e = launch_tcs(t, bidir, y, ticket, ready, deferred, sc, epoch, st);
     if (e != cudaSuccess) return e;
     // The shared-memory opt-in belongs to the kernel in the current context: set on every launch.
     cudaError_t attr_err =

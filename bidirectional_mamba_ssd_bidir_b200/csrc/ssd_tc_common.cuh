@@ -347,11 +347,33 @@ __device__ __forceinline__ unsigned long long ld_acquire(const unsigned long lon
 // block's mid-point keeps every row and column factor within 2^+-(this/2).
 constexpr float kSteepLog2 = 150.f;
 
-// True if, for head h0 or h0 + 1 of batch row b, some 128-token block has
-// |A_h| * log2(e) * sum(dt) above kSteepLog2.  Called by every thread of the
-// CTA (nthreads of them, thread index tid); uses one int of shared memory;
-// returns the same answer in every thread.  Both tensor-core kernels call this
-// same function on the same inputs, so they take the same decision.
+// True if, in memory block blk (128 tokens) of batch row b, head h0 or h0 + 1 has
+// |A_h| * log2(e) * sum(dt) above kSteepLog2 (a0, a1: |A| * log2(e) of the two
+// heads), or a non-number.  Called by the 32 lanes of one warp; every lane gets
+// the answer.  This one function is the test on every path that decides it, so
+// they all take the same decision for every block.
+__device__ __forceinline__ bool block_is_steep(const __nv_bfloat16 *dt, float a0, float a1, int b, int L, int H,
+                                               int h0, int blk, int lane) {
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const size_t t = (size_t)b * L + (size_t)blk * 128 + lane + 32 * i;
+        const uint32_t u = *reinterpret_cast<const uint32_t *>(dt + t * H + h0);
+        s0 += bf16lo(u);
+        s1 += bf16hi(u);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+    }
+    return (a0 * s0 > kSteepLog2) || (a1 * s1 > kSteepLog2) || !(s0 == s0) || !(s1 == s1);
+}
+
+// True if, for head h0 or h0 + 1 of batch row b, some 128-token block is steep
+// (block_is_steep).  Called by every thread of the CTA (nthreads of them,
+// thread index tid); uses one int of shared memory; returns the same answer in
+// every thread.
 __device__ __forceinline__ bool chain_is_steep(const __nv_bfloat16 *dt, const float *A, int b, int L, int H, int h0,
                                                int tid, int nthreads, int *flag) {
     constexpr float kLog2e = 1.4426950408889634f;
@@ -361,22 +383,7 @@ __device__ __forceinline__ bool chain_is_steep(const __nv_bfloat16 *dt, const fl
     const float a0 = fabsf(A[h0]) * kLog2e, a1 = fabsf(A[h0 + 1]) * kLog2e;
     const int nblk = L / 128;
     bool steep = false;
-    for (int blk = warp; blk < nblk; blk += nwarps) {
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const size_t t = (size_t)b * L + (size_t)blk * 128 + lane + 32 * i;
-            const uint32_t u = *reinterpret_cast<const uint32_t *>(dt + t * H + h0);
-            s0 += bf16lo(u);
-            s1 += bf16hi(u);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            s0 += __shfl_xor_sync(0xffffffffu, s0, o);
-            s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-        }
-        steep |= (a0 * s0 > kSteepLog2) || (a1 * s1 > kSteepLog2) || !(s0 == s0) || !(s1 == s1);
-    }
+    for (int blk = warp; blk < nblk; blk += nwarps) steep |= block_is_steep(dt, a0, a1, b, L, H, h0, blk, lane);
     if (steep && lane == 0) atomicOr(flag, 1);
     __syncthreads();
     return *reinterpret_cast<volatile int *>(flag) != 0;

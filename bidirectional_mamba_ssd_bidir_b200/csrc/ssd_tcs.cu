@@ -174,6 +174,12 @@ struct TcsParams {
     int fault;                          // test hook: 1 = the first direction never publishes its part
     const float *s_in;                  // single direction: [batch][H][P][N] state entering the scan, or null
     float *s_out;                       // single direction: [batch][H][P][N] state leaving the scan, or null
+    // sequence segments (nseg > 1): a CTA runs sb blocks of its chain; the state entering its
+    // segment folds the local end states of the segments before it
+    int nseg, sb;
+    const float *sloc;                  // [batch][H][2][nseg][P][N]
+    const float *ldec;                  // [batch][H][2][nseg]: A * (sum of dt over the segment), log2 units
+    const unsigned long long *steep;    // [batch][H/2][2], epoch-tagged: chains left to the exact kernel
 };
 
 struct TcsMaps {
@@ -196,15 +202,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
     const int unit = prm.bidir ? (blockIdx.x >> 1) : blockIdx.x;
     const int slot = prm.bidir ? (blockIdx.x & 1) : 0;
     const int dir = prm.bidir ? (slot == 0 ? 1 : -1) : prm.dir_single;
-    const int b = unit / npairs, hp = unit % npairs;
+    const int seg = unit % prm.nseg, pu = unit / prm.nseg;
+    const int b = pu / npairs, hp = pu % npairs;
     const int h0 = 2 * hp;
-    const int nblk = prm.nblk, L = prm.L;
+    const int nblk_chain = prm.nblk, L = prm.L;
+    // this CTA's blocks: scan-order blocks g0 .. g0 + nblk - 1 of the chain
+    const int g0 = seg * prm.sb;
+    const int nblk = min(prm.sb, nblk_chain - g0);
     const CUtensorMap *map_x = &maps.x[slot], *map_dt = &maps.dt[slot], *map_b = &maps.b[slot],
                       *map_c = &maps.c[slot];
-    const int has_in = prm.s_in != nullptr;   // a state enters the scan (single direction only)
+    // a state enters this CTA's blocks: the caller's (single direction), or a segment's before it
+    const int has_in = prm.s_in != nullptr || seg > 0;
+    float *const s_out = seg == prm.nseg - 1 ? prm.s_out : nullptr;   // left by the chain's last segment
 
-    // A chain with a block too steep for the factorised decay is left to the exact kernel.
-    if (chain_is_steep(prm.d[slot].dt, prm.d[slot].A, b, L, prm.H, h0, threadIdx.x, kThreads, steep_flag)) {
+    // A chain with a block too steep for the factorised decay is left to the exact kernel.  With
+    // segments, the segment-state kernel has run the test on every block of the chain.
+    const bool steep = prm.nseg > 1
+        ? *reinterpret_cast<const volatile unsigned long long *>(prm.steep + ((size_t)b * npairs + hp) * 2 + slot) ==
+              prm.epoch
+        : chain_is_steep(prm.d[slot].dt, prm.d[slot].A, b, L, prm.H, h0, threadIdx.x, kThreads, steep_flag);
+    if (nblk <= 0) return;
+    if (steep) {
         if (threadIdx.x == 0) *reinterpret_cast<volatile unsigned long long *>(prm.deferred) = prm.epoch;
         return;
     }
@@ -234,7 +252,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
     const uint32_t tmem = *tmem_slot;
     SSD_TRACE_CTA(0);
 
-    auto row_of = [&](int jj) { return b * L + (dir > 0 ? jj : nblk - 1 - jj) * kBlk; };
+    // memory block of this CTA's block jj, and its first token row
+    auto mblk_of = [&](int jj) { return dir > 0 ? g0 + jj : nblk_chain - 1 - (g0 + jj); };
+    auto row_of = [&](int jj) { return b * L + mblk_of(jj) * kBlk; };
     if (warp == kWarpLoad) {
         // ---------------------------------------------------------- TMA loads, tables
         // Lane 0 issues the loads as their buffers free up: x of block j once block j-2's
@@ -525,8 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
             bool ok = true;
             for (int j = 0; j < nblk && ok; ++j) {
                 const int st = j & 1;
-                const int cm = dir > 0 ? j : nblk - 1 - j;
-                const size_t pair_slot = ((size_t)b * prm.H + h0) * nblk + cm;
+                const int cm = mblk_of(j);
+                const size_t pair_slot = ((size_t)b * prm.H + h0) * nblk_chain + cm;
                 int sec = 0;
                 if (prm.bidir) {
                     sec = atomicExch(prm.ticket + pair_slot, prm.epoch) == prm.epoch;
@@ -709,10 +729,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
         const size_t sslot = ((size_t)b * prm.H + h) * kP * kN;
         // state entering the scan: scaled by e^{m_0} into TMEM, with its bf16 copy for block 0's Y_off
         auto init_pass = [&]() {
-            const float f = ex2_ftz(tab_s[kTabM2 + hs]);
             float sv[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sv[i] = prm.s_in[sslot + (size_t)(32 * ch + i) * kN + r] * f;
+            for (int i = 0; i < 32; ++i) sv[i] = prm.s_in ? prm.s_in[sslot + (size_t)(32 * ch + i) * kN + r] : 0.f;
+            // S_in(s) = exp(A T_{s-1}) S_in(s-1) + S_loc(s-1), from the first segment on
+            const size_t chain = ((size_t)b * prm.H + h) * 2 + slot;
+            for (int s2 = 0; s2 < seg; ++s2) {
+                const float d2 = ex2_ftz(prm.ldec[chain * prm.nseg + s2]);
+                const float *sl = prm.sloc + (chain * prm.nseg + s2) * kP * kN;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sv[i] = sv[i] * d2 + sl[(size_t)(32 * ch + i) * kN + r];
+            }
+            const float f = ex2_ftz(tab_s[kTabM2 + hs]);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[i] *= f;
             tmem_st32f_nw(tl + kColS + 32 * g, sv);
             uint8_t *stile = sm + kOffS + hs * kTileBytes;
 #pragma unroll
@@ -757,7 +787,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                 // j-1's products had read the stage: placed here, the load has most of a block)
                 if (!cx_pass(j + 1)) break;
                 SSD_TRACE_PT(warp, j, 6);
-            } else if (prm.s_out) {
+            } else if (s_out) {
                 // state leaving the scan: S_out = kappa_last * S (after the last state product)
                 if (!mbar_wait(bar(B_STFULL), j & 1, MASK, abort_flag, prm.status, 49)) break;
                 tc_fence_after();
@@ -765,12 +795,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                 float sv[32];
                 tmem_ld32(tl + kColS + 32 * g, sv);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) prm.s_out[sslot + (size_t)(32 * ch + i) * kN + r] = sv[i] * f;
+                for (int i = 0; i < 32; ++i) s_out[sslot + (size_t)(32 * ch + i) * kN + r] = sv[i] * f;
             }
             // (4) epilogue: y = r Y_j in bf16 into this block's B buffer, which G and the state
             // product have consumed (the state product's completion was awaited in (2), or here
             // for the last block); the store warp writes the tiles to y
-            if (j + 1 == nblk && !prm.s_out && !mbar_wait(bar(B_STFULL), j & 1, MASK, abort_flag, prm.status, 49))
+            if (j + 1 == nblk && !s_out && !mbar_wait(bar(B_STFULL), j & 1, MASK, abort_flag, prm.status, 49))
                 break;
             if (!mbar_wait(bar(B_YFULL), j & 1, MASK, abort_flag, prm.status, 46)) break;
             SSD_TRACE_PT(warp, j, 7);
@@ -835,7 +865,7 @@ extern "C" int ssd_debug_trace(unsigned long long *out, int n) {
 // Launches the shared-score kernel for the chains it can run.  *deferred (in the
 // workspace) is set to `epoch` by any CTA whose chain it left to the exact kernel.
 cudaError_t launch_tcs(const TcArgs &t, bool bidir, void *y, unsigned long long *ticket, unsigned long long *ready,
-                       unsigned long long *deferred, unsigned long long epoch, cudaStream_t st) {
+                       unsigned long long *deferred, const SegScratch &sc, unsigned long long epoch, cudaStream_t st) {
     // The shared-memory opt-in belongs to the kernel in the current context: set on every launch
     // (a host-side call), so it holds in any context the caller makes current.
     cudaError_t e = cudaFuncSetAttribute(k_ssd_tcs, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
@@ -869,7 +899,12 @@ cudaError_t launch_tcs(const TcArgs &t, bool bidir, void *y, unsigned long long 
     p.fault = t.fault;
     p.s_in = bidir ? nullptr : t.s_in;
     p.s_out = bidir ? nullptr : t.s_out;
-    const int grid = t.batch * (t.H / 2) * ndir;
+    p.nseg = t.nseg > 1 ? t.nseg : 1;
+    p.sb = tc_segment_blocks(t.L, p.nseg);
+    p.sloc = sc.sloc;
+    p.ldec = sc.ldec;
+    p.steep = sc.steep;
+    const int grid = t.batch * (t.H / 2) * p.nseg * ndir;
     k_ssd_tcs<<<grid, kThreads, kSmemBytes, st>>>(maps, p);
     return cudaGetLastError();
 }

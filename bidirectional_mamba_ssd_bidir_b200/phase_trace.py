@@ -56,7 +56,7 @@ def library(force_build: bool = False) -> ctypes.CDLL:
     if _trace_lib is None or force_build:
         path = _build.build(force=force_build, trace=True)
         t = ctypes.CDLL(path)
-        for name in ("bidir_ssd", "ssd_workspace_bytes", "ssd_workspace_status"):
+        for name in ("bidir_ssd", "ssd_workspace_bytes", "ssd_workspace_status", "ssd_segments_for"):
             getattr(t, name).argtypes = getattr(_lib, name).argtypes
             getattr(t, name).restype = getattr(_lib, name).restype
         t.ssd_debug_trace.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int]
@@ -96,7 +96,8 @@ def run(fwd: dict, rev: dict, chunk: int = 256):
     cbuf = (ctypes.c_ulonglong * (3 * N_CTA_SLOTS))()
     if t.ssd_debug_cta_times(cbuf, 3 * N_CTA_SLOTS) != N_CTA_SLOTS:
         raise RuntimeError("could not read the CTA times")
-    ncta = min(N_CTA_SLOTS, 2 * shape.batch * (shape.nheads // 2))
+    nseg = max(1, int(t.ssd_segments_for(ctypes.byref(shape), int(chunk))))
+    ncta = min(N_CTA_SLOTS, 2 * shape.batch * (shape.nheads // 2) * nseg)
     ctas = np.array(cbuf[:], dtype=np.int64).reshape(N_CTA_SLOTS, 3)[:ncta]
     return y, phases, ctas
 

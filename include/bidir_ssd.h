@@ -225,6 +225,17 @@ ssd_status ssd_debug_fault(int mode, double wait_limit_seconds);
  * 1 = tensor-core (tcgen05) path, 0 = SIMT path, -1 = refused. */
 int ssd_path_for(const ssd_shape *shape, int chunk);
 
+/* Segments each sequence is cut into on the tensor-core path (SSD / Mamba-2
+ * state passing, "DiffuMamba" technical summary section 2: the scan is linear
+ * in its state, so a sequence split into runs of whole 128-token blocks is
+ * scanned run by run in parallel from the states the runs before it leave).
+ * A call cuts its sequences when batch x heads gives fewer CTAs than the GPU
+ * has SMs: a first kernel forms each segment's local end state, the scan then
+ * runs every segment from the state folded from those before it.  1 = one CTA
+ * walks each whole sequence; 0 on the SIMT path; -1 if the shape is refused.
+ * bidir_ssd_noalloc never segments. */
+int ssd_segments_for(const ssd_shape *shape, int chunk);
+
 #ifdef __cplusplus
 }
 #endif

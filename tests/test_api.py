@@ -133,3 +133,9 @@ def test_python_binding_checks_dtypes():
     with pytest.raises(TypeError):
         ssd.ssd_scan(x, torch.zeros(1, 16, 2), torch.zeros(2), torch.zeros(1, 16, 1, 16),
                      torch.zeros(1, 16, 1, 16), chunk=16)
+
+
+def test_segment_query():
+    # float32 and small head dims take the SIMT path, which never segments; refused shapes say -1
+    assert ssd.segments_for((1, 64, 2, 16, 16, 1), torch.float32, 16) == 0
+    assert ssd.segments_for((1, 60, 2, 16, 16, 1), torch.float32, 16) == -1
