@@ -152,7 +152,7 @@ def _kernel_source_hash() -> str:
     unchanged kernel; the nvcc architecture and flags are part of the key."""
     h = hashlib.sha256()
     pkg = os.path.join(ROOT, "bidirectional_mamba_ssd_bidir_b200")
-    for f in ("ssd_tcs.cu", "ssd_tc.cu", "ssd_tc.cuh", "ssd_tc_common.cuh"):
+    for f in ("ssd_tcs.cu", "ssd_tcs_seg.cu", "ssd_tc.cu", "ssd_tc.cuh", "ssd_tc_common.cuh"):
         h.update(_code_only(open(os.path.join(pkg, "csrc", f), encoding="utf-8").read()).encode())
     import importlib.util
     spec = importlib.util.spec_from_file_location("_ssd_build_flags", os.path.join(pkg, "build.py"))

@@ -173,6 +173,7 @@ ssd_status bidir_run(const ssd_shape *shape, const ssd_params *fwd, const ssd_pa
         t.wait_cycles = wait_cycles_now();
         t.fault = g_fault.load();
         t.nseg = tc_nseg(shape, segments);
+        t.npiece = ssd::tc_state_pieces(shape->batch, shape->seqlen, shape->nheads, t.nseg);
         ssd::tc_set_direction(t, 0, 1, fwd->x, fwd->dt, fwd->A, fwd->B, fwd->C, fwd->D);
         ssd::tc_set_direction(t, 1, -1, rev->x, rev->dt, rev->A, rev->B, rev->C, rev->D);
         cudaError_t e = ssd::launch_tc(t, /*bidir=*/true, y, cs);

@@ -762,9 +762,12 @@ bool tc_supported(bool bf16, int batch, int L, int H, int P, int N, int G, int c
            L % kBlk == 0 && (long long)batch * L <= (1ll << 31) - 1 && get_encode() != nullptr;
 }
 
+namespace {
+constexpr int kTargetCtas = 148;                      // one wave on a B200
+}
+
 int tc_segments(int batch, int L, int H) {
     // CTAs of a bidirectional call without segments: one per (batch row, head pair, direction)
-    constexpr int kTargetCtas = 148;                  // one wave on a B200
     const long long units = (long long)batch * H;
     const int nblk = L / kBlk;
     if (units <= 0 || nblk < 4) return 1;
@@ -782,6 +785,22 @@ int tc_segment_blocks(int L, int nseg) {
     return nseg > 1 ? (nblk + nseg - 1) / nseg : nblk;
 }
 
+int tc_state_pieces(int batch, int L, int H, int nseg) {
+    if (nseg <= 1) return 0;
+    const int sb = tc_segment_blocks(L, nseg);
+    const long long per_piece = (long long)batch * H * (nseg - 1);   // state CTAs per piece of a segment
+    long long m = kTargetCtas / per_piece;
+    if (m < 1) m = 1;
+    if (m > sb) m = sb;
+    const int pb = (sb + (int)m - 1) / (int)m;
+    return (sb + pb - 1) / pb;                          // no empty piece
+}
+
+int tc_piece_blocks(int L, int nseg, int npiece) {
+    const int sb = tc_segment_blocks(L, nseg);
+    return npiece > 0 ? (sb + npiece - 1) / npiece : sb;
+}
+
 namespace {
 size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 // Workspace: epoch-tagged ticket and ready words per (batch, head, block), the epoch-tagged
@@ -791,6 +810,7 @@ struct TcLayout {
     size_t ticket, ready, deferred, steep, ldec, sloc, total;
 };
 TcLayout tc_layout(int batch, int L, int H, int nseg) {
+    const int npieces = nseg > 1 ? (nseg - 1) * tc_state_pieces(batch, L, H, nseg) : 0;
     TcLayout o{};
     const size_t nflags = (size_t)batch * H * (L / kBlk);
     o.ticket = 0;
@@ -800,8 +820,8 @@ TcLayout tc_layout(int batch, int L, int H, int nseg) {
     if (nseg > 1) {
         o.steep = o.total;
         o.ldec = round256(o.steep + (size_t)batch * (H / 2) * 2 * 8);
-        o.sloc = round256(o.ldec + (size_t)batch * H * 2 * nseg * 4);
-        o.total = round256(o.sloc + (size_t)batch * H * 2 * nseg * kP * kN * 4);
+        o.sloc = round256(o.ldec + (size_t)batch * H * 2 * npieces * 4);
+        o.total = round256(o.sloc + (size_t)batch * H * 2 * npieces * kP * kN * 4);
     }
     return o;
 }
@@ -813,6 +833,7 @@ TcArgs make_tc_args(int batch, int L, int H, int chunk, void *ws, int *status) {
     TcArgs t{};
     t.batch = batch; t.L = L; t.H = H; t.chunk = chunk; t.ws = ws; t.status = status;
     t.nseg = tc_segments(batch, L, H);
+    t.npiece = tc_state_pieces(batch, L, H, t.nseg);
     return t;
 }
 

@@ -22,12 +22,13 @@ struct TcArgs {
     const float *s_in;       // single direction only: [batch][H][P][N] state entering the scan, or null
     float *s_out;            // single direction only: [batch][H][P][N] state leaving the scan, or null
     int nseg;                // segments per sequence (1: one CTA walks the whole sequence)
+    int npiece;              // pieces each segment's local end state is formed in (nseg > 1)
 };
 
 // Scratch of a segmented call, inside the path workspace.
 struct SegScratch {
-    float *sloc;                        // [batch][H][2][nseg][P][N] local end states
-    float *ldec;                        // [batch][H][2][nseg] A * (sum of dt per segment), log2 units
+    float *sloc;                        // [batch][H][2][(nseg - 1) npiece][P][N] pieces' local end states
+    float *ldec;                        // [batch][H][2][(nseg - 1) npiece] A * (sum of dt per piece), log2
     unsigned long long *steep;          // [batch][H/2][2] epoch-tagged steep-chain marks
 };
 
@@ -37,6 +38,10 @@ bool tc_supported(bool bf16, int batch, int L, int H, int P, int N, int G, int c
 int tc_segments(int batch, int L, int H);
 // Blocks per segment (the last segment may be shorter).
 int tc_segment_blocks(int L, int nseg);
+// Pieces each of the first nseg - 1 segments is formed in by the segment-state kernel, and
+// blocks per piece (a segment's last piece may be shorter).
+int tc_state_pieces(int batch, int L, int H, int nseg);
+int tc_piece_blocks(int L, int nseg, int npiece);
 size_t tc_workspace_bytes(int batch, int L, int H, int chunk, int nseg);
 TcArgs make_tc_args(int batch, int L, int H, int chunk, void *ws, int *status);
 void tc_set_direction(TcArgs &t, int slot, int dir, const void *x, const void *dt, const float *A,

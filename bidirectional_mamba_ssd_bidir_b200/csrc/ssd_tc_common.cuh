@@ -347,20 +347,20 @@ __device__ __forceinline__ unsigned long long ld_acquire(const unsigned long lon
 // block's mid-point keeps every row and column factor within 2^+-(this/2).
 constexpr float kSteepLog2 = 150.f;
 
-// True if, in memory block blk (128 tokens) of batch row b, head h0 or h0 + 1 has
-// |A_h| * log2(e) * sum(dt) above kSteepLog2 (a0, a1: |A| * log2(e) of the two
-// heads), or a non-number.  Called by the 32 lanes of one warp; every lane gets
-// the answer.  This one function is the test on every path that decides it, so
-// they all take the same decision for every block.
-__device__ __forceinline__ bool block_is_steep(const __nv_bfloat16 *dt, float a0, float a1, int b, int L, int H,
-                                               int h0, int blk, int lane) {
+// The steep-decay test of one 128-token block from its dt values: u[i] holds
+// the bf16 pair (dt of head h0, dt of head h0 + 1) of the block's row
+// lane + 32 i.  True if, for either head, |A_h| * log2(e) * sum(dt) is above
+// kSteepLog2 (a0, a1: |A| * log2(e) of the two heads), or a sum is not a
+// number.  Called by the 32 lanes of one warp; every lane gets the answer.
+// Every path that decides which kernel takes a chain reaches this one
+// function with the same values in the same lanes, so they all sum in the same
+// order and take the same decision for every block.
+__device__ __forceinline__ bool steep_of_block(const uint32_t u[4], float a0, float a1) {
     float s0 = 0.f, s1 = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const size_t t = (size_t)b * L + (size_t)blk * 128 + lane + 32 * i;
-        const uint32_t u = *reinterpret_cast<const uint32_t *>(dt + t * H + h0);
-        s0 += bf16lo(u);
-        s1 += bf16hi(u);
+        s0 += bf16lo(u[i]);
+        s1 += bf16hi(u[i]);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -368,6 +368,18 @@ __device__ __forceinline__ bool block_is_steep(const __nv_bfloat16 *dt, float a0
         s1 += __shfl_xor_sync(0xffffffffu, s1, o);
     }
     return (a0 * s0 > kSteepLog2) || (a1 * s1 > kSteepLog2) || !(s0 == s0) || !(s1 == s1);
+}
+
+// steep_of_block for memory block blk of batch row b, read from global memory.
+__device__ __forceinline__ bool block_is_steep(const __nv_bfloat16 *dt, float a0, float a1, int b, int L, int H,
+                                               int h0, int blk, int lane) {
+    uint32_t u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const size_t t = (size_t)b * L + (size_t)blk * 128 + lane + 32 * i;
+        u[i] = *reinterpret_cast<const uint32_t *>(dt + t * H + h0);
+    }
+    return steep_of_block(u, a0, a1);
 }
 
 // True if, for head h0 or h0 + 1 of batch row b, some 128-token block is steep

@@ -175,10 +175,10 @@ struct TcsParams {
     const float *s_in;                  // single direction: [batch][H][P][N] state entering the scan, or null
     float *s_out;                       // single direction: [batch][H][P][N] state leaving the scan, or null
     // sequence segments (nseg > 1): a CTA runs sb blocks of its chain; the state entering its
-    // segment folds the local end states of the segments before it
-    int nseg, sb;
-    const float *sloc;                  // [batch][H][2][nseg][P][N]
-    const float *ldec;                  // [batch][H][2][nseg]: A * (sum of dt over the segment), log2 units
+    // segment folds the local end states of the pieces (npiece per segment) before it
+    int nseg, sb, npiece;
+    const float *sloc;                  // [batch][H][2][(nseg - 1) npiece][P][N]
+    const float *ldec;                  // [batch][H][2][(nseg - 1) npiece]: A * (sum of dt), log2 units
     const unsigned long long *steep;    // [batch][H/2][2], epoch-tagged: chains left to the exact kernel
 };
 
@@ -732,11 +732,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
             float sv[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) sv[i] = prm.s_in ? prm.s_in[sslot + (size_t)(32 * ch + i) * kN + r] : 0.f;
-            // S_in(s) = exp(A T_{s-1}) S_in(s-1) + S_loc(s-1), from the first segment on
+            // S_in <- exp(A T_piece) S_in + S_loc(piece), over the pieces of the segments before
+            // this one, in scan order
             const size_t chain = ((size_t)b * prm.H + h) * 2 + slot;
-            for (int s2 = 0; s2 < seg; ++s2) {
-                const float d2 = ex2_ftz(prm.ldec[chain * prm.nseg + s2]);
-                const float *sl = prm.sloc + (chain * prm.nseg + s2) * kP * kN;
+            const int npieces = (prm.nseg - 1) * prm.npiece;
+            for (int s2 = 0; s2 < seg * prm.npiece; ++s2) {
+                const float d2 = ex2_ftz(prm.ldec[chain * npieces + s2]);
+                const float *sl = prm.sloc + (chain * npieces + s2) * kP * kN;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) sv[i] = sv[i] * d2 + sl[(size_t)(32 * ch + i) * kN + r];
             }
@@ -901,6 +903,7 @@ cudaError_t launch_tcs(const TcArgs &t, bool bidir, void *y, unsigned long long 
     p.s_out = bidir ? nullptr : t.s_out;
     p.nseg = t.nseg > 1 ? t.nseg : 1;
     p.sb = tc_segment_blocks(t.L, p.nseg);
+    p.npiece = t.npiece;
     p.sloc = sc.sloc;
     p.ldec = sc.ldec;
     p.steep = sc.steep;

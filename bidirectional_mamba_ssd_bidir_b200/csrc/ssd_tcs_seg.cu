@@ -20,15 +20,20 @@
 // block is reached, so one accumulator sums B^T (w x) over the whole segment on
 // the tensor core with no rescaling and nothing that can overflow.
 //
-// One CTA per (batch row, head pair, direction, segment).  Every CTA also runs
-// the steep-decay test (block_is_steep, the one the other kernels use) on its
-// segment's blocks and marks the chain steep in the workspace, so that the
-// scan and the exact kernel agree on which chains the exact kernel takes.  The
-// last segment's CTA does only that (nothing needs its local state).
+// Each segment but the last (nothing needs the last one's local state) is
+// formed in npiece pieces of consecutive blocks, so that the kernel has about
+// as many CTAs as the GPU has SMs: one CTA per (batch row, head pair,
+// direction, piece).  The scan folds the pieces in order.  The CTAs also run
+// the steep-decay test (steep_of_block, the one the other kernels use) on
+// every block of the chain, their own pieces' blocks from the dt tiles they
+// load and a share of the last segment's from global memory, and mark the
+// chain steep in the workspace: the scan and the exact kernel then agree on
+// which chains the exact kernel takes.
 //
-// Warps (320 threads): warp 0 loads x, B and dt (TMA) into three stages; warp 1
-// owns TMEM and issues the MMAs; warps 2-9 weight the rows of x in place (warp
-// 2 + 4 hs + q: head hs, rows 32 q .. 32 q + 31) and read the result out.
+// Warps (576 threads): warp 0 loads x, B and dt (TMA) into three stages; warp 1
+// owns TMEM and issues the MMAs; warps 2-17 weight the rows of x in place
+// (warp 2 + 8 hs + 2 q + c: head hs, rows 32 q .. 32 q + 31, 16-byte chunks
+// 4 c .. 4 c + 3) and read the result out.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -43,7 +48,8 @@ namespace ssd {
 namespace {
 
 constexpr int kBlk = 128, kP = 64, kN = 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
+constexpr int kCw = 16;                                 // weighting warps
 constexpr int kStages = 3;
 constexpr uint32_t kTileBytes = kBlk * 64 * 2;          // [128][64] bf16, 128-byte swizzled
 constexpr uint32_t kPairBytes = 2 * kTileBytes;
@@ -52,7 +58,7 @@ constexpr uint32_t kDtBytes = kBlk * 8 * 2;             // dt box: 128 tokens x 
 constexpr uint32_t kStX = 0, kStB = kPairBytes, kStDt = 2 * kPairBytes;
 constexpr uint32_t kStageBytes = (2 * kPairBytes + kDtBytes + 1023) / 1024 * 1024;
 constexpr uint32_t kOffTab = kStages * kStageBytes;     // per weighting warp: w of the block's 128 rows
-constexpr uint32_t kOffBar = kOffTab + 8 * kBlk * 4;
+constexpr uint32_t kOffBar = kOffTab + kCw * kBlk * 4;
 enum Bar { B_FULL0 = 0, B_EMPTY0 = B_FULL0 + kStages, B_WREADY0 = B_EMPTY0 + kStages, B_DONE = B_WREADY0 + kStages,
            kNumBars };
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;   // tmem slot, abort flag, wait limit
@@ -61,11 +67,11 @@ static_assert(kStageBytes % 1024 == 0 && kSmemBytes <= 232448, "shared memory la
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct SegParams {
-    int batch, L, H, nblk, nseg, sb, bidir, dir_single;
+    int batch, L, H, nblk, nseg, sb, npiece, pb, bidir, dir_single;
     const float *A[2];
     const __nv_bfloat16 *dt[2];
-    float *sloc;                        // [batch][H][2][nseg][P][N]
-    float *ldec;                        // [batch][H][2][nseg]: A T_s, log2 units
+    float *sloc;                        // [batch][H][2][(nseg - 1) npiece][P][N]
+    float *ldec;                        // [batch][H][2][(nseg - 1) npiece]: A T over the piece, log2 units
     unsigned long long *steep;          // [batch][H/2][2], epoch-tagged
     unsigned long long epoch;
     int *status;
@@ -88,32 +94,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_segstate(const __grid_const
     const int slot = prm.bidir ? (blockIdx.x & 1) : 0;
     const int dir = prm.bidir ? (slot == 0 ? 1 : -1) : prm.dir_single;
     const int unit = prm.bidir ? (blockIdx.x >> 1) : blockIdx.x;
-    const int seg = unit % prm.nseg, pu = unit / prm.nseg;
+    const int npieces = (prm.nseg - 1) * prm.npiece;   // pieces of a chain
+    const int piece = unit % npieces, pu = unit / npieces;
     const int npairs = prm.H / 2;
     const int b = pu / npairs, hp = pu % npairs, h0 = 2 * hp;
     const int nblk = prm.nblk, L = prm.L;
-    const int g0 = seg * prm.sb;
-    const int nb = min(prm.sb, nblk - g0);
+    // this piece: scan-order blocks g0 .. g0 + nb - 1 of segment piece / npiece
+    const int g0 = (piece / prm.npiece) * prm.sb + (piece % prm.npiece) * prm.pb;
+    const int nb = min(prm.pb, (piece / prm.npiece + 1) * prm.sb - g0);
     // memory block of scan block g
     auto mblk = [&](int g) { return dir > 0 ? g : nblk - 1 - g; };
+    const float a0 = fabsf(prm.A[slot][h0]) * kLog2e, a1 = fabsf(prm.A[slot][h0 + 1]) * kLog2e;
+    unsigned long long *steep_mark = prm.steep + ((size_t)b * npairs + hp) * 2 + slot;
 
-    // steep-decay test of this segment's blocks (warps 2-9, a block each in turn)
+    // steep-decay test of this CTA's share of the last segment's blocks (the pieces' own blocks
+    // are tested from their dt tiles below)
     if (warp >= 2) {
-        const float a0 = fabsf(prm.A[slot][h0]) * kLog2e, a1 = fabsf(prm.A[slot][h0 + 1]) * kLog2e;
         bool steep = false;
-        for (int i = warp - 2; i < nb; i += 8)
-            steep |= block_is_steep(prm.dt[slot], a0, a1, b, L, prm.H, h0, mblk(g0 + i), lane);
-        if (steep && lane == 0)
-            *reinterpret_cast<volatile unsigned long long *>(prm.steep + ((size_t)b * npairs + hp) * 2 + slot) =
-                prm.epoch;
+        for (int g = (prm.nseg - 1) * prm.sb + piece + npieces * (warp - 2); g < nblk; g += npieces * kCw)
+            steep |= block_is_steep(prm.dt[slot], a0, a1, b, L, prm.H, h0, mblk(g), lane);
+        if (steep && lane == 0) *reinterpret_cast<volatile unsigned long long *>(steep_mark) = prm.epoch;
     }
-    if (seg == prm.nseg - 1 || nb <= 0) return;        // nothing needs the last segment's local state
+    if (nb <= 0) return;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         *reinterpret_cast<volatile long long *>(abort_flag + 1) = prm.wait_cycles;
         for (int i = 0; i < (int)kNumBars; ++i)
-            mbar_init(bar(i), (i >= B_WREADY0 && i < B_WREADY0 + kStages) ? 8 : 1);
+            mbar_init(bar(i), (i >= B_WREADY0 && i < B_WREADY0 + kStages) ? kCw : 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -170,12 +178,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_segstate(const __grid_const
         __syncwarp();
     } else {
         // ---------------------------------------------------------- weights w, rows of x scaled in place
-        const int cw = warp - 2, hs = cw >> 2, q = cw & 3;
+        const int cw = warp - 2, hs = cw >> 3, q = (cw >> 1) & 3, c4 = cw & 1;
         const int h = h0 + hs;
         const float A2 = prm.A[slot][h] * kLog2e;        // log2 units, <= 0
         float *tab = reinterpret_cast<float *>(sm + kOffTab) + cw * kBlk;
-        float carry = 0.f;                               // sum of dt over the blocks after this one
-        bool ok = true;
+        float carry = 0.f;                               // sum of dt over the piece's blocks after this one
+        bool ok = true, steep = false;
         for (int i = 0; i < nb && ok; ++i) {
             const int st = i % kStages;
             if (!mbar_wait(bar(B_FULL0 + st), (i / kStages) & 1, MASK, abort_flag, prm.status, 84)) {
@@ -183,9 +191,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_segstate(const __grid_const
                 break;
             }
             uint8_t *base = sm + st * kStageBytes;
+            const uint8_t *dtt = base + kStDt;           // [128 rows][8 heads] bf16
+            if (i % kCw == cw) {
+                // the steep test of this block, from the tile: row lane + 32 i of the block
+                uint32_t u[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    u[e] = *reinterpret_cast<const uint32_t *>(dtt + (lane + 32 * e) * 16 + (h0 & 7) * 2);
+                steep |= steep_of_block(u, a0, a1);
+            }
             // dt of this head at scan positions 4 lane .. 4 lane + 3 (memory row k forward,
             // 127 - k reverse); suffix sums in scan order
-            const uint8_t *dtt = base + kStDt;
             float d[4];
             int rows[4];
 #pragma unroll
@@ -212,12 +228,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_segstate(const __grid_const
             }
             carry += total;
             __syncwarp();
-            // this warp's rows of its head's x tile, scaled by w in place (fp32 multiply, one rounding)
+            // this warp's rows and chunks of its head's x tile, scaled by w in place (fp32 multiply,
+            // one rounding)
             const int r = q * 32 + lane;
             const float w = tab[r];
             uint8_t *xt = base + kStX + hs * kTileBytes;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int cc = 0; cc < 4; ++cc) {
+                const int c = 4 * c4 + cc;
                 const uint4 v = *reinterpret_cast<const uint4 *>(xt + swz(r, c));
                 const uint32_t xw[4] = {v.x, v.y, v.z, v.w};
                 uint32_t o[4];
@@ -229,20 +247,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_segstate(const __grid_const
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_WREADY0 + st));
         }
-        // read out: TMEM lane quarter warp % 4 (rows n), columns of head hs (p)
+        if (steep && lane == 0) *reinterpret_cast<volatile unsigned long long *>(steep_mark) = prm.epoch;
+        // read out: TMEM lane quarter warp % 4 (rows n), 32 columns of group cw >> 2 (head, p half)
         if (ok && mbar_wait(bar(B_DONE), 0, MASK, abort_flag, prm.status, 85)) {
             tc_fence_after();
-            const int n = (warp & 3) * 32 + lane;
-            const uint32_t ta = tmem + ((uint32_t)((warp & 3) * 32) << 16) + hs * 64;
+            const int n = (warp & 3) * 32 + lane, cg = cw >> 2;
+            const int ho = cg >> 1, p0 = (cg & 1) * 32;
             float v[32];
-            const size_t chain = ((size_t)b * prm.H + h) * 2 + slot;
-            float *out = prm.sloc + (chain * prm.nseg + seg) * kP * kN;
-            for (int half = 0; half < 2; ++half) {
-                tmem_ld32(ta + 32 * half, v);
+            tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + 32 * cg, v);
+            const size_t chain = ((size_t)b * prm.H + h0 + ho) * 2 + slot;
+            float *out = prm.sloc + (chain * npieces + piece) * kP * kN;
 #pragma unroll
-                for (int p = 0; p < 32; ++p) out[(size_t)(32 * half + p) * kN + n] = v[p];
-            }
-            if (q == 0 && lane == 0) prm.ldec[chain * prm.nseg + seg] = A2 * carry;
+            for (int p = 0; p < 32; ++p) out[(size_t)(p0 + p) * kN + n] = v[p];
+            if ((cw & 7) == 0 && lane == 0) prm.ldec[(((size_t)b * prm.H + h) * 2 + slot) * npieces + piece] = A2 * carry;
         }
     }
 
@@ -276,13 +293,14 @@ cudaError_t launch_segstate(const TcArgs &t, bool bidir, const SegScratch &sc, u
     }
     p.batch = t.batch; p.L = t.L; p.H = t.H; p.nblk = t.L / kBlk;
     p.nseg = t.nseg; p.sb = tc_segment_blocks(t.L, t.nseg);
+    p.npiece = t.npiece; p.pb = tc_piece_blocks(t.L, t.nseg, t.npiece);
     p.bidir = bidir ? 1 : 0;
     p.dir_single = t.d[0].dir;
     p.sloc = sc.sloc; p.ldec = sc.ldec; p.steep = sc.steep;
     p.epoch = epoch;
     p.status = t.status;
     p.wait_cycles = t.wait_cycles;
-    const int grid = t.batch * (t.H / 2) * t.nseg * ndir;
+    const int grid = t.batch * (t.H / 2) * (t.nseg - 1) * t.npiece * ndir;
     k_ssd_segstate<<<grid, kThreads, kSmemBytes, st>>>(maps, p);
     return cudaGetLastError();
 }
