@@ -57,10 +57,11 @@ constexpr uint32_t kDtBytes = kBlk * 8 * 2;             // dt box: 128 tokens x 
 // stage: x (two heads) | B (two n halves) | dt
 constexpr uint32_t kStX = 0, kStB = kPairBytes, kStDt = 2 * kPairBytes;
 constexpr uint32_t kStageBytes = (2 * kPairBytes + kDtBytes + 1023) / 1024 * 1024;
-constexpr uint32_t kOffTab = kStages * kStageBytes;     // per weighting warp: w of the block's 128 rows
-constexpr uint32_t kOffBar = kOffTab + kCw * kBlk * 4;
-enum Bar { B_FULL0 = 0, B_EMPTY0 = B_FULL0 + kStages, B_WREADY0 = B_EMPTY0 + kStages, B_DONE = B_WREADY0 + kStages,
-           kNumBars };
+constexpr uint32_t kOffTab = kStages * kStageBytes;     // per stage and head: w of the block's 128 rows
+constexpr uint32_t kOffBar = kOffTab + kStages * 2 * kBlk * 4;
+enum Bar { B_FULL0 = 0, B_EMPTY0 = B_FULL0 + kStages, B_WREADY0 = B_EMPTY0 + kStages,
+           B_TAB0 = B_WREADY0 + kStages,                // [stage][head]
+           B_DONE = B_TAB0 + 2 * kStages, kNumBars };
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;   // tmem slot, abort flag, wait limit
 constexpr uint32_t kSmemBytes = kOffMisc + 32 + 1024;
 static_assert(kStageBytes % 1024 == 0 && kSmemBytes <= 232448, "shared memory layout");
@@ -181,7 +182,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_segstate(const __grid_const
         const int cw = warp - 2, hs = cw >> 3, q = (cw >> 1) & 3, c4 = cw & 1;
         const int h = h0 + hs;
         const float A2 = prm.A[slot][h] * kLog2e;        // log2 units, <= 0
-        float *tab = reinterpret_cast<float *>(sm + kOffTab) + cw * kBlk;
+        // the weights of a block live with its stage: rewritten only once its stage is reloaded,
+        // after every warp has passed the block (B_WREADY, then the MMA, then B_EMPTY)
+        float *tabs = reinterpret_cast<float *>(sm + kOffTab) + hs * kBlk;
         float carry = 0.f;                               // sum of dt over the piece's blocks after this one
         bool ok = true, steep = false;
         for (int i = 0; i < nb && ok; ++i) {
@@ -200,34 +203,44 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_segstate(const __grid_const
                     u[e] = *reinterpret_cast<const uint32_t *>(dtt + (lane + 32 * e) * 16 + (h0 & 7) * 2);
                 steep |= steep_of_block(u, a0, a1);
             }
-            // dt of this head at scan positions 4 lane .. 4 lane + 3 (memory row k forward,
-            // 127 - k reverse); suffix sums in scan order
-            float d[4];
-            int rows[4];
+            float *tab = tabs + st * 2 * kBlk;
+            // one warp per head (rows 0-31, chunks 0-3) builds the head's weights: lane l holds
+            // scan positions l + 32 t (memory row k forward, 127 - k reverse); the suffix sum
+            // of position k is the later columns' totals plus the later lanes of its column
+            if ((cw & 7) == 0) {
+                float d[4];
+                int rows[4];
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                const int k = 4 * lane + t;
-                rows[t] = dir > 0 ? k : kBlk - 1 - k;
-                const __nv_bfloat16 v = *reinterpret_cast<const __nv_bfloat16 *>(dtt + rows[t] * 16 + ((h0 & 7) + hs) * 2);
-                d[t] = __bfloat162float(v);
-            }
-            const float lt = d[0] + d[1] + d[2] + d[3];
-            float incl = lt;
+                for (int t = 0; t < 4; ++t) {
+                    const int k = lane + 32 * t;
+                    rows[t] = dir > 0 ? k : kBlk - 1 - k;
+                    d[t] = __bfloat162float(
+                        *reinterpret_cast<const __nv_bfloat16 *>(dtt + rows[t] * 16 + ((h0 & 7) + hs) * 2));
+                }
+                float incl[4], col[4];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float u = __shfl_up_sync(MASK, incl, o);
-                if (lane >= o) incl += u;
-            }
-            const float total = __shfl_sync(MASK, incl, 31);
-            const float after_lane = total - incl;       // dt of the scan positions beyond this lane's four
-            float sfx = 0.f;                             // dt of this lane's positions after t
+                for (int t = 0; t < 4; ++t) {
+                    incl[t] = d[t];
 #pragma unroll
-            for (int t = 3; t >= 0; --t) {
-                tab[rows[t]] = ex2_ftz(A2 * (carry + after_lane + sfx)) * d[t];
-                sfx += d[t];
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const float u = __shfl_up_sync(MASK, incl[t], o);
+                        if (lane >= o) incl[t] += u;
+                    }
+                    col[t] = __shfl_sync(MASK, incl[t], 31);
+                }
+                float later = carry;                     // dt of the columns after t, and of the blocks after
+#pragma unroll
+                for (int t = 3; t >= 0; --t) {
+                    tab[rows[t]] = ex2_ftz(A2 * (later + col[t] - incl[t])) * d[t];
+                    later += col[t];
+                }
+                carry = later;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_TAB0 + 2 * st + hs));
+            } else if (!mbar_wait(bar(B_TAB0 + 2 * st + hs), (i / kStages) & 1, MASK, abort_flag, prm.status, 86)) {
+                ok = false;
+                break;
             }
-            carry += total;
-            __syncwarp();
             // this warp's rows and chunks of its head's x tile, scaled by w in place (fp32 multiply,
             // one rounding)
             const int r = q * 32 + lane;
