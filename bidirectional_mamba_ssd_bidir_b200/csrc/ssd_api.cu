@@ -308,7 +308,12 @@ ssd_status ssd_scan_bwd(const ssd_shape *shape, const ssd_params *p, int directi
     if (workspace_bytes < need) return fail(SSD_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", workspace_bytes, need);
     ssd::BwdArgs a{};
     a.batch = shape->batch; a.L = shape->seqlen; a.H = shape->nheads; a.P = shape->headdim; a.N = shape->dstate;
-    a.G = shape->ngroups; a.Q = chunk < 64 ? chunk : 64; a.nc = shape->seqlen / a.Q; a.dir = direction;
+    // the tensor-core shapes run the gradients in 128-position chunks on tcgen05; others in chunks
+    // of at most 64 on the CUDA cores
+    const bool tc = choose_path(shape, chunk) == 1;
+    a.G = shape->ngroups; a.Q = tc ? 128 : (chunk < 64 ? chunk : 64); a.nc = shape->seqlen / a.Q; a.dir = direction;
+    a.status = static_cast<int *>(workspace);
+    a.wait_cycles = wait_cycles_now();
     a.x = p->x; a.dt = p->dt; a.B = p->B; a.C = p->C; a.gy = gy; a.A = p->A; a.D = p->D;
     a.gx = gx; a.gdt = gdt; a.gA = gA; a.gB = gB; a.gC = gC; a.gD = gD;
     const size_t nc = a.nc, bh = (size_t)a.batch * a.H, PN = (size_t)a.P * a.N, tokh = (size_t)a.batch * a.L * a.H;

@@ -743,6 +743,9 @@ __global__ void __launch_bounds__(kT) k_bwd_reduce(BwdArgs a) {
 template <typename T, int P, int N>
 cudaError_t bwd_typed(const BwdArgs &a, cudaStream_t st) {
     const int Q = a.Q;
+    // 128-position chunks of the tensor-core shape: chunk sums and per-chunk gradients on tcgen05
+    const bool tc = Q == 128 && bwd_tc_supported(a, sizeof(T) == 2);
+    if (Q > kQm && !tc) return cudaErrorInvalidValue;
     const size_t sm1 = sizeof(float) * (128 + 2 * Q * P + 2 * Q * N);
     const size_t sm3 = sizeof(float) * ChunkSmem<P, N>::kFloats;
     cudaError_t e = cudaFuncSetAttribute(k_bwd_chunk_sums<T, P, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -750,8 +753,12 @@ cudaError_t bwd_typed(const BwdArgs &a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(k_bwd_chunk<T, P, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm3);
     if (e != cudaSuccess) return e;
-    k_bwd_chunk_sums<T, P, N><<<dim3(a.nc, a.H, a.batch), kT, sm1, st>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (tc) {
+        if ((e = launch_bwd_tc_sums(a, st)) != cudaSuccess) return e;
+    } else {
+        k_bwd_chunk_sums<T, P, N><<<dim3(a.nc, a.H, a.batch), kT, sm1, st>>>(a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     static_assert(P * N % (kT * kPassE) == 0 || P * N < kT * kPassE, "pass slicing");
     if constexpr (P * N >= kT * kPassE) {
         k_bwd_pass<P, N><<<dim3(a.H, a.batch, P * N / (kT * kPassE)), kT, 0, st>>>(a);
@@ -759,8 +766,12 @@ cudaError_t bwd_typed(const BwdArgs &a, cudaStream_t st) {
         k_bwd_pass_small<P, N><<<dim3(a.H, a.batch), kT, 0, st>>>(a);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_bwd_chunk<T, P, N><<<dim3(a.nc, a.H, a.batch), kTC, sm3, st>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (tc) {
+        if ((e = launch_bwd_tc_chunk(a, st)) != cudaSuccess) return e;
+    } else {
+        k_bwd_chunk<T, P, N><<<dim3(a.nc, a.H, a.batch), kTC, sm3, st>>>(a);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     k_bwd_dt<T><<<dim3(a.H, a.batch), kT, 0, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const size_t total = (size_t)a.batch * a.L * a.G * a.N;

@@ -65,11 +65,18 @@ struct BwdArgs {
     float *gcs, *u;          // [batch][L][H] dL/dcs and <G_k, x_k B_k^T> per token
     float *gxd;              // [batch][H][nc] per-chunk sum of <gy, x>
     float *gAp, *gDp;        // [batch][H] per-sequence parts of dA and dD
+    int *status;             // workspace status word (bounded waits of the tensor-core kernels)
+    long long wait_cycles;   // bound of every device-side wait, in SM clock cycles
 };
 
 // Launchers (defined in the kernel translation units).  All return the
 // cudaError_t of the launch.
 cudaError_t launch_simt_scan(const ScanArgs &a, bool bf16, cudaStream_t st);
 cudaError_t launch_simt_bwd(const BwdArgs &a, bool bf16, cudaStream_t st);
+// Tensor-core chunk sums and per-chunk gradients (ssd_bwd_tc.cu): bf16, P = 64, N = 128, one
+// group, 128-position chunks (a.Q == 128); launch_simt_bwd uses them in place of its own.
+bool bwd_tc_supported(const BwdArgs &a, bool bf16);
+cudaError_t launch_bwd_tc_sums(const BwdArgs &a, cudaStream_t st);
+cudaError_t launch_bwd_tc_chunk(const BwdArgs &a, cudaStream_t st);
 
 }  // namespace ssd

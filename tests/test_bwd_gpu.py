@@ -26,6 +26,10 @@ CASES = [
     (si.Shape(1, 1024, 2, 64, 128, 1, "bf16"), 128),    # 16 chunks
     (si.Shape(1, 128, 2, 64, 16, 1, "f32"), 32),         # wide x, narrow state, 32-position chunks
     (si.Shape(1, 48, 2, 32, 128, 1, "bf16"), 16),        # 16-position chunks, wide state
+    # tensor-core shapes (bf16, P 64, N 128, heads a multiple of 8): 128-position chunks on tcgen05
+    (si.Shape(2, 256, 8, 64, 128, 1, "bf16"), 256),     # 2 chunks
+    (si.Shape(1, 1024, 8, 64, 128, 1, "bf16"), 128),    # 8 chunks
+    (si.Shape(1, 384, 16, 64, 128, 1, "bf16"), 128),    # 3 chunks, 16 heads
 ]
 
 
@@ -44,6 +48,10 @@ def _ids(v):
 @pytest.mark.parametrize("direction", [1, -1])
 @pytest.mark.parametrize("with_D", [True, False], ids=["D", "noD"])
 def test_gradients_match_oracle(ssd, shape, chunk, direction, with_D):
+    dims = (shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate, shape.ngroups)
+    tc = shape.io == "bf16" and shape.headdim == 64 and shape.dstate == 128 and shape.ngroups == 1 and \
+        shape.nheads % 8 == 0 and chunk % 128 == 0
+    assert ssd.path_for(dims, torch.bfloat16 if shape.io == "bf16" else torch.float32, chunk) == (1 if tc else 0)
     p = si.make_params(shape, seed=41, with_D=with_D)
     dev = torch.device("cuda")
     d = {k: getattr(p, k).torch(dev) for k in ("x", "dt", "A", "B", "C")}
@@ -100,6 +108,7 @@ def test_gradients_at_the_bench_layer_shape(ssd):
     single-threaded oracle; the reverse direction is covered at smaller sizes)."""
     direction = 1
     shape = si.Shape(1, 8192, 64, 64, 128, 1, "bf16")
+    assert ssd.path_for((1, 8192, 64, 64, 128, 1), torch.bfloat16, 256) == 1       # tensor-core gradients
     p = si.make_params(shape, seed=43)
     d = {k: getattr(p, k).torch("cuda") for k in ("x", "dt", "A", "B", "C", "D")}
     gy = torch.randn(d["x"].shape, device="cuda", generator=torch.Generator("cuda").manual_seed(5)).to(torch.bfloat16)
