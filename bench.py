@@ -592,31 +592,51 @@ def run_bwd(args) -> None:
     ms = start.elapsed_time(end) / args.steps
     e = 2 if shape.io == "bf16" else 4
     H, P, N, G = shape.nheads, shape.headdim, shape.dstate, shape.ngroups
-    Q = min(chunk, 64)
+    path = ssd.path_for(dims, fwd["x"].dtype, chunk)
     # per token and direction: read x, dt, B, C, gy; write float32 dx, ddt, dB, dC
     bpt = 2 * (e * (2 * H * P + H + 2 * G * N) + 4 * (H * P + H + 2 * G * N))
-    # float32 multiply-adds of the chunked gradient per token, head and direction: chunk state and
-    # adjoint sums 2PN; pair matrices C.B^T and x.gy^T Q(N + P); the adjoint times B, entering
-    # part PN and causal in-chunk part QP/2; dB and dC, entering parts 2PN and causal in-chunk
-    # parts 2 QN/2
-    macs = 5 * P * N + 2 * Q * N + 1.5 * Q * P
-    fpt = 2 * 2 * H * macs                       # flops per token, both directions
     clocks = clk.summary()
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    mhz = clocks.get("sm_max_mhz") or 1965
-    peak_tf = sms * 128 * 2 * mhz * 1e6 / 1e12   # float32 FMA lanes per SM, 2 flops each
-    achieved = fpt * plan["tokens"] / (ms / 1e3) / 1e12
+    if path == 1:
+        # tensor-core chunks of Q = 128: multiply-adds per token, head and direction of the dense
+        # tiles the kernels compute (the hi/lo operand halves not counted): the pair products
+        # C.B^T, B.C^T (2 Q N) and x.gy^T, gy.x^T (2 Q P); the adjoint times gy and times B
+        # (Q P + N P); dB and dC, in-chunk and entering parts (2 Q N + 2 P N); the chunk sums
+        # (2 P N)
+        Q = 128
+        macs = 2 * Q * N + 2 * Q * P + Q * P + N * P + 2 * Q * N + 2 * P * N + 2 * P * N
+        fpt = 2 * 2 * H * macs
+        peaks = measured_peaks()
+        peak_tf = peaks["bf16_tflops"]
+        achieved = fpt * plan["tokens"] / (ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": achieved / peak_tf, "flops_per_token": fpt,
+                "peak_source": peaks["source"] + " bf16_tflops (dense, burst)",
+                "hbm_bytes_per_token": bpt, "hbm_gbs": bpt * plan["tokens"] / (ms / 1e3) / 1e9,
+                "note": "whole step: the tensor-core chunk kernels with the float32 chunk passes, "
+                        "ddt sums and reductions"}
+    else:
+        Q = min(chunk, 64)
+        # float32 multiply-adds of the chunked gradient per token, head and direction: chunk state
+        # and adjoint sums 2PN; pair matrices C.B^T and x.gy^T Q(N + P); the adjoint times B,
+        # entering part PN and causal in-chunk part QP/2; dB and dC, entering parts 2PN and causal
+        # in-chunk parts 2 QN/2
+        macs = 5 * P * N + 2 * Q * N + 1.5 * Q * P
+        fpt = 2 * 2 * H * macs                       # flops per token, both directions
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        mhz = clocks.get("sm_max_mhz") or 1965
+        peak_tf = sms * 128 * 2 * mhz * 1e6 / 1e12   # float32 FMA lanes per SM, 2 flops each
+        achieved = fpt * plan["tokens"] / (ms / 1e3) / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                "frac": achieved / peak_tf, "flops_per_token": fpt,
+                "peak_source": f"derived: {sms} SMs x 128 float32 lanes x 2 flops x {mhz} MHz",
+                "hbm_bytes_per_token": bpt, "hbm_gbs": bpt * plan["tokens"] / (ms / 1e3) / 1e9}
     line = {"metric": "bidirectional SSD scan gradients tokens/s (both directions)", "op": "bwd",
             "value": plan["tokens"] / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "f32",
             "data": "synthetic", "config": {"workload": args.workload, "global_batch": shape.batch,
-                                             "seq_len": shape.seqlen, "chunk": chunk, "path": "simt"},
-            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
-                         "frac": achieved / peak_tf, "flops_per_token": fpt,
-                         "peak_source": f"derived: {sms} SMs x 128 float32 lanes x 2 flops x {mhz} MHz",
-                         "hbm_bytes_per_token": bpt,
-                         "hbm_gbs": bpt * plan["tokens"] / (ms / 1e3) / 1e9},
-            "gpu_launches": 2 * 5 * args.steps, "clocks": clocks}
+                                             "seq_len": shape.seqlen, "chunk": chunk,
+                                             "path": "tcgen05" if path == 1 else "simt"},
+            "roofline": roof, "gpu_launches": 2 * 5 * args.steps, "clocks": clocks}
     print(json.dumps(line), flush=True)
 
 

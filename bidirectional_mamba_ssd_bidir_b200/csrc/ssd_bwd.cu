@@ -709,9 +709,10 @@ __global__ void __launch_bounds__(kT) k_bwd_dt(BwdArgs a) {
     }
 }
 
-// Step 5: dB, dC summed over the heads of each group; dA, dD summed over the batch.
+// Step 5: dB, dC summed over the heads of each group (unless the per-chunk kernel summed them
+// already: gBh null); dA, dD summed over the batch.
 __global__ void __launch_bounds__(kT) k_bwd_reduce(BwdArgs a) {
-    const size_t total = (size_t)a.batch * a.L * a.G * a.N;
+    const size_t total = a.gBh ? (size_t)a.batch * a.L * a.G * a.N : 0;
     const int per = a.H / a.G;
     for (size_t i = (size_t)blockIdx.x * kT + threadIdx.x; i < total; i += (size_t)gridDim.x * kT) {
         const int n = (int)(i % a.N);
@@ -766,17 +767,19 @@ cudaError_t bwd_typed(const BwdArgs &a, cudaStream_t st) {
         k_bwd_pass_small<P, N><<<dim3(a.H, a.batch), kT, 0, st>>>(a);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    BwdArgs ar = a;
     if (tc) {
         if ((e = launch_bwd_tc_chunk(a, st)) != cudaSuccess) return e;
+        ar.gBh = ar.gCh = nullptr;             // dB, dC already summed over the heads
     } else {
         k_bwd_chunk<T, P, N><<<dim3(a.nc, a.H, a.batch), kTC, sm3, st>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     k_bwd_dt<T><<<dim3(a.H, a.batch), kT, 0, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const size_t total = (size_t)a.batch * a.L * a.G * a.N;
+    const size_t total = ar.gBh ? (size_t)a.batch * a.L * a.G * a.N : 0;
     const int blocks = (int)((total + kT - 1) / kT < 148 * 8 ? (total + kT - 1) / kT : 148 * 8);
-    k_bwd_reduce<<<blocks > 0 ? blocks : 1, kT, 0, st>>>(a);
+    k_bwd_reduce<<<blocks > 0 ? blocks : 1, kT, 0, st>>>(ar);
     return cudaGetLastError();
 }
 

@@ -23,6 +23,11 @@
 // hi = bf16(v) and lo = bf16(v - hi), each its own MMA: about 16 significant
 // bits, so the gradients keep the float32 path's accuracy.
 //
+// dB and dC of the one B/C group are the sums over the heads: each CTA adds its head's part
+// into the (zeroed) outputs with vector float32 reductions in L2, so no per-head copy reaches
+// DRAM; the order of the additions varies, so dB and dC can differ between runs in the last
+// bits.
+//
 // Rows: a chunk is 128 consecutive tokens loaded by TMA in memory order; scan
 // position k of memory row r is r forward, 127 - r reverse.  One CTA per
 // (chunk, head, batch row); every barrier completes once (parity 0), every
@@ -54,7 +59,7 @@ struct BwdTcParams {
     const __nv_bfloat16 *dt;
     const float *A, *D;
     float *sf, *sg, *dec;                     // chunk sums in, states after the passes (per chunk)
-    float *gx, *gBh, *gCh, *gcs, *u, *gxd;
+    float *gx, *gB, *gC, *gcs, *u, *gxd;      // gB, gC: [batch][L][N], zeroed, summed over heads here
     int *status;
     long long wait_cycles;
 };
@@ -70,12 +75,23 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t 
 }
 
 // A [64 p][128 n] float32 state, row-major, into hi and lo bf16 tiles: each is two swizzled
-// [64][64] halves (n 0-63, n 64-127).  Threads tid0 .. tid0 + nthr - 1 share the work.
-__device__ __forceinline__ void stage_state(const float *src, uint8_t *hi, uint8_t *lo, int tid, int nthr) {
-    for (int i = tid; i < kP * kN / 8; i += nthr) {
+// [64][64] halves (n 0-63, n 64-127).  Threads 0 .. NTHR - 1 share the work.
+template <int NTHR>
+__device__ __forceinline__ void stage_state(const float *src, uint8_t *hi, uint8_t *lo, int tid) {
+    constexpr int kIt = kP * kN / 8 / NTHR;
+    static_assert(kIt * NTHR * 8 == kP * kN, "state staging");
+    float4 v[kIt][2];
+#pragma unroll
+    for (int it = 0; it < kIt; ++it) {      // every load in flight before the first conversion
+        const int i = tid + NTHR * it;
+        v[it][0] = *reinterpret_cast<const float4 *>(src + (size_t)i * 8);
+        v[it][1] = *reinterpret_cast<const float4 *>(src + (size_t)i * 8 + 4);
+    }
+#pragma unroll
+    for (int it = 0; it < kIt; ++it) {
+        const int i = tid + NTHR * it;
         const int p = i / (kN / 8), n8 = (i % (kN / 8)) * 8;
-        const float4 v0 = *reinterpret_cast<const float4 *>(src + (size_t)p * kN + n8);
-        const float4 v1 = *reinterpret_cast<const float4 *>(src + (size_t)p * kN + n8 + 4);
+        const float4 v0 = v[it][0], v1 = v[it][1];
         uint4 h, l;
         split2(v0.x, v0.y, h.x, l.x);
         split2(v0.z, v0.w, h.y, l.y);
@@ -259,9 +275,12 @@ constexpr uint32_t kCX = 0, kCG = kTile, kCB = 2 * kTile, kCC = 4 * kTile, kCGH 
 // tables (floats, by memory row): c2 (log2 cs), dt, exp(cl - cs), exp(cs)
 // partials [4 column groups][128]: u, red2, red2b; the diagonal <gy_k, x_k> [128]; its 4 warp sums
 constexpr uint32_t kCPart = kCTab + 4 * kQ * 4;
-constexpr uint32_t kCBar = kCPart + (3 * 4 * kQ + kQ + 4) * 4;
+// dx of the chunk, [128 rows][64 p] float32 with rows kDxS floats apart, for coalesced stores
+constexpr int kDxS = kP + 4;
+constexpr uint32_t kCDx = kCPart + (3 * 4 * kQ + kQ + 4) * 4;
+constexpr uint32_t kCBar = (kCDx + kQ * kDxS * 4 + 7) / 8 * 8;
 enum ChunkBar { CB_FULL = 0, CB_TAB, CB_SREADY, CB_PA, CB_PB, CB_C1, CB_GREAD, CB_C2, CB_DBREAD, CB_C3, CB_FIN,
-                kChunkBars };
+                CB_DX, kChunkBars };
 constexpr uint32_t kCMisc = kCBar + kChunkBars * 8;
 constexpr uint32_t kChunkSmem = kCMisc + 32 + 1024;
 constexpr int kChunkThreads = 576;             // warps 0-15 CUDA cores, 16 loads, 17 MMA
@@ -292,7 +311,7 @@ __global__ void __launch_bounds__(kChunkThreads, 1) k_bwd_tc_chunk(const __grid_
         *reinterpret_cast<volatile long long *>(abort_flag + 1) = prm.wait_cycles;
         for (int i = 0; i < kChunkBars; ++i) {
             uint32_t cnt = 1;
-            if (i == CB_SREADY || i == CB_PB || i == CB_GREAD || i == CB_DBREAD || i == CB_FIN) cnt = 16;
+            if (i == CB_SREADY || i == CB_PB || i == CB_GREAD || i == CB_DBREAD || i == CB_FIN || i == CB_DX) cnt = 16;
             mbar_init(bar(i), cnt);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -456,8 +475,8 @@ __global__ void __launch_bounds__(kChunkThreads, 1) k_bwd_tc_chunk(const __grid_
             if (lane == 0) mbar_arrive(bar(CB_TAB));
         }
         // the entering adjoint and state, split into bf16 hi and lo tiles
-        stage_state(prm.sg + slot, sm + kCGH, sm + kCGL, threadIdx.x, 512);
-        stage_state(prm.sf + slot, sm + kCSH, sm + kCSL, threadIdx.x, 512);
+        stage_state<512>(prm.sg + slot, sm + kCGH, sm + kCGL, threadIdx.x);
+        stage_state<512>(prm.sf + slot, sm + kCSH, sm + kCSL, threadIdx.x);
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(CB_SREADY));
@@ -560,13 +579,27 @@ __global__ void __launch_bounds__(kChunkThreads, 1) k_bwd_tc_chunk(const __grid_
                     }
                 }
             }
-            float *dst = prm.gx + (trow * prm.H + h) * kP + p0;
+            float *dxs = reinterpret_cast<float *>(sm + kCDx) + r * kDxS + p0;
 #pragma unroll
-            for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4 *>(dst + j) = make_float4(dx[j], dx[j + 1], dx[j + 2], dx[j + 3]);
+            for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4 *>(dxs + j) = make_float4(dx[j], dx[j + 1], dx[j + 2], dx[j + 3]);
             pu[cg * kQ + r] = uacc;
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(CB_GREAD));
+        if (lane == 0) {
+            mbar_arrive(bar(CB_GREAD));
+            mbar_arrive(bar(CB_DX));
+        }
+        // dx out: half a warp per row, 256 contiguous bytes (16 lanes x 16 bytes) per row
+        if (ok && mbar_wait(bar(CB_DX), 0, MASK, abort_flag, prm.status, 117)) {
+            const int t = threadIdx.x, c4 = 4 * (t & 15);
+            const float *dxs = reinterpret_cast<const float *>(sm + kCDx);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int rr = (t >> 4) + 32 * i;
+                const float4 v = *reinterpret_cast<const float4 *>(dxs + rr * kDxS + c4);
+                *reinterpret_cast<float4 *>(prm.gx + (((size_t)row0 + rr) * prm.H + h) * kP + c4) = v;
+            }
+        }
         // C2 read-out: dB = dt (dBa + exp(cl - cs_k) dBb) over n = 32 cg .. 32 cg + 31
         ok = ok && mbar_wait(bar(CB_C2), 0, MASK, abort_flag, prm.status, 114);
         if (ok) {
@@ -577,12 +610,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1) k_bwd_tc_chunk(const __grid_
                 float va[16], vb[16];
                 tmem_ld16(tl + kR1 + n0, va);
                 tmem_ld16(tl + kR0 + n0, vb);
-                float *dst = prm.gBh + (trow * prm.H + h) * kN + n0;
+                float *dst = prm.gB + trow * kN + n0;    // one group: summed over the heads here
 #pragma unroll
                 for (int j = 0; j < 16; j += 4)
-                    *reinterpret_cast<float4 *>(dst + j) =
-                        make_float4(dtr * fmaf(el, vb[j], va[j]), dtr * fmaf(el, vb[j + 1], va[j + 1]),
-                                    dtr * fmaf(el, vb[j + 2], va[j + 2]), dtr * fmaf(el, vb[j + 3], va[j + 3]));
+                    red_add_f32x4(dst + j, dtr * fmaf(el, vb[j], va[j]), dtr * fmaf(el, vb[j + 1], va[j + 1]),
+                                  dtr * fmaf(el, vb[j + 2], va[j + 2]), dtr * fmaf(el, vb[j + 3], va[j + 3]));
             }
             tc_fence_before();
         }
@@ -599,12 +631,11 @@ __global__ void __launch_bounds__(kChunkThreads, 1) k_bwd_tc_chunk(const __grid_
                 float va[16], vb[16];
                 tmem_ld16(tl + kR2 + n0, va);
                 tmem_ld16(tl + kR0 + n0, vb);
-                float *dst = prm.gCh + (trow * prm.H + h) * kN + n0;
+                float *dst = prm.gC + trow * kN + n0;
 #pragma unroll
                 for (int j = 0; j < 16; j += 4)
-                    *reinterpret_cast<float4 *>(dst + j) =
-                        make_float4(fmaf(ek, vb[j], va[j]), fmaf(ek, vb[j + 1], va[j + 1]), fmaf(ek, vb[j + 2], va[j + 2]),
-                                    fmaf(ek, vb[j + 3], va[j + 3]));
+                    red_add_f32x4(dst + j, fmaf(ek, vb[j], va[j]), fmaf(ek, vb[j + 1], va[j + 1]),
+                                  fmaf(ek, vb[j + 2], va[j + 2]), fmaf(ek, vb[j + 3], va[j + 3]));
                 // C_k . dCb over these 16 n (C row r, 16-byte chunks of its n half)
                 const uint8_t *cs_ = sm + kCC + (n0 >> 6) * kTile;
 #pragma unroll
@@ -671,7 +702,7 @@ BwdTcParams bwd_params(const BwdArgs &a) {
     p.dt = static_cast<const __nv_bfloat16 *>(a.dt);
     p.A = a.A; p.D = a.D;
     p.sf = a.sf; p.sg = a.sg; p.dec = a.dec;
-    p.gx = a.gx; p.gBh = a.gBh; p.gCh = a.gCh; p.gcs = a.gcs; p.u = a.u; p.gxd = a.gxd;
+    p.gx = a.gx; p.gB = a.gB; p.gC = a.gC; p.gcs = a.gcs; p.u = a.u; p.gxd = a.gxd;
     p.status = a.status; p.wait_cycles = a.wait_cycles;
     return p;
 }
@@ -689,6 +720,10 @@ cudaError_t launch_bwd_tc_sums(const BwdArgs &a, cudaStream_t st) {
 cudaError_t launch_bwd_tc_chunk(const BwdArgs &a, cudaStream_t st) {
     BwdTcMaps m;
     if (!bwd_maps(a, m)) return cudaErrorInvalidValue;
+    const size_t bytes = sizeof(float) * (size_t)a.batch * a.L * kN;   // one group
+    cudaError_t z = cudaMemsetAsync(a.gB, 0, bytes, st);
+    if (z == cudaSuccess) z = cudaMemsetAsync(a.gC, 0, bytes, st);
+    if (z != cudaSuccess) return z;
     cudaError_t e = cudaFuncSetAttribute(k_bwd_tc_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kChunkSmem);
     if (e != cudaSuccess) return e;
     k_bwd_tc_chunk<<<dim3(a.nc, a.H, a.batch), kChunkThreads, kChunkSmem, st>>>(m, bwd_params(a));

@@ -331,6 +331,12 @@ __device__ __forceinline__ void red_add_bf16x8(void *dst, uint4 v) {
                  : "memory");
 }
 
+// 16-byte in-place add of 4 float32 values (performed in L2; dst 16-byte aligned)
+__device__ __forceinline__ void red_add_f32x4(float *dst, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
 __device__ __forceinline__ void st_release(unsigned long long *p, unsigned long long v) {
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
