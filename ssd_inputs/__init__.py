@@ -256,6 +256,72 @@ def make_gate(seed: int = 0, step: int = 0) -> float:
     return float(np.float32(0.5 * u))
 
 
+# ------------------------------------------------------------- the Mamba-2 mixer around the scan
+
+MIXER_U_ID = 200            # the layer input, shared by both layers
+MIXER_IDS = {"W_in": 201, "conv_w": 202, "conv_b": 203, "dt_bias": 204, "A": 205, "D": 206, "norm_w": 207,
+             "W_out": 208}
+MIXER_REV_OFFSET = 16
+
+
+@dataclass
+class MixerShape:
+    batch: int
+    seqlen: int
+    d_model: int
+    nheads: int
+    headdim: int = 64
+    dstate: int = 128
+    ngroups: int = 1
+    d_conv: int = 4
+
+    @property
+    def d_inner(self) -> int:
+        return self.nheads * self.headdim
+
+    @property
+    def conv_dim(self) -> int:
+        return self.d_inner + 2 * self.ngroups * self.dstate
+
+    @property
+    def d_in_proj(self) -> int:
+        return 2 * self.d_inner + 2 * self.ngroups * self.dstate + self.nheads
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.seqlen
+
+
+def make_mixer_input(shape: MixerShape, seed: int = 0) -> Stored:
+    """The layer input u [b, L, d_model] ~ N(0, 1), bf16."""
+    return _gen_tensor(seed, MIXER_U_ID, (shape.batch, shape.seqlen, shape.d_model), "bf16", True)
+
+
+def make_mixer_layer(shape: MixerShape, seed: int = 0, offset: int = 0) -> dict:
+    """One Mamba-2 layer's weights.  Projections bf16 (N(0, 1/fan_in)); conv taps U(-1/2, 1/2) and
+    bias 0.1 N(0, 1), float32; dt_bias the inverse softplus of dt ~ exp(U(ln 1e-3, ln 1e-1));
+    A = -exp(U(0, ln 16)); D ~ U(0, 1); norm weight 1 + 0.1 N(0, 1)."""
+    t = {k: v + offset for k, v in MIXER_IDS.items()}
+    H, dm, di, cd, K = shape.nheads, shape.d_model, shape.d_inner, shape.conv_dim, shape.d_conv
+    dt0 = np.exp(math.log(1e-3) + uniform(seed, t["dt_bias"], H) * (math.log(1e-1) - math.log(1e-3)))
+    return {
+        "W_in": _gen_tensor(seed, t["W_in"], (shape.d_in_proj, dm), "bf16", True, lambda z: z / math.sqrt(dm)),
+        "conv_w": _store(uniform(seed, t["conv_w"], cd * K) - 0.5, "f32", (cd, K)),
+        "conv_b": _store(0.1 * normal(seed, t["conv_b"], cd), "f32", (cd,)),
+        "dt_bias": _store(dt0 + np.log(-np.expm1(-dt0)), "f32", (H,)),
+        "A": _store(-np.exp(uniform(seed, t["A"], H) * math.log(16.0)), "f32", (H,)),
+        "D": _store(uniform(seed, t["D"], H), "f32", (H,)),
+        "norm_w": _store(1.0 + 0.1 * normal(seed, t["norm_w"], di), "f32", (di,)),
+        "W_out": _gen_tensor(seed, t["W_out"], (dm, di), "bf16", True, lambda z: z / math.sqrt(di)),
+    }
+
+
+def make_mixer(shape: MixerShape, seed: int = 0):
+    """Input and the forward and reverse layers' weights (two independent layers)."""
+    return (make_mixer_input(shape, seed), make_mixer_layer(shape, seed, 0),
+            make_mixer_layer(shape, seed, MIXER_REV_OFFSET))
+
+
 # ------------------------------------------------------------- workloads
 
 # The five workloads: a tiny fp32 case the oracle checks exhaustively, two
