@@ -25,7 +25,7 @@ import os
 import torch
 
 __all__ = ["ssd_scan", "ssd_scan_state", "ssd_scan_bwd", "bidir_ssd", "r2l_block_scan", "bidir_ssd_noalloc", "noalloc_status", "NoallocArea", "workspace_bytes", "path_for",
-           "segments_for", "kernel_launches", "workspace_status", "SSDError", "library_path", "lib"]
+           "segments_for", "kernel_launches", "mixer_bidir", "mixer_workspace_bytes", "gemm_bf16", "workspace_status", "SSDError", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libbidirssd.so")
@@ -52,7 +52,23 @@ class _Params(ctypes.Structure):
                 ("B", ctypes.c_void_p), ("C", ctypes.c_void_p), ("D", ctypes.c_void_p)]
 
 
+class _MixerShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("batch", "seqlen", "d_model", "nheads", "headdim", "dstate", "ngroups",
+                                            "d_conv")]
+
+
+class _MixerLayer(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("W_in", "conv_w", "conv_b", "dt_bias", "A", "D", "norm_w", "W_out")]
+
+
 _SP, _PP, _VP, _SZ = ctypes.POINTER(_Shape), ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_size_t
+_MSP, _MLP = ctypes.POINTER(_MixerShape), ctypes.POINTER(_MixerLayer)
+lib.ssd_mixer_workspace_bytes.argtypes = [_MSP]
+lib.ssd_mixer_workspace_bytes.restype = _SZ
+lib.mamba2_mixer_bidir.argtypes = [_MSP, _VP, _MLP, _MLP, _VP, _VP, _SZ, _VP]
+lib.mamba2_mixer_bidir.restype = ctypes.c_int
+lib.ssd_gemm_bf16.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _VP, _VP, _VP, _VP, _SZ, _VP]
+lib.ssd_gemm_bf16.restype = ctypes.c_int
 lib.ssd_workspace_bytes.argtypes = [_SP, ctypes.c_int]
 lib.ssd_workspace_bytes.restype = _SZ
 lib.ssd_path_for.argtypes = [_SP, ctypes.c_int]
@@ -257,6 +273,58 @@ def r2l_block_scan(p: dict, s: float, residual, chunk: int = 32, out=None, works
     ws, nbytes = _workspace(shape, chunk, p["x"].device, workspace)
     _check(lib.r2l_block_scan(ctypes.byref(shape), ctypes.byref(prm), ctypes.c_float(s), residual.data_ptr(),
                               int(chunk), o.data_ptr(), ws.data_ptr(), nbytes, _stream(p["x"].device)))
+    return o
+
+
+_MIXER_KEYS = ("W_in", "conv_w", "conv_b", "dt_bias", "A", "D", "norm_w", "W_out")
+
+
+def _mixer_layer(layer: dict) -> _MixerLayer:
+    for k in ("W_in", "W_out"):
+        if layer[k].dtype != torch.bfloat16 or not layer[k].is_contiguous():
+            raise ValueError(f"{k} must be contiguous bf16")
+    for k in ("conv_w", "conv_b", "dt_bias", "A", "D", "norm_w"):
+        if layer[k].dtype != torch.float32 or not layer[k].is_contiguous():
+            raise ValueError(f"{k} must be contiguous float32")
+    return _MixerLayer(*(layer[k].data_ptr() for k in _MIXER_KEYS))
+
+
+def mixer_workspace_bytes(batch: int, seqlen: int, d_model: int, nheads: int, headdim: int = 64,
+                          dstate: int = 128, ngroups: int = 1, d_conv: int = 4) -> int:
+    s = _MixerShape(batch, seqlen, d_model, nheads, headdim, dstate, ngroups, d_conv)
+    return int(lib.ssd_mixer_workspace_bytes(ctypes.byref(s)))
+
+
+def mixer_bidir(u, fwd: dict, rev: dict, nheads: int, headdim: int = 64, dstate: int = 128, d_conv: int = 4,
+                out=None, workspace=None):
+    """The DiffuMamba mixer: two independent Mamba-2 layers (forward, and on the reversed sequence), summed.
+
+    u [batch, seqlen, d_model] bf16; each layer a dict of W_in, conv_w, conv_b, dt_bias, A, D, norm_w, W_out."""
+    if u.dtype != torch.bfloat16 or u.dim() != 3 or not u.is_contiguous():
+        raise ValueError("u must be contiguous bf16 [batch, seqlen, d_model]")
+    b, L, dm = u.shape
+    s = _MixerShape(b, L, dm, nheads, headdim, dstate, 1, d_conv)
+    need = int(lib.ssd_mixer_workspace_bytes(ctypes.byref(s)))
+    if need == 0:
+        raise SSDError(2)
+    o = torch.empty_like(u) if out is None else out
+    if workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=u.device)
+    f, r = _mixer_layer(fwd), _mixer_layer(rev)
+    _check(lib.mamba2_mixer_bidir(ctypes.byref(s), u.data_ptr(), ctypes.byref(f), ctypes.byref(r), o.data_ptr(),
+                                  workspace.data_ptr(), workspace.numel(), _stream(u.device)))
+    return o
+
+
+def gemm_bf16(A, W, out=None):
+    """A [M, K] @ W[N, K]^T on the tensor core (bf16 in and out, float32 accumulation)."""
+    if A.dtype != torch.bfloat16 or W.dtype != torch.bfloat16 or not A.is_contiguous() or not W.is_contiguous():
+        raise ValueError("A and W must be contiguous bf16")
+    M, K = A.shape
+    N = W.shape[0]
+    o = torch.empty(M, N, dtype=torch.bfloat16, device=A.device) if out is None else out
+    ws = torch.zeros(256, dtype=torch.uint8, device=A.device)
+    _check(lib.ssd_gemm_bf16(M, N, K, A.data_ptr(), W.data_ptr(), o.data_ptr(), ws.data_ptr(), 256, _stream(A.device)))
     return o
 
 

@@ -7,6 +7,7 @@
 #include <string>
 
 #include "../../include/bidir_ssd.h"
+#include "mixer.cuh"
 #include "ssd_internal.cuh"
 #include "ssd_tc.cuh"
 
@@ -456,3 +457,125 @@ ssd_status bidir_ssd_noalloc(const ssd_shape *shape, const ssd_params *fwd, cons
 
 }  // extern "C"
 
+// ---------------------------------------------------------------- the mixer around the scan
+
+namespace {
+
+struct MixerLayout {
+    int chunk;
+    ssd_shape scan;
+    size_t scan_ws, zx, x, b, c, dt, y, ynf, ynr, total;
+};
+
+ssd_status mixer_layout(const ssd_mixer_shape *s, MixerLayout *lo) {
+    if (!s) return fail(SSD_ERR_INVALID_ARG, "shape is NULL");
+    if (s->batch < 0 || s->seqlen < 0 || s->d_model <= 0 || s->nheads <= 0)
+        return fail(SSD_ERR_INVALID_ARG, "negative or zero size in mixer shape");
+    if (s->headdim != 64 || s->dstate != 128 || s->ngroups != 1 || s->nheads % 8 != 0)
+        return fail(SSD_ERR_UNSUPPORTED, "mixer needs headdim 64, dstate 128, one group, heads a multiple of 8");
+    if (s->d_model % 64 != 0 || s->seqlen % 128 != 0 || s->d_conv < 1 || s->d_conv > 8)
+        return fail(SSD_ERR_UNSUPPORTED, "mixer needs d_model %% 64 == 0, seqlen %% 128 == 0, d_conv in 1..8");
+    const int di = s->nheads * s->headdim;
+    if (di % 256 != 0 || di > 8192) return fail(SSD_ERR_UNSUPPORTED, "d_inner %d not a multiple of 256 up to 8192", di);
+    lo->chunk = s->seqlen % 256 == 0 ? 256 : 128;
+    lo->scan = ssd_shape{s->batch, s->seqlen, s->nheads, s->headdim, s->dstate, s->ngroups, SSD_BF16};
+    const size_t M = (size_t)s->batch * s->seqlen, N = (size_t)s->ngroups * s->dstate;
+    const size_t dinp = 2 * (size_t)di + 2 * N + s->nheads;
+    lo->scan_ws = round_up(path_ws_bytes(&lo->scan, lo->chunk));
+    size_t o = lo->scan_ws;
+    auto take = [&](size_t bytes) { const size_t at = o; o += round_up(bytes); return at; };
+    lo->zx = take(M * dinp * 2);
+    lo->x = take(M * di * 2);
+    lo->b = take(M * N * 2);
+    lo->c = take(M * N * 2);
+    lo->dt = take(M * s->nheads * 2);
+    lo->y = take(M * di * 2);
+    lo->ynf = take(M * di * 2);
+    lo->ynr = take(M * di * 2);
+    lo->total = o;
+    return SSD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ssd_mixer_workspace_bytes(const ssd_mixer_shape *shape) {
+    MixerLayout lo;
+    return mixer_layout(shape, &lo) == SSD_OK ? lo.total : 0;
+}
+
+ssd_status ssd_gemm_bf16(int M, int N, int K, const void *A, const void *W, void *D, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    g_err.clear();
+    if (M < 0 || N < 0 || K < 0) return fail(SSD_ERR_INVALID_ARG, "negative GEMM size");
+    if (M == 0 || N == 0) return SSD_OK;
+    if (!ssd::mixer_gemm_supported(M, N, K))
+        return fail(SSD_ERR_UNSUPPORTED, "GEMM needs M %% 128 == 0, K %% 64 == 0, N %% 8 == 0 (and the TMA encoder)");
+    if (!aligned16(A) || !aligned16(W) || !aligned16(D)) return fail(SSD_ERR_INVALID_ARG, "A, W, D must be 16-byte aligned");
+    if (!workspace || workspace_bytes < kStatusBytes) return fail(SSD_ERR_INVALID_ARG, "workspace of 256 bytes needed");
+    ssd::GemmArgs g{};
+    g.M = M; g.N = N; g.k1 = K; g.k2 = 0; g.A1 = A; g.W1 = W; g.D = D;
+    g.status = static_cast<int *>(workspace);
+    g.wait_cycles = wait_cycles_now();
+    cudaError_t e = ssd::launch_gemm_bf16(g, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, "GEMM launch");
+}
+
+ssd_status mamba2_mixer_bidir(const ssd_mixer_shape *shape, const void *u, const ssd_mixer_layer *fwd,
+                              const ssd_mixer_layer *rev, void *out, void *workspace, size_t workspace_bytes,
+                              void *stream) {
+    g_err.clear();
+    MixerLayout lo;
+    ssd_status st = mixer_layout(shape, &lo);
+    if (st != SSD_OK) return st;
+    if (shape->batch == 0 || shape->seqlen == 0) return SSD_OK;
+    if (!aligned16(u) || !aligned16(out)) return fail(SSD_ERR_INVALID_ARG, "u and out must be 16-byte aligned");
+    if (!fwd || !rev) return fail(SSD_ERR_INVALID_ARG, "layer weights are NULL");
+    for (const ssd_mixer_layer *l : {fwd, rev})
+        if (!aligned16(l->W_in) || !aligned16(l->W_out) || !l->conv_w || !l->conv_b || !l->dt_bias || !l->A || !l->D ||
+            !l->norm_w)
+            return fail(SSD_ERR_INVALID_ARG, "a layer weight is NULL (or a projection not 16-byte aligned)");
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)))
+        return fail(SSD_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+    if (workspace_bytes < lo.total) return fail(SSD_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", workspace_bytes, lo.total);
+    if (!ssd::mixer_gemm_supported(shape->batch * shape->seqlen, 8, shape->d_model))
+        return fail(SSD_ERR_UNSUPPORTED, "tensor-core GEMM unavailable for this shape");
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    const int M = shape->batch * shape->seqlen, di = shape->nheads * shape->headdim, N = shape->dstate;
+    const int cd = di + 2 * N, dinp = 2 * di + 2 * N + shape->nheads;
+    auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16 *>(ws + off); };
+    int *status = static_cast<int *>(workspace);   // the scan's status word: one for the whole call
+    const long long wc = wait_cycles_now();
+    cudaError_t e;
+    for (int li = 0; li < 2; ++li) {
+        const ssd_mixer_layer *L_ = li ? rev : fwd;
+        ssd::GemmArgs g{};
+        g.M = M; g.N = dinp; g.k1 = shape->d_model; g.k2 = 0; g.A1 = u; g.W1 = L_->W_in; g.D = bf(lo.zx);
+        g.status = status; g.wait_cycles = wc;
+        if ((e = ssd::launch_gemm_bf16(g, cs)) != cudaSuccess) return cuda_fail(e, "input projection");
+        ssd::MixerConvArgs ca{};
+        ca.batch = shape->batch; ca.L = shape->seqlen; ca.d_inner = di; ca.N = N; ca.H = shape->nheads;
+        ca.conv_dim = cd; ca.d_in_proj = dinp; ca.K = shape->d_conv; ca.dir = li ? -1 : 1;
+        ca.zxbcdt = bf(lo.zx); ca.conv_w = L_->conv_w; ca.conv_b = L_->conv_b; ca.dt_bias = L_->dt_bias;
+        ca.x = bf(lo.x); ca.B = bf(lo.b); ca.C = bf(lo.c); ca.dt = bf(lo.dt);
+        if ((e = ssd::launch_conv_silu_dt(ca, cs)) != cudaSuccess) return cuda_fail(e, "convolution");
+        const ssd_params p{bf(lo.x), bf(lo.dt), L_->A, bf(lo.b), bf(lo.c), L_->D};
+        if ((st = ssd_scan(&lo.scan, &p, li ? -1 : 1, lo.chunk, bf(lo.y), workspace, lo.scan_ws, stream)) != SSD_OK)
+            return st;
+        ssd::MixerNormArgs na{};
+        na.batch = shape->batch; na.L = shape->seqlen; na.d_inner = di; na.d_in_proj = dinp; na.eps = 1e-5f;
+        na.y = bf(lo.y); na.zxbcdt = bf(lo.zx); na.w = L_->norm_w; na.out = bf(li ? lo.ynr : lo.ynf);
+        if ((e = ssd::launch_gated_norm(na, cs)) != cudaSuccess) return cuda_fail(e, "gated norm");
+    }
+    ssd::GemmArgs g{};
+    g.M = M; g.N = shape->d_model; g.k1 = di; g.k2 = di;
+    g.A1 = bf(lo.ynf); g.W1 = fwd->W_out; g.A2 = bf(lo.ynr); g.W2 = rev->W_out; g.D = out;
+    g.status = status; g.wait_cycles = wc;
+    if ((e = ssd::launch_gemm_bf16(g, cs)) != cudaSuccess) return cuda_fail(e, "output projection");
+    g_err.clear();
+    return SSD_OK;
+}
+
+}  // extern "C"

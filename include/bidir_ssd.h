@@ -236,6 +236,58 @@ int ssd_path_for(const ssd_shape *shape, int chunk);
  * bidir_ssd_noalloc never segments. */
 int ssd_segments_for(const ssd_shape *shape, int chunk);
 
+/* ------------------------------------------------------------------------
+ * The Mamba-2 mixer around the scan.
+ *
+ * "DiffuMamba: High-Throughput Diffusion LMs with Mamba Backbone", technical
+ * summary section 2: the mixer is two independent Mamba-2 layers, one run
+ * forward and one on the reversed sequence, summed.  The page does not spell
+ * out a layer; it is read as the standard Mamba-2 block:
+ *
+ *   zxbcdt = u W_in^T                      (no bias; z | xBC | dt_raw)
+ *   xBC    = silu(conv(xBC) + conv_b)      (depthwise, width d_conv, causal in the layer's order)
+ *   dt     = softplus(dt_raw + dt_bias)
+ *   y      = ssd_scan(x, dt, A, B, C, D)   (x, B, C split from xBC)
+ *   out    = (rmsnorm(y * silu(z)) * norm_w) W_out^T     (mean over d_inner, eps 1e-5)
+ *
+ * and the mixer output is layer_fwd(u) + flip(layer_rev(flip(u))).
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int batch, seqlen;       /* tokens: batch x seqlen, seqlen a multiple of 128 */
+    int d_model;             /* a multiple of 64 */
+    int nheads, headdim, dstate, ngroups;   /* headdim 64, dstate 128, ngroups 1, nheads % 8 == 0 */
+    int d_conv;              /* 1 .. 8 */
+} ssd_mixer_shape;
+
+/* One layer's weights; device pointers, row-major.  d_inner = nheads * headdim,
+ * conv_dim = d_inner + 2 ngroups dstate, d_in_proj = 2 d_inner + 2 ngroups dstate + nheads. */
+typedef struct {
+    const void *W_in;        /* bf16 [d_in_proj][d_model] */
+    const float *conv_w;     /* [conv_dim][d_conv]; tap k multiplies token t + k - (d_conv - 1) of the layer's order */
+    const float *conv_b;     /* [conv_dim] */
+    const float *dt_bias;    /* [nheads] */
+    const float *A, *D;      /* [nheads]; D may not be NULL */
+    const float *norm_w;     /* [d_inner] */
+    const void *W_out;       /* bf16 [d_model][d_inner] */
+} ssd_mixer_layer;
+
+/* Workspace for mamba2_mixer_bidir (0 if the shape is refused).  Its first
+ * 256 bytes are the status word (read with ssd_workspace_status). */
+size_t ssd_mixer_workspace_bytes(const ssd_mixer_shape *shape);
+
+/* out [batch][seqlen][d_model] (bf16) = the bidirectional mixer on u (bf16, same
+ * shape).  Stream-ordered, asynchronous; the workspace status word must be
+ * zero on entry (as for bidir_ssd).  SSD_ERR_UNSUPPORTED for other shapes. */
+ssd_status mamba2_mixer_bidir(const ssd_mixer_shape *shape, const void *u, const ssd_mixer_layer *fwd,
+                              const ssd_mixer_layer *rev, void *out, void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/* D [M][N] = A [M][K] W [N][K]^T on the tensor core: bf16 in and out, float32
+ * accumulation; M a multiple of 128, K of 64, N of 8.  The workspace is the
+ * 256-byte status area (zero on entry). */
+ssd_status ssd_gemm_bf16(int M, int N, int K, const void *A, const void *W, void *D, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
