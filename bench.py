@@ -26,8 +26,9 @@ rendezvous); ``--dry-run`` runs only the host logic of the ranks (gloo
 process group, shards, MAX reduction), without a GPU.
 ``--workload r2l_block_L32`` times the R2L sidecar decode: one step is 256
 back-to-back denoising-step calls on fresh inputs, reported per call.
-``--op bwd`` times the gradients of both directions (its own JSON line, with
-a roofline against the float32 ALU peak).  ``--batch`` replaces the batch
+``--op bwd`` times the gradients of both directions (its own JSON line);
+``--op mixer`` the whole Mamba-2 mixer layer around the scan (projections,
+conv, scans, norms), against the bf16 tensor peak.  ``--batch`` replaces the batch
 size, for small ncu captures.
 """
 from __future__ import annotations
@@ -391,6 +392,95 @@ def run_ours(args) -> None:
         dist.destroy_process_group()
 
 
+def run_mixer(args) -> None:
+    """The whole DiffuMamba mixer layer (two Mamba-2 layers around the scan), one GPU, device-timed,
+    plus the same call end to end from pinned host memory."""
+    import torch
+    import bidirectional_mamba_ssd_bidir_b200 as ssd
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    w = si.WORKLOADS[args.workload]
+    base = w["shape"]
+    batch = base.batch if args.batch is None else args.batch
+    H, P, N = base.nheads, base.headdim, base.dstate
+    ms_ = si.MixerShape(batch=batch, seqlen=base.seqlen, d_model=H * P // 2, nheads=H, headdim=P, dstate=N)
+    u, f, r = si.make_mixer(ms_, seed=0)
+    u_h = u.torch().pin_memory()
+    u_d = u_h.to(dev)
+    fd = {k: v.torch(dev) for k, v in f.items()}
+    rd = {k: v.torch(dev) for k, v in r.items()}
+    ws = torch.zeros(ssd.mixer_workspace_bytes(ms_.batch, ms_.seqlen, ms_.d_model, H), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(u_d)
+
+    def step():
+        ssd.mixer_bidir(u_d, fd, rd, H, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    with ClockSampler(0) as clk:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize()
+    ssd.workspace_status(ws)
+    ms = start.elapsed_time(end) / args.steps
+    tokens = ms_.tokens
+    # end to end: u in from pinned host memory, the output back, every step
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_steps = max(2, min(args.steps, 10))
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(e2e_steps):
+        u_d.copy_(u_h, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+    e2.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = s2.elapsed_time(e2) / e2e_steps
+    # tensor work per token: both layers' input projections, the output projection over both
+    # layers' inner dimension, and the scan's products (16.8 MFLOP per 128 tokens and head pair
+    # per direction, shared scores)
+    dm, di, dinp = ms_.d_model, ms_.d_inner, ms_.d_in_proj
+    fpt = 2 * 2 * dinp * dm + 2 * dm * 2 * di + 2 * (H // 2) * 16.8e6 / 128
+    peaks = measured_peaks()
+    achieved = fpt * tokens / (ms / 1e3) / 1e12
+    line = {"metric": f"DiffuMamba bidirectional Mamba-2 mixer layer tokens/s, {args.workload} (d_model {dm})",
+            "op": "mixer", "value": tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "global_batch": batch, "seq_len": ms_.seqlen, "d_model": dm,
+                       "d_inner": di, "nheads": H, "dstate": N, "d_conv": ms_.d_conv, "path": "tcgen05"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"], "flops_per_token": fpt,
+                         "peak_source": peaks["source"] + " bf16_tflops (dense, burst)",
+                         "note": "whole layer: two input projections, conv, two scans, two norms, output projection"},
+            "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": u_h.numel() * 2, "d2h_bytes_per_step": out_h.numel() * 2,
+                    "overlap": "none: copy-in, call and copy-out in order on one stream"},
+            "gpu_launches": args.steps * (2 * (3 + ssd.kernel_launches(
+                (batch, ms_.seqlen, H, P, N, 1), torch.bfloat16, 256 if ms_.seqlen % 256 == 0 else 128, "scan")) + 1),
+            "clocks": clk.summary()}
+    if not args.no_cpu_baseline:
+        import oracle
+        from oracle import mixer as om
+        Ls = min(ms_.seqlen, 512)
+        small = si.MixerShape(batch=1, seqlen=Ls, d_model=dm, nheads=H, headdim=P, dstate=N)
+        uf = u.f64()[:1, :Ls]
+        ff, rf = om.layer_to_f64(f), om.layer_to_f64(r)
+        t0 = time.perf_counter()
+        om.mixer_bidir_f64(uf, ff, rf, small)
+        cpu_s = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": Ls / cpu_s, "unit": "tokens/s", "cores": oracle.default_threads(),
+                                "kind": "oracle",
+                                "sample": f"float64 mixer (numpy projections, C recurrence), batch 0, first {Ls} tokens"}
+    print(json.dumps(line), flush=True)
+
+
 def run_r2l(args) -> None:
     """R2L sidecar decode: 256 denoising steps back to back, each a fresh block of inputs.
 
@@ -711,8 +801,9 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(si.WORKLOADS))
     ap.add_argument("--batch", type=int, default=None,
                     help="replace the workload's batch size (a smaller case of the same shape, for profiling)")
-    ap.add_argument("--op", choices=["fwd", "bwd"], default="fwd",
-                    help="bwd: time the gradients of both directions instead (an extra line, one GPU)")
+    ap.add_argument("--op", choices=["fwd", "bwd", "mixer"], default="fwd",
+                    help="bwd: the gradients of both directions; mixer: the whole Mamba-2 mixer layer around the "
+                         "scan (extra lines, one GPU)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU work of the oracle baseline sample")
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds for the reference arm's steps")
@@ -731,6 +822,8 @@ def main(argv=None):
         run_reference(args)
     elif args.op == "bwd":
         run_bwd(args)
+    elif args.op == "mixer":
+        run_mixer(args)
     elif si.WORKLOADS[args.workload]["kind"] == "r2l":
         run_r2l(args)
     else:

@@ -154,96 +154,225 @@ __global__ void __launch_bounds__(kGemmThreads, 2) k_gemm_bf16(const __grid_cons
 
 // ------------------------------------------------------------------ conv + SiLU, dt softplus
 
-// One thread: 8 consecutive channels of xBC (or 8 heads of dt) of one token.  Taps of the
-// forward layer: token t + k - (K - 1); of the reverse layer: t - k + (K - 1); zero outside the
-// sequence.
-__global__ void __launch_bounds__(256) k_conv_silu_dt(MixerConvArgs a) {
-    const int groups_xbc = a.conv_dim / 8, groups_dt = a.H / 8, groups = groups_xbc + groups_dt;
-    const long long total = (long long)a.batch * a.L * groups;
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-         i += (long long)gridDim.x * blockDim.x) {
-        const int gidx = (int)(i % groups);
-        const long long tok = i / groups;                 // b * L + t
-        const int t = (int)(tok % a.L);
-        const __nv_bfloat16 *row = a.zxbcdt + tok * a.d_in_proj;
-        if (gidx < groups_xbc) {
-            const int c0 = 8 * gidx;
-            float acc[8];
+// One thread: 8 consecutive channels of xBC (or 8 heads of dt) over a run of kConvT tokens of
+// one sequence.  The thread first copies every input row it needs (16 bytes each) into its own
+// column of shared memory with cp.async, so all of them are in flight at once and none holds a
+// register; it reads back only what it copied itself, so no barrier is needed.  The taps and
+// bias stay in registers and the inputs slide through a window.  Taps of the forward layer:
+// token t + k - (K - 1); of the reverse layer: t - k + (K - 1) (the run is walked backwards);
+// zero outside the sequence.
+constexpr int kConvT = 32, kConvKMax = 8, kConvThreads = 128;
+
+// Pairs of float32 through the packed f32x2 instructions of sm_100 (one instruction per pair).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 unpack2(uint32_t w) { return make_float2(bf16lo(w), bf16hi(w)); }
+
+// silu(v) = v / (1 + exp(-v)) on a pair: exp(-v) = 2^(-v log2 e) and the reciprocal on the
+// special-function unit (approximate, a few ulp).  Very negative v gives 2^(+big) = inf and a
+// reciprocal of 0, so the result is 0 there without a branch.
+__device__ __forceinline__ float2 silu2(float2 v) {
+    const float2 t = mul2(v, make_float2(-1.4426950408889634f, -1.4426950408889634f));
+    float e0, e1, r0, r1;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(t.x));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(t.y));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(1.f + e0));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r1) : "f"(1.f + e1));
+    return mul2(v, make_float2(r0, r1));
+}
+
+__device__ __forceinline__ void conv_out(const MixerConvArgs &a, long long tok, int c0, const float2 (&acc)[4]) {
+    uint32_t o[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = a.conv_b[c0 + e];
-            for (int k = 0; k < a.K; ++k) {
-                const int tt = a.dir > 0 ? t + k - (a.K - 1) : t - k + (a.K - 1);
-                if (tt < 0 || tt >= a.L) continue;
-                const uint4 v = *reinterpret_cast<const uint4 *>(row + (long long)(tt - t) * a.d_in_proj + a.d_inner + c0);
-                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    acc[2 * e] = fmaf(a.conv_w[(c0 + 2 * e) * a.K + k], bf16lo(w4[e]), acc[2 * e]);
-                    acc[2 * e + 1] = fmaf(a.conv_w[(c0 + 2 * e + 1) * a.K + k], bf16hi(w4[e]), acc[2 * e + 1]);
-                }
+    for (int p = 0; p < 4; ++p) {
+        const float2 s_ = silu2(acc[p]);
+        o[p] = pack_bf16(s_.x, s_.y);
+    }
+    __nv_bfloat16 *dst;
+    if (c0 < a.d_inner) dst = a.x + tok * a.d_inner + c0;
+    else if (c0 < a.d_inner + a.N) dst = a.B + tok * a.N + (c0 - a.d_inner);
+    else dst = a.C + tok * a.N + (c0 - a.d_inner - a.N);
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8]) {
+    f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+    f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+}
+__device__ __forceinline__ void unpack4x2(const uint4 &v, float2 (&f)[4]) {
+    f[0] = unpack2(v.x); f[1] = unpack2(v.y); f[2] = unpack2(v.z); f[3] = unpack2(v.w);
+}
+
+// KT > 0: the conv width, fixed at compile time; KT = 0: the width a.K (at most kConvKMax)
+template <int KT>
+__global__ void __launch_bounds__(kConvThreads) k_conv_silu_dt(MixerConvArgs a) {
+    constexpr int KM = KT > 0 ? KT : kConvKMax;
+    extern __shared__ uint4 conv_stage[];   // [kConvT + KM - 1][kConvThreads]
+    const int K = KT > 0 ? KT : a.K;
+    const int groups_xbc = a.conv_dim / 8, groups = groups_xbc + a.H / 8;
+    const int gidx = blockIdx.x * kConvThreads + threadIdx.x;
+    if (gidx >= groups) return;
+    const int runs = a.L / kConvT;
+    const int b = blockIdx.y / runs, t0 = (blockIdx.y % runs) * kConvT;
+    const long long seq0 = (long long)b * a.L;
+    const bool is_dt = gidx >= groups_xbc;
+    const int c0 = is_dt ? 8 * (gidx - groups_xbc) : 8 * gidx;          // channel (or head) of xBC (or dt)
+    const int col = is_dt ? a.d_inner + a.conv_dim + c0 : a.d_inner + c0;  // its column in zxbcdt
+    const int halo = is_dt ? 0 : K - 1;
+    const int step = (is_dt || a.dir > 0) ? 1 : -1;
+    const int first = step > 0 ? t0 : t0 + kConvT - 1;
+    // row r of the column: the input at token first + step * (r - halo), zero outside the sequence
+    // Two copy groups: the halo and the first half of the run, then the second half, so the
+    // first half is computed while the second is still in flight.
+    uint4 *mine = conv_stage + threadIdx.x;
+    auto copy_rows = [&](int r0, int r1) {
+        for (int r = r0; r < r1; ++r) {
+            const int t = first + step * (r - halo);
+            uint4 *dst = mine + r * kConvThreads;
+            if (t < 0 || t >= a.L) {
+                *dst = make_uint4(0u, 0u, 0u, 0u);
+            } else {
+                const __nv_bfloat16 *src = a.zxbcdt + (seq0 + t) * a.d_in_proj + col;
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
             }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    copy_rows(0, halo + kConvT / 2);
+    copy_rows(halo + kConvT / 2, halo + kConvT);
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+    if (is_dt) {
+        float bias[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) bias[e] = a.dt_bias[c0 + e];
+#pragma unroll 4
+        for (int i = 0; i < kConvT; ++i) {
+            if (i == kConvT / 2) asm volatile("cp.async.wait_group 0;" ::: "memory");
+            float v[8];
+            unpack8(mine[i * kConvThreads], v);
             uint32_t o[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float s0 = acc[2 * e] / (1.f + __expf(-acc[2 * e]));
-                const float s1 = acc[2 * e + 1] / (1.f + __expf(-acc[2 * e + 1]));
-                o[e] = pack_bf16(s0, s1);
-            }
-            __nv_bfloat16 *dst;
-            if (c0 < a.d_inner) dst = a.x + tok * a.d_inner + c0;
-            else if (c0 < a.d_inner + a.N) dst = a.B + tok * a.N + (c0 - a.d_inner);
-            else dst = a.C + tok * a.N + (c0 - a.d_inner - a.N);
-            *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
-        } else {
-            const int h0 = 8 * (gidx - groups_xbc);
-            const uint4 v = *reinterpret_cast<const uint4 *>(row + a.d_inner + a.conv_dim + h0);
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-            uint32_t o[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float r0 = bf16lo(w4[e]) + a.dt_bias[h0 + 2 * e], r1 = bf16hi(w4[e]) + a.dt_bias[h0 + 2 * e + 1];
+                const float r0 = v[2 * e] + bias[2 * e], r1 = v[2 * e + 1] + bias[2 * e + 1];
                 // softplus, with the linear branch above 20 (exp would dominate 1 there)
                 const float s0 = r0 > 20.f ? r0 : log1pf(__expf(r0));
                 const float s1 = r1 > 20.f ? r1 : log1pf(__expf(r1));
                 o[e] = pack_bf16(s0, s1);
             }
-            *reinterpret_cast<uint4 *>(a.dt + tok * a.H + h0) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4 *>(a.dt + (seq0 + t0 + i) * a.H + c0) = make_uint4(o[0], o[1], o[2], o[3]);
         }
+        return;
+    }
+    // wr[p][j]: the taps of channels (2p, 2p + 1) that multiply the input j steps back
+    // (tap K - 1 - j), 0 past the width
+    float2 wr[4][KM], bias[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        bias[p] = make_float2(a.conv_b[c0 + 2 * p], a.conv_b[c0 + 2 * p + 1]);
+#pragma unroll
+        for (int j = 0; j < KM; ++j)
+            wr[p][j] = j < K ? make_float2(a.conv_w[(c0 + 2 * p) * K + (K - 1 - j)],
+                                           a.conv_w[(c0 + 2 * p + 1) * K + (K - 1 - j)])
+                             : make_float2(0.f, 0.f);
+    }
+    // win[j]: the input j steps back in the layer's order.  Before the first token's shift it
+    // holds the token j + 1 steps back (rows halo - 1 down to 0, then zeros).
+    float2 win[KM][4];
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+        if (j < halo) unpack4x2(mine[(halo - 1 - j) * kConvThreads], win[j]);
+        else {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) win[j][p] = make_float2(0.f, 0.f);
+        }
+    }
+    // unrolled by 4 only: a fully unrolled run does not fit the instruction cache
+#pragma unroll 4
+    for (int i = 0; i < kConvT; ++i) {
+        if (i == kConvT / 2) asm volatile("cp.async.wait_group 0;" ::: "memory");
+#pragma unroll
+        for (int j = KM - 1; j > 0; --j)
+#pragma unroll
+            for (int p = 0; p < 4; ++p) win[j][p] = win[j - 1][p];
+        unpack4x2(mine[(halo + i) * kConvThreads], win[0]);
+        float2 acc[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            float2 s_ = bias[p];
+#pragma unroll
+            for (int j = 0; j < KM; ++j) s_ = fma2(wr[p][j], win[j][p], s_);
+            acc[p] = s_;
+        }
+        conv_out(a, seq0 + first + step * i, c0, acc);
     }
 }
 
 // ------------------------------------------------------------------ gated RMS norm
 
-// One CTA per token, one thread per 8 channels (d_inner / 8 threads, whole warps):
-// g = y * silu(z) over d_inner, g / sqrt(mean(g^2) + eps) * w.
+// One CTA per token, d_inner / (8 U) threads, each with U chunks of 8 channels (U loads of y
+// and of z in flight): g = y * silu(z), computed once and kept in registers, then
+// g / sqrt(mean(g^2) + eps) * w.  norm_w is read as float4 (16-byte aligned).
+template <int U>
 __global__ void __launch_bounds__(1024) k_gated_norm(MixerNormArgs a) {
     __shared__ float part[32];
     const long long tok = blockIdx.x;
-    const int c0 = threadIdx.x * 8;
-    const uint4 yv = *reinterpret_cast<const uint4 *>(a.y + tok * a.d_inner + c0);
-    const uint4 zv = *reinterpret_cast<const uint4 *>(a.zxbcdt + tok * a.d_in_proj + c0);
-    const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w}, zw[4] = {zv.x, zv.y, zv.z, zv.w};
-    float g[8];
-    float ss = 0.f;
+    const int stride = 8 * blockDim.x;
+    const __nv_bfloat16 *yrow = a.y + tok * a.d_inner, *zrow = a.zxbcdt + tok * a.d_in_proj;
+    uint4 yv[U], zv[U];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float z0 = bf16lo(zw[e]), z1 = bf16hi(zw[e]);
-        g[2 * e] = bf16lo(yw[e]) * (z0 / (1.f + __expf(-z0)));
-        g[2 * e + 1] = bf16hi(yw[e]) * (z1 / (1.f + __expf(-z1)));
-        ss = fmaf(g[2 * e], g[2 * e], fmaf(g[2 * e + 1], g[2 * e + 1], ss));
+    for (int u = 0; u < U; ++u) {
+        yv[u] = *reinterpret_cast<const uint4 *>(yrow + 8 * threadIdx.x + u * stride);
+        zv[u] = *reinterpret_cast<const uint4 *>(zrow + 8 * threadIdx.x + u * stride);
     }
+    float2 g[U][4], ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        float2 yf[4], zf[4];
+        unpack4x2(yv[u], yf);
+        unpack4x2(zv[u], zf);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            g[u][p] = mul2(yf[p], silu2(zf[p]));
+            ss2 = fma2(g[u][p], g[u][p], ss2);
+        }
+    }
+    float ss = ss2.x + ss2.y;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const int nw = blockDim.x >> 5;
     if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
     __syncthreads();
     float tot = 0.f;
-    for (int w = 0; w < nw; ++w) tot += part[w];
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += part[w];
     const float inv = rsqrtf(tot / a.d_inner + a.eps);
-    uint32_t o[4];
+    const float2 inv2 = make_float2(inv, inv);
+    __nv_bfloat16 *orow = a.out + tok * a.d_inner;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o[e] = pack_bf16(g[2 * e] * inv * a.w[c0 + 2 * e], g[2 * e + 1] * inv * a.w[c0 + 2 * e + 1]);
-    *reinterpret_cast<uint4 *>(a.out + tok * a.d_inner + c0) = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int u = 0; u < U; ++u) {
+        const int c0 = 8 * threadIdx.x + u * stride;
+        const float4 w0 = *reinterpret_cast<const float4 *>(a.w + c0);
+        const float4 w1 = *reinterpret_cast<const float4 *>(a.w + c0 + 4);
+        const float2 wp[4] = {make_float2(w0.x, w0.y), make_float2(w0.z, w0.w), make_float2(w1.x, w1.y),
+                              make_float2(w1.z, w1.w)};
+        uint32_t o[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float2 v = mul2(mul2(g[u][p], inv2), wp[p]);
+            o[p] = pack_bf16(v.x, v.y);
+        }
+        *reinterpret_cast<uint4 *>(orow + c0) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
 }
 
 }  // namespace
@@ -274,15 +403,32 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, cudaStream_t st) {
 }
 
 cudaError_t launch_conv_silu_dt(const MixerConvArgs &a, cudaStream_t st) {
-    const long long total = (long long)a.batch * a.L * (a.conv_dim / 8 + a.H / 8);
-    const int blocks = (int)((total + 255) / 256 < 148 * 16 ? (total + 255) / 256 : 148 * 16);
-    k_conv_silu_dt<<<blocks > 0 ? blocks : 1, 256, 0, st>>>(a);
-    return cudaGetLastError();
+    if (a.L % kConvT != 0 || a.K < 1 || a.K > kConvKMax) return cudaErrorInvalidValue;
+    const int groups = a.conv_dim / 8 + a.H / 8;
+    dim3 grid((groups + kConvThreads - 1) / kConvThreads, (unsigned)((long long)a.batch * (a.L / kConvT)));
+    auto run = [&](auto kernel, int km) -> cudaError_t {
+        const int smem = (kConvT + km - 1) * kConvThreads * (int)sizeof(uint4);
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        kernel<<<grid, kConvThreads, smem, st>>>(a);
+        return cudaGetLastError();
+    };
+    switch (a.K) {
+        case 2: return run(k_conv_silu_dt<2>, 2);
+        case 3: return run(k_conv_silu_dt<3>, 3);
+        case 4: return run(k_conv_silu_dt<4>, 4);
+        default: return run(k_conv_silu_dt<0>, kConvKMax);
+    }
 }
 
 cudaError_t launch_gated_norm(const MixerNormArgs &a, cudaStream_t st) {
-    if (a.d_inner % 256 != 0 || a.d_inner > 8192) return cudaErrorInvalidValue;
-    k_gated_norm<<<(unsigned)((long long)a.batch * a.L), a.d_inner / 8, 0, st>>>(a);
+    if (a.d_inner % 512 != 0 || a.d_inner > 16384 || (reinterpret_cast<uintptr_t>(a.w) & 15) != 0)
+        return cudaErrorInvalidValue;
+    const unsigned tokens = (unsigned)((long long)a.batch * a.L);
+    if (a.d_inner % 1024 == 0 && a.d_inner <= 8192)
+        k_gated_norm<4><<<tokens, a.d_inner / 32, 0, st>>>(a);
+    else
+        k_gated_norm<2><<<tokens, a.d_inner / 16, 0, st>>>(a);
     return cudaGetLastError();
 }
 

@@ -475,8 +475,8 @@ ssd_status mixer_layout(const ssd_mixer_shape *s, MixerLayout *lo) {
         return fail(SSD_ERR_UNSUPPORTED, "mixer needs headdim 64, dstate 128, one group, heads a multiple of 8");
     if (s->d_model % 64 != 0 || s->seqlen % 128 != 0 || s->d_conv < 1 || s->d_conv > 8)
         return fail(SSD_ERR_UNSUPPORTED, "mixer needs d_model %% 64 == 0, seqlen %% 128 == 0, d_conv in 1..8");
-    const int di = s->nheads * s->headdim;
-    if (di % 256 != 0 || di > 8192) return fail(SSD_ERR_UNSUPPORTED, "d_inner %d not a multiple of 256 up to 8192", di);
+    if (s->nheads > 256) return fail(SSD_ERR_UNSUPPORTED, "mixer takes at most 256 heads (d_inner 16384)");
+    const int di = s->nheads * s->headdim;   // a multiple of 512
     lo->chunk = s->seqlen % 256 == 0 ? 256 : 128;
     lo->scan = ssd_shape{s->batch, s->seqlen, s->nheads, s->headdim, s->dstate, s->ngroups, SSD_BF16};
     const size_t M = (size_t)s->batch * s->seqlen, N = (size_t)s->ngroups * s->dstate;
@@ -534,8 +534,8 @@ ssd_status mamba2_mixer_bidir(const ssd_mixer_shape *shape, const void *u, const
     if (!fwd || !rev) return fail(SSD_ERR_INVALID_ARG, "layer weights are NULL");
     for (const ssd_mixer_layer *l : {fwd, rev})
         if (!aligned16(l->W_in) || !aligned16(l->W_out) || !l->conv_w || !l->conv_b || !l->dt_bias || !l->A || !l->D ||
-            !l->norm_w)
-            return fail(SSD_ERR_INVALID_ARG, "a layer weight is NULL (or a projection not 16-byte aligned)");
+            !aligned16(l->norm_w))
+            return fail(SSD_ERR_INVALID_ARG, "a layer weight is NULL (or W_in, W_out, norm_w not 16-byte aligned)");
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)))
         return fail(SSD_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
     if (workspace_bytes < lo.total) return fail(SSD_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", workspace_bytes, lo.total);

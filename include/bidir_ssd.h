@@ -255,7 +255,7 @@ int ssd_segments_for(const ssd_shape *shape, int chunk);
 typedef struct {
     int batch, seqlen;       /* tokens: batch x seqlen, seqlen a multiple of 128 */
     int d_model;             /* a multiple of 64 */
-    int nheads, headdim, dstate, ngroups;   /* headdim 64, dstate 128, ngroups 1, nheads % 8 == 0 */
+    int nheads, headdim, dstate, ngroups;   /* headdim 64, dstate 128, ngroups 1, nheads % 8 == 0, <= 256 */
     int d_conv;              /* 1 .. 8 */
 } ssd_mixer_shape;
 
@@ -267,7 +267,7 @@ typedef struct {
     const float *conv_b;     /* [conv_dim] */
     const float *dt_bias;    /* [nheads] */
     const float *A, *D;      /* [nheads]; D may not be NULL */
-    const float *norm_w;     /* [d_inner] */
+    const float *norm_w;     /* [d_inner], 16-byte aligned */
     const void *W_out;       /* bf16 [d_model][d_inner] */
 } ssd_mixer_layer;
 

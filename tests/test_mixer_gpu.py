@@ -39,6 +39,10 @@ def test_gemm_matches_float64(ssd, M, N, K):
 SHAPES = [
     si.MixerShape(batch=2, seqlen=256, d_model=256, nheads=8),       # d_in_proj 1288: a ragged last N tile
     si.MixerShape(batch=1, seqlen=384, d_model=512, nheads=16),      # 3 blocks of 128, 16 heads
+    si.MixerShape(batch=1, seqlen=256, d_model=256, nheads=8, d_conv=2),   # other compiled conv widths
+    si.MixerShape(batch=1, seqlen=256, d_model=256, nheads=8, d_conv=3),
+    si.MixerShape(batch=1, seqlen=256, d_model=256, nheads=8, d_conv=6),   # the run-time width path
+    si.MixerShape(batch=1, seqlen=256, d_model=256, nheads=8, d_conv=1),
 ]
 
 
@@ -46,12 +50,13 @@ def _dev_layer(layer):
     return {k: v.torch("cuda") for k, v in layer.items()}
 
 
-@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"b{s.batch}L{s.seqlen}dm{s.d_model}H{s.nheads}")
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"b{s.batch}L{s.seqlen}dm{s.d_model}H{s.nheads}K{s.d_conv}")
 def test_mixer_matches_oracle(ssd, shape):
     u, f, r = si.make_mixer(shape, seed=7)
     ws = torch.zeros(ssd.mixer_workspace_bytes(shape.batch, shape.seqlen, shape.d_model, shape.nheads),
                      dtype=torch.uint8, device="cuda")
-    out = ssd.mixer_bidir(u.torch("cuda"), _dev_layer(f), _dev_layer(r), shape.nheads, workspace=ws)
+    out = ssd.mixer_bidir(u.torch("cuda"), _dev_layer(f), _dev_layer(r), shape.nheads, d_conv=shape.d_conv,
+                          workspace=ws)
     torch.cuda.synchronize()
     ssd.workspace_status(ws)
     ref = om.mixer_bidir_f64(u.f64(), om.layer_to_f64(f), om.layer_to_f64(r), shape)
