@@ -156,10 +156,12 @@ ssd_status run_simt(const ssd_shape *s, const ssd_params *p, int dir, int chunk,
     return e == cudaSuccess ? SSD_OK : cuda_fail(e, "SIMT scan launch");
 }
 
-// The bidirectional mixer; `segments` lets the tensor-core path cut sequences into segments
-// (the no-allocation entry point keeps one CTA per sequence: its scratch is fixed).
+// The bidirectional mixer.  `fixed_scratch` is the no-allocation entry point: one CTA per
+// sequence (its scratch has a fixed size) and every kernel on the caller's stream (no side
+// stream is made for it).
 ssd_status bidir_run(const ssd_shape *shape, const ssd_params *fwd, const ssd_params *rev, int chunk, void *y,
-                     void *workspace, size_t workspace_bytes, void *stream, bool segments) {
+                     void *workspace, size_t workspace_bytes, void *stream, bool fixed_scratch) {
+    const bool segments = !fixed_scratch;
     g_err.clear();
     bool empty = false;
     ssd_status st = common_checks(shape, chunk, y, workspace, workspace_bytes, &empty, segments);
@@ -175,6 +177,7 @@ ssd_status bidir_run(const ssd_shape *shape, const ssd_params *fwd, const ssd_pa
         t.fault = g_fault.load();
         t.nseg = tc_nseg(shape, segments);
         t.npiece = ssd::tc_state_pieces(shape->batch, shape->seqlen, shape->nheads, t.nseg);
+        t.concurrent = !fixed_scratch;
         ssd::tc_set_direction(t, 0, 1, fwd->x, fwd->dt, fwd->A, fwd->B, fwd->C, fwd->D);
         ssd::tc_set_direction(t, 1, -1, rev->x, rev->dt, rev->A, rev->B, rev->C, rev->D);
         cudaError_t e = ssd::launch_tc(t, /*bidir=*/true, y, cs);
@@ -336,7 +339,7 @@ ssd_status ssd_scan_bwd(const ssd_shape *shape, const ssd_params *p, int directi
 
 ssd_status bidir_ssd(const ssd_shape *shape, const ssd_params *fwd, const ssd_params *rev, int chunk, void *y,
                      void *workspace, size_t workspace_bytes, void *stream) {
-    return bidir_run(shape, fwd, rev, chunk, y, workspace, workspace_bytes, stream, true);
+    return bidir_run(shape, fwd, rev, chunk, y, workspace, workspace_bytes, stream, /*fixed_scratch=*/false);
 }
 
 ssd_status r2l_block_scan(const ssd_shape *shape, const ssd_params *p, float s, const void *residual, int chunk,
@@ -450,7 +453,7 @@ ssd_status bidir_ssd_noalloc(const ssd_shape *shape, const ssd_params *fwd, cons
     const size_t clear = choose_path(shape, chunk) == 1 ? need : kStatusBytes;
     cudaError_t e = cudaMemsetAsync(ws, 0, clear, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "scratch clear");
-    st = bidir_run(shape, fwd, rev, chunk, y, ws, (size_t)SSD_NOALLOC_MAX_SCRATCH_BYTES, stream, false);
+    st = bidir_run(shape, fwd, rev, chunk, y, ws, (size_t)SSD_NOALLOC_MAX_SCRATCH_BYTES, stream, /*fixed_scratch=*/true);
     if (st == SSD_OK && status_area) *status_area = ws;
     return st;
 }

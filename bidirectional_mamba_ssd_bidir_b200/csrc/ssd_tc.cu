@@ -146,9 +146,6 @@ struct TcParams {
     int fault;                          // test hook: 1 = the first direction never publishes its part
     const float *s_in;                  // single direction: [batch][H][P][N] state entering the scan, or null
     float *s_out;                       // single direction: [batch][H][P][N] state leaving the scan, or null
-    // Non-null: run only the chains the shared-score kernel left to this one.  A CTA then
-    // returns at once unless *deferred == epoch and its own chain fails the same steep test.
-    const unsigned long long *deferred;
 };
 
 struct TcMaps {
@@ -181,12 +178,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
     const CUtensorMap *map_x = &maps.x[slot], *map_dt = &maps.dt[slot], *map_b = &maps.b[slot],
                       *map_c = &maps.c[slot];
 
-    if (prm.deferred != nullptr) {
-        if (*reinterpret_cast<const volatile unsigned long long *>(prm.deferred) != prm.epoch) return;
-        if (!chain_is_steep(prm.d[slot].dt, prm.d[slot].A, b, L, prm.H, h0, threadIdx.x, kThreads,
-                            reinterpret_cast<int *>(sm + kOffMisc + 16)))
-            return;
+    // The CTA past the last chain: wait for the shared-score grid this launch may overlap, so
+    // that this grid completes after it (a no-op when launched in plain stream order).
+    if ((int)blockIdx.x == (prm.bidir ? 2 : 1) * prm.batch * npairs) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        return;
     }
+    // This kernel runs only the chains the shared-score kernel leaves: those that fail the steep
+    // test, which both kernels take with the same function on the same inputs.
+    if (!chain_is_steep(prm.d[slot].dt, prm.d[slot].A, b, L, prm.H, h0, threadIdx.x, kThreads,
+                        reinterpret_cast<int *>(sm + kOffMisc + 16)))
+        return;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -803,11 +805,10 @@ int tc_piece_blocks(int L, int nseg, int npiece) {
 
 namespace {
 size_t round256(size_t v) { return (v + 255) / 256 * 256; }
-// Workspace: epoch-tagged ticket and ready words per (batch, head, block), the epoch-tagged
-// word that tells the exact kernel some chain was left to it; with segments, the steep marks,
-// the per-segment decays and local end states.
+// Workspace: epoch-tagged ticket and ready words per (batch, head, block); with segments, the
+// steep marks, the per-segment decays and local end states.
 struct TcLayout {
-    size_t ticket, ready, deferred, steep, ldec, sloc, total;
+    size_t ticket, ready, steep, ldec, sloc, total;
 };
 TcLayout tc_layout(int batch, int L, int H, int nseg) {
     const int npieces = nseg > 1 ? (nseg - 1) * tc_state_pieces(batch, L, H, nseg) : 0;
@@ -815,8 +816,7 @@ TcLayout tc_layout(int batch, int L, int H, int nseg) {
     const size_t nflags = (size_t)batch * H * (L / kBlk);
     o.ticket = 0;
     o.ready = nflags * 8;
-    o.deferred = 2 * nflags * 8;
-    o.total = round256(o.deferred + 8);
+    o.total = round256(2 * nflags * 8);
     if (nseg > 1) {
         o.steep = o.total;
         o.ldec = round256(o.steep + (size_t)batch * (H / 2) * 2 * 8);
@@ -834,6 +834,7 @@ TcArgs make_tc_args(int batch, int L, int H, int chunk, void *ws, int *status) {
     t.batch = batch; t.L = L; t.H = H; t.chunk = chunk; t.ws = ws; t.status = status;
     t.nseg = tc_segments(batch, L, H);
     t.npiece = tc_state_pieces(batch, L, H, t.nseg);
+    t.concurrent = true;
     return t;
 }
 
@@ -855,7 +856,6 @@ cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
     char *ws = static_cast<char *>(t.ws);
     unsigned long long *ticket = reinterpret_cast<unsigned long long *>(ws + lo.ticket);
     unsigned long long *ready = reinterpret_cast<unsigned long long *>(ws + lo.ready);
-    unsigned long long *deferred = reinterpret_cast<unsigned long long *>(ws + lo.deferred);
     SegScratch sc{};
     if (nseg > 1) {
         sc.sloc = reinterpret_cast<float *>(ws + lo.sloc);
@@ -864,15 +864,11 @@ cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
     }
     const unsigned long long epoch = next_epoch();
     const bool with_state = !bidir && (t.s_in || t.s_out);
-    cudaError_t e = cudaSuccess;
-    if (nseg > 1 && (e = launch_segstate(t, bidir, sc, epoch, st)) != cudaSuccess) return e;
-    e = launch_tcs(t, bidir, y, ticket, ready, deferred, sc, epoch, st);
-    if (e != cudaSuccess) return e;
     // The shared-memory opt-in belongs to the kernel in the current context: set on every launch.
-    cudaError_t attr_err =
+    cudaError_t e =
         cudaFuncSetAttribute(with_state ? k_ssd_tc<true> : k_ssd_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes);
-    if (attr_err != cudaSuccess) return attr_err;
+    if (e != cudaSuccess) return e;
     const int ndir = bidir ? 2 : 1;
     const uint64_t rows = (uint64_t)t.batch * t.L;
     TcMaps maps;
@@ -896,18 +892,33 @@ cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
     p.status = t.status;
     p.ticket = ticket;
     p.ready = ready;
-    p.deferred = deferred;
     p.epoch = epoch;
     p.wait_cycles = t.wait_cycles;
     p.fault = t.fault;
     p.s_in = bidir ? nullptr : t.s_in;
     p.s_out = bidir ? nullptr : t.s_out;
     const int grid = t.batch * (t.H / 2) * ndir;
-    if (p.s_in || p.s_out)
-        k_ssd_tc<true><<<grid, kThreads, kSmemBytes, st>>>(maps, p);
-    else
-        k_ssd_tc<false><<<grid, kThreads, kSmemBytes, st>>>(maps, p);
-    return cudaGetLastError();
+    if (nseg > 1 && (e = launch_segstate(t, bidir, sc, epoch, st)) != cudaSuccess) return e;
+    if ((e = launch_tcs(t, bidir, y, ticket, ready, sc, epoch, st)) != cudaSuccess) return e;
+    // The exact kernel may start while the shared-score kernel still runs (programmatic
+    // dependent launch: that kernel lets its dependents go as each CTA starts), so the steep
+    // chains, each one long single-CTA walk, overlap the rest of the call.  Its last CTA only
+    // waits for the shared-score grid to complete, so that work queued after this call sees
+    // both kernels done.
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3(grid + 1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    if (t.concurrent) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return with_state ? cudaLaunchKernelEx(&cfg, k_ssd_tc<true>, maps, p)
+                      : cudaLaunchKernelEx(&cfg, k_ssd_tc<false>, maps, p);
 }
 
 }  // namespace ssd

@@ -23,6 +23,7 @@ struct TcArgs {
     float *s_out;            // single direction only: [batch][H][P][N] state leaving the scan, or null
     int nseg;                // segments per sequence (1: one CTA walks the whole sequence)
     int npiece;              // pieces each segment's local end state is formed in (nseg > 1)
+    bool concurrent;         // run the exact kernel on a side stream beside the shared-score kernel
 };
 
 // Scratch of a segmented call, inside the path workspace.
@@ -50,7 +51,7 @@ int tc_launches(bool bidir, int nseg);
 cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st);
 // the shared-score kernel (ssd_tcs.cu); launch_tc runs it first for calls without a carried state
 cudaError_t launch_tcs(const TcArgs &t, bool bidir, void *y, unsigned long long *ticket, unsigned long long *ready,
-                       unsigned long long *deferred, const SegScratch &sc, unsigned long long epoch, cudaStream_t st);
+                       const SegScratch &sc, unsigned long long epoch, cudaStream_t st);
 // the segment-state kernel (ssd_tcs_seg.cu): local end states and steep marks, before launch_tcs
 cudaError_t launch_segstate(const TcArgs &t, bool bidir, const SegScratch &sc, unsigned long long epoch,
                             cudaStream_t st);

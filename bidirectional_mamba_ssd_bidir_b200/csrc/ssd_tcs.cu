@@ -168,7 +168,6 @@ struct TcsParams {
     int *status;
     unsigned long long *ticket;         // [batch][H][nblk], epoch-tagged (bidir only)
     unsigned long long *ready;          // [batch][H][nblk], epoch-tagged (bidir only)
-    unsigned long long *deferred;       // set to epoch when a chain is left to the exact kernel
     unsigned long long epoch;
     long long wait_cycles;              // bound of every device-side wait
     int fault;                          // test hook: 1 = the first direction never publishes its part
@@ -188,6 +187,9 @@ struct TcsMaps {
 
 __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__ TcsMaps maps,
                                                          const __grid_constant__ TcsParams prm) {
+    // Dependents launched programmatically behind this grid (the exact kernel for the steep
+    // chains) may start as soon as every CTA of it has started.
+    asm volatile("griddepcontrol.launch_dependents;");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
@@ -222,10 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
               prm.epoch
         : chain_is_steep(prm.d[slot].dt, prm.d[slot].A, b, L, prm.H, h0, threadIdx.x, kThreads, steep_flag);
     if (nblk <= 0) return;
-    if (steep) {
-        if (threadIdx.x == 0) *reinterpret_cast<volatile unsigned long long *>(prm.deferred) = prm.epoch;
-        return;
-    }
+    if (steep) return;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -864,10 +863,10 @@ extern "C" int ssd_debug_trace(unsigned long long *out, int n) {
 }
 #endif
 
-// Launches the shared-score kernel for the chains it can run.  *deferred (in the
-// workspace) is set to `epoch` by any CTA whose chain it left to the exact kernel.
+// Launches the shared-score kernel for the chains it can run (the steep ones are the exact
+// kernel's).
 cudaError_t launch_tcs(const TcArgs &t, bool bidir, void *y, unsigned long long *ticket, unsigned long long *ready,
-                       unsigned long long *deferred, const SegScratch &sc, unsigned long long epoch, cudaStream_t st) {
+                       const SegScratch &sc, unsigned long long epoch, cudaStream_t st) {
     // The shared-memory opt-in belongs to the kernel in the current context: set on every launch
     // (a host-side call), so it holds in any context the caller makes current.
     cudaError_t e = cudaFuncSetAttribute(k_ssd_tcs, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
@@ -895,7 +894,6 @@ cudaError_t launch_tcs(const TcArgs &t, bool bidir, void *y, unsigned long long 
     p.status = t.status;
     p.ticket = ticket;
     p.ready = ready;
-    p.deferred = deferred;
     p.epoch = epoch;
     p.wait_cycles = t.wait_cycles;
     p.fault = t.fault;
