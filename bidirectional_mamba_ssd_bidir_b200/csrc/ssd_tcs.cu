@@ -382,9 +382,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                 SSD_TRACE_PT(kWarpLoad, j, 0);
                 if (lane == 0) {
                     mbar_expect_tx(bar(B_XFULL0 + sx), kPairBytes);
+                    // x is read by this CTA only: first out of L2 (B, C and dt are shared by the
+                    // head pairs of a batch row and keep the default priority)
+                    const uint64_t pol = l2_evict_first();
                     for (int h = 0; h < 2; ++h)
-                        tma_load_2d(sbase + kOffX + sx * kPairBytes + h * kTileBytes, map_x, (h0 + h) * kP,
-                                    row_of(j), bar(B_XFULL0 + sx));
+                        tma_load_2d_hint(sbase + kOffX + sx * kPairBytes + h * kTileBytes, map_x, (h0 + h) * kP,
+                                         row_of(j), bar(B_XFULL0 + sx), pol);
                 }
                 x_issued = j + 1;
             }
@@ -574,12 +577,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                 SSD_TRACE_BLK(j, 1);
                 const uint32_t tile = sbase + kOffB + st * kPairBytes;
                 if (!sec) {
-                    for (int hs = 0; hs < 2; ++hs)
-                        tma_store_2d(&maps.y, tile + hs * kTileBytes, (h0 + hs) * kP, b * L + cm * kBlk);
+                    if (prm.bidir) {
+                        // the other direction adds its part to this one later: keep it in L2
+                        const uint64_t pol = l2_evict_last();
+                        for (int hs = 0; hs < 2; ++hs)
+                            tma_store_2d_hint(&maps.y, tile + hs * kTileBytes, (h0 + hs) * kP, b * L + cm * kBlk,
+                                              pol);
+                    } else {
+                        for (int hs = 0; hs < 2; ++hs)
+                            tma_store_2d(&maps.y, tile + hs * kTileBytes, (h0 + hs) * kP, b * L + cm * kBlk);
+                    }
                 } else {
                     asm volatile("fence.proxy.async.global;" ::: "memory");
+                    const uint64_t pol = l2_evict_first();   // the finished sum
                     for (int hs = 0; hs < 2; ++hs)
-                        tma_reduce_add_2d(&maps.y, tile + hs * kTileBytes, (h0 + hs) * kP, b * L + cm * kBlk);
+                        tma_reduce_add_2d_hint(&maps.y, tile + hs * kTileBytes, (h0 + hs) * kP, b * L + cm * kBlk,
+                                               pol);
                 }
                 bulk_commit();
                 bulk_wait_read0();                        // the tiles may be overwritten from here on
