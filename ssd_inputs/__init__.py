@@ -322,6 +322,45 @@ def make_mixer(shape: MixerShape, seed: int = 0):
             make_mixer_layer(shape, seed, MIXER_REV_OFFSET))
 
 
+# ------------------------------------------------------------- the DiffuMamba-H attention mixer
+
+ATTN_IDS = {"q": 300, "k": 301, "v": 302, "u": 303, "W_qkv": 304, "W_o": 305}
+
+
+@dataclass
+class AttnShape:
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int = 128
+    d_model: int = 0          # the block's width (0: nheads * headdim)
+
+    @property
+    def width(self) -> int:
+        return self.nheads * self.headdim
+
+    @property
+    def model(self) -> int:
+        return self.d_model or self.width
+
+
+def make_attention(shape: AttnShape, seed: int = 0):
+    """q, k, v [b, L, H, D] ~ N(0, 1), bf16: projections of unit-variance activations, so the
+    scaled scores q.k / sqrt(D) have unit variance."""
+    dims = (shape.batch, shape.seqlen, shape.nheads, shape.headdim)
+    return tuple(_gen_tensor(seed, ATTN_IDS[n], dims, "bf16", True) for n in ("q", "k", "v"))
+
+
+def make_attention_layer(shape: AttnShape, seed: int = 0):
+    """The block input u [b, L, d_model] ~ N(0, 1) and its weights W_qkv [3 H D, d_model],
+    W_o [d_model, H D] ~ N(0, 1/fan_in), all bf16."""
+    dm, w = shape.model, shape.width
+    u = _gen_tensor(seed, ATTN_IDS["u"], (shape.batch, shape.seqlen, dm), "bf16", True)
+    wqkv = _gen_tensor(seed, ATTN_IDS["W_qkv"], (3 * w, dm), "bf16", True, lambda z: z / math.sqrt(dm))
+    wo = _gen_tensor(seed, ATTN_IDS["W_o"], (dm, w), "bf16", True, lambda z: z / math.sqrt(w))
+    return u, wqkv, wo
+
+
 # ------------------------------------------------------------- workloads
 
 # The five workloads: a tiny fp32 case the oracle checks exhaustively, two
