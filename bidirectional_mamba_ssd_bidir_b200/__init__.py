@@ -25,7 +25,8 @@ import os
 import torch
 
 __all__ = ["ssd_scan", "ssd_scan_state", "ssd_scan_bwd", "bidir_ssd", "r2l_block_scan", "bidir_ssd_noalloc", "noalloc_status", "NoallocArea", "workspace_bytes", "path_for",
-           "segments_for", "kernel_launches", "mixer_bidir", "mixer_workspace_bytes", "gemm_bf16", "workspace_status", "SSDError", "library_path", "lib"]
+           "segments_for", "kernel_launches", "mixer_bidir", "mixer_workspace_bytes", "gemm_bf16", "attention",
+           "attention_block", "attention_block_workspace_bytes", "workspace_status", "SSDError", "library_path", "lib"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libbidirssd.so")
@@ -61,7 +62,18 @@ class _MixerLayer(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("W_in", "conv_w", "conv_b", "dt_bias", "A", "D", "norm_w", "W_out")]
 
 
+class _AttnShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("batch", "seqlen", "nheads", "headdim")]
+
+
 _SP, _PP, _VP, _SZ = ctypes.POINTER(_Shape), ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_size_t
+_ASP, _LL = ctypes.POINTER(_AttnShape), ctypes.c_longlong
+lib.ssd_attention.argtypes = [_ASP, _VP, _LL, _VP, _LL, _VP, _LL, _VP, _LL, ctypes.c_float, _VP, _SZ, _VP]
+lib.ssd_attention.restype = ctypes.c_int
+lib.ssd_attention_block_workspace_bytes.argtypes = [_ASP]
+lib.ssd_attention_block_workspace_bytes.restype = _SZ
+lib.attention_block.argtypes = [_ASP, ctypes.c_int, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]
+lib.attention_block.restype = ctypes.c_int
 _MSP, _MLP = ctypes.POINTER(_MixerShape), ctypes.POINTER(_MixerLayer)
 lib.ssd_mixer_workspace_bytes.argtypes = [_MSP]
 lib.ssd_mixer_workspace_bytes.restype = _SZ
@@ -325,6 +337,49 @@ def gemm_bf16(A, W, out=None):
     o = torch.empty(M, N, dtype=torch.bfloat16, device=A.device) if out is None else out
     ws = torch.zeros(256, dtype=torch.uint8, device=A.device)
     _check(lib.ssd_gemm_bf16(M, N, K, A.data_ptr(), W.data_ptr(), o.data_ptr(), ws.data_ptr(), 256, _stream(A.device)))
+    return o
+
+
+def attention(q, k, v, out=None, scale: float = 0.0, workspace=None):
+    """Unmasked multi-head softmax attention on the tensor core: q, k, v [batch, seqlen, nheads,
+    headdim] bf16 (headdim 64 or 128; the last two dimensions contiguous, tokens any multiple of 8
+    elements apart, so q, k, v may be views of one packed projection).  scale 0: 1/sqrt(headdim)."""
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or t.dim() != 4 or t.stride(3) != 1 or t.stride(2) != t.shape[3]:
+            raise ValueError("q, k, v must be bf16 [batch, seqlen, nheads, headdim] with contiguous heads")
+        if t.shape != q.shape or (t.shape[0] > 1 and t.stride(0) != t.shape[1] * t.stride(1)):
+            raise ValueError("q, k, v must have one shape and sequences one after another")
+    b, L, H, D = q.shape
+    o = torch.empty(b, L, H, D, dtype=torch.bfloat16, device=q.device) if out is None else out
+    if workspace is None:
+        workspace = torch.zeros(256, dtype=torch.uint8, device=q.device)
+    s = _AttnShape(b, L, H, D)
+    _check(lib.ssd_attention(ctypes.byref(s), q.data_ptr(), q.stride(1), k.data_ptr(), k.stride(1), v.data_ptr(),
+                             v.stride(1), o.data_ptr(), o.stride(1), float(scale), workspace.data_ptr(),
+                             workspace.numel(), _stream(q.device)))
+    return o
+
+
+def attention_block_workspace_bytes(batch: int, seqlen: int, nheads: int, headdim: int) -> int:
+    s = _AttnShape(batch, seqlen, nheads, headdim)
+    return int(lib.ssd_attention_block_workspace_bytes(ctypes.byref(s)))
+
+
+def attention_block(u, W_qkv, W_o, nheads: int, headdim: int = 128, out=None, workspace=None):
+    """The DiffuMamba-H attention block: out = attention(split(u W_qkv^T)) W_o^T; u [batch, seqlen,
+    d_model] bf16, W_qkv [3 nheads headdim, d_model], W_o [d_model, nheads headdim]."""
+    if u.dtype != torch.bfloat16 or u.dim() != 3 or not u.is_contiguous():
+        raise ValueError("u must be contiguous bf16 [batch, seqlen, d_model]")
+    b, L, dm = u.shape
+    s = _AttnShape(b, L, nheads, headdim)
+    need = int(lib.ssd_attention_block_workspace_bytes(ctypes.byref(s)))
+    if need == 0:
+        raise SSDError(2)
+    o = torch.empty_like(u) if out is None else out
+    if workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=u.device)
+    _check(lib.attention_block(ctypes.byref(s), dm, u.data_ptr(), W_qkv.data_ptr(), W_o.data_ptr(), o.data_ptr(),
+                               workspace.data_ptr(), workspace.numel(), _stream(u.device)))
     return o
 
 

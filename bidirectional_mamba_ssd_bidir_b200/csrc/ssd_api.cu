@@ -7,6 +7,7 @@
 #include <string>
 
 #include "../../include/bidir_ssd.h"
+#include "attention.cuh"
 #include "mixer.cuh"
 #include "ssd_internal.cuh"
 #include "ssd_tc.cuh"
@@ -577,6 +578,102 @@ ssd_status mamba2_mixer_bidir(const ssd_mixer_shape *shape, const void *u, const
     g.A1 = bf(lo.ynf); g.W1 = fwd->W_out; g.A2 = bf(lo.ynr); g.W2 = rev->W_out; g.D = out;
     g.status = status; g.wait_cycles = wc;
     if ((e = ssd::launch_gemm_bf16(g, cs)) != cudaSuccess) return cuda_fail(e, "output projection");
+    g_err.clear();
+    return SSD_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- the DiffuMamba-H attention mixer
+
+namespace {
+
+ssd_status attn_checks(const ssd_attn_shape *s) {
+    if (!s) return fail(SSD_ERR_INVALID_ARG, "shape is NULL");
+    if (s->batch < 0 || s->seqlen < 0 || s->nheads <= 0 || s->headdim <= 0)
+        return fail(SSD_ERR_INVALID_ARG, "negative or zero size in attention shape");
+    if (s->batch > 65535 || s->nheads > 65535) return fail(SSD_ERR_UNSUPPORTED, "batch and heads up to 65535");
+    if (!ssd::attention_supported(s->headdim))
+        return fail(SSD_ERR_UNSUPPORTED, "attention needs headdim 64 or 128 (and the TMA encoder)");
+    return SSD_OK;
+}
+
+ssd_status attn_run(const ssd_attn_shape *s, const void *q, long long ldq, const void *k, long long ldk,
+                    const void *v, long long ldv, void *out, long long ldo, float scale, int *status,
+                    cudaStream_t cs) {
+    const long long w = (long long)s->nheads * s->headdim;
+    for (long long ld : {ldq, ldk, ldv, ldo})
+        if (ld < w || ld % 8 != 0) return fail(SSD_ERR_INVALID_ARG, "row strides must be >= nheads*headdim and multiples of 8");
+    ssd::AttnArgs a{};
+    a.batch = s->batch; a.L = s->seqlen; a.H = s->nheads; a.D = s->headdim;
+    a.q = q; a.k = k; a.v = v; a.o = out;
+    a.ldq = ldq; a.ldk = ldk; a.ldv = ldv; a.ldo = ldo;
+    a.scale = scale != 0.f ? scale : 1.f / sqrtf((float)s->headdim);
+    a.status = status;
+    a.wait_cycles = wait_cycles_now();
+    cudaError_t e = ssd::launch_attention(a, cs);
+    return e == cudaSuccess ? SSD_OK : cuda_fail(e, "attention launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+ssd_status ssd_attention(const ssd_attn_shape *shape, const void *q, long long ldq, const void *k, long long ldk,
+                         const void *v, long long ldv, void *out, long long ldo, float scale, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+    g_err.clear();
+    ssd_status st = attn_checks(shape);
+    if (st != SSD_OK) return st;
+    if (shape->batch == 0 || shape->seqlen == 0) return SSD_OK;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return fail(SSD_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
+    if (!workspace || workspace_bytes < kStatusBytes) return fail(SSD_ERR_INVALID_ARG, "workspace of 256 bytes needed");
+    return attn_run(shape, q, ldq, k, ldk, v, ldv, out, ldo, scale, static_cast<int *>(workspace),
+                    static_cast<cudaStream_t>(stream));
+}
+
+size_t ssd_attention_block_workspace_bytes(const ssd_attn_shape *shape) {
+    if (attn_checks(shape) != SSD_OK) return 0;
+    const size_t M = (size_t)shape->batch * shape->seqlen, w = (size_t)shape->nheads * shape->headdim;
+    return kStatusBytes + round_up(M * 3 * w * 2) + round_up(M * w * 2);
+}
+
+ssd_status attention_block(const ssd_attn_shape *shape, int d_model, const void *u, const void *W_qkv,
+                           const void *W_o, void *out, void *workspace, size_t workspace_bytes, void *stream) {
+    g_err.clear();
+    ssd_status st = attn_checks(shape);
+    if (st != SSD_OK) return st;
+    if (shape->batch == 0 || shape->seqlen == 0) return SSD_OK;
+    const int M = shape->batch * shape->seqlen, w = shape->nheads * shape->headdim;
+    if (d_model <= 0 || d_model % 64 != 0 || M % 128 != 0)
+        return fail(SSD_ERR_UNSUPPORTED, "attention block needs d_model %% 64 == 0 and batch*seqlen %% 128 == 0");
+    if (!ssd::mixer_gemm_supported(M, 3 * w, d_model) || !ssd::mixer_gemm_supported(M, d_model, w))
+        return fail(SSD_ERR_UNSUPPORTED, "tensor-core GEMM unavailable for this shape");
+    if (!aligned16(u) || !aligned16(W_qkv) || !aligned16(W_o) || !aligned16(out))
+        return fail(SSD_ERR_INVALID_ARG, "u, W_qkv, W_o and out must be 16-byte aligned");
+    const size_t need = ssd_attention_block_workspace_bytes(shape);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)))
+        return fail(SSD_ERR_INVALID_ARG, "workspace must be non-NULL and 256-byte aligned");
+    if (workspace_bytes < need) return fail(SSD_ERR_INVALID_ARG, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+    int *status = static_cast<int *>(workspace);
+    __nv_bfloat16 *qkv = reinterpret_cast<__nv_bfloat16 *>(ws + kStatusBytes);
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(ws + kStatusBytes + round_up((size_t)M * 3 * w * 2));
+    const long long wc = wait_cycles_now();
+    cudaError_t e;
+    ssd::GemmArgs g{};
+    g.M = M; g.N = 3 * w; g.k1 = d_model; g.A1 = u; g.W1 = W_qkv; g.D = qkv;
+    g.status = status; g.wait_cycles = wc;
+    if ((e = ssd::launch_gemm_bf16(g, cs)) != cudaSuccess) return cuda_fail(e, "q/k/v projection");
+    // q, k, v: column blocks of the projection, 3 w elements between tokens
+    if ((st = attn_run(shape, qkv, 3LL * w, qkv + w, 3LL * w, qkv + 2 * w, 3LL * w, o, w, 0.f, status, cs)) != SSD_OK)
+        return st;
+    ssd::GemmArgs g2{};
+    g2.M = M; g2.N = d_model; g2.k1 = w; g2.A1 = o; g2.W1 = W_o; g2.D = out;
+    g2.status = status; g2.wait_cycles = wc;
+    if ((e = ssd::launch_gemm_bf16(g2, cs)) != cudaSuccess) return cuda_fail(e, "output projection");
     g_err.clear();
     return SSD_OK;
 }

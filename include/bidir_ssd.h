@@ -288,6 +288,51 @@ ssd_status mamba2_mixer_bidir(const ssd_mixer_shape *shape, const void *u, const
 ssd_status ssd_gemm_bf16(int M, int N, int K, const void *A, const void *W, void *D, void *workspace,
                          size_t workspace_bytes, void *stream);
 
+/* ------------------------------------------------------------------------
+ * The attention mixer of DiffuMamba-H.
+ *
+ * "DiffuMamba: High-Throughput Diffusion LMs with Mamba Backbone", technical
+ * summary section 2: DiffuMamba-H inserts one Transformer block (an attention
+ * mixer) after every five Mamba blocks.  The page does not spell the attention
+ * out; it is read as the attention of a diffusion language model, where every
+ * token sees the whole sequence (no mask):
+ *
+ *   O[b, i, h, :] = sum_j softmax_j(scale q[b, i, h, :] . k[b, j, h, :]) v[b, j, h, :]
+ *
+ * and the block around it as  out = attention(split(u W_qkv^T)) W_o^T  (no
+ * bias, no positional encoding: the page names none).
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int batch, seqlen;       /* any seqlen >= 0 for ssd_attention */
+    int nheads, headdim;     /* headdim 64 or 128; batch and nheads up to 65535 */
+} ssd_attn_shape;
+
+/* out = attention(q, k, v) on the tensor core; bf16 in and out, float32 softmax
+ * and accumulation.  Element d of head h of token t of sequence b is at
+ * [(b seqlen + t) ld + h headdim + d] for each of q, k, v (ldq, ldk, ldv) and out
+ * (ldo): row strides in elements, >= nheads*headdim and multiples of 8, so q, k
+ * and v may be column blocks of one packed projection.  scale 0 means
+ * 1/sqrt(headdim).  Device pointers, 16-byte aligned, owned by the caller; the
+ * workspace is the 256-byte status area (zero on entry; read it with
+ * ssd_workspace_status).  Stream-ordered, asynchronous.  SSD_ERR_UNSUPPORTED
+ * for another headdim, SSD_ERR_INVALID_ARG for bad pointers or strides. */
+ssd_status ssd_attention(const ssd_attn_shape *shape, const void *q, long long ldq, const void *k, long long ldk,
+                         const void *v, long long ldv, void *out, long long ldo, float scale, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/* Workspace for attention_block (0 if the shape is refused): the status area,
+ * the packed q/k/v projection and the attention output. */
+size_t ssd_attention_block_workspace_bytes(const ssd_attn_shape *shape);
+
+/* The attention block: qkv = u W_qkv^T (u bf16 [batch][seqlen][d_model], W_qkv
+ * bf16 [3 nheads headdim][d_model], q, k, v its three column blocks in that
+ * order), o = attention(q, k, v) with scale 1/sqrt(headdim), out = o W_o^T
+ * (W_o bf16 [d_model][nheads headdim], out bf16 [batch][seqlen][d_model]).
+ * batch*seqlen a multiple of 128, d_model of 64.  Workspace 256-byte aligned,
+ * of ssd_attention_block_workspace_bytes, status word zero on entry. */
+ssd_status attention_block(const ssd_attn_shape *shape, int d_model, const void *u, const void *W_qkv,
+                           const void *W_o, void *out, void *workspace, size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
