@@ -163,22 +163,6 @@ __global__ void __launch_bounds__(kGemmThreads, 2) k_gemm_bf16(const __grid_cons
 // zero outside the sequence.
 constexpr int kConvT = 32, kConvKMax = 8, kConvThreads = 128;
 
-// Pairs of float32 through the packed f32x2 instructions of sm_100 (one instruction per pair).
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float2 unpack2(uint32_t w) { return make_float2(bf16lo(w), bf16hi(w)); }
 
 // silu(v) = v / (1 + exp(-v)) on a pair: exp(-v) = 2^(-v log2 e) and the reciprocal on the
 // special-function unit (approximate, a few ulp).  Very negative v gives 2^(+big) = inf and a
