@@ -481,6 +481,114 @@ def run_mixer(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_attention(args) -> None:
+    """The DiffuMamba-H attention block (q/k/v projection, unmasked softmax attention, output
+    projection), one GPU, device-timed, plus the attention kernel alone for its roofline and the
+    block end to end from pinned host memory."""
+    import torch
+    import bidirectional_mamba_ssd_bidir_b200 as ssd
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    base = si.WORKLOADS[args.workload]["shape"]
+    batch = base.batch if args.batch is None else args.batch
+    dm = base.nheads * base.headdim // 2            # the layer width of the model the workload belongs to
+    D = 128
+    shape = si.AttnShape(batch, base.seqlen, dm // D, D, d_model=dm)
+    H, L = shape.nheads, shape.seqlen
+    u, wqkv, wo = si.make_attention_layer(shape, seed=0)
+    u_h = u.torch().pin_memory()
+    u_d, wqkv_d, wo_d = u_h.to(dev), wqkv.torch(dev), wo.torch(dev)
+    ws = torch.zeros(ssd.attention_block_workspace_bytes(batch, L, H, D), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(u_d)
+
+    def step():
+        ssd.attention_block(u_d, wqkv_d, wo_d, H, D, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    with ClockSampler(0) as clk:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize()
+    ssd.workspace_status(ws)
+    ms = start.elapsed_time(end) / args.steps
+    tokens = batch * L
+    # the attention kernel alone, on the block's own q/k/v (the packed projection in the workspace)
+    qkv = ws[256:256 + tokens * 3 * H * D * 2].view(torch.bfloat16).view(batch, L, 3, H, D)
+    q, k, v = qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2]
+    o = torch.empty(batch, L, H, D, dtype=torch.bfloat16, device=dev)
+    aws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        ssd.attention(q, k, v, out=o, workspace=aws)
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(args.steps):
+        ssd.attention(q, k, v, out=o, workspace=aws)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    ssd.workspace_status(aws)
+    attn_ms = a0.elapsed_time(a1) / args.steps
+    # end to end: u in from pinned host memory, the output back, every step
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2e_steps = max(2, min(args.steps, 10))
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(e2e_steps):
+        u_d.copy_(u_h, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+    e2.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = s2.elapsed_time(e2) / e2e_steps
+    attn_flops = 4.0 * batch * H * L * L * D          # Q K^T and P V, multiply-adds counted twice
+    peaks = measured_peaks()
+    achieved = attn_flops / (attn_ms / 1e3) / 1e12
+    line = {"metric": f"DiffuMamba-H attention block tokens/s, {args.workload} shape (d_model {dm}, {H} heads x {D})",
+            "op": "attention", "value": tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{args.workload} attention block", "global_batch": batch, "seq_len": L,
+                       "d_model": dm, "nheads": H, "headdim": D, "mask": "none (bidirectional)", "path": "tcgen05"},
+            "roofline": {"bound": "tensor", "kernel": "k_attention", "achieved": achieved,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "flops_per_launch": attn_flops, "launch_ms": attn_ms,
+                         "peak_source": peaks["source"] + " bf16_tflops (dense, burst)"},
+            "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": u_h.numel() * 2, "d2h_bytes_per_step": out_h.numel() * 2,
+                    "overlap": "none: copy-in, call and copy-out in order on one stream"},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clk.summary()}
+    if not args.no_cpu_baseline:
+        import numpy as np
+        import oracle
+        from oracle import attention as oa
+        R = 256
+        uf, wq, wof = u.f64()[0], wqkv.f64(), wo.f64()
+        t0 = time.perf_counter()
+        kv = uf @ wq[H * D:].T                              # keys and values of all L tokens
+        t1 = time.perf_counter()
+        qr = (uf[:R] @ wq[:H * D].T).reshape(1, R, H, D)
+        kk = kv[:, :H * D].reshape(1, L, H, D)
+        vv = kv[:, H * D:].reshape(1, L, H, D)
+        rows = oa.attention_rows_f64(qr, kk, vv, [(0, i, h) for i in range(R) for h in range(H)])
+        np.asarray(rows).reshape(R, H * D) @ wof.T
+        t2 = time.perf_counter()
+        per_token = (t1 - t0) / L + (t2 - t1) / R
+        line["cpu_baseline"] = {"value": 1.0 / per_token, "unit": "tokens/s", "cores": oracle.default_threads(),
+                                "kind": "oracle",
+                                "sample": f"float64 block on batch 0: k/v projection of all {L} tokens (cost per "
+                                          f"token) + q projection, attention rows over {L} keys and output "
+                                          f"projection of the first {R} tokens (cost per token)"}
+    print(json.dumps(line), flush=True)
+
+
 def run_r2l(args) -> None:
     """R2L sidecar decode: 256 denoising steps back to back, each a fresh block of inputs.
 
@@ -801,9 +909,9 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(si.WORKLOADS))
     ap.add_argument("--batch", type=int, default=None,
                     help="replace the workload's batch size (a smaller case of the same shape, for profiling)")
-    ap.add_argument("--op", choices=["fwd", "bwd", "mixer"], default="fwd",
+    ap.add_argument("--op", choices=["fwd", "bwd", "mixer", "attention"], default="fwd",
                     help="bwd: the gradients of both directions; mixer: the whole Mamba-2 mixer layer around the "
-                         "scan (extra lines, one GPU)")
+                         "scan; attention: the DiffuMamba-H attention block (extra lines, one GPU)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU work of the oracle baseline sample")
     ap.add_argument("--ref-budget", type=float, default=90.0, help="seconds for the reference arm's steps")
@@ -824,6 +932,8 @@ def main(argv=None):
         run_bwd(args)
     elif args.op == "mixer":
         run_mixer(args)
+    elif args.op == "attention":
+        run_attention(args)
     elif si.WORKLOADS[args.workload]["kind"] == "r2l":
         run_r2l(args)
     else:
