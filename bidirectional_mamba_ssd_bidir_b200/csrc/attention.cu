@@ -100,6 +100,22 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t sr
                  : "memory");
 }
 
+// Optional hand-off timeline for the tracing build (-DSSD_TRACE): SM-clock stamps of CTA 0 for
+// its first kATraceTiles key tiles, [point][tile]: 0/1 PV_t issued (t = 0, 1), 2/3 S_t(j + 1)
+// issued, 4/5 the softmax of tile t started (its S arrived; warp of lane quarter 2), 6/7 that
+// warp handed its P over.
+#ifdef SSD_TRACE
+constexpr int kATraceTiles = 32, kATracePts = 8;
+__device__ unsigned long long g_attn_trace[kATracePts * kATraceTiles];
+__device__ __forceinline__ void attn_pt(int k, int j) {
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && j < kATraceTiles && (threadIdx.x & 31) == 0)
+        g_attn_trace[k * kATraceTiles + j] = clock64();
+}
+#define ATTN_PT(k, j) attn_pt(k, j)
+#else
+#define ATTN_PT(k, j) ((void)0)
+#endif
+
 template <int D>
 __global__ void __launch_bounds__(kAThreads, 1) k_attention(const __grid_constant__ AttnMaps maps,
                                                             const __grid_constant__ AttnParams prm) {
@@ -210,6 +226,7 @@ __global__ void __launch_bounds__(kAThreads, 1) k_attention(const __grid_constan
                 for (int ks = 0; ks < kAKeys / 16; ++ks)
                     mma_ts_w(tmem + col_o(t), tmem + col_s(t) + 16 * ks, dv.at(ks * 2048), id_o, (j | ks) != 0);
                 mma_commit_w(bar(AB_ODONE0 + t));
+                ATTN_PT(t, j);
                 if (t == kATiles - 1) mma_commit_w(bar(AB_KVEMPTY0 + s));
                 if (j + 1 < nt) {
                     if (!(ok = mbar_wait(bar(AB_KFULL0 + s1), ((j + 1) / kAStages) & 1, MASK, abort_flag, prm.status,
@@ -218,6 +235,7 @@ __global__ void __launch_bounds__(kAThreads, 1) k_attention(const __grid_constan
                     if (!(ok = mbar_wait(bar(AB_ODONE0 + t), j & 1, MASK, abort_flag, prm.status, 137))) break;
                     tc_fence_after();
                     issue_s(t, j + 1);
+                    ATTN_PT(2 + t, j);
                 }
             }
         }
@@ -236,6 +254,7 @@ __global__ void __launch_bounds__(kAThreads, 1) k_attention(const __grid_constan
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
             if (!(ok = mbar_wait(bar(AB_SFULL0 + t), j & 1, MASK, abort_flag, prm.status, 138))) break;
+            if (quarter == 2) ATTN_PT(4 + t, j);
             tc_fence_after();
             float x[128];
             tmem_ld32x2(tl + cs, tl + cs + 32, x, x + 32);
@@ -306,6 +325,7 @@ __global__ void __launch_bounds__(kAThreads, 1) k_attention(const __grid_constan
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(AB_PREADY0 + t));
+            if (quarter == 2) ATTN_PT(6 + t, j);
         }
         if (ok) ok = mbar_wait(bar(AB_ODONE0 + t), (nt - 1) & 1, MASK, abort_flag, prm.status, 140);
         uint8_t *qt = sm + Lo::kOffQ + t * Lo::kTile;
@@ -388,6 +408,14 @@ cudaError_t launch_typed(const AttnArgs &a, cudaStream_t st) {
 }
 
 }  // namespace
+
+#ifdef SSD_TRACE
+extern "C" int attn_debug_trace(unsigned long long *out, int n) {
+    const int total = kATracePts * kATraceTiles;
+    if (n < total) return -1;
+    return cudaMemcpyFromSymbol(out, g_attn_trace, sizeof(unsigned long long) * total) == cudaSuccess ? total : -2;
+}
+#endif
 
 bool attention_supported(int D) { return (D == 64 || D == 128) && get_encode() != nullptr; }
 
