@@ -30,26 +30,46 @@ namespace {
 
 // ------------------------------------------------------------------ GEMM: D[M][N] = A[M][K] W[N][K]^T
 
-constexpr int kGM = 128, kGN = 128, kGK = 64;   // tile; K step of one 128-byte swizzled row
-constexpr int kGStages = 3;
-constexpr uint32_t kGTile = kGM * kGK * 2;      // 16 KB (A tile and W tile alike)
-constexpr uint32_t kGStage = 2 * kGTile;
-constexpr uint32_t kGBar = kGStages * kGStage;
-enum GemmBar { GB_FULL0 = 0, GB_EMPTY0 = GB_FULL0 + kGStages, GB_DONE = GB_EMPTY0 + kGStages, kGemmBars };
+// Persistent: one CTA per SM walks output tiles of 128 x 256 (tile t: rows 128 (t / nN), columns
+// 256 (t % nN); CTAs that run together share an A row block, and W stays in L2).  Warp 0 feeds a
+// 4-stage TMA ring (A box 128 x 64, W box 256 x 64, both K-major, 128-byte swizzle); warp 1 issues
+// the MMAs (M 128, N 256, K 16) into one of two TMEM accumulators (256 columns each), so the
+// epilogue warps 2-5 drain tile i while tile i + 1 accumulates.  The epilogue converts to bf16
+// and stages each 128-column half of the tile in shared memory for a TMA store.
+constexpr int kGM = 128, kGN = 256, kGK = 64;   // tile; K step of one 128-byte swizzled row
+constexpr int kGStages = 4;
+constexpr uint32_t kGATile = kGM * kGK * 2;     // 16 KB
+constexpr uint32_t kGWTile = kGN * kGK * 2;     // 32 KB
+constexpr uint32_t kGStage = kGATile + kGWTile;
+constexpr uint32_t kGBox = 128 * 128;           // one [128 rows][64 bf16] output box, 16 KB
+constexpr uint32_t kGOut = kGStages * kGStage;  // output staging: two boxes (half a tile)
+constexpr uint32_t kGBar = kGOut + 2 * kGBox;
+enum GemmBar {
+    GB_FULL0 = 0,
+    GB_EMPTY0 = GB_FULL0 + kGStages,
+    GB_ACCFULL0 = GB_EMPTY0 + kGStages,         // two accumulators
+    GB_ACCEMPTY0 = GB_ACCFULL0 + 2,
+    GB_STAGED = GB_ACCEMPTY0 + 2,               // the four epilogue warps wrote the half tile
+    GB_STAGEFREE,                               // the TMA store has read it
+    GB_DONE,
+    kGemmBars
+};
 constexpr uint32_t kGMisc = kGBar + kGemmBars * 8;
 constexpr uint32_t kGemmSmem = kGMisc + 32 + 1024;
 constexpr int kGemmThreads = 192;               // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+static_assert(kGemmSmem <= 232448, "shared memory budget");
 
 struct GemmMaps {
     CUtensorMap a[2], w[2], d;                  // two (A, W) pairs summed over K; D the output
 };
 struct GemmParams {
     int M, N, k1, k2;                           // K of the first pair and of the second (0: none)
+    int ntiles, ntn;                            // output tiles, tiles along N
     int *status;
     long long wait_cycles;
 };
 
-__global__ void __launch_bounds__(kGemmThreads, 2) k_gemm_bf16(const __grid_constant__ GemmMaps maps,
+__global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_bf16(const __grid_constant__ GemmMaps maps,
                                                                const __grid_constant__ GemmParams prm) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -58,18 +78,18 @@ __global__ void __launch_bounds__(kGemmThreads, 2) k_gemm_bf16(const __grid_cons
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kGMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kGMisc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * kGN, m0 = blockIdx.y * kGM;
     const int nk1 = prm.k1 / kGK, nk = nk1 + prm.k2 / kGK;
     const uint32_t MASK = 0xffffffffu;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         *reinterpret_cast<volatile long long *>(abort_flag + 1) = prm.wait_cycles;
-        for (int i = 0; i < kGemmBars; ++i) mbar_init(bar(i), 1);
+        for (int i = 0; i < kGemmBars; ++i)
+            mbar_init(bar(i), (i == GB_ACCEMPTY0 || i == GB_ACCEMPTY0 + 1 || i == GB_STAGED) ? 4u : 1u);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 128;" ::"r"(smem_u32(tmem_slot)));
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(tmem_slot)));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc_fence_before();
@@ -78,77 +98,125 @@ __global__ void __launch_bounds__(kGemmThreads, 2) k_gemm_bf16(const __grid_cons
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
+        // ------------------------------------------------------------ TMA loads
         if (lane == 0) {
-            int issued = 0;
-            for (int kt = 0; kt < nk; ++kt) {
-                const int st = kt % kGStages;
-                if (kt >= kGStages &&
-                    !mbar_wait(bar(GB_EMPTY0 + st), ((kt / kGStages) - 1) & 1, 1u, abort_flag, prm.status, 121))
-                    break;
-                const int pr = kt < nk1 ? 0 : 1, kc = (kt < nk1 ? kt : kt - nk1) * kGK;
-                const uint32_t base = sbase + st * kGStage;
-                mbar_expect_tx(bar(GB_FULL0 + st), kGStage);
-                tma_load_2d(base, &maps.a[pr], kc, m0, bar(GB_FULL0 + st));
-                tma_load_2d(base + kGTile, &maps.w[pr], kc, n0, bar(GB_FULL0 + st));
-                issued = kt + 1;
+            long long g = 0;                                  // k-steps issued so far, over all tiles
+            bool ok = true;
+            for (int t = blockIdx.x; t < prm.ntiles && ok; t += gridDim.x) {
+                const int m0 = (t / prm.ntn) * kGM, n0 = (t % prm.ntn) * kGN;
+                for (int kt = 0; kt < nk; ++kt, ++g) {
+                    const int st = (int)(g % kGStages);
+                    if (g >= kGStages &&
+                        !(ok = mbar_wait(bar(GB_EMPTY0 + st), (uint32_t)((g / kGStages) - 1) & 1, 1u, abort_flag,
+                                         prm.status, 121)))
+                        break;
+                    const int pr = kt < nk1 ? 0 : 1, kc = (kt < nk1 ? kt : kt - nk1) * kGK;
+                    const uint32_t base = sbase + st * kGStage;
+                    mbar_expect_tx(bar(GB_FULL0 + st), kGStage);
+                    tma_load_2d(base, &maps.a[pr], kc, m0, bar(GB_FULL0 + st));
+                    tma_load_2d(base + kGATile, &maps.w[pr], kc, n0, bar(GB_FULL0 + st));
+                }
             }
             if (*abort_flag)
-                for (int kt = issued - 1; kt >= 0 && kt >= issued - kGStages; --kt)
-                    mbar_drain(bar(GB_FULL0 + kt % kGStages), (kt / kGStages) & 1, prm.wait_cycles);
+                for (long long q = g - 1; q >= 0 && q >= g - kGStages; --q)
+                    mbar_drain(bar(GB_FULL0 + (int)(q % kGStages)), (uint32_t)(q / kGStages) & 1, prm.wait_cycles);
         }
         __syncwarp();
     } else if (warp == 1) {
+        // ------------------------------------------------------------ MMAs (one elected lane)
         const uint32_t id = idesc(kGN, 0, 0);
+        long long g = 0;
+        int tc = 0;                                           // tiles of this CTA so far
         bool ok = true;
-        for (int kt = 0; kt < nk && ok; ++kt) {
-            const int st = kt % kGStages;
-            if (!(ok = mbar_wait(bar(GB_FULL0 + st), (kt / kGStages) & 1, MASK, abort_flag, prm.status, 122))) break;
+        for (int t = blockIdx.x; t < prm.ntiles && ok; t += gridDim.x, ++tc) {
+            const int acc = tc & 1;
+            // the accumulator is free once the epilogue has read tile tc - 2 out of it
+            if (tc >= 2 &&
+                !(ok = mbar_wait(bar(GB_ACCEMPTY0 + acc), ((tc >> 1) - 1) & 1, MASK, abort_flag, prm.status, 122)))
+                break;
             tc_fence_after();
-            const uint32_t base = sbase + st * kGStage;
-            const SDesc da = make_sdesc(base, kGTile, 1024), dw = make_sdesc(base + kGTile, kGTile, 1024);
+            for (int kt = 0; kt < nk; ++kt, ++g) {
+                const int st = (int)(g % kGStages);
+                if (!(ok = mbar_wait(bar(GB_FULL0 + st), (uint32_t)(g / kGStages) & 1, MASK, abort_flag, prm.status,
+                                     123)))
+                    break;
+                tc_fence_after();
+                const uint32_t base = sbase + st * kGStage;
+                const SDesc da = make_sdesc(base, 16, 1024), dw = make_sdesc(base + kGATile, 16, 1024);
 #pragma unroll
-            for (int ks = 0; ks < kGK / 16; ++ks) mma_ss_w(tmem, da.at(ks * 32), dw.at(ks * 32), id, (kt | ks) != 0);
-            mma_commit_w(bar(GB_EMPTY0 + st));
+                for (int ks = 0; ks < kGK / 16; ++ks)
+                    mma_ss_w(tmem + 256u * acc, da.at(ks * 32), dw.at(ks * 32), id, (kt | ks) != 0);
+                mma_commit_w(bar(GB_EMPTY0 + st));
+            }
+            if (!ok) break;
+            mma_commit_w(bar(GB_ACCFULL0 + acc));
         }
+        // every MMA issued has completed before TMEM is released
         mma_commit_w(bar(GB_DONE));
-        if (lane == 0 && !ok) mbar_drain(bar(GB_DONE), 0, prm.wait_cycles);
+        if (lane == 0) mbar_drain(bar(GB_DONE), 0, prm.wait_cycles);
         __syncwarp();
     } else {
-        // epilogue: TMEM lane quarter warp % 4 (rows), all 128 columns; bf16 into two swizzled
-        // [128][64] halves (the pipeline stages are free once every MMA has completed), then TMA
-        if (mbar_wait(bar(GB_DONE), 0, MASK, abort_flag, prm.status, 123)) {
+        // ------------------------------------------------------------ epilogue: TMEM -> bf16 -> TMA store
+        const int q = warp & 3, r = 32 * q + lane;
+        const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
+        const bool storer = warp == 2 && lane == 0;
+        int tc = 0, h = 0;                                    // tiles, half tiles staged so far
+        bool ok = true;
+        for (int t = blockIdx.x; t < prm.ntiles && ok; t += gridDim.x, ++tc) {
+            const int acc = tc & 1;
+            const int m0 = (t / prm.ntn) * kGM, n0 = (t % prm.ntn) * kGN;
+            if (!(ok = mbar_wait(bar(GB_ACCFULL0 + acc), (tc >> 1) & 1, MASK, abort_flag, prm.status, 124))) break;
             tc_fence_after();
-            const int q = warp & 3, r = 32 * q + lane;
-            const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
+            for (int half = 0; half < 2 && ok; ++half, ++h) {
+                // the staging buffer is free once the previous half's store has read it
+                if (h >= 1 && !(ok = mbar_wait(bar(GB_STAGEFREE), (h - 1) & 1, MASK, abort_flag, prm.status, 125)))
+                    break;
 #pragma unroll 1
-            for (int c0 = 0; c0 < kGN; c0 += 32) {
-                float v[32];
-                tmem_ld32(tl + c0, v);
-                uint8_t *half = sm + (c0 >> 6) * kGTile;
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    float v[32];
+                    tmem_ld32(tl + 256u * acc + 128u * half + c0, v);
+                    uint8_t *box = sm + kGOut + (c0 >> 6) * kGBox;
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    uint4 o;
-                    o.x = pack_bf16(v[8 * qq + 0], v[8 * qq + 1]);
-                    o.y = pack_bf16(v[8 * qq + 2], v[8 * qq + 3]);
-                    o.z = pack_bf16(v[8 * qq + 4], v[8 * qq + 5]);
-                    o.w = pack_bf16(v[8 * qq + 6], v[8 * qq + 7]);
-                    *reinterpret_cast<uint4 *>(half + swz(r, ((c0 & 63) >> 3) + qq)) = o;
+                    for (int qq = 0; qq < 4; ++qq) {
+                        uint4 o;
+                        o.x = pack_bf16(v[8 * qq + 0], v[8 * qq + 1]);
+                        o.y = pack_bf16(v[8 * qq + 2], v[8 * qq + 3]);
+                        o.z = pack_bf16(v[8 * qq + 4], v[8 * qq + 5]);
+                        o.w = pack_bf16(v[8 * qq + 6], v[8 * qq + 7]);
+                        *reinterpret_cast<uint4 *>(box + swz(r, ((c0 & 63) >> 3) + qq)) = o;
+                    }
                 }
+                if (half == 1) {
+                    // the whole accumulator has been read: the MMA warp may reuse it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(GB_ACCEMPTY0 + acc));
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(GB_STAGED));
+                if (storer) {
+                    if ((ok = mbar_wait(bar(GB_STAGED), h & 1, 1u, abort_flag, prm.status, 126))) {
+                        for (int x = 0; x < 2; ++x) {
+                            const int nc = n0 + 128 * half + 64 * x;
+                            if (nc < prm.N) tma_store_2d(&maps.d, sbase + kGOut + x * kGBox, nc, m0);
+                        }
+                        bulk_commit();
+                        bulk_wait_read0();
+                    }
+                    mbar_arrive(bar(GB_STAGEFREE));
+                }
+                ok = __shfl_sync(MASK, ok ? 1 : 0, 0) != 0 && ok;
             }
-            fence_async_smem();
         }
+        if (storer) bulk_wait0();
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 64 && !*abort_flag) {
-        for (int hf = 0; hf < 2; ++hf)
-            if (n0 + 64 * hf < prm.N) tma_store_2d(&maps.d, sbase + hf * kGTile, n0 + 64 * hf, m0);
-        bulk_commit();
-        bulk_wait0();
-    }
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 128;" ::"r"(tmem));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
     }
 }
 
@@ -372,16 +440,21 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, cudaStream_t st) {
     for (int p = 0; p < (g.k2 ? 2 : 1); ++p) {
         const int K = p ? g.k2 : g.k1;
         if (!make_map(&maps.a[p], p ? g.A2 : g.A1, g.M, K, 64, true) ||
-            !make_map(&maps.w[p], p ? g.W2 : g.W1, g.N, K, 64, true))
+            !make_map(&maps.w[p], p ? g.W2 : g.W1, g.N, K, 64, true, kGN))
             return cudaErrorInvalidValue;
     }
     if (!make_map(&maps.d, g.D, g.M, g.N, 64, true)) return cudaErrorInvalidValue;
     GemmParams p{};
     p.M = g.M; p.N = g.N; p.k1 = g.k1; p.k2 = g.k2;
+    p.ntn = (g.N + kGN - 1) / kGN;
+    p.ntiles = (g.M / kGM) * p.ntn;
     p.status = g.status; p.wait_cycles = g.wait_cycles;
     cudaError_t e = cudaFuncSetAttribute(k_gemm_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
     if (e != cudaSuccess) return e;
-    dim3 grid((g.N + kGN - 1) / kGN, g.M / kGM);
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const int grid = p.ntiles < sms ? p.ntiles : sms;
     k_gemm_bf16<<<grid, kGemmThreads, kGemmSmem, st>>>(maps, p);
     return cudaGetLastError();
 }
