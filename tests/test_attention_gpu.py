@@ -120,6 +120,17 @@ def test_attention_block_matches_oracle(ssd):
     _check(out, ref)
 
 
+def test_attention_block_at_width_2048(ssd):
+    """The 1.3B block width (d_model 2048, 16 heads x 128) on one 2048-token sequence: both
+    projections run several 128 x 256 tiles per persistent GEMM CTA."""
+    shape = si.AttnShape(1, 2048, 16, 128, d_model=2048)
+    u, wqkv, wo = si.make_attention_layer(shape, 17)
+    out = ssd.attention_block(u.torch("cuda"), wqkv.torch("cuda"), wo.torch("cuda"), shape.nheads, shape.headdim)
+    torch.cuda.synchronize()
+    ref = oa.attention_layer_f64(u.f64(), wqkv.f64(), wo.f64(), shape.nheads)
+    _check(out, ref)
+
+
 def test_refuses_other_head_sizes(ssd):
     q = torch.zeros(1, 128, 2, 96, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(ssd.SSDError):

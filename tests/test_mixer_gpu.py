@@ -23,7 +23,11 @@ def ssd():
     return m
 
 
-@pytest.mark.parametrize("M,N,K", [(256, 1288, 256), (384, 200, 128), (128, 64, 64), (512, 8512, 2048)])
+# The GEMM is persistent over 128 x 256 output tiles (one CTA per SM, two TMEM accumulators in
+# turn): shapes with fewer tiles than SMs, with one or two tiles per CTA (8192 x 1024), and with
+# about fourteen per CTA (32768 x 2048), plus ragged last column tiles (N = 8, 200, 264, 1288, 8512).
+@pytest.mark.parametrize("M,N,K", [(256, 1288, 256), (384, 200, 128), (128, 64, 64), (512, 8512, 2048),
+                                   (128, 8, 64), (256, 264, 192), (8192, 1024, 256), (32768, 2048, 128)])
 def test_gemm_matches_float64(ssd, M, N, K):
     g = torch.Generator().manual_seed(M + N + K)
     A = torch.randn(M, K, generator=g).to(torch.bfloat16)
