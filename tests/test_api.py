@@ -139,3 +139,26 @@ def test_segment_query():
     # float32 and small head dims take the SIMT path, which never segments; refused shapes say -1
     assert ssd.segments_for((1, 64, 2, 16, 16, 1), torch.float32, 16) == 0
     assert ssd.segments_for((1, 60, 2, 16, 16, 1), torch.float32, 16) == -1
+
+
+def test_mixer_and_attention_refusals():
+    """Host-side refusals of the mixer, attention and GEMM entry points (no kernel is launched)."""
+    ms = ssd._MixerShape(1, 256, 256, 8, 64, 128, 1, 4)
+    assert ssd.lib.ssd_mixer_workspace_bytes(ctypes.byref(ms)) > 0
+    for bad in (ssd._MixerShape(1, 256, 256, 8, 32, 128, 1, 4),      # headdim 32
+                ssd._MixerShape(1, 200, 256, 8, 64, 128, 1, 4),      # seqlen not a multiple of 128
+                ssd._MixerShape(1, 256, 256, 12, 64, 128, 1, 4),     # heads not a multiple of 8
+                ssd._MixerShape(1, 256, 256, 264, 64, 128, 1, 4),    # more than 256 heads
+                ssd._MixerShape(1, 256, 256, 8, 64, 128, 1, 9)):     # conv wider than 8
+        assert ssd.lib.ssd_mixer_workspace_bytes(ctypes.byref(bad)) == 0
+    good = 1 << 20
+    a = ssd._AttnShape(1, 128, 2, 96)                                  # headdim 96: refused
+    assert ssd.lib.ssd_attention(ctypes.byref(a), good, 192, good, 192, good, 192, good, 192, 0.0, good, 256,
+                                 None) == 2
+    assert ssd.lib.ssd_attention_block_workspace_bytes(ctypes.byref(a)) == 0
+    assert ssd.lib.ssd_attention(None, good, 256, good, 256, good, 256, good, 256, 0.0, good, 256, None) == 1
+    neg = ssd._AttnShape(-1, 128, 2, 128)
+    assert ssd.lib.ssd_attention(ctypes.byref(neg), good, 256, good, 256, good, 256, good, 256, 0.0, good, 256,
+                                 None) == 1
+    assert ssd.lib.ssd_gemm_bf16(-1, 8, 64, good, good, good, good, 256, None) == 1
+    assert ssd.lib.ssd_gemm_bf16(0, 8, 64, good, good, good, good, 256, None) == 0     # empty: a no-op
