@@ -100,7 +100,7 @@ constexpr uint32_t kOffBar = kOffDT + 3 * kDtBytes;
 enum Bar {
     B_XFULL0 = 0, B_XFULL1, B_XEMPTY0, B_XEMPTY1, B_BFULL0, B_BFULL1, B_CFULL, B_CEMPTY,
     B_DTFULL0, B_DTFULL1, B_DTFULL2, B_GFULL, B_GCREADY, B_CXREADY0,
-    B_CXREADY1, B_STFULL, B_SREADY, B_YOFFDONE, B_YFULL, B_YEMPTY, B_TABREADY0, B_TABREADY1, B_TABREADY2,
+    B_CXREADY1, B_STFULL, B_SREADY, B_YOFFDONE, B_YFULL, B_TABREADY0, B_TABREADY1, B_TABREADY2,
     B_TABFREE0, B_TABFREE1, B_TABFREE2, B_TILE0, B_TILE1, B_DONEA, B_DONEB, kNumBars
 };
 // misc: tmem base, abort flag, wait limit, steep flag
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
             // arrivals: 16 = one per CUDA-core warp, 1 = one thread or one MMA commit (TMA
             // completions count bytes)
             uint32_t cnt = 1;
-            if (i == B_GCREADY || i == B_CXREADY0 || i == B_CXREADY1 || i == B_SREADY || i == B_YEMPTY) cnt = 16;
+            if (i == B_GCREADY || i == B_CXREADY0 || i == B_CXREADY1 || i == B_SREADY) cnt = 16;
             if (i == B_TILE0 || i == B_TILE1 || (i >= B_TABFREE0 && i <= B_TABFREE2)) cnt = 16;
             // read by both MMA streams: a commit from each
             if (i == B_XEMPTY0 || i == B_XEMPTY1 || i == B_CEMPTY) cnt = 2;
@@ -632,8 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
             const int st = jj & 1, sl = jj % 3;
             if (!mbar_wait(bar(B_TABREADY0 + sl), (jj / 3) & 1, MASK, abort_flag, prm.status, 41)) return false;
             if (!mbar_wait(bar(B_XFULL0 + st), (jj >> 1) & 1, MASK, abort_flag, prm.status, 42)) return false;
-            // Y buffer st was last read by block jj-2's epilogue
-            if (jj >= 2 && !mbar_wait(bar(B_YEMPTY), (jj - 2) & 1, MASK, abort_flag, prm.status, 43)) return false;
+            // Y buffer st was last read by block jj-2's epilogue, which this warp ran before this
+            // pass, on the same TMEM lanes and columns it writes here (each warp its own slice)
             const float *tb = tab_s + sl * kTabFloats;
             const float cf = tb[kTabCF + hs * kBlk + r], dr = tb[kTabDR + hs * kBlk + r];
             uint8_t *xt = sm + kOffX + st * kPairBytes + hs * kTileBytes;
@@ -797,10 +797,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                 tc_fence_after();
                 if (!state_pass(j + 1, k2)) break;
                 SSD_TRACE_PT(warp, j, 5);
-                // (3) the next block's cX and Y starting value (its x stage was loaded once block
-                // j-1's products had read the stage: placed here, the load has most of a block)
-                if (!cx_pass(j + 1)) break;
-                SSD_TRACE_PT(warp, j, 6);
             } else if (s_out) {
                 // state leaving the scan: S_out = kappa_last * S (after the last state product)
                 if (!mbar_wait(bar(B_STFULL), j & 1, MASK, abort_flag, prm.status, 49)) break;
@@ -811,9 +807,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
 #pragma unroll
                 for (int i = 0; i < 32; ++i) s_out[sslot + (size_t)(32 * ch + i) * kN + r] = sv[i] * f;
             }
-            // (4) epilogue: y = r Y_j in bf16 into this block's B buffer, which G and the state
+            // (3) epilogue: y = r Y_j in bf16 into this block's B buffer, which G and the state
             // product have consumed (the state product's completion was awaited in (2), or here
-            // for the last block); the store warp writes the tiles to y
+            // for the last block); the store warp writes the tiles to y.  It comes before the next
+            // block's cX pass: the sooner the tiles leave, the sooner B of block j+2 can be loaded
+            // into this buffer, and the next G waits for that B.
             if (j + 1 == nblk && !s_out && !mbar_wait(bar(B_STFULL), j & 1, MASK, abort_flag, prm.status, 49))
                 break;
             if (!mbar_wait(bar(B_YFULL), j & 1, MASK, abort_flag, prm.status, 46)) break;
@@ -838,11 +836,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(bar(B_YEMPTY));            // the Y accumulator has been read
                 mbar_arrive(bar(B_TABFREE0 + sl));     // and the block's tables, for the last time
                 mbar_arrive(bar(B_TILE0 + st));
             }
             SSD_TRACE_PT(warp, j, 8);
+            if (j + 1 < nblk) {
+                // (4) the next block's cX and Y starting value (its x stage was loaded once block
+                // j-1's products had read the stage: placed here, the load has most of a block)
+                if (!cx_pass(j + 1)) break;
+                SSD_TRACE_PT(warp, j, 6);
+            }
         }
     }
 

@@ -35,7 +35,7 @@ WARP_MMA = WARP_MMA_A
 # the points each role records, in program order within a block
 COMPUTE_POINTS = [(0, "block start"), (1, "scores G ready"), (2, "masked scores Gc written"),
                   (3, "tables two blocks ahead built"), (4, "state product done"), (5, "state hand-off done"),
-                  (6, "next block's cX and Y start written"), (7, "Y ready"), (8, "epilogue done")]
+                  (7, "Y ready"), (8, "epilogue done"), (6, "next block's cX and Y start written")]
 # (warp, point): stream A (warp 17) issues G and the state product, stream B (warp 19) Y_off and Y_diag
 MMA_POINTS = [(17, 0, "G issued"), (19, 1, "Y_off issued"), (17, 2, "state product issued"), (19, 3, "Y_diag issued")]
 # (warp, point, name) of the load and hand-off warps
