@@ -518,7 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
         // both heads' y tiles into the block's B buffer: first direction, TMA store; second,
         // TMA bf16 reduce-add (in L2) onto the published part.  As soon as the tiles have been
         // read, B of block j+2 is loaded into the buffer.  A first part is published once its
-        // writes have completed, checked after the next block's store is issued; before this
+        // writes have completed, at the start of the next block's turn (before that block's
+        // tiles are ready, so the fence and the release cost the store nothing); before this
         // direction waits on a block the other direction took, it publishes what it has
         // pending.  So a publication depends on nothing the other direction still has to do,
         // and the two cannot wait on each other.  One ticket covers both heads.
@@ -550,8 +551,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                 const int cm = mblk_of(j);
                 const size_t pair_slot = ((size_t)b * prm.H + h0) * nblk_chain + cm;
                 int sec = 0;
+                SSD_TRACE_PT(kWarpStore, j, 3);
                 if (prm.bidir) {
                     sec = atomicExch(prm.ticket + pair_slot, prm.epoch) == prm.epoch;
+                    SSD_TRACE_PT(kWarpStore, j, 4);
                     if (sec) {
                         if (pend >= 0) {
                             bulk_wait0();
@@ -571,6 +574,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                         }
                         if (!ok) break;
                     }
+                }
+                if (pend >= 0) {
+                    // the previous block's first part, while the CUDA-core warps still write this
+                    // block's tiles: its store has completed by now or soon
+                    bulk_wait0();
+                    SSD_TRACE_PT(kWarpStore, j, 5);
+                    publish();
                 }
                 if (!mbar_wait(bar(B_TILE0 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 61)) break;
                 SSD_TRACE_PT(kWarpStore, j, 0);
@@ -599,10 +609,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
                 SSD_TRACE_PT(kWarpStore, j, 2);
                 SSD_TRACE_BLK(j, 2);
                 if (j + 2 < nblk) load_b(j + 2);
-                if (pend >= 0) {
-                    bulk_wait1();                         // every store group but this block's is done
-                    publish();
-                }
                 if (prm.bidir && !sec) {
                     pend = j;
                     pend_slot = pair_slot;

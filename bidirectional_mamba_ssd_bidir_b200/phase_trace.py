@@ -41,8 +41,9 @@ MMA_POINTS = [(17, 0, "G issued"), (19, 1, "Y_off issued"), (17, 2, "state produ
 # (warp, point, name) of the load and hand-off warps
 LOAD_POINTS = [(16, 0, "x stage free, x loads issued"), (16, 1, "B loads issued (store warp)"),
                (16, 2, "C buffer free, C loads issued"), (16, 3, "decay tables built"),
+               (18, 3, "iteration start (ticket next)"), (18, 4, "ticket taken"),
                (18, 0, "y tiles written, store issued"), (18, 2, "y tiles read"),
-               (18, 1, "first part published")]
+               (18, 5, "previous store completed"), (18, 1, "first part published")]
 # per-block timeline of CTAs 0 and 1, every block (see block_times)
 BLOCK_POINTS = ["G issued", "y store issued", "y tiles read", "B load issued"]
 N_ALL_BLOCKS = 1024
