@@ -194,13 +194,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
         *abort_flag = 0;
         *reinterpret_cast<volatile long long *>(abort_flag + 1) = prm.wait_cycles;
         // arrival counts: 16 = one per CUDA-core warp, 8 = one per warp of a head's two
-        // warpgroups, 2 = one per store warp, 1 = one thread / one MMA commit
+        // warpgroups, 1 = one thread (the store warp's, for the x stages) / one MMA commit
         constexpr uint32_t k16 = (1u << B_WXREADY) | (1u << B_SPREADY) | (1u << B_MREADY) | (1u << B_YEMPTY) |
                                  (1u << B_TABREADY0) | (1u << B_TABREADY1) | (1u << B_DTEMPTY0) | (1u << B_DTEMPTY1);
         constexpr uint32_t k8 = (1u << B_TILE00) | (1u << B_TILE01) | (1u << B_TILE10) | (1u << B_TILE11);
-        constexpr uint32_t k2 = (1u << B_XEMPTY0) | (1u << B_XEMPTY1);
-        for (int i = 0; i < (int)kNumBars; ++i)
-            mbar_init(bar(i), (k16 >> i) & 1 ? 16 : (k8 >> i) & 1 ? 8 : (k2 >> i) & 1 ? 2 : 1);
+        for (int i = 0; i < (int)kNumBars; ++i) mbar_init(bar(i), (k16 >> i) & 1 ? 16 : (k8 >> i) & 1 ? 8 : 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == kWarpMma) {
@@ -324,25 +322,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
             mma_commit(bar(B_DONE));
             mbar_drain(bar(B_DONE), 0, prm.wait_cycles);
         }
-    } else if (warp == kWarpStore || warp == kWarpStore + 1) {
-        // ---------------------------------------------------------- y stores, one warp per head
+    } else if (warp == kWarpStore) {
+        // ---------------------------------------------------------- y stores of both heads
+        // The two directions of a head pair take one ticket per output block, at the pair's
+        // first head: the same word the shared-score kernel takes, so a pair whose two chains
+        // run in different kernels (one direction steep, the other not) still meets once per
+        // block.  The first direction stores both heads' tiles and publishes the pair once both
+        // have landed; the second waits for that and adds both.  (Warp kWarpStore + 1 has no
+        // part in this.)
         const uint32_t MASK = 0xffffffffu;
-        const int hs = warp - kWarpStore;
-        const int h = h0 + hs;
-        const size_t flag_base = ((size_t)b * prm.H + h) * nblk;
+        const size_t pair_base = ((size_t)b * prm.H + h0) * nblk;
         for (int j = 0; j < nblk; ++j) {
             const int st = j & 1;
             const int cm = dir > 0 ? j : nblk - 1 - j;
-            if (!mbar_wait(bar(B_TILE00 + 2 * hs + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 61)) break;
-            const uint32_t tile = sbase + kOffX + st * kStageBytes + hs * kTileBytes;
+            if (!mbar_wait(bar(B_TILE00 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 61)) break;
+            if (!mbar_wait(bar(B_TILE10 + st), (j >> 1) & 1, MASK, abort_flag, prm.status, 62)) break;
+            const uint32_t tile = sbase + kOffX + st * kStageBytes;
             int sec = 0;
             if (prm.bidir) {
                 if (lane == 0) {
                     // this direction's part of the block is complete: first or second?
-                    sec = atomicExch(prm.ticket + flag_base + cm, prm.epoch) == prm.epoch;
+                    sec = atomicExch(prm.ticket + pair_base + cm, prm.epoch) == prm.epoch;
                     if (sec) {
-                        // the other direction's store warp took the block first and is storing it
-                        const unsigned long long *rp = prm.ready + flag_base + cm;
+                        // the other direction took the block first and is storing it
+                        const unsigned long long *rp = prm.ready + pair_base + cm;
                         const long long t0 = clock64();
                         while (ld_acquire(rp) != prm.epoch) {
                             if (*abort_flag) { sec = 2; break; }
@@ -359,34 +362,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
                 sec = __shfl_sync(MASK, sec, 0);
                 if (sec == 2) break;
             }
-            if (sec == 0) {
-                if (lane == 0) {
-                    tma_store_2d(&maps.y, tile, h * kP, b * L + cm * kBlk);
-                    bulk_commit();
-                    bulk_wait_read0();                    // the tile may be overwritten from here on
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(bar(B_XEMPTY0 + st));
-                    if (prm.bidir) {
-                        bulk_wait0();                     // this part of y is in global memory
-                        asm volatile("fence.proxy.async.global;" ::: "memory");
-                        if (prm.fault != 1) st_release(prm.ready + flag_base + cm, prm.epoch);
-                    }
-                }
-            } else {
-                // y += this part: a bulk tensor reduction (bf16 add in L2) onto the published part
-                if (lane == 0) {
+            if (lane == 0) {
+                if (sec == 0) {
+                    for (int hs = 0; hs < 2; ++hs)
+                        tma_store_2d(&maps.y, tile + hs * kTileBytes, (h0 + hs) * kP, b * L + cm * kBlk);
+                } else {
+                    // y += this part: bulk tensor reductions (bf16 add in L2) onto the published part
                     asm volatile("fence.proxy.async.global;" ::: "memory");
-                    tma_reduce_add_2d(&maps.y, tile, h * kP, b * L + cm * kBlk);
-                    bulk_commit();
-                    bulk_wait_read0();
+                    for (int hs = 0; hs < 2; ++hs)
+                        tma_reduce_add_2d(&maps.y, tile + hs * kTileBytes, (h0 + hs) * kP, b * L + cm * kBlk);
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_XEMPTY0 + st));
+                bulk_commit();
+                bulk_wait_read0();                        // the tiles may be overwritten from here on
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(B_XEMPTY0 + st));
+                if (prm.bidir && sec == 0) {
+                    bulk_wait0();                         // both heads' parts are in global memory
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                    if (prm.fault != 1) st_release(prm.ready + pair_base + cm, prm.epoch);
+                }
             }
         }
         if (lane == 0) bulk_wait0();                      // every store has landed before the CTA exits
+    } else if (warp == kWarpStore + 1) {
+        // no work: the store warp above writes both heads
     } else {
         // ---------------------------------------------------------- CUDA-core work
         // Four warpgroups: g = 2 * head + half.  Each handles one head's rows and one half

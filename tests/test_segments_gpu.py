@@ -116,3 +116,25 @@ def test_segmented_steep_chain_goes_to_the_exact_kernel(ssd):
     torch.cuda.synchronize()
     ref = oracle.bidir_f64(oracle.params_f64(pf), oracle.params_f64(pr))
     assert oracle.rel_err(y.double().cpu().numpy(), ref) <= 2e-2
+
+
+def test_bidir_with_one_direction_steep(ssd):
+    """The forward layer has a head pair too steep for the factorised kernel, the reverse layer
+    does not: the exact kernel runs that pair's forward chain while the shared-score kernel runs
+    its reverse chain, and the two parts of every output block still meet once (both kernels take
+    the same ticket per head pair and block).  Segmented (bidir_ssd) and whole-sequence
+    (bidir_ssd_noalloc) calls."""
+    shape, chunk = si.Shape(1, 1024, 8, 64, 128, 1, "bf16"), 256
+    pf, pr = si.make_bidir(shape, seed=7)
+    A = pf.A.data.copy()
+    A[2] = -60.0                # head pair 1 of the forward layer only
+    pf.A.data[:] = A
+    ref = oracle.bidir_f64(oracle.params_f64(pf), oracle.params_f64(pr))
+    y = ssd.bidir_ssd(_dev(pf), _dev(pr), chunk=chunk)
+    torch.cuda.synchronize()
+    assert oracle.rel_err(y.double().cpu().numpy(), ref) <= 2e-2
+    out = torch.empty_like(y)
+    area = ssd.bidir_ssd_noalloc(_dev(pf), _dev(pr), out, chunk=chunk)
+    torch.cuda.synchronize()
+    ssd.noalloc_status(area)
+    assert oracle.rel_err(out.double().cpu().numpy(), ref) <= 2e-2
