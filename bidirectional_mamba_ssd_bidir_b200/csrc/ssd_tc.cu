@@ -133,6 +133,7 @@ struct TcDirParams {
 };
 
 struct TcParams {
+    const unsigned long long *steep;    // [batch][H/2][2], epoch-tagged: the chains this kernel runs
     int batch, L, H, nblk;
     int bidir;                          // 1: slot = blockIdx & 1, forward/reverse hand-off through flags
     int dir_single;                     // direction of slot 0 when bidir == 0
@@ -184,10 +185,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tc(const __grid_constant__ 
         asm volatile("griddepcontrol.wait;" ::: "memory");
         return;
     }
-    // This kernel runs only the chains the shared-score kernel leaves: those that fail the steep
-    // test, which both kernels take with the same function on the same inputs.
-    if (!chain_is_steep(prm.d[slot].dt, prm.d[slot].A, b, L, prm.H, h0, threadIdx.x, kThreads,
-                        reinterpret_cast<int *>(sm + kOffMisc + 16)))
+    // This kernel runs only the chains the shared-score kernel leaves: those the steep-decay
+    // marks of this call name (one pass, before both kernels, decides for every chain)
+    if (*reinterpret_cast<const volatile unsigned long long *>(prm.steep + ((size_t)b * npairs + h0 / 2) * 2 + slot) !=
+        prm.epoch)
         return;
 
     if (threadIdx.x == 0) {
@@ -806,8 +807,8 @@ int tc_piece_blocks(int L, int nseg, int npiece) {
 
 namespace {
 size_t round256(size_t v) { return (v + 255) / 256 * 256; }
-// Workspace: epoch-tagged ticket and ready words per (batch, head, block); with segments, the
-// steep marks, the per-segment decays and local end states.
+// Workspace: epoch-tagged ticket and ready words per (batch, head, block), the epoch-tagged steep
+// marks per chain; with segments, the per-segment decays and local end states.
 struct TcLayout {
     size_t ticket, ready, steep, ldec, sloc, total;
 };
@@ -817,10 +818,10 @@ TcLayout tc_layout(int batch, int L, int H, int nseg) {
     const size_t nflags = (size_t)batch * H * (L / kBlk);
     o.ticket = 0;
     o.ready = nflags * 8;
-    o.total = round256(2 * nflags * 8);
+    o.steep = round256(2 * nflags * 8);
+    o.total = round256(o.steep + (size_t)batch * (H / 2) * 2 * 8);
     if (nseg > 1) {
-        o.steep = o.total;
-        o.ldec = round256(o.steep + (size_t)batch * (H / 2) * 2 * 8);
+        o.ldec = o.total;
         o.sloc = round256(o.ldec + (size_t)batch * H * 2 * npieces * 4);
         o.total = round256(o.sloc + (size_t)batch * H * 2 * npieces * kP * kN * 4);
     }
@@ -847,7 +848,69 @@ void tc_set_direction(TcArgs &t, int slot, int dir, const void *x, const void *d
 // Every call runs the shared-score kernel and then the exact kernel for the chains it left
 // (which returns at once when there are none); a segmented call runs the segment-state kernel
 // first.
-int tc_launches(bool, int nseg) { return nseg > 1 ? 3 : 2; }
+int tc_launches(bool, int) { return 3; }   // steep marks (or segment states), scan, exact kernel
+
+namespace {
+// Steep-decay marks of a whole-sequence call (a segmented call's state kernel makes them): for
+// each chain (batch row, head pair, direction) with a 128-token block whose decay passes
+// kSteepLog2 for either head (log2 units, or is not a number), marks[(b H/2 + pair) 2 + slot] =
+// epoch.  Nothing else decides which kernel runs a chain of the call, so the shared-score kernel
+// and the exact kernel agree by construction.  One CTA per (block, batch row, direction), one
+// thread per token: the thread reads its token's whole dt row (16-byte loads, so each row is
+// read once for all heads), a warp butterfly sums 8 heads at a time, the 4 warps' sums meet
+// in shared memory.
+struct SteepArgs {
+    const __nv_bfloat16 *dt[2];
+    const float *A[2];
+    unsigned long long *marks;
+    unsigned long long epoch;
+    int L, H;
+};
+
+__global__ void __launch_bounds__(128) k_ssd_steep_marks(const __grid_constant__ SteepArgs a) {
+    extern __shared__ float part[];                     // [4 warps][H] per-warp sums
+    const int blk = blockIdx.x, b = blockIdx.y, slot = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t row = (size_t)b * a.L + (size_t)blk * kBlk + threadIdx.x;
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.dt[slot] + row * a.H);
+    for (int g = 0; g < a.H / 8; ++g) {
+        const uint4 v = src[g];
+        float d[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
+                      bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) d[e] += __shfl_xor_sync(0xffffffffu, d[e], o);
+        if (lane == 0)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) part[warp * a.H + 8 * g + e] = d[e];
+    }
+    __syncthreads();
+    for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
+        const float sum = (part[h] + part[a.H + h]) + (part[2 * a.H + h] + part[3 * a.H + h]);
+        const float ah = fabsf(a.A[slot][h]) * 1.4426950408889634f;
+        if (ah * sum > kSteepLog2 || !(sum == sum))
+            *reinterpret_cast<volatile unsigned long long *>(a.marks + ((size_t)b * (a.H / 2) + h / 2) * 2 + slot) =
+                a.epoch;
+    }
+}
+
+cudaError_t launch_steep_marks(const TcArgs &t, bool bidir, unsigned long long *marks, unsigned long long epoch,
+                               cudaStream_t st) {
+    SteepArgs a{};
+    for (int s = 0; s < (bidir ? 2 : 1); ++s) {
+        a.dt[s] = static_cast<const __nv_bfloat16 *>(t.d[s].dt);
+        a.A[s] = t.d[s].A;
+    }
+    a.marks = marks;
+    a.epoch = epoch;
+    a.L = t.L;
+    a.H = t.H;
+    dim3 grid((unsigned)(t.L / kBlk), (unsigned)t.batch, bidir ? 2u : 1u);
+    k_ssd_steep_marks<<<grid, kBlk, 4 * t.H * (int)sizeof(float), st>>>(a);
+    return cudaGetLastError();
+}
+}  // namespace
 
 
 
@@ -858,10 +921,10 @@ cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
     unsigned long long *ticket = reinterpret_cast<unsigned long long *>(ws + lo.ticket);
     unsigned long long *ready = reinterpret_cast<unsigned long long *>(ws + lo.ready);
     SegScratch sc{};
+    sc.steep = reinterpret_cast<unsigned long long *>(ws + lo.steep);
     if (nseg > 1) {
         sc.sloc = reinterpret_cast<float *>(ws + lo.sloc);
         sc.ldec = reinterpret_cast<float *>(ws + lo.ldec);
-        sc.steep = reinterpret_cast<unsigned long long *>(ws + lo.steep);
     }
     const unsigned long long epoch = next_epoch();
     const bool with_state = !bidir && (t.s_in || t.s_out);
@@ -899,7 +962,13 @@ cudaError_t launch_tc(const TcArgs &t, bool bidir, void *y, cudaStream_t st) {
     p.s_in = bidir ? nullptr : t.s_in;
     p.s_out = bidir ? nullptr : t.s_out;
     const int grid = t.batch * (t.H / 2) * ndir;
-    if (nseg > 1 && (e = launch_segstate(t, bidir, sc, epoch, st)) != cudaSuccess) return e;
+    p.steep = sc.steep;
+    // the steep marks: the state kernel makes them for a segmented call, one pass otherwise
+    if (nseg > 1) {
+        if ((e = launch_segstate(t, bidir, sc, epoch, st)) != cudaSuccess) return e;
+    } else if ((e = launch_steep_marks(t, bidir, sc.steep, epoch, st)) != cudaSuccess) {
+        return e;
+    }
     if ((e = launch_tcs(t, bidir, y, ticket, ready, sc, epoch, st)) != cudaSuccess) return e;
     // The exact kernel may start while the shared-score kernel still runs (programmatic
     // dependent launch: that kernel lets its dependents go as each CTA starts), so the steep

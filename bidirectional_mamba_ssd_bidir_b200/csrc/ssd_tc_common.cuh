@@ -415,9 +415,7 @@ constexpr float kSteepLog2 = 150.f;
 // lane + 32 i.  True if, for either head, |A_h| * log2(e) * sum(dt) is above
 // kSteepLog2 (a0, a1: |A| * log2(e) of the two heads), or a sum is not a
 // number.  Called by the 32 lanes of one warp; every lane gets the answer.
-// Every path that decides which kernel takes a chain reaches this one
-// function with the same values in the same lanes, so they all sum in the same
-// order and take the same decision for every block.
+// The state kernel of a segmented call marks steep chains with it.
 __device__ __forceinline__ bool steep_of_block(const uint32_t u[4], float a0, float a1) {
     float s0 = 0.f, s1 = 0.f;
 #pragma unroll
@@ -443,25 +441,6 @@ __device__ __forceinline__ bool block_is_steep(const __nv_bfloat16 *dt, float a0
         u[i] = *reinterpret_cast<const uint32_t *>(dt + t * H + h0);
     }
     return steep_of_block(u, a0, a1);
-}
-
-// True if, for head h0 or h0 + 1 of batch row b, some 128-token block is steep
-// (block_is_steep).  Called by every thread of the CTA (nthreads of them,
-// thread index tid); uses one int of shared memory; returns the same answer in
-// every thread.
-__device__ __forceinline__ bool chain_is_steep(const __nv_bfloat16 *dt, const float *A, int b, int L, int H, int h0,
-                                               int tid, int nthreads, int *flag) {
-    constexpr float kLog2e = 1.4426950408889634f;
-    const int warp = tid >> 5, lane = tid & 31, nwarps = nthreads >> 5;
-    if (tid == 0) *reinterpret_cast<volatile int *>(flag) = 0;
-    __syncthreads();
-    const float a0 = fabsf(A[h0]) * kLog2e, a1 = fabsf(A[h0 + 1]) * kLog2e;
-    const int nblk = L / 128;
-    bool steep = false;
-    for (int blk = warp; blk < nblk; blk += nwarps) steep |= block_is_steep(dt, a0, a1, b, L, H, h0, blk, lane);
-    if (steep && lane == 0) atomicOr(flag, 1);
-    __syncthreads();
-    return *reinterpret_cast<volatile int *>(flag) != 0;
 }
 
 // ------------------------------------------------------------------ host side

@@ -103,7 +103,7 @@ enum Bar {
     B_CXREADY1, B_STFULL, B_SREADY, B_YOFFDONE, B_YFULL, B_TABREADY0, B_TABREADY1, B_TABREADY2,
     B_TABFREE0, B_TABFREE1, B_TABFREE2, B_TILE0, B_TILE1, B_DONEA, B_DONEB, kNumBars
 };
-// misc: tmem base, abort flag, wait limit, steep flag
+// misc: tmem base, abort flag, wait limit
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 32 + 1024;   // + alignment slack
 static_assert(kPairBytes % 1024 == 0, "tiles must stay 1024-byte aligned");
@@ -196,7 +196,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
     auto bar = [&](int i) { return sbase + kOffBar + 8u * i; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffMisc + 4);   // limit at +8
-    int *steep_flag = reinterpret_cast<int *>(sm + kOffMisc + 16);
     float *tab_s = reinterpret_cast<float *>(sm + kOffTab);         // [3 buffers][kTabFloats]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -217,12 +216,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_ssd_tcs(const __grid_constant__
     const int has_in = prm.s_in != nullptr || seg > 0;
     float *const s_out = seg == prm.nseg - 1 ? prm.s_out : nullptr;   // left by the chain's last segment
 
-    // A chain with a block too steep for the factorised decay is left to the exact kernel.  With
-    // segments, the segment-state kernel has run the test on every block of the chain.
-    const bool steep = prm.nseg > 1
-        ? *reinterpret_cast<const volatile unsigned long long *>(prm.steep + ((size_t)b * npairs + hp) * 2 + slot) ==
-              prm.epoch
-        : chain_is_steep(prm.d[slot].dt, prm.d[slot].A, b, L, prm.H, h0, threadIdx.x, kThreads, steep_flag);
+    // A chain with a block too steep for the factorised decay is left to the exact kernel: the
+    // call's steep marks (made by the state kernel when segmented, by one pass otherwise) say which.
+    const bool steep =
+        *reinterpret_cast<const volatile unsigned long long *>(prm.steep + ((size_t)b * npairs + hp) * 2 + slot) ==
+        prm.epoch;
     if (nblk <= 0) return;
     if (steep) return;
 

@@ -45,7 +45,7 @@ def test_segment_policy(ssd):
     assert ssd.segments_for((1, 1024, 8, 64, 128, 1), bf, 256) == 4        # 8 blocks, 2 per segment
     assert ssd.segments_for((1, 1408, 8, 64, 128, 1), bf, 128) == 4        # 11 blocks: 3, 3, 3, 2
     assert ssd.segments_for((1, 128, 8, 64, 128, 1), bf, 128) == 1        # a single block
-    assert ssd.kernel_launches((4, 8192, 64, 64, 128, 1), bf, 256, "bidir") == 2
+    assert ssd.kernel_launches((4, 8192, 64, 64, 128, 1), bf, 256, "bidir") == 3     # marks, scan, exact
 
 
 CASES = [
