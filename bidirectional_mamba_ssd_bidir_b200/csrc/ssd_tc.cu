@@ -873,17 +873,33 @@ __global__ void __launch_bounds__(128) k_ssd_steep_marks(const __grid_constant__
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t row = (size_t)b * a.L + (size_t)blk * kBlk + threadIdx.x;
     const uint4 *src = reinterpret_cast<const uint4 *>(a.dt[slot] + row * a.H);
-    for (int g = 0; g < a.H / 8; ++g) {
-        const uint4 v = src[g];
-        float d[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
-                      bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
+    const int ng = a.H / 8;
+    for (int g0 = 0; g0 < ng; g0 += 8) {
+        uint4 v[8];                                     // up to eight groups of 8 heads in flight
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
+        for (int i = 0; i < 8; ++i)
+            if (g0 + i < ng) v[i] = src[g0 + i];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) d[e] += __shfl_xor_sync(0xffffffffu, d[e], o);
-        if (lane == 0)
+        for (int i = 0; i < 8; ++i) {
+            if (g0 + i >= ng) break;
+            const float d[8] = {bf16lo(v[i].x), bf16hi(v[i].x), bf16lo(v[i].y), bf16hi(v[i].y),
+                                bf16lo(v[i].z), bf16hi(v[i].z), bf16lo(v[i].w), bf16hi(v[i].w)};
+            // Sums over the warp's 32 rows by a reduce-scatter butterfly: each level hands the
+            // partner lane the half of the heads it keeps and adds the half it receives, so lane l
+            // ends with the sum of head (l >> 2) & 7 (9 shuffles for the 8 heads).
+            const bool b4 = (lane >> 4) & 1, b3 = (lane >> 3) & 1, b2 = (lane >> 2) & 1;
+            float e4[4], e2[2];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) part[warp * a.H + 8 * g + e] = d[e];
+            for (int k = 0; k < 4; ++k)
+                e4[k] = (b4 ? d[k + 4] : d[k]) + __shfl_xor_sync(0xffffffffu, b4 ? d[k] : d[k + 4], 16);
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+                e2[k] = (b3 ? e4[k + 2] : e4[k]) + __shfl_xor_sync(0xffffffffu, b3 ? e4[k] : e4[k + 2], 8);
+            float e1 = (b2 ? e2[1] : e2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? e2[0] : e2[1], 4);
+            e1 += __shfl_xor_sync(0xffffffffu, e1, 2);
+            e1 += __shfl_xor_sync(0xffffffffu, e1, 1);
+            if ((lane & 3) == 0) part[warp * a.H + 8 * (g0 + i) + ((lane >> 2) & 7)] = e1;
+        }
     }
     __syncthreads();
     for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
