@@ -142,6 +142,26 @@ def _shape_of(x, B) -> _Shape:
 
 
 def _params(x, dt, A, B, C, D) -> _Params:
+    """The six parameter pointers, after checking shapes, dtypes, device and layout.
+
+    The common case is checked with few tensor calls (a per-call cost of decode-sized
+    launches); if anything is off, the checks run one by one for the error message."""
+    b, L, H, P = x.shape
+    io, dev = x.dtype, x.get_device()
+    if (dev >= 0 and dt.shape == (b, L, H) and B.dim() == 4 and C.shape == B.shape and B.shape[:2] == (b, L)
+            and dt.dtype is io and B.dtype is io and C.dtype is io
+            and A.dtype is torch.float32 and A.shape == (H,)
+            and (D is None or (D.dtype is torch.float32 and D.shape == (H,)))
+            and dt.get_device() == dev and A.get_device() == dev and B.get_device() == dev
+            and C.get_device() == dev and (D is None or D.get_device() == dev)
+            and x.is_contiguous() and dt.is_contiguous() and A.is_contiguous() and B.is_contiguous()
+            and C.is_contiguous() and (D is None or D.is_contiguous())):
+        return _Params(x.data_ptr(), dt.data_ptr(), A.data_ptr(), B.data_ptr(), C.data_ptr(),
+                       D.data_ptr() if D is not None else None)
+    return _params_checked(x, dt, A, B, C, D)
+
+
+def _params_checked(x, dt, A, B, C, D) -> _Params:
     b, L, H, P = x.shape
     io = x.dtype
     for name, t, shp in (("dt", dt, (b, L, H)), ("B", B, None), ("C", C, tuple(B.shape))):
@@ -167,7 +187,13 @@ def _params(x, dt, A, B, C, D) -> _Params:
                    D.data_ptr() if D is not None else None)
 
 
+# the current stream's handle without building a torch Stream object (about 2 us a call less)
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(dev) -> int:
+    if _raw_stream is not None:
+        return int(_raw_stream(dev.index if dev.index is not None else torch.cuda.current_device()))
     return torch.cuda.current_stream(dev).cuda_stream
 
 

@@ -279,14 +279,201 @@ __global__ void __launch_bounds__(kThreads) k_chunk_output(ScanArgs a, int have_
     }
 }
 
+// ---------------------------------------------------------------- single-chunk calls
+// A call whose sequence is one chunk of at most 64 tokens with no state in or out (the R2L
+// block of the Bifocal sidecar is one): nothing crosses a chunk, so one CTA per (head, batch
+// row) runs its head's whole scan after a single round of global loads (x, B, C as 16-byte
+// vectors, dt, and the residual or the output that the result is added to), instead of the
+// several dependent load phases of k_chunk_output.  Same arithmetic: the decays by the same
+// prefix sum, the scores C_k . B_s e^(cs_k - cs_s) dt_s for s <= k, their product with x,
+// D x and the output mode, in float32.
+constexpr int kOneQ = 64;    // longest chunk taken
+
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4 &v, float *f);
+template <>
+__device__ __forceinline__ void unpack16<float>(const uint4 &v, float *f) {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+}
+template <>
+__device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4 &v, float *f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// shared floats of one CTA: cs, dt, B and C (rows padded to N + 1), x, the masked scores
+__host__ __device__ constexpr size_t one_chunk_floats(int Q, int P, int N) {
+    return 2 * (size_t)kOneQ + 2 * (size_t)Q * (N + 1) + (size_t)Q * P + (size_t)Q * Q;
+}
+
+template <typename T, int P, int N>
+__global__ void __launch_bounds__(kThreads) k_one_chunk(ScanArgs a) {
+    constexpr int V = 16 / (int)sizeof(T);                        // elements per 16-byte vector
+    constexpr int NB = (kOneQ * N / V + kThreads - 1) / kThreads;  // B (and C) vectors per thread, at most
+    constexpr int NX = (kOneQ * P / V + kThreads - 1) / kThreads;  // x vectors per thread, at most
+    constexpr int H2 = P / 2;                                      // a thread's two outputs: p and p + P/2
+    constexpr int NO = (kOneQ * H2 + kThreads - 1) / kThreads;     // output pairs per thread, at most
+    constexpr int NP = N + 1;
+    __shared__ float warp_tot[kOneQ / 32];
+    const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int Q = a.Q, g = h / (a.H / a.G);
+    const T *x = (const T *)a.x, *Bm = (const T *)a.B, *Cm = (const T *)a.C;
+    extern __shared__ float sm[];
+    float *cs = sm, *dts = cs + kOneQ, *Bs = dts + kOneQ, *Cs = Bs + Q * NP, *xs = Cs + Q * NP, *Ms = xs + Q * P;
+
+    // every global load first
+    uint4 vb[NB], vc[NB], vx[NX];
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+        const int i = tid + kThreads * j;
+        if (i < Q * (N / V)) {
+            const int s = i / (N / V), cv = i % (N / V);
+            const size_t off = (((size_t)b * a.L + tok(s, a.L, a.dir)) * a.G + g) * N + cv * V;
+            vb[j] = __ldg(reinterpret_cast<const uint4 *>(Bm + off));
+            vc[j] = __ldg(reinterpret_cast<const uint4 *>(Cm + off));
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < NX; ++j) {
+        const int i = tid + kThreads * j;
+        if (i < Q * (P / V)) {
+            const int s = i / (P / V), cv = i % (P / V);
+            const size_t off = (((size_t)b * a.L + tok(s, a.L, a.dir)) * a.H + h) * P + cv * V;
+            vx[j] = __ldg(reinterpret_cast<const uint4 *>(x + off));
+        }
+    }
+    float dtv = 0.f;
+    if (tid < Q) dtv = ldf<T>((const T *)a.dt, ((size_t)b * a.L + tok(tid, a.L, a.dir)) * a.H + h);
+    // what the result is added to: the residual (OUT_GATE) or the output so far (OUT_ACCUM)
+    const T *addend = a.mode == OUT_GATE ? (const T *)a.residual : a.mode == OUT_ACCUM ? (const T *)a.y : nullptr;
+    float add0[NO], add1[NO];
+#pragma unroll
+    for (int j = 0; j < NO; ++j) {
+        const int o = tid + kThreads * j;
+        add0[j] = add1[j] = 0.f;
+        if (addend && o < Q * H2) {
+            const size_t row = (((size_t)b * a.L + tok(o / H2, a.L, a.dir)) * a.H + h) * P + o % H2;
+            add0[j] = ldf<T>(addend, row);
+            add1[j] = ldf<T>(addend, row + H2);
+        }
+    }
+
+    // cs = A * inclusive prefix sum of dt in scan order: warp scans, then the warps in order
+    // (the additions of chunk_cumsum, so the same values)
+    float sc = dtv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, sc, o);
+        if (lane >= o) sc += u;
+    }
+    if (lane == 31 && warp < kOneQ / 32) warp_tot[warp] = sc;
+    if (tid < Q) dts[tid] = dtv;
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+        const int i = tid + kThreads * j;
+        if (i < Q * (N / V)) {
+            const int s = i / (N / V), cv = i % (N / V);
+            float f[V];
+            unpack16<T>(vb[j], f);
+#pragma unroll
+            for (int e = 0; e < V; ++e) Bs[s * NP + cv * V + e] = f[e];
+            unpack16<T>(vc[j], f);
+#pragma unroll
+            for (int e = 0; e < V; ++e) Cs[s * NP + cv * V + e] = f[e];
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < NX; ++j) {
+        const int i = tid + kThreads * j;
+        if (i < Q * (P / V)) {
+            float f[V];
+            unpack16<T>(vx[j], f);
+#pragma unroll
+            for (int e = 0; e < V; ++e) xs[i * V + e] = f[e];
+        }
+    }
+    __syncthreads();
+    if (tid < Q) {
+        float base = 0.f;
+        for (int w = 0; w < warp; ++w) base += warp_tot[w];
+        cs[tid] = a.A[h] * (base + sc);
+    }
+    __syncthreads();
+
+    // decayed scores M[k][s] for the Q (Q + 1) / 2 pairs s <= k only (pair e: row k with
+    // k (k + 1) / 2 <= e < (k + 1) (k + 2) / 2, column s = e - k (k + 1) / 2)
+    const int npair = Q * (Q + 1) / 2;
+#pragma unroll 1
+    for (int e = tid; e < npair; e += kThreads) {
+        int k = (int)((sqrtf(8.f * (float)e + 1.f) - 1.f) * 0.5f);
+        while (k * (k + 1) / 2 > e) --k;
+        while ((k + 1) * (k + 2) / 2 <= e) ++k;
+        const int s = e - k * (k + 1) / 2;
+        float d0 = 0.f, d1 = 0.f;
+#pragma unroll 8
+        for (int n = 0; n < N; n += 2) {
+            d0 = fmaf(Cs[k * NP + n], Bs[s * NP + n], d0);
+            d1 = fmaf(Cs[k * NP + n + 1], Bs[s * NP + n + 1], d1);
+        }
+        Ms[k * Q + s] = (d0 + d1) * expf(cs[k] - cs[s]) * dts[s];
+    }
+    __syncthreads();
+
+    // y[k][p] = sum_{s <= k} M[k][s] x[s][p] + D x[k][p] for p and p + P/2, then the output mode
+    const float dh = a.D ? a.D[h] : 0.f;
+    T *y = (T *)a.y;
+#pragma unroll
+    for (int j = 0; j < NO; ++j) {
+        const int o = tid + kThreads * j;
+        if (o < Q * H2) {
+            const int k = o / H2, p = o % H2;
+            float y0 = 0.f, y1 = 0.f;
+#pragma unroll 2
+            for (int s = 0; s <= k; ++s) {
+                const float m = Ms[k * Q + s];
+                y0 = fmaf(m, xs[s * P + p], y0);
+                y1 = fmaf(m, xs[s * P + p + H2], y1);
+            }
+            const float v0 = fmaf(dh, xs[k * P + p], y0), v1 = fmaf(dh, xs[k * P + p + H2], y1);
+            const size_t idx = (((size_t)b * a.L + tok(k, a.L, a.dir)) * a.H + h) * P + p;
+            if (a.mode == OUT_WRITE) {
+                stf<T>(y, idx, v0);
+                stf<T>(y, idx + H2, v1);
+            } else if (a.mode == OUT_ACCUM) {
+                stf<T>(y, idx, add0[j] + v0);
+                stf<T>(y, idx + H2, add1[j] + v1);
+            } else {
+                stf<T>(y, idx, fmaf(a.gate, v0, add0[j]));
+                stf<T>(y, idx + H2, fmaf(a.gate, v1, add1[j]));
+            }
+        }
+    }
+}
+
 template <typename T, int P, int N>
 cudaError_t launch_typed(const ScanArgs &a, cudaStream_t st) {
     // the state kernels run whenever a state crosses a chunk or the call boundary
     const bool multi = a.nc > 1 || a.s_in || a.s_out;
+    cudaError_t e;
+    if (!multi && a.Q <= kOneQ) {
+        const size_t bytes = sizeof(float) * one_chunk_floats(a.Q, P, N);
+        if (bytes > 48 * 1024) {
+            e = cudaFuncSetAttribute(k_one_chunk<T, P, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+            if (e != cudaSuccess) return e;
+        }
+        k_one_chunk<T, P, N><<<dim3(a.H, a.batch), kThreads, bytes, st>>>(a);
+        return cudaGetLastError();
+    }
     const size_t sm_state = sizeof(float) * (2 * a.Q + kSTile * P + kSTile * N);
     const size_t sm_out = sizeof(float) * (2 * a.Q + kRows * N + (multi ? P * (N + 1) : 0) +
                                            kSTile * (N + 1) + kSTile * P + kRows * kSTile);
-    cudaError_t e;
     if (multi) {
         e = cudaFuncSetAttribute(k_chunk_state<T, P, N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_state);
         if (e != cudaSuccess) return e;

@@ -321,3 +321,39 @@ def test_workspace_needs_only_its_status_word_zeroed(ssd, dims, chunk):
             torch.cuda.synchronize()
             ssd.workspace_status(ws)
             assert torch.equal(y, y_ref)
+
+
+ONE_CHUNK = [
+    # sequences of one chunk (seqlen == chunk <= 64) with no state: the single-chunk kernel
+    (si.Shape(2, 16, 3, 16, 16, 1, "f32"), 16),
+    (si.Shape(2, 32, 4, 64, 128, 2, "f32"), 32),
+    (si.Shape(3, 64, 4, 64, 128, 1, "bf16"), 64),
+    (si.Shape(1, 64, 6, 32, 64, 3, "bf16"), 64),
+    (si.Shape(2, 32, 5, 16, 128, 1, "bf16"), 32),
+]
+
+
+@pytest.mark.parametrize("shape,chunk", ONE_CHUNK, ids=lambda v: str(v) if isinstance(v, int) else
+                         f"b{v.batch}L{v.seqlen}H{v.nheads}P{v.headdim}N{v.dstate}G{v.ngroups}{v.io}")
+def test_single_chunk_calls(ssd, shape, chunk):
+    """Every output mode of a one-chunk call: each direction alone (write), the bidirectional sum
+    (write, then add) and the R2L gate (residual + s y_rev), with and without the skip term."""
+    io = torch.bfloat16 if shape.io == "bf16" else torch.float32
+    assert ssd.path_for(_dims(shape), io, chunk) == 0
+    tol = TOL[shape.io]
+    for with_D in (True, False):
+        assert _bidir_case(ssd, shape, chunk, with_D, seed=21) <= tol
+        p = si.make_params(shape, seed=22, with_D=with_D)
+        q = oracle.params_f64(p)
+        for direction in (1, -1):
+            y = ssd.ssd_scan(**_dev(p, with_D), direction=direction, chunk=chunk)
+            torch.cuda.synchronize()
+            ref = oracle.ssd_scan_f64(q["x"], q["dt"], q["A"], q["B"], q["C"], q.get("D"), direction)
+            assert oracle.rel_err(_f64(y), ref) <= tol, (with_D, direction)
+        gate = 0.37
+        res = si.make_residual(shape, seed=23)
+        for r_dev, r_ref in ((res.torch("cuda"), res.f64()),
+                             (torch.zeros(res.torch().shape, dtype=io, device="cuda"), np.zeros(res.torch().shape))):
+            out = ssd.r2l_block_scan(_dev(p, with_D), gate, r_dev, chunk=chunk)
+            torch.cuda.synchronize()
+            assert oracle.rel_err(_f64(out), oracle.r2l_block_f64(q, gate, r_ref)) <= tol, with_D
