@@ -222,19 +222,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_gemm_bf16(const __grid_cons
 
 // ------------------------------------------------------------------ conv + SiLU, dt softplus
 
-// One thread: 8 consecutive channels of xBC (or 8 heads of dt) over a run of kConvT tokens of
-// one sequence.  The thread first copies every input row it needs (16 bytes each) into its own
+// One thread: 4 consecutive channels of xBC (or 4 heads of dt) over a run of kConvT tokens of
+// one sequence.  The thread first copies every input row it needs (8 bytes each) into its own
 // column of shared memory with cp.async, so all of them are in flight at once and none holds a
 // register; it reads back only what it copied itself, so no barrier is needed.  The taps and
 // bias stay in registers and the inputs slide through a window.  Taps of the forward layer:
 // token t + k - (K - 1); of the reverse layer: t - k + (K - 1) (the run is walked backwards);
-// zero outside the sequence.
+// zero outside the sequence.  Four channels a thread (not eight) halve the staging a thread
+// holds, so twice as many warps fit beside the same shared memory: the kernel is bound by
+// latency, not by its arithmetic.
 constexpr int kConvT = 32, kConvKMax = 8, kConvThreads = 128;
 
-
-// silu(v) = v / (1 + exp(-v)) on a pair: exp(-v) = 2^(-v log2 e) and the reciprocal on the
-// special-function unit (approximate, a few ulp).  Very negative v gives 2^(+big) = inf and a
-// reciprocal of 0, so the result is 0 there without a branch.
 __device__ __forceinline__ float2 silu2(float2 v) {
     const float2 t = mul2(v, make_float2(-1.4426950408889634f, -1.4426950408889634f));
     float e0, e1, r0, r1;
@@ -245,10 +243,10 @@ __device__ __forceinline__ float2 silu2(float2 v) {
     return mul2(v, make_float2(r0, r1));
 }
 
-__device__ __forceinline__ void conv_out(const MixerConvArgs &a, long long tok, int c0, const float2 (&acc)[4]) {
-    uint32_t o[4];
+__device__ __forceinline__ void conv_out(const MixerConvArgs &a, long long tok, int c0, const float2 (&acc)[2]) {
+    uint32_t o[2];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
+    for (int p = 0; p < 2; ++p) {
         const float2 s_ = silu2(acc[p]);
         o[p] = pack_bf16(s_.x, s_.y);
     }
@@ -256,12 +254,12 @@ __device__ __forceinline__ void conv_out(const MixerConvArgs &a, long long tok, 
     if (c0 < a.d_inner) dst = a.x + tok * a.d_inner + c0;
     else if (c0 < a.d_inner + a.N) dst = a.B + tok * a.N + (c0 - a.d_inner);
     else dst = a.C + tok * a.N + (c0 - a.d_inner - a.N);
-    *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(o[0], o[1]);
 }
 
-__device__ __forceinline__ void unpack8(const uint4 &v, float (&f)[8]) {
-    f[0] = bf16lo(v.x); f[1] = bf16hi(v.x); f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
-    f[4] = bf16lo(v.z); f[5] = bf16hi(v.z); f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+__device__ __forceinline__ void unpack2x2(const uint2 &v, float2 (&f)[2]) {
+    f[0] = unpack2(v.x);
+    f[1] = unpack2(v.y);
 }
 __device__ __forceinline__ void unpack4x2(const uint4 &v, float2 (&f)[4]) {
     f[0] = unpack2(v.x); f[1] = unpack2(v.y); f[2] = unpack2(v.z); f[3] = unpack2(v.w);
@@ -271,16 +269,16 @@ __device__ __forceinline__ void unpack4x2(const uint4 &v, float2 (&f)[4]) {
 template <int KT>
 __global__ void __launch_bounds__(kConvThreads) k_conv_silu_dt(MixerConvArgs a) {
     constexpr int KM = KT > 0 ? KT : kConvKMax;
-    extern __shared__ uint4 conv_stage[];   // [kConvT + KM - 1][kConvThreads]
+    extern __shared__ uint2 conv_stage[];   // [kConvT + KM - 1][kConvThreads]
     const int K = KT > 0 ? KT : a.K;
-    const int groups_xbc = a.conv_dim / 8, groups = groups_xbc + a.H / 8;
+    const int groups_xbc = a.conv_dim / 4, groups = groups_xbc + a.H / 4;
     const int gidx = blockIdx.x * kConvThreads + threadIdx.x;
     if (gidx >= groups) return;
     const int runs = a.L / kConvT;
     const int b = blockIdx.y / runs, t0 = (blockIdx.y % runs) * kConvT;
     const long long seq0 = (long long)b * a.L;
     const bool is_dt = gidx >= groups_xbc;
-    const int c0 = is_dt ? 8 * (gidx - groups_xbc) : 8 * gidx;          // channel (or head) of xBC (or dt)
+    const int c0 = is_dt ? 4 * (gidx - groups_xbc) : 4 * gidx;          // channel (or head) of xBC (or dt)
     const int col = is_dt ? a.d_inner + a.conv_dim + c0 : a.d_inner + c0;  // its column in zxbcdt
     const int halo = is_dt ? 0 : K - 1;
     const int step = (is_dt || a.dir > 0) ? 1 : -1;
@@ -288,16 +286,16 @@ __global__ void __launch_bounds__(kConvThreads) k_conv_silu_dt(MixerConvArgs a) 
     // row r of the column: the input at token first + step * (r - halo), zero outside the sequence
     // Two copy groups: the halo and the first half of the run, then the second half, so the
     // first half is computed while the second is still in flight.
-    uint4 *mine = conv_stage + threadIdx.x;
+    uint2 *mine = conv_stage + threadIdx.x;
     auto copy_rows = [&](int r0, int r1) {
         for (int r = r0; r < r1; ++r) {
             const int t = first + step * (r - halo);
-            uint4 *dst = mine + r * kConvThreads;
+            uint2 *dst = mine + r * kConvThreads;
             if (t < 0 || t >= a.L) {
-                *dst = make_uint4(0u, 0u, 0u, 0u);
+                *dst = make_uint2(0u, 0u);
             } else {
                 const __nv_bfloat16 *src = a.zxbcdt + (seq0 + t) * a.d_in_proj + col;
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
             }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
@@ -306,32 +304,32 @@ __global__ void __launch_bounds__(kConvThreads) k_conv_silu_dt(MixerConvArgs a) 
     copy_rows(halo + kConvT / 2, halo + kConvT);
     asm volatile("cp.async.wait_group 1;" ::: "memory");
     if (is_dt) {
-        float bias[8];
+        float bias[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) bias[e] = a.dt_bias[c0 + e];
+        for (int e = 0; e < 4; ++e) bias[e] = a.dt_bias[c0 + e];
 #pragma unroll 4
         for (int i = 0; i < kConvT; ++i) {
             if (i == kConvT / 2) asm volatile("cp.async.wait_group 0;" ::: "memory");
-            float v[8];
-            unpack8(mine[i * kConvThreads], v);
-            uint32_t o[4];
+            float2 v[2];
+            unpack2x2(mine[i * kConvThreads], v);
+            uint32_t o[2];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float r0 = v[2 * e] + bias[2 * e], r1 = v[2 * e + 1] + bias[2 * e + 1];
+            for (int e = 0; e < 2; ++e) {
+                const float r0 = v[e].x + bias[2 * e], r1 = v[e].y + bias[2 * e + 1];
                 // softplus, with the linear branch above 20 (exp would dominate 1 there)
                 const float s0 = r0 > 20.f ? r0 : log1pf(__expf(r0));
                 const float s1 = r1 > 20.f ? r1 : log1pf(__expf(r1));
                 o[e] = pack_bf16(s0, s1);
             }
-            *reinterpret_cast<uint4 *>(a.dt + (seq0 + t0 + i) * a.H + c0) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint2 *>(a.dt + (seq0 + t0 + i) * a.H + c0) = make_uint2(o[0], o[1]);
         }
         return;
     }
     // wr[p][j]: the taps of channels (2p, 2p + 1) that multiply the input j steps back
     // (tap K - 1 - j), 0 past the width
-    float2 wr[4][KM], bias[4];
+    float2 wr[2][KM], bias[2];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
+    for (int p = 0; p < 2; ++p) {
         bias[p] = make_float2(a.conv_b[c0 + 2 * p], a.conv_b[c0 + 2 * p + 1]);
 #pragma unroll
         for (int j = 0; j < KM; ++j)
@@ -341,13 +339,13 @@ __global__ void __launch_bounds__(kConvThreads) k_conv_silu_dt(MixerConvArgs a) 
     }
     // win[j]: the input j steps back in the layer's order.  Before the first token's shift it
     // holds the token j + 1 steps back (rows halo - 1 down to 0, then zeros).
-    float2 win[KM][4];
+    float2 win[KM][2];
 #pragma unroll
     for (int j = 0; j < KM; ++j) {
-        if (j < halo) unpack4x2(mine[(halo - 1 - j) * kConvThreads], win[j]);
+        if (j < halo) unpack2x2(mine[(halo - 1 - j) * kConvThreads], win[j]);
         else {
 #pragma unroll
-            for (int p = 0; p < 4; ++p) win[j][p] = make_float2(0.f, 0.f);
+            for (int p = 0; p < 2; ++p) win[j][p] = make_float2(0.f, 0.f);
         }
     }
     // unrolled by 4 only: a fully unrolled run does not fit the instruction cache
@@ -357,11 +355,11 @@ __global__ void __launch_bounds__(kConvThreads) k_conv_silu_dt(MixerConvArgs a) 
 #pragma unroll
         for (int j = KM - 1; j > 0; --j)
 #pragma unroll
-            for (int p = 0; p < 4; ++p) win[j][p] = win[j - 1][p];
-        unpack4x2(mine[(halo + i) * kConvThreads], win[0]);
-        float2 acc[4];
+            for (int p = 0; p < 2; ++p) win[j][p] = win[j - 1][p];
+        unpack2x2(mine[(halo + i) * kConvThreads], win[0]);
+        float2 acc[2];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
+        for (int p = 0; p < 2; ++p) {
             float2 s_ = bias[p];
 #pragma unroll
             for (int j = 0; j < KM; ++j) s_ = fma2(wr[p][j], win[j][p], s_);
@@ -461,10 +459,10 @@ cudaError_t launch_gemm_bf16(const GemmArgs &g, cudaStream_t st) {
 
 cudaError_t launch_conv_silu_dt(const MixerConvArgs &a, cudaStream_t st) {
     if (a.L % kConvT != 0 || a.K < 1 || a.K > kConvKMax) return cudaErrorInvalidValue;
-    const int groups = a.conv_dim / 8 + a.H / 8;
+    const int groups = a.conv_dim / 4 + a.H / 4;
     dim3 grid((groups + kConvThreads - 1) / kConvThreads, (unsigned)((long long)a.batch * (a.L / kConvT)));
     auto run = [&](auto kernel, int km) -> cudaError_t {
-        const int smem = (kConvT + km - 1) * kConvThreads * (int)sizeof(uint4);
+        const int smem = (kConvT + km - 1) * kConvThreads * (int)sizeof(uint2);
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         kernel<<<grid, kConvThreads, smem, st>>>(a);
