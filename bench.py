@@ -685,7 +685,7 @@ def run_r2l(args) -> None:
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                          "algorithmic_bytes_per_launch": alg_bytes, "bytes_per_token": bpt,
                          "launch_us": us_per_call, "peak_source": peaks["source"] + " hbm_gbs",
-                         "note": "latency-bound: a few MB per call; per-call launch latency dominates"},
+                         "note": "latency-bound: a few MB per call, one launch of the single-chunk kernel per call"},
             "e2e": {"value": e2e_us, "unit": "us", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": nsteps, "overlap": "none: each call's copies and call in order on one stream"},
             "gpu_launches": per_call * nsteps * args.steps,
